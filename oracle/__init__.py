@@ -1,0 +1,133 @@
+"""fp64 CPU oracle for exact attention (forward and backward).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+the benchmark's CPU-baseline / reference leg may import this package.  The
+CUDA product path never calls it and has no CPU fallback.
+
+All functions take float64 arrays shaped (B, H, N, d) (or (BH, N, d)) and
+return float64 results; the C routines are in ``attn_oracle.c`` (see its
+header for the passages each routine follows).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        lp = ctypes.POINTER(ctypes.c_int64)
+        i64, ci, cd = ctypes.c_int64, ctypes.c_int, ctypes.c_double
+        L.oracle_fwd.argtypes = [dp, dp, dp, dp, dp, i64, i64, i64, ci, cd]
+        L.oracle_fwd.restype = None
+        L.oracle_fwd_rows.argtypes = [dp, dp, dp, i64, i64, i64, ci, cd, lp, i64, dp, dp]
+        L.oracle_fwd_rows.restype = None
+        L.oracle_fwd_online.argtypes = [dp, dp, dp, dp, dp, i64, i64, i64, ci, cd, i64]
+        L.oracle_fwd_online.restype = None
+        L.oracle_bwd_heads.argtypes = [dp, dp, dp, dp, i64, i64, i64, ci, cd, lp, i64, dp, dp, dp]
+        L.oracle_bwd_heads.restype = None
+        L.oracle_num_threads.argtypes = []
+        L.oracle_num_threads.restype = ci
+        L.oracle_set_num_threads.argtypes = [ci]
+        L.oracle_set_num_threads.restype = None
+        _lib = L
+    return _lib
+
+
+def _f64(a):
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _p(a, t=ctypes.c_double):
+    return a.ctypes.data_as(ctypes.POINTER(t))
+
+
+def _dims(q):
+    if q.ndim == 4:
+        B, H, N, d = q.shape
+        return B * H, N, d
+    if q.ndim == 3:
+        return q.shape
+    raise ValueError("expected (B,H,N,d) or (BH,N,d)")
+
+
+def num_threads() -> int:
+    return lib().oracle_num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    lib().oracle_set_num_threads(int(n))
+
+
+def fwd(q, k, v, causal: bool, scale: float):
+    """Two-pass exact forward: returns (O, LSE) shaped like q and q.shape[:-1]."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    BH, N, d = _dims(q)
+    o = np.empty_like(q)
+    lse = np.empty(q.shape[:-1], dtype=np.float64)
+    lib().oracle_fwd(_p(q), _p(k), _p(v), _p(o), _p(lse), BH, N, d, int(bool(causal)), float(scale))
+    return o, lse
+
+
+def fwd_rows(q, k, v, causal: bool, scale: float, rows):
+    """Forward for selected rows; ``rows`` are flat indices bh*N + i.
+
+    Returns (O_rows (len, d), LSE_rows (len,))."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    BH, N, d = _dims(q)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    if rows.size and (rows.min() < 0 or rows.max() >= BH * N):
+        raise IndexError("row index out of range")
+    o = np.empty((rows.size, d), dtype=np.float64)
+    lse = np.empty(rows.size, dtype=np.float64)
+    lib().oracle_fwd_rows(_p(q), _p(k), _p(v), BH, N, d, int(bool(causal)), float(scale),
+                          _p(rows, ctypes.c_int64), rows.size, _p(o), _p(lse))
+    return o, lse
+
+
+def fwd_online(q, k, v, causal: bool, scale: float, block: int):
+    """The per-block online-softmax pseudo-code in fp64 (self-check only)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    BH, N, d = _dims(q)
+    o = np.empty_like(q)
+    lse = np.empty(q.shape[:-1], dtype=np.float64)
+    lib().oracle_fwd_online(_p(q), _p(k), _p(v), _p(o), _p(lse), BH, N, d, int(bool(causal)),
+                            float(scale), int(block))
+    return o, lse
+
+
+def bwd_heads(q, k, v, dout, causal: bool, scale: float, heads=None):
+    """Exact gradients of sum(O * dO) for the listed flat heads (bh indices).
+
+    Returns (dQ, dK, dV), each (len(heads), N, d)."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    BH, N, d = _dims(q)
+    if heads is None:
+        heads = np.arange(BH)
+    heads = np.ascontiguousarray(heads, dtype=np.int64)
+    if heads.size and (heads.min() < 0 or heads.max() >= BH):
+        raise IndexError("head index out of range")
+    shp = (heads.size, N, d)
+    dq, dk, dv = np.empty(shp), np.empty(shp), np.empty(shp)
+    lib().oracle_bwd_heads(_p(q), _p(k), _p(v), _p(dout), BH, N, d, int(bool(causal)),
+                           float(scale), _p(heads, ctypes.c_int64), heads.size,
+                           _p(dq), _p(dk), _p(dv))
+    return dq, dk, dv
+
+
+def bwd(q, k, v, dout, causal: bool, scale: float):
+    """Exact gradients for every head, shaped like q."""
+    shape = np.shape(q)
+    dq, dk, dv = bwd_heads(q, k, v, dout, causal, scale)
+    return dq.reshape(shape), dk.reshape(shape), dv.reshape(shape)

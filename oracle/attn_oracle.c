@@ -1,0 +1,253 @@
+/*
+ * fp64 CPU oracle for exact scaled-dot-product attention, forward and
+ * backward.  TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the
+ * benchmark's CPU-baseline leg may call it; the CUDA product path never does.
+ * It shares no code, header or constant with the GPU library.
+ *
+ * Sources (titles of the pages, section named):
+ *  - "Is a full day of context better than ten minutes? FlashAttention and the
+ *    sequence-length question" (marketmaker.cc), section "why attention is
+ *    bound by memory": O = softmax(Q K^T / sqrt(d_k)) V.
+ *    Same page, "online softmax recurrence": a naive softmax takes two passes
+ *    over a row, one for the maximum and one to exponentiate and normalise;
+ *    the tiled method is algebraically the same result.
+ *    Same page, "causal masking": a query never attends to a later key.
+ *    Same page, "Flash Attention algorithm" (the per-block pseudo-code):
+ *    restated by oracle_fwd_online below as a self-check only.
+ *    Same page, "backward: recompute instead of store": gradients need P,
+ *    rebuilt from the stored statistics.
+ *  - "Performance optimisation with Flash-Attention 2" (Medium), section
+ *    "Flash Attention 2": one statistic L (the log-sum-exp) is kept per row.
+ *
+ * The forward is the plain definition, row by row, in two passes (maximum,
+ * then exponentiate/normalise); the score row is the only O(N) scratch.  The
+ * backward is the analytic chain rule of L = sum(O * dO), row by row, with no
+ * N x N storage; rows run in parallel (OpenMP) with per-thread dK/dV partials
+ * that are summed at the end of each head.
+ *
+ * Conventions: every tensor is contiguous (BH, N, d) float64, LSE is (BH, N);
+ * key j is visible to query i iff !causal || j <= i; LSE is natural-log.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static double dot(const double* a, const double* b, int64_t d) {
+    double s = 0.0;
+    for (int64_t k = 0; k < d; ++k) s += a[k] * b[k];
+    return s;
+}
+
+/* One query row: fills s[0..nvis) with probabilities, returns LSE, writes O. */
+static double row_forward(const double* qi, const double* K, const double* V, int64_t nvis,
+                          int64_t d, double scale, double* s, double* oi) {
+    double M = -INFINITY;
+    for (int64_t j = 0; j < nvis; ++j) {          /* scores and pass 1: max */
+        s[j] = scale * dot(qi, K + j * d, d);
+        if (s[j] > M) M = s[j];
+    }
+    double Z = 0.0;
+    for (int64_t j = 0; j < nvis; ++j) {          /* pass 2: exponentiate, sum */
+        s[j] = exp(s[j] - M);
+        Z += s[j];
+    }
+    for (int64_t k = 0; k < d; ++k) oi[k] = 0.0;
+    for (int64_t j = 0; j < nvis; ++j) {          /* normalise, weight V */
+        s[j] /= Z;
+        const double* vj = V + j * d;
+        for (int64_t k = 0; k < d; ++k) oi[k] += s[j] * vj[k];
+    }
+    return M + log(Z);
+}
+
+static int64_t visible(int64_t i, int64_t N, int causal) { return causal ? i + 1 : N; }
+
+/* Forward on a list of rows; rows[r] = bh * N + i.  o_rows is (nrows, d). */
+void oracle_fwd_rows(const double* q, const double* k, const double* v, int64_t BH, int64_t N,
+                     int64_t d, int causal, double scale, const int64_t* rows, int64_t nrows,
+                     double* o_rows, double* lse_rows) {
+    (void)BH;
+#pragma omp parallel
+    {
+        double* s = (double*)malloc((size_t)N * sizeof(double));
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t r = 0; r < nrows; ++r) {
+            int64_t bh = rows[r] / N, i = rows[r] % N;
+            const double* base_k = k + bh * N * d;
+            const double* base_v = v + bh * N * d;
+            lse_rows[r] = row_forward(q + rows[r] * d, base_k, base_v, visible(i, N, causal), d,
+                                      scale, s, o_rows + r * d);
+        }
+        free(s);
+    }
+}
+
+/* Full forward: O (BH, N, d), LSE (BH, N). */
+void oracle_fwd(const double* q, const double* k, const double* v, double* o, double* lse,
+                int64_t BH, int64_t N, int64_t d, int causal, double scale) {
+#pragma omp parallel
+    {
+        double* s = (double*)malloc((size_t)N * sizeof(double));
+#pragma omp for collapse(2) schedule(dynamic, 16)
+        for (int64_t bh = 0; bh < BH; ++bh)
+            for (int64_t i = 0; i < N; ++i) {
+                int64_t row = bh * N + i;
+                lse[row] = row_forward(q + row * d, k + bh * N * d, v + bh * N * d,
+                                       visible(i, N, causal), d, scale, s, o + row * d);
+            }
+        free(s);
+    }
+}
+
+/*
+ * The page's per-block pseudo-code, literally: for each query row, walk the
+ * key/value blocks of width Bc, keep (m, l) and an O that is normalised after
+ * every block (FA1 form).  Blocks lying entirely in the future of the row are
+ * skipped, as the causal-masking section describes.  Self-check only.
+ */
+void oracle_fwd_online(const double* q, const double* k, const double* v, double* o, double* lse,
+                       int64_t BH, int64_t N, int64_t d, int causal, double scale, int64_t Bc) {
+#pragma omp parallel
+    {
+        double* p = (double*)malloc((size_t)Bc * sizeof(double));
+        double* pv = (double*)malloc((size_t)d * sizeof(double));
+#pragma omp for collapse(2) schedule(dynamic, 16)
+        for (int64_t bh = 0; bh < BH; ++bh)
+            for (int64_t i = 0; i < N; ++i) {
+                const double* qi = q + (bh * N + i) * d;
+                double* oi = o + (bh * N + i) * d;
+                double m = -INFINITY, l = 0.0;
+                for (int64_t t = 0; t < d; ++t) oi[t] = 0.0;
+                for (int64_t j0 = 0; j0 < N; j0 += Bc) {
+                    if (causal && j0 > i) break;           /* whole block in the future */
+                    int64_t j1 = j0 + Bc < N ? j0 + Bc : N;
+                    double mij = -INFINITY;
+                    for (int64_t j = j0; j < j1; ++j) {    /* S_ij and its row max */
+                        int vis = !causal || j <= i;
+                        p[j - j0] = vis ? scale * dot(qi, k + (bh * N + j) * d, d) : -INFINITY;
+                        if (p[j - j0] > mij) mij = p[j - j0];
+                    }
+                    double lij = 0.0;
+                    for (int64_t j = j0; j < j1; ++j) {    /* P_ij = exp(S_ij - m_ij), l_ij */
+                        p[j - j0] = exp(p[j - j0] - mij);
+                        lij += p[j - j0];
+                    }
+                    for (int64_t t = 0; t < d; ++t) pv[t] = 0.0;
+                    for (int64_t j = j0; j < j1; ++j) {    /* P_ij V_j */
+                        const double* vj = v + (bh * N + j) * d;
+                        for (int64_t t = 0; t < d; ++t) pv[t] += p[j - j0] * vj[t];
+                    }
+                    double mnew = m > mij ? m : mij;
+                    double a = exp(m - mnew), b = exp(mij - mnew);
+                    double lnew = l * a + lij * b;
+                    for (int64_t t = 0; t < d; ++t)
+                        oi[t] = oi[t] * (l * a / lnew) + pv[t] * (b / lnew);
+                    m = mnew;
+                    l = lnew;
+                }
+                lse[bh * N + i] = m + log(l);
+            }
+        free(pv);
+        free(p);
+    }
+}
+
+/*
+ * Backward of L = sum(O * dO) for the heads listed in heads[0..nheads):
+ * dq/dk/dv are (nheads, N, d), in the order of heads[].  The forward
+ * quantities (P row, O row, D_i) are recomputed here in fp64 from q, k, v, so
+ * the result is the exact gradient of the definition.
+ *
+ *   P_ij = softmax_j(s_ij),  s_ij = scale q_i.k_j (visible j only)
+ *   D_i  = sum_t dO_it O_it            ( = sum_j P_ij dP_ij )
+ *   dP_ij = dO_i . v_j,  dS_ij = P_ij (dP_ij - D_i)
+ *   dq_i = scale sum_j dS_ij k_j,  dk_j += scale dS_ij q_i,  dv_j += P_ij dO_i
+ */
+void oracle_bwd_heads(const double* q, const double* k, const double* v, const double* dout,
+                      int64_t BH, int64_t N, int64_t d, int causal, double scale,
+                      const int64_t* heads, int64_t nheads, double* dq, double* dk, double* dv) {
+    (void)BH;
+    int nthr = 1;
+#ifdef _OPENMP
+    nthr = omp_get_max_threads();
+#endif
+    size_t nd = (size_t)N * (size_t)d;
+    double* part = (double*)calloc((size_t)nthr * 2 * nd, sizeof(double));
+    for (int64_t hh = 0; hh < nheads; ++hh) {
+        int64_t bh = heads[hh];
+        const double* Q = q + bh * N * d;
+        const double* K = k + bh * N * d;
+        const double* V = v + bh * N * d;
+        const double* dO = dout + bh * N * d;
+        double* dQ = dq + hh * N * d;
+        memset(part, 0, (size_t)nthr * 2 * nd * sizeof(double));
+#pragma omp parallel
+        {
+            int tid = 0;
+#ifdef _OPENMP
+            tid = omp_get_thread_num();
+#endif
+            double* dKp = part + (size_t)tid * 2 * nd;
+            double* dVp = dKp + nd;
+            double* p = (double*)malloc((size_t)N * sizeof(double));
+            double* oi = (double*)malloc((size_t)d * sizeof(double));
+#pragma omp for schedule(dynamic, 8)
+            for (int64_t i = 0; i < N; ++i) {
+                int64_t nv = visible(i, N, causal);
+                const double* qi = Q + i * d;
+                const double* doi = dO + i * d;
+                row_forward(qi, K, V, nv, d, scale, p, oi);
+                double Di = dot(doi, oi, d);
+                double* dqi = dQ + i * d;
+                for (int64_t t = 0; t < d; ++t) dqi[t] = 0.0;
+                for (int64_t j = 0; j < nv; ++j) {
+                    const double* vj = V + j * d;
+                    const double* kj = K + j * d;
+                    double dpij = dot(doi, vj, d);
+                    double dsij = p[j] * (dpij - Di);
+                    double* dkj = dKp + j * d;
+                    double* dvj = dVp + j * d;
+                    for (int64_t t = 0; t < d; ++t) {
+                        dqi[t] += scale * dsij * kj[t];
+                        dkj[t] += scale * dsij * qi[t];
+                        dvj[t] += p[j] * doi[t];
+                    }
+                }
+            }
+            free(oi);
+            free(p);
+        }
+        double* dK = dk + hh * N * d;
+        double* dV = dv + hh * N * d;
+        for (size_t e = 0; e < nd; ++e) {
+            double sk = 0.0, sv = 0.0;
+            for (int t = 0; t < nthr; ++t) {
+                sk += part[(size_t)t * 2 * nd + e];
+                sv += part[(size_t)t * 2 * nd + nd + e];
+            }
+            dK[e] = sk;
+            dV[e] = sv;
+        }
+    }
+    free(part);
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
