@@ -1,0 +1,130 @@
+/*
+ * attn.h — C ABI of libattn.so: exact scaled-dot-product attention on B200
+ * (sm_100a), forward with the online-softmax recurrence and a backward that
+ * recomputes the probabilities from the stored output and log-sum-exp.
+ *
+ * The operation (web pages on IO-aware exact attention):
+ *  - O = softmax(Q K^T / sqrt(d) [+ causal mask]) V — "Is a full day of
+ *    context better than ten minutes? FlashAttention and the sequence-length
+ *    question" (marketmaker.cc), section "why attention is bound by memory";
+ *    tensors are (batch, heads, seq, head_dim), half precision, and the causal
+ *    mask is built inside the kernel — same page, section "integration is
+ *    eight lines".
+ *  - The N x N score matrix never reaches device memory: tiles of Q, K, V are
+ *    staged on chip and the softmax is renormalised block by block — same
+ *    page, sections "Flash Attention algorithm" and "online softmax
+ *    recurrence".  Blocks wholly in the future of a query block are skipped —
+ *    section "causal masking".
+ *  - The backward keeps only O and one softmax statistic per row and
+ *    recomputes P tile by tile — same page, section "backward: recompute
+ *    instead of store"; the statistic is the log-sum-exp L — "Performance
+ *    optimisation with Flash-Attention 2" (Medium), section "Flash Attention 2".
+ *
+ * Conventions shared by every entry point
+ *  - Layout: q, k, v, o, dout, dq, dk, dv are contiguous (B, H, N, d) arrays of
+ *    the same element type (bf16 or fp16); lse is a contiguous (B, H, N) fp32
+ *    array holding the natural-log log-sum-exp of the scaled scores of each
+ *    query row: lse = ln sum_j exp(scale * q_i . k_j) over the visible keys.
+ *  - Key j is visible to query i iff causal == 0 or j <= i.
+ *  - d must be 64 or 128; 1 <= N; 1 <= B, H; B * H * N * d < 2^31 elements;
+ *    every pointer must be device memory aligned to 16 bytes.
+ *  - scale is the score multiplier, usually 1/sqrt(d); it must be finite and > 0.
+ *  - Ownership: the caller allocates and frees every buffer (torch or
+ *    cudaMalloc).  The library never allocates or frees device memory inside
+ *    these calls and never materialises an N x N array; it caches tensor-map
+ *    descriptors per call only (they are kernel parameters).
+ *  - Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *    All launches are asynchronous on it; outputs are valid once the stream
+ *    reaches the end of the call.
+ *  - Errors: argument errors are returned synchronously and nothing is
+ *    launched; launch failures map to ATTN_ERR_LAUNCH.  Every wait inside a
+ *    kernel is bounded in time; a wait that runs out sets a device error word
+ *    and the kernel frees its tensor memory and returns, after which
+ *    attn_last_device_status() reports ATTN_ERR_TIMEOUT.  No exception or
+ *    abort crosses the ABI.
+ *  - Inputs must be finite; NaN/Inf inputs are outside the contract.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { ATTN_BF16 = 0, ATTN_FP16 = 1 } attn_dtype_t;
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_NULL = -1,     /* a required pointer is NULL */
+    ATTN_ERR_SHAPE = -2,    /* B, H or N < 1, or the tensor is too large */
+    ATTN_ERR_HEADDIM = -3,  /* d not in {64, 128} */
+    ATTN_ERR_ALIGN = -4,    /* a pointer is not 16-byte aligned */
+    ATTN_ERR_DTYPE = -5,    /* dtype not bf16/fp16 */
+    ATTN_ERR_DEVICE = -6,   /* no sm_100 device current, or a pointer is not device memory */
+    ATTN_ERR_LAUNCH = -7,   /* the CUDA runtime rejected a launch */
+    ATTN_ERR_TIMEOUT = -8,  /* a bounded in-kernel wait ran out (device status) */
+    ATTN_ERR_ARG = -9       /* scale not finite and positive, or another bad scalar */
+} attn_status_t;
+
+/*
+ * Forward.  Reads q, k, v; writes o (same dtype, rounded to nearest even) and
+ * lse (fp32).  Computes, for every (b, h) and query row i, the exact softmax
+ * weights over the visible keys and their weighted sum of v rows, one query
+ * tile of 128 rows at a time, streaming 128-key tiles of k and v through
+ * shared memory with the running max / running sum recurrence.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+             int B, int H, int N, int d, int causal, float scale,
+             attn_dtype_t dtype, void* stream);
+
+/*
+ * Bytes of device scratch attn_bwd needs: D (B*H*N fp32, the row dot products
+ * of dO and O) followed by the fp32 dQ accumulator (B*H*N*d), each section
+ * 256-byte aligned.  Returns 0 for invalid sizes.
+ */
+size_t attn_bwd_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * Backward of the forward above for an upstream gradient dout.  Reads q, k, v,
+ * o and lse exactly as attn_fwd wrote them (the probabilities are recomputed
+ * from lse, never stored), and dout; writes dq, dk, dv (same dtype as q).
+ * `workspace` is caller-owned device memory of attn_bwd_workspace_bytes()
+ * bytes, 256-byte aligned; its contents on entry do not matter and are
+ * overwritten.  dq accumulates across key tiles in fp32 by atomic addition,
+ * so its last bits may differ between runs; dk and dv are deterministic.
+ */
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+             const void* dout, void* dq, void* dk, void* dv, void* workspace,
+             int B, int H, int N, int d, int causal, float scale,
+             attn_dtype_t dtype, void* stream);
+
+/*
+ * Synchronises `stream`, then returns ATTN_OK, ATTN_ERR_TIMEOUT if a kernel
+ * of this library recorded a wait that ran out since the last call, or
+ * ATTN_ERR_LAUNCH if the stream reported a CUDA error.  Clears the device
+ * error word of the current device.
+ */
+int attn_last_device_status(void* stream);
+
+/*
+ * Diagnostic: launches one block that waits on a shared-memory barrier that
+ * nothing ever completes, with the library's bounded wait and the given
+ * limit in microseconds (1 .. 10^7).  The wait runs out, the kernel records
+ * ATTN_ERR_TIMEOUT in the device error word and returns; the context stays
+ * usable.  Lets tests exercise the timeout path without a fault or a hang.
+ */
+int attn_selftest_wait_timeout(unsigned timeout_us, void* stream);
+
+/* Static description of a status code. */
+const char* attn_strerror(int status);
+
+/* Library version, e.g. "0.1.0". */
+const char* attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

@@ -1,0 +1,173 @@
+"""Python binding of libattn.so — argument marshalling only.
+
+Every step of the attention path runs in the library's CUDA kernels; this
+module converts torch tensors to pointers and sizes, passes the current CUDA
+stream, and raises on a non-zero status.  There is no CPU fallback: if the
+library is missing or the device is not sm_100, calls raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libattn.so")
+
+ATTN_BF16, ATTN_FP16 = 0, 1
+_DTYPES = {torch.bfloat16: ATTN_BF16, torch.float16: ATTN_FP16}
+
+STATUS = {
+    0: "ATTN_OK", -1: "ATTN_ERR_NULL", -2: "ATTN_ERR_SHAPE", -3: "ATTN_ERR_HEADDIM",
+    -4: "ATTN_ERR_ALIGN", -5: "ATTN_ERR_DTYPE", -6: "ATTN_ERR_DEVICE", -7: "ATTN_ERR_LAUNCH",
+    -8: "ATTN_ERR_TIMEOUT", -9: "ATTN_ERR_ARG",
+}
+
+# Every symbol include/attn.h declares.
+EXPORTS = ("attn_fwd", "attn_bwd", "attn_bwd_workspace_bytes", "attn_last_device_status",
+           "attn_selftest_wait_timeout", "attn_strerror", "attn_version")
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({strerror(status)})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libattn.so from the package directory (never from elsewhere)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built: run `python -m io_aware_exact_30_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, ci, cf, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp]
+        L.attn_fwd.restype = ci
+        L.attn_bwd.argtypes = [vp] * 10 + [ci, ci, ci, ci, ci, cf, ci, vp]
+        L.attn_bwd.restype = ci
+        L.attn_bwd_workspace_bytes.argtypes = [ci, ci, ci, ci]
+        L.attn_bwd_workspace_bytes.restype = sz
+        L.attn_last_device_status.argtypes = [vp]
+        L.attn_last_device_status.restype = ci
+        L.attn_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
+        L.attn_selftest_wait_timeout.restype = ci
+        L.attn_strerror.argtypes = [ci]
+        L.attn_strerror.restype = ctypes.c_char_p
+        L.attn_version.argtypes = []
+        L.attn_version.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def strerror(status: int) -> str:
+    return lib().attn_strerror(int(status)).decode()
+
+
+def version() -> str:
+    return lib().attn_version().decode()
+
+
+def _stream(device, stream):
+    if stream is not None:
+        return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise AttnError(rc, where)
+
+
+def _shape(q):
+    if q.dim() != 4:
+        raise ValueError("q must be (B, H, N, d)")
+    return q.shape
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _dtype(q):
+    if q.dtype not in _DTYPES:
+        raise TypeError(f"dtype must be bfloat16 or float16, got {q.dtype}")
+    return _DTYPES[q.dtype]
+
+
+def _same(ref, *ts, names):
+    for t, n in zip(ts, names):
+        if t.dtype != ref.dtype or t.shape != ref.shape or not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous with the shape and dtype of q")
+
+
+def attn_fwd(q, k, v, o, lse, causal: bool, scale: float | None = None, stream=None) -> None:
+    """O, LSE <- attention(q, k, v); all tensors caller-allocated, (B, H, N, d) / (B, H, N)."""
+    B, H, N, d = _shape(q)
+    _same(q, k, v, o, names=("k", "v", "o"))
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 (B, H, N) tensor")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, int(bool(causal)),
+                        scale, _dtype(q), ctypes.c_void_p(_stream(q.device, stream)))
+    _check(rc, "attn_fwd")
+
+
+def attn_bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(lib().attn_bwd_workspace_bytes(B, H, N, d))
+
+
+def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, causal: bool,
+             scale: float | None = None, stream=None) -> None:
+    """dQ, dK, dV <- gradients of sum(O * dout), recomputing P from lse."""
+    B, H, N, d = _shape(q)
+    _same(q, k, v, o, dout, dq, dk, dv, names=("k", "v", "o", "dout", "dq", "dk", "dv"))
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 (B, H, N) tensor")
+    need = attn_bwd_workspace_bytes(B, H, N, d)
+    if workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace needs {need} bytes")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+                        _ptr(dv), _ptr(workspace), B, H, N, d, int(bool(causal)), scale, _dtype(q),
+                        ctypes.c_void_p(_stream(q.device, stream)))
+    _check(rc, "attn_bwd")
+
+
+def attn_last_device_status(stream=None, device=None) -> int:
+    st = _stream(device or torch.cuda.current_device(), stream)
+    return int(lib().attn_last_device_status(ctypes.c_void_p(st)))
+
+
+def attn_selftest_wait_timeout(timeout_us: int, stream=None) -> None:
+    st = _stream(torch.cuda.current_device(), stream)
+    _check(lib().attn_selftest_wait_timeout(int(timeout_us), ctypes.c_void_p(st)),
+           "attn_selftest_wait_timeout")
+
+
+# ------------------------------------------------------------ conveniences --
+def forward(q, k, v, causal: bool = False, scale: float | None = None):
+    """Allocates O and LSE with torch and runs attn_fwd; returns (o, lse)."""
+    B, H, N, d = _shape(q)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    attn_fwd(q, k, v, o, lse, causal, scale)
+    return o, lse
+
+
+def backward(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None,
+             workspace=None):
+    """Allocates dQ, dK, dV (and the workspace if not given); returns (dq, dk, dv)."""
+    B, H, N, d = _shape(q)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if workspace is None:
+        workspace = torch.empty(attn_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8,
+                                device=q.device)
+    attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, causal, scale)
+    return dq, dk, dv

@@ -1,0 +1,89 @@
+"""Shared test helpers: seeded inputs for both paths and the parity bars.
+
+Tolerances (for bf16/fp16 inputs, against the fp64 oracle):
+forward O max-abs <= 1e-2 and relative L2 <= 5e-3; LSE max-abs <= 1e-3;
+dQ, dK, dV relative L2 <= 1e-2.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+from io_aware_exact_30_b200 import synth
+
+O_MAX_ABS = 1e-2
+O_REL_L2 = 5e-3
+LSE_MAX_ABS = 1e-3
+GRAD_REL_L2 = 1e-2
+
+# The five workloads: (B, H, N, d, causal, dtype, sigma, backward?)
+CONFIGS = {
+    "tiny": (1, 2, 256, 64, False, "bf16", 1.0, False),
+    "bert_large": (8, 16, 512, 64, False, "bf16", 1.0, False),
+    "gpt2_causal": (8, 12, 1024, 64, True, "bf16", 1.0, True),
+    "long_day": (1, 12, 23400, 64, True, "fp16", 0.5, False),
+    "large_head": (4, 16, 4096, 128, True, "bf16", 1.0, True),
+}
+
+
+def inputs(B, H, N, d, dtype="bf16", sigma=1.0, seed=0, with_dout=False):
+    """Storage arrays from the seeded generator plus their exact f64 values."""
+    arrs = synth.attention_inputs(B, H, N, d, seed=seed, sigma=sigma, dtype=dtype,
+                                  with_dout=with_dout)
+    return arrs, [synth.to_f64(a, dtype) for a in arrs]
+
+
+def to_device(arr, dtype):
+    import torch
+    if dtype == "bf16":
+        t = torch.from_numpy(arr.view(np.int16)).view(torch.bfloat16)
+    else:
+        t = torch.from_numpy(arr)
+    return t.cuda().contiguous()
+
+
+def rel_l2(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def max_abs(a, b):
+    return float(np.max(np.abs(np.asarray(a, np.float64) - np.asarray(b, np.float64)))) if np.size(a) else 0.0
+
+
+def check_fwd(o_gpu, lse_gpu, o_ref, lse_ref, label=""):
+    ma, rl, la = max_abs(o_gpu, o_ref), rel_l2(o_gpu, o_ref), max_abs(lse_gpu, lse_ref)
+    assert np.all(np.isfinite(o_gpu)) and np.all(np.isfinite(lse_gpu)), label
+    assert ma <= O_MAX_ABS, f"{label} O max-abs {ma}"
+    assert rl <= O_REL_L2, f"{label} O rel-L2 {rl}"
+    assert la <= LSE_MAX_ABS, f"{label} LSE max-abs {la}"
+    return ma, rl, la
+
+
+def check_grads(g_gpu, g_ref, label=""):
+    errs = []
+    for name, a, b in zip(("dQ", "dK", "dV"), g_gpu, g_ref):
+        assert np.all(np.isfinite(a)), f"{label} {name} not finite"
+        e = rel_l2(a, b)
+        assert e <= GRAD_REL_L2, f"{label} {name} rel-L2 {e}"
+        errs.append(e)
+    return errs
+
+
+def sample_rows(BH, N, per_head=24, seed=1):
+    """Flat row indices bh*N + i: tile edges, first/last rows and random rows."""
+    rng = np.random.default_rng(seed)
+    edge = {0, 1, 127, 128, 129, N // 2, N - 129, N - 128, N - 2, N - 1}
+    edge = sorted(i for i in edge if 0 <= i < N)
+    rows = []
+    for bh in range(BH):
+        extra = rng.choice(N, size=min(N, per_head), replace=False)
+        rows.extend(bh * N + i for i in sorted(set(edge) | set(int(x) for x in extra)))
+    return np.array(rows, dtype=np.int64)
+
+
+def default_scale(d):
+    return 1.0 / math.sqrt(d)
