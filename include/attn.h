@@ -81,8 +81,9 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 
 /*
  * Bytes of device scratch attn_bwd needs: D (B*H*N fp32, the row dot products
- * of dO and O) followed by the fp32 dQ accumulator (B*H*N*d), each section
- * 256-byte aligned.  Returns 0 for invalid sizes.
+ * of dO and O), the fp32 dQ accumulator (B*H*N*d) and one int32 completion
+ * counter per (b, h), each section 256-byte aligned.  Returns 0 for invalid
+ * sizes.
  */
 size_t attn_bwd_workspace_bytes(int B, int H, int N, int d);
 
@@ -99,6 +100,28 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
              const void* dout, void* dq, void* dk, void* dv, void* workspace,
              int B, int H, int N, int d, int causal, float scale,
              attn_dtype_t dtype, void* stream);
+
+/*
+ * The two phases attn_bwd runs, for callers that want to schedule or time them
+ * separately; calling attn_bwd_prep then attn_bwd_main on the same stream
+ * and workspace is exactly attn_bwd.
+ *
+ * attn_bwd_prep: D_i = sum_t dout_it * o_it (fp32, one per query row) into the
+ * workspace, and clears the workspace's fp32 dQ accumulator and per-head
+ * completion counters.  Reads o and dout only.
+ *
+ * attn_bwd_main: for every 128-key tile, recomputes S and P per 128-query tile
+ * from q, k and lse (never storing P), forms dV, dK in tensor memory and adds
+ * the dQ contributions into the workspace accumulator; the last tile of each
+ * head to finish converts that head's dQ into dq.  Requires the workspace as
+ * attn_bwd_prep left it.
+ */
+int attn_bwd_prep(const void* o, const void* dout, void* workspace, int B, int H, int N, int d,
+                  attn_dtype_t dtype, void* stream);
+
+int attn_bwd_main(const void* q, const void* k, const void* v, const float* lse,
+                  const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H,
+                  int N, int d, int causal, float scale, attn_dtype_t dtype, void* stream);
 
 /*
  * Synchronises `stream`, then returns ATTN_OK, ATTN_ERR_TIMEOUT if a kernel

@@ -186,29 +186,87 @@ size_t attn_bwd_workspace_bytes(int B, int H, int N, int d) {
     return attn::bwd_workspace_bytes(B, H, N, d);
 }
 
-int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-             const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H, int N,
-             int d, int causal, float scale, attn_dtype_t dtype, void* stream) {
-    if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
-        return ATTN_ERR_NULL;
+namespace {
+int bwd_common_checks(const void* const* ptrs, int nptr, const void* workspace, int B, int H,
+                      int N, int d, attn_dtype_t dtype, float scale, int* dev) {
+    for (int i = 0; i < nptr; ++i)
+        if (!ptrs[i]) return ATTN_ERR_NULL;
     int rc = check_shape(B, H, N, d, dtype, scale);
     if (rc) return rc;
-    const void* ptrs[10] = {q, k, v, o, lse, dout, dq, dk, dv, workspace};
-    for (const void* ptr : ptrs)
-        if (!aligned16(ptr)) return ATTN_ERR_ALIGN;
+    for (int i = 0; i < nptr; ++i)
+        if (!aligned16(ptrs[i])) return ATTN_ERR_ALIGN;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_ALIGN;
-    int dev;
-    if ((rc = check_device(&dev))) return rc;
-    for (const void* ptr : ptrs)
-        if (!on_device(ptr, dev)) return ATTN_ERR_DEVICE;
+    if ((rc = check_device(dev))) return rc;
+    for (int i = 0; i < nptr; ++i)
+        if (!on_device(ptrs[i], *dev)) return ATTN_ERR_DEVICE;
+    return ATTN_OK;
+}
+
+int bwd_prep_dispatch(const void* o, const void* dout, void* workspace, int B, int H, int N,
+                      int d, attn_dtype_t dtype, cudaStream_t st) {
+    const bool bf = dtype == ATTN_BF16;
+    if (d == 64)
+        return bf ? attn::bwd_prep_launch<64, true>(o, dout, workspace, B, H, N, st)
+                  : attn::bwd_prep_launch<64, false>(o, dout, workspace, B, H, N, st);
+    return bf ? attn::bwd_prep_launch<128, true>(o, dout, workspace, B, H, N, st)
+              : attn::bwd_prep_launch<128, false>(o, dout, workspace, B, H, N, st);
+}
+
+int bwd_main_dispatch(const void* q, const void* k, const void* v, const float* lse,
+                      const void* dout, void* dq, void* dk, void* dv, void* workspace, int B,
+                      int H, int N, int d, int causal, float scale, attn_dtype_t dtype,
+                      cudaStream_t st) {
     const int BH = B * H;
     CUtensorMap mq, mk, mv, mdo;
     if (!make_map(&mq, q, dtype, BH, N, d) || !make_map(&mk, k, dtype, BH, N, d) ||
         !make_map(&mv, v, dtype, BH, N, d) || !make_map(&mdo, dout, dtype, BH, N, d))
         return ATTN_ERR_LAUNCH;
-    return attn::bwd_launch(mq, mk, mv, mdo, o, lse, dout, dq, dk, dv, workspace, BH, N, d,
-                            causal ? 1 : 0, scale, dtype == ATTN_BF16,
-                            static_cast<cudaStream_t>(stream));
+    const bool bf = dtype == ATTN_BF16;
+    const int c = causal ? 1 : 0;
+    if (d == 64)
+        return bf ? attn::bwd_main_launch<64, true>(mq, mk, mv, mdo, lse, dq, dk, dv, workspace, B,
+                                                    H, N, c, scale, st)
+                  : attn::bwd_main_launch<64, false>(mq, mk, mv, mdo, lse, dq, dk, dv, workspace,
+                                                     B, H, N, c, scale, st);
+    return bf ? attn::bwd_main_launch<128, true>(mq, mk, mv, mdo, lse, dq, dk, dv, workspace, B, H,
+                                                 N, c, scale, st)
+              : attn::bwd_main_launch<128, false>(mq, mk, mv, mdo, lse, dq, dk, dv, workspace, B,
+                                                  H, N, c, scale, st);
+}
+}  // namespace
+
+int attn_bwd_prep(const void* o, const void* dout, void* workspace, int B, int H, int N, int d,
+                  attn_dtype_t dtype, void* stream) {
+    const void* ptrs[3] = {o, dout, workspace};
+    int dev;
+    int rc = bwd_common_checks(ptrs, 3, workspace, B, H, N, d, dtype, 1.f, &dev);
+    if (rc) return rc;
+    return bwd_prep_dispatch(o, dout, workspace, B, H, N, d, dtype,
+                             static_cast<cudaStream_t>(stream));
+}
+
+int attn_bwd_main(const void* q, const void* k, const void* v, const float* lse,
+                  const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H,
+                  int N, int d, int causal, float scale, attn_dtype_t dtype, void* stream) {
+    const void* ptrs[9] = {q, k, v, lse, dout, dq, dk, dv, workspace};
+    int dev;
+    int rc = bwd_common_checks(ptrs, 9, workspace, B, H, N, d, dtype, scale, &dev);
+    if (rc) return rc;
+    return bwd_main_dispatch(q, k, v, lse, dout, dq, dk, dv, workspace, B, H, N, d, causal, scale,
+                             dtype, static_cast<cudaStream_t>(stream));
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+             const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H, int N,
+             int d, int causal, float scale, attn_dtype_t dtype, void* stream) {
+    const void* ptrs[10] = {q, k, v, o, lse, dout, dq, dk, dv, workspace};
+    int dev;
+    int rc = bwd_common_checks(ptrs, 10, workspace, B, H, N, d, dtype, scale, &dev);
+    if (rc) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((rc = bwd_prep_dispatch(o, dout, workspace, B, H, N, d, dtype, st))) return rc;
+    return bwd_main_dispatch(q, k, v, lse, dout, dq, dk, dv, workspace, B, H, N, d, causal, scale,
+                             dtype, st);
 }
 
 int attn_last_device_status(void* stream) {

@@ -1,4 +1,37 @@
-// Backward kernels (placeholder until the recompute backward lands).
+// Backward kernels: gradients of sum(O * dO) for exact attention, with the
+// probabilities recomputed tile by tile from the stored log-sum-exp instead
+// of being stored by the forward.
+//
+// Method: "Is a full day of context better than ten minutes? FlashAttention
+// and the sequence-length question" (marketmaker.cc), section "backward:
+// recompute instead of store" (only O and the per-row softmax statistic are
+// kept, P is rebuilt from Q, K per tile — gradient checkpointing at tile
+// granularity) and section "causal masking" (key/query tile pairs wholly in
+// the future are skipped); the statistic is the log-sum-exp L —
+// "Performance optimisation with Flash-Attention 2" (Medium), section
+// "Flash Attention 2".  The chain rule itself is not on the pages; with
+// s_ij = scale q_i.k_j, P_ij = exp(s_ij - L_i), D_i = sum_t dO_it O_it:
+//   dV_j = sum_i P_ij dO_i,  dP_ij = dO_i.v_j,  dS_ij = P_ij (dP_ij - D_i),
+//   dK_j = scale sum_i dS_ij q_i,  dQ_i = scale sum_j dS_ij k_j.
+//
+// Kernels
+//   attn_bwd_prep_kernel  D_i = rowdot(dO_i, O_i) (fp32), zero the fp32 dQ
+//                         accumulator and the per-head completion counters.
+//   attn_bwd_main_kernel  one CTA per (head, 128-key tile j): K_j, V_j stay in
+//                         shared memory; for every query tile i the MMAs form
+//                         S^T = K_j Q_i^T and dP^T = V_j dO_i^T in tensor
+//                         memory, the compute warps turn them into P^T and
+//                         dS^T (bf16/fp16, shared memory), and the MMAs
+//                         accumulate dV_j += P^T dO_i, dK_j += dS^T Q_i in
+//                         tensor memory and form dQ_i = dS K_j, which the
+//                         compute warps add into the fp32 accumulator with
+//                         vector atomics.  The last CTA of a head to finish
+//                         converts that head's dQ to the output type.
+//
+// Roles (192 threads): warps 0-3 compute (thread t = TMEM lane t: key row t
+// for P^T/dS^T/dK/dV, query row t for dQ), warp 4 TMA, warp 5 MMA + TMEM.
+// Tensor memory (512 columns): S^T at 0 (reused for dQ once S^T is consumed),
+// dP^T at 128, dV at 256, dK at 256 + D.
 #pragma once
 
 #include "ptx.cuh"
@@ -7,17 +40,451 @@ namespace attn {
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Workspace: D (BH*N fp32) | dQ accumulator (BH*N*d fp32) | counters (BH int32).
+inline size_t bwd_ws_off_dq(int B, int H, int N) {
+    return align256(static_cast<size_t>(B) * H * N * 4);
+}
+inline size_t bwd_ws_off_cnt(int B, int H, int N, int d) {
+    return bwd_ws_off_dq(B, H, N) + align256(static_cast<size_t>(B) * H * N * d * 4);
+}
 inline size_t bwd_workspace_bytes(int B, int H, int N, int d) {
-    const size_t rows = static_cast<size_t>(B) * H * N;
-    return align256(rows * 4) + align256(rows * d * 4);
+    return bwd_ws_off_cnt(B, H, N, d) + align256(static_cast<size_t>(B) * H * 4);
 }
 
-inline bool bwd_set_attributes() { return true; }
+// ------------------------------------------------------------------ prep --
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const uint4* __restrict__ o,
+                                                            const uint4* __restrict__ dout,
+                                                            float* __restrict__ dvec,
+                                                            float4* __restrict__ dqacc,
+                                                            int* __restrict__ counters,
+                                                            long long rows, int BH) {
+    constexpr int TPR = D / 8;  // threads per row, 8 elements (16 bytes) each
+    const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const long long row = gid / TPR;
+    const int part = static_cast<int>(gid % TPR);
+    float acc = 0.f;
+    if (row < rows) {
+        const uint4 a = o[row * TPR + part];
+        const uint4 b = dout[row * TPR + part];
+        const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const float2 x = unpack2<BF16>(av[t]), y = unpack2<BF16>(bv[t]);
+            acc = fmaf(x.x, y.x, acc);
+            acc = fmaf(x.y, y.y, acc);
+        }
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        dqacc[row * (D / 4) + 2 * part] = z;
+        dqacc[row * (D / 4) + 2 * part + 1] = z;
+    }
+#pragma unroll
+    for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (row < rows && part == 0) dvec[row] = acc;
+    if (gid < BH) counters[gid] = 0;
+}
 
-inline int bwd_launch(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                      const CUtensorMap&, const void*, const float*, const void*, void*, void*,
-                      void*, void*, int, int, int, int, float, bool, cudaStream_t) {
-    return -7;
+// ------------------------------------------------------------------ main --
+struct BwdParams {
+    const float* lse;
+    const float* dvec;
+    float* dqacc;
+    int* counters;
+    void* dq;
+    void* dk;
+    void* dv;
+    int BH;
+    int N;
+    int n_qtiles;
+    int n_ktiles;
+    int causal;
+    float scale;
+    float scale_log2;
+};
+
+template <int D>
+struct BwdCfg {
+    static constexpr int KB = D / 64;
+    static constexpr uint32_t TILE = 128u * D * 2u;
+    static constexpr uint32_t OFF_K = 0;
+    static constexpr uint32_t OFF_V = OFF_K + TILE;
+    static constexpr uint32_t OFF_Q = OFF_V + TILE;
+    static constexpr uint32_t OFF_DO = OFF_Q + TILE;
+    static constexpr uint32_t OFF_PT = OFF_DO + TILE;        // 128 x 128 half
+    static constexpr uint32_t OFF_DST = OFF_PT + 32768u;     // 128 x 128 half
+    static constexpr uint32_t OFF_L = OFF_DST + 32768u;      // 4 warps x 128 fp32 (log2 LSE)
+    static constexpr uint32_t OFF_DD = OFF_L + 2048u;        // 4 warps x 128 fp32 (D)
+    static constexpr uint32_t OFF_BAR = OFF_DD + 2048u;
+    static constexpr int B_KV = 0, B_Q = 1, B_DO = 2, B_QE = 3, B_SF = 4, B_DPF = 5, B_DSF = 6,
+                         B_DQF = 7, B_DQE = 8, B_FIN = 9, B_DR = 10, B_ENDA = 11, B_ENDB = 12,
+                         NBAR = 13;
+    static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
+    static constexpr int NTHREADS = 192;
+};
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(192, 1)
+    attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
+                         const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV,
+                         const __grid_constant__ CUtensorMap tmDO, const BwdParams p) {
+    using C = BwdCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // Work item: head-major, the heaviest key tile (j = 0 under the causal mask) first.
+    const int bh = static_cast<int>(blockIdx.x) / p.n_ktiles;
+    const int j = static_cast<int>(blockIdx.x) % p.n_ktiles;
+    const int i_begin = p.causal ? j : 0;
+    const int n_it = p.n_qtiles - i_begin;
+
+    const uint32_t bar0 = base + C::OFF_BAR;
+#define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + C::OFF_MISC);
+    volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(gbase + C::OFF_MISC + 4);
+    volatile uint32_t* last_flag = reinterpret_cast<volatile uint32_t*>(gbase + C::OFF_MISC + 8);
+    float* sL = reinterpret_cast<float*>(gbase + C::OFF_L);
+    float* sDD = reinterpret_cast<float*>(gbase + C::OFF_DD);
+
+    if (threadIdx.x == 0) {
+        mbar_init(BAR(C::B_KV), 1);
+        mbar_init(BAR(C::B_Q), 1);
+        mbar_init(BAR(C::B_DO), 1);
+        mbar_init(BAR(C::B_QE), 1);
+        mbar_init(BAR(C::B_SF), 1);
+        mbar_init(BAR(C::B_DPF), 1);
+        mbar_init(BAR(C::B_DSF), 128);
+        mbar_init(BAR(C::B_DQF), 1);
+        mbar_init(BAR(C::B_DQE), 128);
+        mbar_init(BAR(C::B_FIN), 1);
+        mbar_init(BAR(C::B_DR), 1);
+        mbar_init(BAR(C::B_ENDA), 128);
+        mbar_init(BAR(C::B_ENDB), 1);
+        *abort_flag = 0u;
+        *last_flag = 0u;
+        fence_mbar_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(base + C::OFF_MISC, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 4) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            tma_prefetch_desc(&tmDO);
+            mbar_arrive_expect_tx(BAR(C::B_KV), 2 * C::TILE);
+#pragma unroll
+            for (int kb = 0; kb < C::KB; ++kb) {
+                tma_load_3d(base + C::OFF_K + kb * 16384u, &tmK, BAR(C::B_KV), kb * 64, j * 128, bh);
+                tma_load_3d(base + C::OFF_V + kb * 16384u, &tmV, BAR(C::B_KV), kb * 64, j * 128, bh);
+            }
+            int issued = 0;
+            for (int it = 0; it < n_it; ++it) {
+                const int i = i_begin + it;
+                if (!wait_bounded(BAR(C::B_QE), (it & 1) ^ 1, abort_flag)) break;
+                mbar_arrive_expect_tx(BAR(C::B_Q), C::TILE);
+#pragma unroll
+                for (int kb = 0; kb < C::KB; ++kb)
+                    tma_load_3d(base + C::OFF_Q + kb * 16384u, &tmQ, BAR(C::B_Q), kb * 64, i * 128, bh);
+                mbar_arrive_expect_tx(BAR(C::B_DO), C::TILE);
+#pragma unroll
+                for (int kb = 0; kb < C::KB; ++kb)
+                    tma_load_3d(base + C::OFF_DO + kb * 16384u, &tmDO, BAR(C::B_DO), kb * 64, i * 128,
+                                bh);
+                issued = it + 1;
+            }
+            if (*abort_flag) {
+                wait_drain(BAR(C::B_KV), 0);
+                if (issued > 0) {
+                    wait_drain(BAR(C::B_Q), (issued - 1) & 1);
+                    wait_drain(BAR(C::B_DO), (issued - 1) & 1);
+                }
+            }
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t ID_SS = idesc_f16(BF16, 128, 128, false, false);
+            constexpr uint32_t ID_KV = idesc_f16(BF16, 128, D, false, true);
+            constexpr uint32_t ID_Q = idesc_f16(BF16, 128, D, true, true);
+            const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sQ = base + C::OFF_Q,
+                           sDO = base + C::OFF_DO, sPT = base + C::OFF_PT, sDST = base + C::OFF_DST;
+            bool ok = wait_bounded(BAR(C::B_KV), 0, abort_flag);
+            for (int it = 0; ok && it < n_it; ++it) {
+                const uint32_t ph = it & 1;
+                if (!(ok = wait_bounded(BAR(C::B_Q), ph, abort_flag))) break;
+                if (!(ok = wait_bounded(BAR(C::B_DQE), ph ^ 1, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {  // S^T = K Q^T
+                    const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                    mma_ss(tmem + C::COL_S, sdesc_sw128(sK + off, 16, 1024),
+                           sdesc_sw128(sQ + off, 16, 1024), ID_SS, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(BAR(C::B_SF));
+                if (!(ok = wait_bounded(BAR(C::B_DO), ph, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {  // dP^T = V dO^T
+                    const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                    mma_ss(tmem + C::COL_DP, sdesc_sw128(sV + off, 16, 1024),
+                           sdesc_sw128(sDO + off, 16, 1024), ID_SS, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(BAR(C::B_DPF));
+                if (!(ok = wait_bounded(BAR(C::B_DSF), ph, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {  // dV += P^T dO ; dK += dS^T Q
+                    const uint32_t offa = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                    const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+                    mma_ss(tmem + C::COL_DV, sdesc_sw128(sPT + offa, 16, 1024),
+                           sdesc_sw128(sDO + kk * 2048u, 16384, 1024), ID_KV, acc);
+                    mma_ss(tmem + C::COL_DK, sdesc_sw128(sDST + offa, 16, 1024),
+                           sdesc_sw128(sQ + kk * 2048u, 16384, 1024), ID_KV, acc);
+                }
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)  // dQ = dS K  (A = dS^T read MN-major)
+                    mma_ss(tmem + C::COL_S, sdesc_sw128(sDST + kk * 2048u, 16384, 1024),
+                           sdesc_sw128(sK + kk * 2048u, 16384, 1024), ID_Q, kk > 0 ? 1u : 0u);
+                mma_commit(BAR(C::B_QE));
+                mma_commit(BAR(C::B_DQF));
+            }
+            if (ok) mma_commit(BAR(C::B_FIN));
+            if (*abort_flag) {
+                mma_commit(BAR(C::B_DR));
+                wait_drain(BAR(C::B_DR), 0);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------- compute
+        const int r = threadIdx.x;
+        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        const int key = j * 128 + r;
+        const bool key_valid = key < p.N;
+        const float sl = p.scale_log2;
+        const size_t head_row0 = static_cast<size_t>(bh) * p.N;
+        bool ok = true;
+        for (int it = 0; it < n_it; ++it) {
+            const int i = i_begin + it;
+            const int q0 = i * 128;
+            const uint32_t ph = it & 1;
+            // Stage this tile's 128 statistics in the warp's own slice (no
+            // cross-warp barrier): lane e loads queries q0 + e + 32 t.
+            float* L = sL + warp * 128;
+            float* Dd = sDD + warp * 128;
+            __syncwarp();
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const int c = lane + 32 * t, qr = q0 + c;
+                L[c] = qr < p.N ? p.lse[head_row0 + qr] * 1.4426950408889634f : INFINITY;
+                Dd[c] = qr < p.N ? p.dvec[head_row0 + qr] : 0.f;
+            }
+            __syncwarp();
+            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SF), ph, abort_flag));
+            if (ok) ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_DPF), ph, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            // mask: causal keys after the query, and key rows past N
+            int limit = key_valid ? 128 : 0;  // columns c < limit may be visible
+            int lo = 0;                       // columns c < lo are masked (causal)
+            if (p.causal && i == j) lo = r;   // query q0 + c sees key j*128 + r iff c >= r
+            const uint32_t sPT = base + C::OFF_PT, sDST = base + C::OFF_DST;
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                uint32_t sv[32], dpv[32];
+                tmem_ld32(lane_addr + C::COL_S + c4 * 32u, sv);
+                tmem_ld32(lane_addr + C::COL_DP + c4 * 32u, dpv);
+                tmem_ld_wait();
+                reg_fence32(sv);
+                reg_fence32(dpv);
+                float pv[32], dsv[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int c = c4 * 32 + e;
+                    float pe = ex2(fmaf(__uint_as_float(sv[e]), sl, -L[c]));
+                    if (c < lo || c >= limit) pe = 0.f;
+                    pv[e] = pe;
+                    dsv[e] = pe * (__uint_as_float(dpv[e]) - Dd[c]);
+                }
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const int c = c4 * 4 + g;  // 16-byte chunk index (8 columns)
+                    const uint32_t off = (c >> 3) * 16384u + sw128_off(r, c & 7);
+                    st_shared_v4(sPT + off, pack2<BF16>(pv[8 * g + 0], pv[8 * g + 1]),
+                                 pack2<BF16>(pv[8 * g + 2], pv[8 * g + 3]),
+                                 pack2<BF16>(pv[8 * g + 4], pv[8 * g + 5]),
+                                 pack2<BF16>(pv[8 * g + 6], pv[8 * g + 7]));
+                    st_shared_v4(sDST + off, pack2<BF16>(dsv[8 * g + 0], dsv[8 * g + 1]),
+                                 pack2<BF16>(dsv[8 * g + 2], dsv[8 * g + 3]),
+                                 pack2<BF16>(dsv[8 * g + 4], dsv[8 * g + 5]),
+                                 pack2<BF16>(dsv[8 * g + 6], dsv[8 * g + 7]));
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(BAR(C::B_DSF));
+
+            // dQ_i partial: thread r holds query row q0 + r of dS K_j
+            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_DQF), ph, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            const int qr = q0 + r;
+            float4* dst = reinterpret_cast<float4*>(p.dqacc + (head_row0 + qr) * D);
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(lane_addr + C::COL_S + c * 32u, v);
+                tmem_ld_wait();
+                reg_fence32(v);
+                if (qr < p.N) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        atomicAdd(dst + c * 8 + e,
+                                  make_float4(__uint_as_float(v[4 * e]) * p.scale,
+                                              __uint_as_float(v[4 * e + 1]) * p.scale,
+                                              __uint_as_float(v[4 * e + 2]) * p.scale,
+                                              __uint_as_float(v[4 * e + 3]) * p.scale));
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(BAR(C::B_DQE));
+        }
+        if (ok) ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_FIN), 0, abort_flag));
+        if (ok) {  // dK_j, dV_j rows: thread r holds key row j*128 + r
+            tc_fence_after();
+            const size_t rowoff = (head_row0 + key) * (D * 2);
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                uint8_t* out = static_cast<uint8_t*>(which ? p.dv : p.dk) + rowoff;
+                const uint32_t col = which ? C::COL_DV : C::COL_DK;
+                const float mul = which ? 1.f : p.scale;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(lane_addr + col + c * 32u, v);
+                    tmem_ld_wait();
+                    reg_fence32(v);
+                    uint32_t h[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        h[e] = pack2<BF16>(__uint_as_float(v[2 * e]) * mul,
+                                           __uint_as_float(v[2 * e + 1]) * mul);
+                    if (key_valid) {
+                        uint4* d4 = reinterpret_cast<uint4*>(out + c * 64);
+                        d4[0] = make_uint4(h[0], h[1], h[2], h[3]);
+                        d4[1] = make_uint4(h[4], h[5], h[6], h[7]);
+                        d4[2] = make_uint4(h[8], h[9], h[10], h[11]);
+                        d4[3] = make_uint4(h[12], h[13], h[14], h[15]);
+                    }
+                }
+            }
+            // The last CTA of this head to finish converts the head's dQ.
+            // Bounded mbarrier syncs (not bar.sync): a warp that gave up
+            // cannot leave the others waiting for ever.
+            __threadfence();
+            mbar_arrive(BAR(C::B_ENDA));
+            if (r == 0) {
+                if (wait_bounded(BAR(C::B_ENDA), 0, abort_flag)) {
+                    const int done = atomicAdd(p.counters + bh, 1);
+                    *last_flag = (done == p.n_ktiles - 1) ? 1u : 0u;
+                }
+                mbar_arrive(BAR(C::B_ENDB));
+            }
+            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_ENDB), 0, abort_flag));
+            if (ok && *last_flag) {
+                __threadfence();
+                const float4* src = reinterpret_cast<const float4*>(p.dqacc + head_row0 * D);
+                uint2* out = reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.dq) + head_row0 * D * 2);
+                const long long n4 = static_cast<long long>(p.N) * D / 4;
+                for (long long e = r; e < n4; e += 128) {
+                    const float4 x = __ldcg(src + e);
+                    out[e] = make_uint2(pack2<BF16>(x.x, x.y), pack2<BF16>(x.z, x.w));
+                }
+            }
+        }
+    }
+#undef BAR
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+inline bool bwd_set_attributes() {
+    bool ok = true;
+    ok &= cudaFuncSetAttribute(attn_bwd_main_kernel<64, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               BwdCfg<64>::SMEM_BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn_bwd_main_kernel<64, false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               BwdCfg<64>::SMEM_BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn_bwd_main_kernel<128, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               BwdCfg<128>::SMEM_BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn_bwd_main_kernel<128, false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               BwdCfg<128>::SMEM_BYTES) == cudaSuccess;
+    return ok;
+}
+
+template <int D, bool BF16>
+int bwd_prep_launch(const void* o, const void* dout, void* ws, int B, int H, int N,
+                    cudaStream_t st) {
+    const long long rows = 1LL * B * H * N;
+    const long long threads = rows * (D / 8);
+    const long long blocks = (threads + 255) / 256;
+    if (blocks >= (1LL << 31)) return -2;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    attn_bwd_prep_kernel<D, BF16><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        static_cast<const uint4*>(o), static_cast<const uint4*>(dout), reinterpret_cast<float*>(w),
+        reinterpret_cast<float4*>(w + bwd_ws_off_dq(B, H, N)),
+        reinterpret_cast<int*>(w + bwd_ws_off_cnt(B, H, N, D)), rows, B * H);
+    return cudaGetLastError() == cudaSuccess ? 0 : -7;
+}
+
+template <int D, bool BF16>
+int bwd_main_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                    const CUtensorMap& mdo, const float* lse, void* dq, void* dk, void* dv,
+                    void* ws, int B, int H, int N, int causal, float scale, cudaStream_t st) {
+    BwdParams p;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    p.lse = lse;
+    p.dvec = reinterpret_cast<const float*>(w);
+    p.dqacc = reinterpret_cast<float*>(w + bwd_ws_off_dq(B, H, N));
+    p.counters = reinterpret_cast<int*>(w + bwd_ws_off_cnt(B, H, N, D));
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    p.BH = B * H;
+    p.N = N;
+    p.n_qtiles = (N + 127) / 128;
+    p.n_ktiles = (N + 127) / 128;
+    p.causal = causal;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    const long long nblocks = 1LL * p.n_ktiles * p.BH;
+    if (nblocks >= (1LL << 31)) return -2;
+    attn_bwd_main_kernel<D, BF16><<<static_cast<unsigned>(nblocks), BwdCfg<D>::NTHREADS,
+                                    BwdCfg<D>::SMEM_BYTES, st>>>(mq, mk, mv, mdo, p);
+    return cudaGetLastError() == cudaSuccess ? 0 : -7;
 }
 
 }  // namespace attn

@@ -70,12 +70,6 @@ struct FwdCfg {
     static constexpr int NTHREADS = 192;
 };
 
-// Bounded wait used only while draining after an abort: ignores the abort flag.
-__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
-    uint32_t never = 0;
-    wait_bounded(bar, parity, &never, 200000000ull);
-}
-
 template <int D, bool BF16>
 __global__ void __launch_bounds__(192, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -88,9 +82,11 @@ __global__ void __launch_bounds__(192, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Work item: heaviest query tiles (largest index under the causal mask) first.
-    const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x) / p.BH;
-    const int bh = static_cast<int>(blockIdx.x) % p.BH;
+    // Work item: head-major, so the CTAs resident at one time share a few
+    // heads' K/V in L2; within a head the heaviest query tile (largest index
+    // under the causal mask) goes first.
+    const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x) % p.n_qtiles;
+    const int bh = static_cast<int>(blockIdx.x) / p.n_qtiles;
     const int n_kv_all = (p.N + 127) >> 7;
     const int nkv = p.causal ? min(n_kv_all, qt + 1) : n_kv_all;
 

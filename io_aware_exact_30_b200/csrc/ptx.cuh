@@ -77,6 +77,12 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
+// Bounded wait used only while draining after an abort: ignores the abort flag.
+__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
+    uint32_t never = 0;
+    wait_bounded(bar, parity, &never, 200000000ull);
+}
+
 // ---------------------------------------------------------------- proxies --
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
