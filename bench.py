@@ -137,6 +137,27 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(mhz)}
 
 
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own instance of the workload (weak scaling)."""
+    return seed + rank
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (the job is as slow as its slowest rank)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flop_per_rank_step: float, world: int, max_ms_per_step: float) -> float:
+    """Whole-job throughput: every rank's work over the slowest rank's time."""
+    return world * flop_per_rank_step / (max_ms_per_step * 1e-3) / 1e12
+
+
 def host_inputs(wl, seed):
     B, H, N, d, causal, dtype, sigma, passes = WORKLOADS[wl]
     arrs = synth.attention_inputs(B, H, N, d, seed=seed, sigma=sigma, dtype=dtype,
@@ -157,7 +178,7 @@ def run_ours(args, rank, world, local_rank):
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float16
     scale = 1.0 / math.sqrt(d)
 
-    arrs = host_inputs(args.workload, seed=args.seed + rank)
+    arrs = host_inputs(args.workload, seed=rank_seed(args.seed, rank))
     pinned = []
     for a in arrs:
         t = torch.from_numpy(a.view(np.int16)).view(tdt) if dtype == "bf16" else torch.from_numpy(a)
@@ -226,10 +247,7 @@ def run_ours(args, rank, world, local_rank):
         main_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in per_step)
 
     # whole-job time = slowest rank
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = reduce_max(total_ms, world, dev)
     clk = clocks.stop() if rank == 0 else None
 
     # ---- end to end through the public API with host buffers -------------
@@ -259,10 +277,7 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    te = torch.tensor([e0.elapsed_time(e1) / e2e_steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / e2e_steps, world, dev)
     h2d = sum(t.numel() * t.element_size() for t in pinned)
     d2h = sum(t.numel() * t.element_size() for t in host_out) + (
         0 if passes == "fwdbwd" else host_lse.numel() * 4)
@@ -274,7 +289,7 @@ def run_ours(args, rank, world, local_rank):
     f_fwd, f_bwd = flops(B, H, N, d, causal)
     f_step = f_fwd + (f_bwd if passes == "fwdbwd" else 0.0)
     ms_step = max_ms / args.steps
-    value = world * f_step / (ms_step * 1e-3) / 1e12
+    value = job_tflops(f_step, world, ms_step)
     burst, sustained, hbm, src = peaks()
     if passes == "fwdbwd":
         dom = ("attn_bwd_main", f_bwd, main_ms)
@@ -318,7 +333,7 @@ def run_ours(args, rank, world, local_rank):
             "frac": round(achieved / sustained, 4),
             "traffic": None,
         },
-        "e2e": {"value": round(world * f_step / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+        "e2e": {"value": round(job_tflops(f_step, world, e2e_ms), 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": n_launch * args.steps,
