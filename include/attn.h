@@ -65,7 +65,8 @@ typedef enum {
     ATTN_ERR_DEVICE = -6,   /* no sm_100 device current, or a pointer is not device memory */
     ATTN_ERR_LAUNCH = -7,   /* the CUDA runtime rejected a launch */
     ATTN_ERR_TIMEOUT = -8,  /* a bounded in-kernel wait ran out (device status) */
-    ATTN_ERR_ARG = -9       /* scale not finite and positive, or another bad scalar */
+    ATTN_ERR_ARG = -9,      /* scale not finite and positive, or another bad scalar */
+    ATTN_ERR_SCRATCH = -10  /* attn_bwd_noalloc: problem exceeds the built-in scratch */
 } attn_status_t;
 
 /*
@@ -122,6 +123,36 @@ int attn_bwd_prep(const void* o, const void* dout, void* workspace, int B, int H
 int attn_bwd_main(const void* q, const void* k, const void* v, const float* lse,
                   const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H,
                   int N, int d, int causal, float scale, attn_dtype_t dtype, void* stream);
+
+/*
+ * Backward that allocates nothing, for callers that cannot get device memory
+ * for a workspace: for example a plugin inside a host framework that owns
+ * every device allocation through its own pool and hands the plugin only the
+ * input and output tensors, or a latency-critical loop that may not call
+ * cudaMalloc (which can synchronise the whole device) once it is running.
+ * The papers describe no such entry point; it exists only for these callers.
+ *
+ * Same arguments, semantics and results as attn_bwd, minus `workspace`: the
+ * scratch (D, the fp32 dQ accumulator and the per-head counters) lives in a
+ * fixed array of ATTN_NOALLOC_SCRATCH_BYTES bytes that every device which
+ * loads this library holds until the process exits.  The caller still passes
+ * every input and output buffer.  Problems whose attn_bwd_workspace_bytes()
+ * exceed that size are rejected with ATTN_ERR_SCRATCH before any launch.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture.
+ *  - All calls share the one array and it keeps what the last call left;
+ *    each call clears what must start at zero.  Calls whose kernels overlap
+ *    on the GPU (two streams, or two host threads) race on the array: order
+ *    them on one stream or synchronise between them.
+ *  - No cudaMalloc, cudaFree or other allocating routine is called.
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                     const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                     int B, int H, int N, int d, int causal, float scale,
+                     attn_dtype_t dtype, void* stream);
 
 /*
  * Synchronises `stream`, then returns ATTN_OK, ATTN_ERR_TIMEOUT if a kernel

@@ -23,7 +23,7 @@ _DTYPES = {torch.bfloat16: ATTN_BF16, torch.float16: ATTN_FP16}
 STATUS = {
     0: "ATTN_OK", -1: "ATTN_ERR_NULL", -2: "ATTN_ERR_SHAPE", -3: "ATTN_ERR_HEADDIM",
     -4: "ATTN_ERR_ALIGN", -5: "ATTN_ERR_DTYPE", -6: "ATTN_ERR_DEVICE", -7: "ATTN_ERR_LAUNCH",
-    -8: "ATTN_ERR_TIMEOUT", -9: "ATTN_ERR_ARG",
+    -8: "ATTN_ERR_TIMEOUT", -9: "ATTN_ERR_ARG", -10: "ATTN_ERR_SCRATCH",
 }
 
 # Kernel launches one attn_bwd call makes (D preprocess, main backward).
@@ -31,7 +31,11 @@ BWD_LAUNCHES = 2
 
 # Every symbol include/attn.h declares.
 EXPORTS = ("attn_fwd", "attn_bwd", "attn_bwd_prep", "attn_bwd_main", "attn_bwd_workspace_bytes",
-           "attn_last_device_status", "attn_selftest_wait_timeout", "attn_strerror", "attn_version")
+           "attn_bwd_noalloc", "attn_last_device_status", "attn_selftest_wait_timeout",
+           "attn_strerror", "attn_version")
+
+# Size of the built-in scratch attn_bwd_noalloc uses (bytes, per device).
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 class AttnError(RuntimeError):
@@ -59,6 +63,8 @@ def lib() -> ctypes.CDLL:
         L.attn_bwd_prep.restype = ci
         L.attn_bwd_main.argtypes = [vp] * 9 + [ci, ci, ci, ci, ci, cf, ci, vp]
         L.attn_bwd_main.restype = ci
+        L.attn_bwd_noalloc.argtypes = [vp] * 9 + [ci, ci, ci, ci, ci, cf, ci, vp]
+        L.attn_bwd_noalloc.restype = ci
         L.attn_bwd_workspace_bytes.argtypes = [ci, ci, ci, ci]
         L.attn_bwd_workspace_bytes.restype = sz
         L.attn_last_device_status.argtypes = [vp]
@@ -174,6 +180,23 @@ def attn_bwd_main(q, k, v, o, lse, dout, dq, dk, dv, workspace, causal: bool,
                              _ptr(dv), _ptr(workspace), B, H, N, d, int(bool(causal)), scale,
                              _dtype(q), ctypes.c_void_p(_stream(q.device, stream)))
     _check(rc, "attn_bwd_main")
+
+
+def attn_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, causal: bool,
+                     scale: float | None = None, stream=None) -> None:
+    """attn_bwd without a workspace argument: the library uses its own fixed
+    device array (``NOALLOC_SCRATCH_BYTES`` per device) and allocates nothing.
+    For callers that have their inputs and outputs but no way to obtain
+    scratch memory.  Calls that overlap on the GPU share that array and race."""
+    B, H, N, d = _shape(q)
+    _same(q, k, v, o, dout, dq, dk, dv, names=("k", "v", "o", "dout", "dq", "dk", "dv"))
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 (B, H, N) tensor")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib().attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
+                                _ptr(dk), _ptr(dv), B, H, N, d, int(bool(causal)), scale, _dtype(q),
+                                ctypes.c_void_p(_stream(q.device, stream)))
+    _check(rc, "attn_bwd_noalloc")
 
 
 def attn_last_device_status(stream=None, device=None) -> int:

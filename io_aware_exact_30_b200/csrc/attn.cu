@@ -146,6 +146,30 @@ __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
     __syncthreads();
 }
 
+// Built-in backward scratch for attn_bwd_noalloc: one copy per device that
+// loads this library, held until the process exits.  Host code must not pass
+// `g_bwd_scratch` itself to a kernel (on the host it names a stand-in, not the
+// device copy); the device address is looked up with cudaGetSymbolAddress,
+// once per device, with that device current.
+__device__ __align__(256) unsigned char g_bwd_scratch[ATTN_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices];
+
+int scratch_address(int dev, void** out) {
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_bwd_scratch) != cudaSuccess || ptr == nullptr) {
+            cudaGetLastError();
+            return ATTN_ERR_DEVICE;
+        }
+        g_scratch_addr[dev] = ptr;
+    }
+    *out = g_scratch_addr[dev];
+    return ATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -269,6 +293,33 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
                              dtype, st);
 }
 
+int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                     const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                     int H, int N, int d, int causal, float scale, attn_dtype_t dtype,
+                     void* stream) {
+    const void* ptrs[9] = {q, k, v, o, lse, dout, dq, dk, dv};
+    for (const void* ptr : ptrs)
+        if (!ptr) return ATTN_ERR_NULL;
+    int rc = check_shape(B, H, N, d, dtype, scale);
+    if (rc) return rc;
+    if (attn::bwd_workspace_bytes(B, H, N, d) > ATTN_NOALLOC_SCRATCH_BYTES)
+        return ATTN_ERR_SCRATCH;
+    for (const void* ptr : ptrs)
+        if (!aligned16(ptr)) return ATTN_ERR_ALIGN;
+    int dev;
+    if ((rc = check_device(&dev))) return rc;
+    for (const void* ptr : ptrs)
+        if (!on_device(ptr, dev)) return ATTN_ERR_DEVICE;
+    void* scratch = nullptr;
+    if ((rc = scratch_address(dev, &scratch))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // The prep kernel rewrites D and clears the dQ accumulator and counters,
+    // so whatever the previous call left in the scratch does not matter.
+    if ((rc = bwd_prep_dispatch(o, dout, scratch, B, H, N, d, dtype, st))) return rc;
+    return bwd_main_dispatch(q, k, v, lse, dout, dq, dk, dv, scratch, B, H, N, d, causal, scale,
+                             dtype, st);
+}
+
 int attn_last_device_status(void* stream) {
     int dev;
     if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -306,6 +357,7 @@ const char* attn_strerror(int status) {
         case ATTN_ERR_LAUNCH: return "the CUDA runtime rejected a launch or reported an error";
         case ATTN_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
         case ATTN_ERR_ARG: return "scale must be finite and > 0 (or a scalar argument is out of range)";
+        case ATTN_ERR_SCRATCH: return "problem needs more backward scratch than the built-in array holds";
         default: return "unknown status";
     }
 }
