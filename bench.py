@@ -208,10 +208,10 @@ def run_ours(args, rank, world, local_rank):
         if evs:
             evs[1].record(stream)
         if passes == "fwdbwd":
-            attn.attn_bwd_prep(o, do, ws, causal)
+            attn.attn_bwd_prep(o, do, lse, ws)
             if evs:
                 evs[2].record(stream)
-            attn.attn_bwd_main(q, k, v, o, lse, do, dq, dk, dv, ws, causal, scale)
+            attn.attn_bwd_main(q, k, v, do, dq, dk, dv, ws, causal, scale)
             if evs:
                 evs[3].record(stream)
 

@@ -81,10 +81,10 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              attn_dtype_t dtype, void* stream);
 
 /*
- * Bytes of device scratch attn_bwd needs: D (B*H*N fp32, the row dot products
- * of dO and O), the fp32 dQ accumulator (B*H*N*d) and one int32 completion
- * counter per (b, h), each section 256-byte aligned.  Returns 0 for invalid
- * sizes.
+ * Bytes of device scratch attn_bwd needs: the log2-scaled LSE and D (the row
+ * dot products of dO and O), B*H*Np fp32 each with Np = N rounded up to 128,
+ * the fp32 dQ accumulator (B*H*N*d) and one int32 completion counter per
+ * (b, h), each section 256-byte aligned.  Returns 0 for invalid sizes.
  */
 size_t attn_bwd_workspace_bytes(int B, int H, int N, int d);
 
@@ -107,22 +107,23 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
  * separately; calling attn_bwd_prep then attn_bwd_main on the same stream
  * and workspace is exactly attn_bwd.
  *
- * attn_bwd_prep: D_i = sum_t dout_it * o_it (fp32, one per query row) into the
- * workspace, and clears the workspace's fp32 dQ accumulator and per-head
- * completion counters.  Reads o and dout only.
+ * attn_bwd_prep: reads o, dout and lse; writes into the workspace D_i =
+ * sum_t dout_it * o_it and lse_i * log2(e) (fp32, per head padded to a
+ * multiple of 128 rows), and clears the fp32 dQ accumulator and the per-head
+ * completion counters.
  *
  * attn_bwd_main: for every 128-key tile, recomputes S and P per 128-query tile
- * from q, k and lse (never storing P), forms dV, dK in tensor memory and adds
- * the dQ contributions into the workspace accumulator; the last tile of each
- * head to finish converts that head's dQ into dq.  Requires the workspace as
- * attn_bwd_prep left it.
+ * from q, k and the statistics attn_bwd_prep staged (never storing P), forms
+ * dV, dK in tensor memory and adds the dQ contributions into the workspace
+ * accumulator; the last tile of each head to finish converts that head's dQ
+ * into dq.  Requires the workspace as attn_bwd_prep left it.
  */
-int attn_bwd_prep(const void* o, const void* dout, void* workspace, int B, int H, int N, int d,
-                  attn_dtype_t dtype, void* stream);
+int attn_bwd_prep(const void* o, const void* dout, const float* lse, void* workspace, int B,
+                  int H, int N, int d, attn_dtype_t dtype, void* stream);
 
-int attn_bwd_main(const void* q, const void* k, const void* v, const float* lse,
-                  const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H,
-                  int N, int d, int causal, float scale, attn_dtype_t dtype, void* stream);
+int attn_bwd_main(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                  void* dk, void* dv, void* workspace, int B, int H, int N, int d, int causal,
+                  float scale, attn_dtype_t dtype, void* stream);
 
 /*
  * Backward that allocates nothing, for callers that cannot get device memory

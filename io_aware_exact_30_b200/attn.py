@@ -59,9 +59,9 @@ def lib() -> ctypes.CDLL:
         L.attn_fwd.restype = ci
         L.attn_bwd.argtypes = [vp] * 10 + [ci, ci, ci, ci, ci, cf, ci, vp]
         L.attn_bwd.restype = ci
-        L.attn_bwd_prep.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, vp]
+        L.attn_bwd_prep.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, vp]
         L.attn_bwd_prep.restype = ci
-        L.attn_bwd_main.argtypes = [vp] * 9 + [ci, ci, ci, ci, ci, cf, ci, vp]
+        L.attn_bwd_main.argtypes = [vp] * 8 + [ci, ci, ci, ci, ci, cf, ci, vp]
         L.attn_bwd_main.restype = ci
         L.attn_bwd_noalloc.argtypes = [vp] * 9 + [ci, ci, ci, ci, ci, cf, ci, vp]
         L.attn_bwd_noalloc.restype = ci
@@ -153,32 +153,32 @@ def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, causal: bool,
     _check(rc, "attn_bwd")
 
 
-def attn_bwd_prep(o, dout, workspace, causal: bool = False, stream=None) -> None:
-    """D = rowdot(dout, o) into the workspace; clears the dQ accumulator."""
+def attn_bwd_prep(o, dout, lse, workspace, stream=None) -> None:
+    """Stage D = rowdot(dout, o) and lse * log2(e) in the workspace; clear the dQ accumulator."""
     B, H, N, d = _shape(o)
     _same(o, dout, names=("dout",))
-    need = attn_bwd_workspace_bytes(B, H, N, d)
-    if workspace.numel() * workspace.element_size() < need:
-        raise ValueError(f"workspace needs {need} bytes")
-    rc = lib().attn_bwd_prep(_ptr(o), _ptr(dout), _ptr(workspace), B, H, N, d, _dtype(o),
-                             ctypes.c_void_p(_stream(o.device, stream)))
-    _check(rc, "attn_bwd_prep")
-
-
-def attn_bwd_main(q, k, v, o, lse, dout, dq, dk, dv, workspace, causal: bool,
-                  scale: float | None = None, stream=None) -> None:
-    """Recompute backward after attn_bwd_prep (``o`` is accepted for symmetry, unused)."""
-    B, H, N, d = _shape(q)
-    _same(q, k, v, dout, dq, dk, dv, names=("k", "v", "dout", "dq", "dk", "dv"))
     if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous float32 (B, H, N) tensor")
     need = attn_bwd_workspace_bytes(B, H, N, d)
     if workspace.numel() * workspace.element_size() < need:
         raise ValueError(f"workspace needs {need} bytes")
+    rc = lib().attn_bwd_prep(_ptr(o), _ptr(dout), _ptr(lse), _ptr(workspace), B, H, N, d, _dtype(o),
+                             ctypes.c_void_p(_stream(o.device, stream)))
+    _check(rc, "attn_bwd_prep")
+
+
+def attn_bwd_main(q, k, v, dout, dq, dk, dv, workspace, causal: bool,
+                  scale: float | None = None, stream=None) -> None:
+    """Recompute backward on a workspace prepared by attn_bwd_prep."""
+    B, H, N, d = _shape(q)
+    _same(q, k, v, dout, dq, dk, dv, names=("k", "v", "dout", "dq", "dk", "dv"))
+    need = attn_bwd_workspace_bytes(B, H, N, d)
+    if workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace needs {need} bytes")
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    rc = lib().attn_bwd_main(_ptr(q), _ptr(k), _ptr(v), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
-                             _ptr(dv), _ptr(workspace), B, H, N, d, int(bool(causal)), scale,
-                             _dtype(q), ctypes.c_void_p(_stream(q.device, stream)))
+    rc = lib().attn_bwd_main(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                             _ptr(workspace), B, H, N, d, int(bool(causal)), scale, _dtype(q),
+                             ctypes.c_void_p(_stream(q.device, stream)))
     _check(rc, "attn_bwd_main")
 
 

@@ -226,20 +226,19 @@ int bwd_common_checks(const void* const* ptrs, int nptr, const void* workspace, 
     return ATTN_OK;
 }
 
-int bwd_prep_dispatch(const void* o, const void* dout, void* workspace, int B, int H, int N,
-                      int d, attn_dtype_t dtype, cudaStream_t st) {
+int bwd_prep_dispatch(const void* o, const void* dout, const float* lse, void* workspace, int B,
+                      int H, int N, int d, attn_dtype_t dtype, cudaStream_t st) {
     const bool bf = dtype == ATTN_BF16;
     if (d == 64)
-        return bf ? attn::bwd_prep_launch<64, true>(o, dout, workspace, B, H, N, st)
-                  : attn::bwd_prep_launch<64, false>(o, dout, workspace, B, H, N, st);
-    return bf ? attn::bwd_prep_launch<128, true>(o, dout, workspace, B, H, N, st)
-              : attn::bwd_prep_launch<128, false>(o, dout, workspace, B, H, N, st);
+        return bf ? attn::bwd_prep_launch<64, true>(o, dout, lse, workspace, B, H, N, st)
+                  : attn::bwd_prep_launch<64, false>(o, dout, lse, workspace, B, H, N, st);
+    return bf ? attn::bwd_prep_launch<128, true>(o, dout, lse, workspace, B, H, N, st)
+              : attn::bwd_prep_launch<128, false>(o, dout, lse, workspace, B, H, N, st);
 }
 
-int bwd_main_dispatch(const void* q, const void* k, const void* v, const float* lse,
-                      const void* dout, void* dq, void* dk, void* dv, void* workspace, int B,
-                      int H, int N, int d, int causal, float scale, attn_dtype_t dtype,
-                      cudaStream_t st) {
+int bwd_main_dispatch(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                      void* dk, void* dv, void* workspace, int B, int H, int N, int d, int causal,
+                      float scale, attn_dtype_t dtype, cudaStream_t st) {
     const int BH = B * H;
     CUtensorMap mq, mk, mv, mdo;
     if (!make_map(&mq, q, dtype, BH, N, d) || !make_map(&mk, k, dtype, BH, N, d) ||
@@ -248,35 +247,35 @@ int bwd_main_dispatch(const void* q, const void* k, const void* v, const float* 
     const bool bf = dtype == ATTN_BF16;
     const int c = causal ? 1 : 0;
     if (d == 64)
-        return bf ? attn::bwd_main_launch<64, true>(mq, mk, mv, mdo, lse, dq, dk, dv, workspace, B,
-                                                    H, N, c, scale, st)
-                  : attn::bwd_main_launch<64, false>(mq, mk, mv, mdo, lse, dq, dk, dv, workspace,
-                                                     B, H, N, c, scale, st);
-    return bf ? attn::bwd_main_launch<128, true>(mq, mk, mv, mdo, lse, dq, dk, dv, workspace, B, H,
-                                                 N, c, scale, st)
-              : attn::bwd_main_launch<128, false>(mq, mk, mv, mdo, lse, dq, dk, dv, workspace, B,
-                                                  H, N, c, scale, st);
+        return bf ? attn::bwd_main_launch<64, true>(mq, mk, mv, mdo, dq, dk, dv, workspace, B, H,
+                                                    N, c, scale, st)
+                  : attn::bwd_main_launch<64, false>(mq, mk, mv, mdo, dq, dk, dv, workspace, B, H,
+                                                     N, c, scale, st);
+    return bf ? attn::bwd_main_launch<128, true>(mq, mk, mv, mdo, dq, dk, dv, workspace, B, H, N,
+                                                 c, scale, st)
+              : attn::bwd_main_launch<128, false>(mq, mk, mv, mdo, dq, dk, dv, workspace, B, H, N,
+                                                  c, scale, st);
 }
 }  // namespace
 
-int attn_bwd_prep(const void* o, const void* dout, void* workspace, int B, int H, int N, int d,
-                  attn_dtype_t dtype, void* stream) {
-    const void* ptrs[3] = {o, dout, workspace};
+int attn_bwd_prep(const void* o, const void* dout, const float* lse, void* workspace, int B,
+                  int H, int N, int d, attn_dtype_t dtype, void* stream) {
+    const void* ptrs[4] = {o, dout, lse, workspace};
     int dev;
-    int rc = bwd_common_checks(ptrs, 3, workspace, B, H, N, d, dtype, 1.f, &dev);
+    int rc = bwd_common_checks(ptrs, 4, workspace, B, H, N, d, dtype, 1.f, &dev);
     if (rc) return rc;
-    return bwd_prep_dispatch(o, dout, workspace, B, H, N, d, dtype,
+    return bwd_prep_dispatch(o, dout, lse, workspace, B, H, N, d, dtype,
                              static_cast<cudaStream_t>(stream));
 }
 
-int attn_bwd_main(const void* q, const void* k, const void* v, const float* lse,
-                  const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H,
-                  int N, int d, int causal, float scale, attn_dtype_t dtype, void* stream) {
-    const void* ptrs[9] = {q, k, v, lse, dout, dq, dk, dv, workspace};
+int attn_bwd_main(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                  void* dk, void* dv, void* workspace, int B, int H, int N, int d, int causal,
+                  float scale, attn_dtype_t dtype, void* stream) {
+    const void* ptrs[8] = {q, k, v, dout, dq, dk, dv, workspace};
     int dev;
-    int rc = bwd_common_checks(ptrs, 9, workspace, B, H, N, d, dtype, scale, &dev);
+    int rc = bwd_common_checks(ptrs, 8, workspace, B, H, N, d, dtype, scale, &dev);
     if (rc) return rc;
-    return bwd_main_dispatch(q, k, v, lse, dout, dq, dk, dv, workspace, B, H, N, d, causal, scale,
+    return bwd_main_dispatch(q, k, v, dout, dq, dk, dv, workspace, B, H, N, d, causal, scale,
                              dtype, static_cast<cudaStream_t>(stream));
 }
 
@@ -288,8 +287,8 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
     int rc = bwd_common_checks(ptrs, 10, workspace, B, H, N, d, dtype, scale, &dev);
     if (rc) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if ((rc = bwd_prep_dispatch(o, dout, workspace, B, H, N, d, dtype, st))) return rc;
-    return bwd_main_dispatch(q, k, v, lse, dout, dq, dk, dv, workspace, B, H, N, d, causal, scale,
+    if ((rc = bwd_prep_dispatch(o, dout, lse, workspace, B, H, N, d, dtype, st))) return rc;
+    return bwd_main_dispatch(q, k, v, dout, dq, dk, dv, workspace, B, H, N, d, causal, scale,
                              dtype, st);
 }
 
@@ -315,8 +314,8 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // The prep kernel rewrites D and clears the dQ accumulator and counters,
     // so whatever the previous call left in the scratch does not matter.
-    if ((rc = bwd_prep_dispatch(o, dout, scratch, B, H, N, d, dtype, st))) return rc;
-    return bwd_main_dispatch(q, k, v, lse, dout, dq, dk, dv, scratch, B, H, N, d, causal, scale,
+    if ((rc = bwd_prep_dispatch(o, dout, lse, scratch, B, H, N, d, dtype, st))) return rc;
+    return bwd_main_dispatch(q, k, v, dout, dq, dk, dv, scratch, B, H, N, d, causal, scale,
                              dtype, st);
 }
 

@@ -15,23 +15,32 @@
 //   dK_j = scale sum_i dS_ij q_i,  dQ_i = scale sum_j dS_ij k_j.
 //
 // Kernels
-//   attn_bwd_prep_kernel  D_i = rowdot(dO_i, O_i) (fp32), zero the fp32 dQ
-//                         accumulator and the per-head completion counters.
-//   attn_bwd_main_kernel  one CTA per (head, 128-key tile j): K_j, V_j stay in
-//                         shared memory; for every query tile i the MMAs form
-//                         S^T = K_j Q_i^T and dP^T = V_j dO_i^T in tensor
-//                         memory, the compute warps turn them into P^T and
-//                         dS^T (bf16/fp16, shared memory), and the MMAs
-//                         accumulate dV_j += P^T dO_i, dK_j += dS^T Q_i in
-//                         tensor memory and form dQ_i = dS K_j, which the
-//                         compute warps add into the fp32 accumulator with
-//                         vector atomics.  The last CTA of a head to finish
-//                         converts that head's dQ to the output type.
+//   attn_bwd_prep_kernel  D_i = rowdot(dO_i, O_i) and L2_i = LSE_i * log2(e),
+//                         both fp32 in a per-head array padded to a multiple of
+//                         128 rows (padding: D = 0, L2 = +inf so P = 0); zeroes
+//                         the fp32 dQ accumulator and the per-head counters.
+//   attn_bwd_main_kernel  one CTA per (head, 128-key tile j); K_j, V_j stay in
+//                         shared memory while the 128-query tiles i stream
+//                         through (Q double-buffered).  Per query tile:
+//                           S^T  = K_j Q_i^T          (tensor memory)
+//                           dP^T = V_j dO_i^T         (tensor memory)
+//                           P^T  = exp2(S^T log2e scale - L2_i), written back
+//                                  into tensor memory as bf16/fp16 over S^T
+//                           dV  += P^T dO_i           (A read from tensor memory)
+//                           dS^T = P^T (dP^T - D_i)   (shared memory, half)
+//                           dK  += dS^T Q_i
+//                           dQ_i partial = dS K_j, added to the fp32
+//                                  accumulator with non-returning reductions
+//                         The last CTA of a head to finish converts that head's
+//                         dQ to the output type.
 //
-// Roles (192 threads): warps 0-3 compute (thread t = TMEM lane t: key row t
-// for P^T/dS^T/dK/dV, query row t for dQ), warp 4 TMA, warp 5 MMA + TMEM.
-// Tensor memory (512 columns): S^T at 0 (reused for dQ once S^T is consumed),
-// dP^T at 128, dV at 256, dK at 256 + D.
+// Roles (192 threads): warps 0-3 compute (thread t = TMEM lane t), warp 4
+// TMA producer, warp 5 MMA issuer and TMEM owner.
+// Tensor memory (512 columns): S^T/P^T at 0, dP^T at 128, dV at 256, dK at
+// 256 + D.  For D = 128 the dQ tile is formed transposed, dQ^T = K^T dS^T
+// (lane = feature, column = query), in the dP^T columns once dS^T has been
+// read out, so each warp's reductions cover 32 consecutive floats of one
+// query row.  For D = 64 it is dQ = dS K (lane = query) in columns 384..447.
 #pragma once
 
 #include "ptx.cuh"
@@ -40,10 +49,13 @@ namespace attn {
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Workspace: D (BH*N fp32) | dQ accumulator (BH*N*d fp32) | counters (BH int32).
-inline size_t bwd_ws_off_dq(int B, int H, int N) {
-    return align256(static_cast<size_t>(B) * H * N * 4);
+// Workspace: L2 (BH*Np fp32) | D (BH*Np fp32) | dQ accumulator (BH*N*d fp32) |
+// counters (BH int32), Np = N rounded up to 128; sections 256-byte aligned.
+inline size_t bwd_np(int N) { return (static_cast<size_t>(N) + 127) / 128 * 128; }
+inline size_t bwd_ws_off_d(int B, int H, int N) {
+    return align256(static_cast<size_t>(B) * H * bwd_np(N) * 4);
 }
+inline size_t bwd_ws_off_dq(int B, int H, int N) { return 2 * bwd_ws_off_d(B, H, N); }
 inline size_t bwd_ws_off_cnt(int B, int H, int N, int d) {
     return bwd_ws_off_dq(B, H, N) + align256(static_cast<size_t>(B) * H * N * d * 4);
 }
@@ -53,18 +65,20 @@ inline size_t bwd_workspace_bytes(int B, int H, int N, int d) {
 
 // ------------------------------------------------------------------ prep --
 template <int D, bool BF16>
-__global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const uint4* __restrict__ o,
-                                                            const uint4* __restrict__ dout,
-                                                            float* __restrict__ dvec,
-                                                            float4* __restrict__ dqacc,
-                                                            int* __restrict__ counters,
-                                                            long long rows, int BH) {
+__global__ void __launch_bounds__(256) attn_bwd_prep_kernel(
+    const uint4* __restrict__ o, const uint4* __restrict__ dout, const float* __restrict__ lse,
+    float* __restrict__ l2pad, float* __restrict__ dpad, float4* __restrict__ dqacc,
+    int* __restrict__ counters, int N, int Np, long long rows_padded, int BH) {
     constexpr int TPR = D / 8;  // threads per row, 8 elements (16 bytes) each
     const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const long long row = gid / TPR;
+    const long long prow = gid / TPR;  // padded row: bh * Np + i
     const int part = static_cast<int>(gid % TPR);
+    const long long bh = prow / Np;
+    const int i = static_cast<int>(prow - bh * Np);
+    const bool real = prow < rows_padded && i < N;
+    const long long row = bh * N + i;
     float acc = 0.f;
-    if (row < rows) {
+    if (real) {
         const uint4 a = o[row * TPR + part];
         const uint4 b = dout[row * TPR + part];
         const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
@@ -80,14 +94,17 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const uint4* __restr
     }
 #pragma unroll
     for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (row < rows && part == 0) dvec[row] = acc;
+    if (prow < rows_padded && part == 0) {
+        dpad[prow] = real ? acc : 0.f;
+        l2pad[prow] = real ? lse[row] * 1.4426950408889634f : INFINITY;
+    }
     if (gid < BH) counters[gid] = 0;
 }
 
 // ------------------------------------------------------------------ main --
 struct BwdParams {
-    const float* lse;
-    const float* dvec;
+    const float* l2pad;
+    const float* dpad;
     float* dqacc;
     int* counters;
     void* dq;
@@ -95,6 +112,7 @@ struct BwdParams {
     void* dv;
     int BH;
     int N;
+    int Np;
     int n_qtiles;
     int n_ktiles;
     int causal;
@@ -106,22 +124,26 @@ template <int D>
 struct BwdCfg {
     static constexpr int KB = D / 64;
     static constexpr uint32_t TILE = 128u * D * 2u;
+    static constexpr int QST = 2;
+    static constexpr int DOST = D == 128 ? 1 : 2;
     static constexpr uint32_t OFF_K = 0;
     static constexpr uint32_t OFF_V = OFF_K + TILE;
     static constexpr uint32_t OFF_Q = OFF_V + TILE;
-    static constexpr uint32_t OFF_DO = OFF_Q + TILE;
-    static constexpr uint32_t OFF_PT = OFF_DO + TILE;        // 128 x 128 half
-    static constexpr uint32_t OFF_DST = OFF_PT + 32768u;     // 128 x 128 half
-    static constexpr uint32_t OFF_L = OFF_DST + 32768u;      // 4 warps x 128 fp32 (log2 LSE)
-    static constexpr uint32_t OFF_DD = OFF_L + 2048u;        // 4 warps x 128 fp32 (D)
-    static constexpr uint32_t OFF_BAR = OFF_DD + 2048u;
-    static constexpr int B_KV = 0, B_Q = 1, B_DO = 2, B_QE = 3, B_SF = 4, B_DPF = 5, B_DSF = 6,
-                         B_DQF = 7, B_DQE = 8, B_FIN = 9, B_DR = 10, B_ENDA = 11, B_ENDB = 12,
-                         NBAR = 13;
+    static constexpr uint32_t OFF_DO = OFF_Q + QST * TILE;
+    static constexpr uint32_t OFF_DST = OFF_DO + DOST * TILE;   // 128 x 128 half
+    static constexpr uint32_t OFF_LD = OFF_DST + 32768u;       // QST x (128 L2 + 128 D) fp32
+    static constexpr uint32_t OFF_BAR = OFF_LD + QST * 1024u;
+    static constexpr int B_KV = 0, B_QF = 1, B_QE = B_QF + QST, B_DOF = B_QE + QST,
+                         B_DOE = B_DOF + DOST, B_SF = B_DOE + DOST, B_DPF = B_SF + 1,
+                         B_PTF = B_DPF + 1, B_DVD = B_PTF + 1, B_DSF = B_DVD + 1,
+                         B_DQF = B_DSF + 1, B_DQE = B_DQF + 1, B_FIN = B_DQE + 1,
+                         B_DR = B_FIN + 1, B_ENDA = B_DR + 1, B_ENDB = B_ENDA + 1,
+                         NBAR = B_ENDB + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
+    static constexpr uint32_t COL_DQ = D == 128 ? COL_DP : 384;
     static constexpr int NTHREADS = 192;
 };
 
@@ -150,16 +172,22 @@ __global__ void __launch_bounds__(192, 1)
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + C::OFF_MISC);
     volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(gbase + C::OFF_MISC + 4);
     volatile uint32_t* last_flag = reinterpret_cast<volatile uint32_t*>(gbase + C::OFF_MISC + 8);
-    float* sL = reinterpret_cast<float*>(gbase + C::OFF_L);
-    float* sDD = reinterpret_cast<float*>(gbase + C::OFF_DD);
+    const float* sLD = reinterpret_cast<const float*>(gbase + C::OFF_LD);
 
     if (threadIdx.x == 0) {
         mbar_init(BAR(C::B_KV), 1);
-        mbar_init(BAR(C::B_Q), 1);
-        mbar_init(BAR(C::B_DO), 1);
-        mbar_init(BAR(C::B_QE), 1);
+        for (int s = 0; s < C::QST; ++s) {
+            mbar_init(BAR(C::B_QF + s), 1);
+            mbar_init(BAR(C::B_QE + s), 1);
+        }
+        for (int s = 0; s < C::DOST; ++s) {
+            mbar_init(BAR(C::B_DOF + s), 1);
+            mbar_init(BAR(C::B_DOE + s), 1);
+        }
         mbar_init(BAR(C::B_SF), 1);
         mbar_init(BAR(C::B_DPF), 1);
+        mbar_init(BAR(C::B_PTF), 128);
+        mbar_init(BAR(C::B_DVD), 1);
         mbar_init(BAR(C::B_DSF), 128);
         mbar_init(BAR(C::B_DQF), 1);
         mbar_init(BAR(C::B_DQE), 128);
@@ -193,27 +221,38 @@ __global__ void __launch_bounds__(192, 1)
                 tma_load_3d(base + C::OFF_K + kb * 16384u, &tmK, BAR(C::B_KV), kb * 64, j * 128, bh);
                 tma_load_3d(base + C::OFF_V + kb * 16384u, &tmV, BAR(C::B_KV), kb * 64, j * 128, bh);
             }
-            int issued = 0;
+            int q_issued[C::QST], do_issued[C::DOST];
+            for (int s = 0; s < C::QST; ++s) q_issued[s] = 0;
+            for (int s = 0; s < C::DOST; ++s) do_issued[s] = 0;
+            const size_t ld_row0 = static_cast<size_t>(bh) * p.Np;
             for (int it = 0; it < n_it; ++it) {
                 const int i = i_begin + it;
-                if (!wait_bounded(BAR(C::B_QE), (it & 1) ^ 1, abort_flag)) break;
-                mbar_arrive_expect_tx(BAR(C::B_Q), C::TILE);
+                const int qs = it % C::QST, qn = it / C::QST;
+                const int ds = it % C::DOST, dn = it / C::DOST;
+                if (!wait_bounded(BAR(C::B_QE + qs), (qn & 1) ^ 1, abort_flag)) break;
+                const uint32_t sq = base + C::OFF_Q + qs * C::TILE;
+                const uint32_t sld = base + C::OFF_LD + qs * 1024u;
+                mbar_arrive_expect_tx(BAR(C::B_QF + qs), C::TILE + 1024u);
 #pragma unroll
                 for (int kb = 0; kb < C::KB; ++kb)
-                    tma_load_3d(base + C::OFF_Q + kb * 16384u, &tmQ, BAR(C::B_Q), kb * 64, i * 128, bh);
-                mbar_arrive_expect_tx(BAR(C::B_DO), C::TILE);
+                    tma_load_3d(sq + kb * 16384u, &tmQ, BAR(C::B_QF + qs), kb * 64, i * 128, bh);
+                bulk_load(sld, p.l2pad + ld_row0 + i * 128, 512u, BAR(C::B_QF + qs));
+                bulk_load(sld + 512u, p.dpad + ld_row0 + i * 128, 512u, BAR(C::B_QF + qs));
+                q_issued[qs] = qn + 1;
+                if (!wait_bounded(BAR(C::B_DOE + ds), (dn & 1) ^ 1, abort_flag)) break;
+                const uint32_t sdo = base + C::OFF_DO + ds * C::TILE;
+                mbar_arrive_expect_tx(BAR(C::B_DOF + ds), C::TILE);
 #pragma unroll
                 for (int kb = 0; kb < C::KB; ++kb)
-                    tma_load_3d(base + C::OFF_DO + kb * 16384u, &tmDO, BAR(C::B_DO), kb * 64, i * 128,
-                                bh);
-                issued = it + 1;
+                    tma_load_3d(sdo + kb * 16384u, &tmDO, BAR(C::B_DOF + ds), kb * 64, i * 128, bh);
+                do_issued[ds] = dn + 1;
             }
             if (*abort_flag) {
                 wait_drain(BAR(C::B_KV), 0);
-                if (issued > 0) {
-                    wait_drain(BAR(C::B_Q), (issued - 1) & 1);
-                    wait_drain(BAR(C::B_DO), (issued - 1) & 1);
-                }
+                for (int s = 0; s < C::QST; ++s)
+                    if (q_issued[s] > 0) wait_drain(BAR(C::B_QF + s), (q_issued[s] - 1) & 1);
+                for (int s = 0; s < C::DOST; ++s)
+                    if (do_issued[s] > 0) wait_drain(BAR(C::B_DOF + s), (do_issued[s] - 1) & 1);
             }
         }
     } else if (warp == 5) {
@@ -221,47 +260,74 @@ __global__ void __launch_bounds__(192, 1)
         if (lane == 0) {
             constexpr uint32_t ID_SS = idesc_f16(BF16, 128, 128, false, false);
             constexpr uint32_t ID_KV = idesc_f16(BF16, 128, D, false, true);
-            constexpr uint32_t ID_Q = idesc_f16(BF16, 128, D, true, true);
-            const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sQ = base + C::OFF_Q,
-                           sDO = base + C::OFF_DO, sPT = base + C::OFF_PT, sDST = base + C::OFF_DST;
+            constexpr uint32_t ID_DQT = idesc_f16(BF16, 128, 128, true, true);  // D == 128
+            constexpr uint32_t ID_DQ = idesc_f16(BF16, 128, D, true, true);     // D == 64
+            const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sDST = base + C::OFF_DST;
             bool ok = wait_bounded(BAR(C::B_KV), 0, abort_flag);
             for (int it = 0; ok && it < n_it; ++it) {
                 const uint32_t ph = it & 1;
-                if (!(ok = wait_bounded(BAR(C::B_Q), ph, abort_flag))) break;
-                if (!(ok = wait_bounded(BAR(C::B_DQE), ph ^ 1, abort_flag))) break;
+                const int qs = it % C::QST, qn = it / C::QST;
+                const int ds = it % C::DOST, dn = it / C::DOST;
+                const uint32_t sQ = base + C::OFF_Q + qs * C::TILE;
+                const uint32_t sDO = base + C::OFF_DO + ds * C::TILE;
+                // S^T = K Q^T; the S/P columns must be free: dV(it-1) has read P^T(it-1)
+                if (!(ok = wait_bounded(BAR(C::B_QF + qs), qn & 1, abort_flag))) break;
+                if (it > 0 && !(ok = wait_bounded(BAR(C::B_DVD), ph ^ 1, abort_flag))) break;
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {  // S^T = K Q^T
+                for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
                     mma_ss(tmem + C::COL_S, sdesc_sw128(sK + off, 16, 1024),
                            sdesc_sw128(sQ + off, 16, 1024), ID_SS, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(BAR(C::B_SF));
-                if (!(ok = wait_bounded(BAR(C::B_DO), ph, abort_flag))) break;
+                // dP^T = V dO^T; for D = 128 the columns hold dQ^T(it-1) until drained
+                if (!(ok = wait_bounded(BAR(C::B_DOF + ds), dn & 1, abort_flag))) break;
+                if (D == 128 && it > 0 && !(ok = wait_bounded(BAR(C::B_DQE), ph ^ 1, abort_flag)))
+                    break;
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {  // dP^T = V dO^T
+                for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
                     mma_ss(tmem + C::COL_DP, sdesc_sw128(sV + off, 16, 1024),
                            sdesc_sw128(sDO + off, 16, 1024), ID_SS, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(BAR(C::B_DPF));
-                if (!(ok = wait_bounded(BAR(C::B_DSF), ph, abort_flag))) break;
+                // dV += P^T dO with P^T read from tensor memory
+                if (!(ok = wait_bounded(BAR(C::B_PTF), ph, abort_flag))) break;
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {  // dV += P^T dO ; dK += dS^T Q
-                    const uint32_t offa = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                    const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                    mma_ss(tmem + C::COL_DV, sdesc_sw128(sPT + offa, 16, 1024),
-                           sdesc_sw128(sDO + kk * 2048u, 16384, 1024), ID_KV, acc);
-                    mma_ss(tmem + C::COL_DK, sdesc_sw128(sDST + offa, 16, 1024),
-                           sdesc_sw128(sQ + kk * 2048u, 16384, 1024), ID_KV, acc);
-                }
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + C::COL_DV, tmem + C::COL_S + kk * 8u,
+                           sdesc_sw128(sDO + kk * 2048u, 16384, 1024), ID_KV,
+                           (it > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(BAR(C::B_DVD));
+                mma_commit(BAR(C::B_DOE + ds));
+                // dK += dS^T Q ; dQ partial
+                if (!(ok = wait_bounded(BAR(C::B_DSF), ph, abort_flag))) break;
+                if (D == 64 && it > 0 && !(ok = wait_bounded(BAR(C::B_DQE), ph ^ 1, abort_flag)))
+                    break;
+                tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)  // dQ = dS K  (A = dS^T read MN-major)
-                    mma_ss(tmem + C::COL_S, sdesc_sw128(sDST + kk * 2048u, 16384, 1024),
-                           sdesc_sw128(sK + kk * 2048u, 16384, 1024), ID_Q, kk > 0 ? 1u : 0u);
-                mma_commit(BAR(C::B_QE));
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(tmem + C::COL_DK,
+                           sdesc_sw128(sDST + (kk >> 2) * 16384u + (kk & 3) * 32u, 16, 1024),
+                           sdesc_sw128(sQ + kk * 2048u, 16384, 1024), ID_KV,
+                           (it > 0 || kk > 0) ? 1u : 0u);
+                if constexpr (D == 128) {
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)  // dQ^T = K^T dS^T: A = K (MN-major), B = dS^T (MN-major)
+                        mma_ss(tmem + C::COL_DQ, sdesc_sw128(sK + kk * 2048u, 16384, 1024),
+                               sdesc_sw128(sDST + kk * 2048u, 16384, 1024), ID_DQT,
+                               kk > 0 ? 1u : 0u);
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)  // dQ = dS K: A = dS^T read MN-major, B = K MN-major
+                        mma_ss(tmem + C::COL_DQ, sdesc_sw128(sDST + kk * 2048u, 16384, 1024),
+                               sdesc_sw128(sK + kk * 2048u, 16384, 1024), ID_DQ,
+                               kk > 0 ? 1u : 0u);
+                }
+                mma_commit(BAR(C::B_QE + qs));
                 mma_commit(BAR(C::B_DQF));
             }
             if (ok) mma_commit(BAR(C::B_FIN));
@@ -273,64 +339,73 @@ __global__ void __launch_bounds__(192, 1)
         __syncwarp();
     } else {
         // ---------------------------------------------------------- compute
-        const int r = threadIdx.x;
+        const int r = threadIdx.x;  // TMEM lane
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
         const int key = j * 128 + r;
         const bool key_valid = key < p.N;
         const float sl = p.scale_log2;
         const size_t head_row0 = static_cast<size_t>(bh) * p.N;
+        const uint32_t sDST = base + C::OFF_DST;
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
             const int i = i_begin + it;
             const int q0 = i * 128;
             const uint32_t ph = it & 1;
-            // Stage this tile's 128 statistics in the warp's own slice (no
-            // cross-warp barrier): lane e loads queries q0 + e + 32 t.
-            float* L = sL + warp * 128;
-            float* Dd = sDD + warp * 128;
-            __syncwarp();
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const int c = lane + 32 * t, qr = q0 + c;
-                L[c] = qr < p.N ? p.lse[head_row0 + qr] * 1.4426950408889634f : INFINITY;
-                Dd[c] = qr < p.N ? p.dvec[head_row0 + qr] : 0.f;
-            }
-            __syncwarp();
-            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SF), ph, abort_flag));
-            if (ok) ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_DPF), ph, abort_flag));
+            const float* L = sLD + (it % C::QST) * 256;
+            const float* Dd = L + 128;
+
+            // ---- P^T = exp2(S^T scale log2e - L2), into tensor memory over S^T
+            // (wait on the load barrier too: it makes the bulk-copied L2/D visible)
+            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_QF + it % C::QST),
+                                                      (it / C::QST) & 1, abort_flag));
+            if (ok) ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SF), ph, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            // mask: causal keys after the query, and key rows past N
-            int limit = key_valid ? 128 : 0;  // columns c < limit may be visible
-            int lo = 0;                       // columns c < lo are masked (causal)
-            if (p.causal && i == j) lo = r;   // query q0 + c sees key j*128 + r iff c >= r
-            const uint32_t sPT = base + C::OFF_PT, sDST = base + C::OFF_DST;
+            float pv[128];
+            {
+                uint32_t sv[4][32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + C::COL_S + c * 32u, sv[c]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < 4; ++c) reg_fence32(sv[c]);
+                // causal: on the diagonal tile query q0 + c sees key j*128 + r iff c >= r
+                const int lo = (p.causal && i == j) ? r : 0;
+                const int hi = key_valid ? 128 : 0;
+#pragma unroll
+                for (int c = 0; c < 128; ++c) {
+                    const float e = ex2(fmaf(__uint_as_float(sv[c >> 5][c & 31]), sl, -L[c]));
+                    pv[c] = (c < lo || c >= hi) ? 0.f : e;
+                }
+                uint32_t ph2[2][32];
+#pragma unroll
+                for (int c = 0; c < 64; ++c) ph2[c >> 5][c & 31] = pack2<BF16>(pv[2 * c], pv[2 * c + 1]);
+                tmem_st32(lane_addr + C::COL_S, ph2[0]);
+                tmem_st32(lane_addr + C::COL_S + 32u, ph2[1]);
+                tmem_st_wait();
+            }
+            tc_fence_before();
+            mbar_arrive(BAR(C::B_PTF));
+
+            // ---- dS^T = P^T (dP^T - D), half, into shared memory
+            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_DPF), ph, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) {
-                uint32_t sv[32], dpv[32];
-                tmem_ld32(lane_addr + C::COL_S + c4 * 32u, sv);
+                uint32_t dpv[32];
                 tmem_ld32(lane_addr + C::COL_DP + c4 * 32u, dpv);
                 tmem_ld_wait();
-                reg_fence32(sv);
                 reg_fence32(dpv);
-                float pv[32], dsv[32];
+                float dsv[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int c = c4 * 32 + e;
-                    float pe = ex2(fmaf(__uint_as_float(sv[e]), sl, -L[c]));
-                    if (c < lo || c >= limit) pe = 0.f;
-                    pv[e] = pe;
-                    dsv[e] = pe * (__uint_as_float(dpv[e]) - Dd[c]);
-                }
+                for (int e = 0; e < 32; ++e)
+                    dsv[e] = pv[c4 * 32 + e] * (__uint_as_float(dpv[e]) - Dd[c4 * 32 + e]);
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
                     const int c = c4 * 4 + g;  // 16-byte chunk index (8 columns)
-                    const uint32_t off = (c >> 3) * 16384u + sw128_off(r, c & 7);
-                    st_shared_v4(sPT + off, pack2<BF16>(pv[8 * g + 0], pv[8 * g + 1]),
-                                 pack2<BF16>(pv[8 * g + 2], pv[8 * g + 3]),
-                                 pack2<BF16>(pv[8 * g + 4], pv[8 * g + 5]),
-                                 pack2<BF16>(pv[8 * g + 6], pv[8 * g + 7]));
-                    st_shared_v4(sDST + off, pack2<BF16>(dsv[8 * g + 0], dsv[8 * g + 1]),
+                    st_shared_v4(sDST + (c >> 3) * 16384u + sw128_off(r, c & 7),
+                                 pack2<BF16>(dsv[8 * g + 0], dsv[8 * g + 1]),
                                  pack2<BF16>(dsv[8 * g + 2], dsv[8 * g + 3]),
                                  pack2<BF16>(dsv[8 * g + 4], dsv[8 * g + 5]),
                                  pack2<BF16>(dsv[8 * g + 6], dsv[8 * g + 7]));
@@ -340,26 +415,46 @@ __global__ void __launch_bounds__(192, 1)
             tc_fence_before();
             mbar_arrive(BAR(C::B_DSF));
 
-            // dQ_i partial: thread r holds query row q0 + r of dS K_j
+            // ---- dQ partial into the fp32 accumulator
             ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_DQF), ph, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            const int qr = q0 + r;
-            float4* dst = reinterpret_cast<float4*>(p.dqacc + (head_row0 + qr) * D);
+            if constexpr (D == 128) {
+                // lane r holds feature r of dQ for the tile's 128 queries
+                float* col = p.dqacc + head_row0 * D + r;
+                const int nq = min(128, p.N - q0);
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t v[32];
-                tmem_ld32(lane_addr + C::COL_S + c * 32u, v);
-                tmem_ld_wait();
-                reg_fence32(v);
-                if (qr < p.N) {
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    uint32_t v[32];
+                    tmem_ld32(lane_addr + C::COL_DQ + c4 * 32u, v);
+                    tmem_ld_wait();
+                    reg_fence32(v);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        atomicAdd(dst + c * 8 + e,
-                                  make_float4(__uint_as_float(v[4 * e]) * p.scale,
-                                              __uint_as_float(v[4 * e + 1]) * p.scale,
-                                              __uint_as_float(v[4 * e + 2]) * p.scale,
-                                              __uint_as_float(v[4 * e + 3]) * p.scale));
+                    for (int e = 0; e < 32; ++e) {
+                        const int qc = c4 * 32 + e;
+                        if (qc < nq)
+                            red_add_f32(col + static_cast<size_t>(q0 + qc) * D,
+                                        __uint_as_float(v[e]) * p.scale);
+                    }
+                }
+            } else {
+                // lane r holds query row q0 + r of dQ (64 features)
+                const int qr = q0 + r;
+                float* row = p.dqacc + (head_row0 + qr) * D;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(lane_addr + C::COL_DQ + c * 32u, v);
+                    tmem_ld_wait();
+                    reg_fence32(v);
+                    if (qr < p.N) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            red_add_v4_f32(row + c * 32 + 4 * e, __uint_as_float(v[4 * e]) * p.scale,
+                                           __uint_as_float(v[4 * e + 1]) * p.scale,
+                                           __uint_as_float(v[4 * e + 2]) * p.scale,
+                                           __uint_as_float(v[4 * e + 3]) * p.scale);
+                    }
                 }
             }
             tc_fence_before();
@@ -446,28 +541,30 @@ inline bool bwd_set_attributes() {
 }
 
 template <int D, bool BF16>
-int bwd_prep_launch(const void* o, const void* dout, void* ws, int B, int H, int N,
-                    cudaStream_t st) {
-    const long long rows = 1LL * B * H * N;
-    const long long threads = rows * (D / 8);
+int bwd_prep_launch(const void* o, const void* dout, const float* lse, void* ws, int B, int H,
+                    int N, cudaStream_t st) {
+    const int Np = static_cast<int>(bwd_np(N));
+    const long long rows_padded = 1LL * B * H * Np;
+    const long long threads = rows_padded * (D / 8);
     const long long blocks = (threads + 255) / 256;
     if (blocks >= (1LL << 31)) return -2;
     uint8_t* w = static_cast<uint8_t*>(ws);
     attn_bwd_prep_kernel<D, BF16><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-        static_cast<const uint4*>(o), static_cast<const uint4*>(dout), reinterpret_cast<float*>(w),
+        static_cast<const uint4*>(o), static_cast<const uint4*>(dout), lse,
+        reinterpret_cast<float*>(w), reinterpret_cast<float*>(w + bwd_ws_off_d(B, H, N)),
         reinterpret_cast<float4*>(w + bwd_ws_off_dq(B, H, N)),
-        reinterpret_cast<int*>(w + bwd_ws_off_cnt(B, H, N, D)), rows, B * H);
+        reinterpret_cast<int*>(w + bwd_ws_off_cnt(B, H, N, D)), N, Np, rows_padded, B * H);
     return cudaGetLastError() == cudaSuccess ? 0 : -7;
 }
 
 template <int D, bool BF16>
 int bwd_main_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                    const CUtensorMap& mdo, const float* lse, void* dq, void* dk, void* dv,
-                    void* ws, int B, int H, int N, int causal, float scale, cudaStream_t st) {
+                    const CUtensorMap& mdo, void* dq, void* dk, void* dv, void* ws, int B, int H,
+                    int N, int causal, float scale, cudaStream_t st) {
     BwdParams p;
     uint8_t* w = static_cast<uint8_t*>(ws);
-    p.lse = lse;
-    p.dvec = reinterpret_cast<const float*>(w);
+    p.l2pad = reinterpret_cast<const float*>(w);
+    p.dpad = reinterpret_cast<const float*>(w + bwd_ws_off_d(B, H, N));
     p.dqacc = reinterpret_cast<float*>(w + bwd_ws_off_dq(B, H, N));
     p.counters = reinterpret_cast<int*>(w + bwd_ws_off_cnt(B, H, N, D));
     p.dq = dq;
@@ -475,6 +572,7 @@ int bwd_main_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensor
     p.dv = dv;
     p.BH = B * H;
     p.N = N;
+    p.Np = static_cast<int>(bwd_np(N));
     p.n_qtiles = (N + 127) / 128;
     p.n_ktiles = (N + 127) / 128;
     p.causal = causal;

@@ -37,10 +37,10 @@ def test_host_side_errors_without_device_work():
     assert L.attn_fwd(ctypes.c_void_p(17), p, p, p, p, 1, 1, 16, 64, 0, 0.125, 0, None) == -4
     assert L.attn_fwd(p, p, p, p, p, 1 << 16, 1 << 16, 16, 64, 0, 0.125, 0, None) == -2
     assert L.attn_bwd(*([None] * 10), 1, 1, 16, 64, 0, 0.125, 0, None) == -1
-    # sizes: D (B*H*N fp32) + dQ accumulator (B*H*N*d fp32) + counters (B*H int32),
-    # each 256-byte aligned
-    assert attn.attn_bwd_workspace_bytes(1, 1, 1, 64) == 256 * 3
-    assert attn.attn_bwd_workspace_bytes(4, 16, 4096, 128) == 4 * 16 * 4096 * 4 * (1 + 128) + 256
+    # sizes: L2 and D (B*H*Np fp32 each, Np = N rounded up to 128) + dQ accumulator
+    # (B*H*N*d fp32) + counters (B*H int32), each section 256-byte aligned
+    assert attn.attn_bwd_workspace_bytes(1, 1, 1, 64) == 512 + 512 + 256 + 256
+    assert attn.attn_bwd_workspace_bytes(4, 16, 4096, 128) == 2 * 64 * 4096 * 4 + 64 * 4096 * 128 * 4 + 256
     assert attn.attn_bwd_workspace_bytes(1, 1, 16, 96) == 0
     for s in attn.STATUS:
         assert attn.strerror(s)

@@ -25,8 +25,8 @@ def gpu_fwd_bwd(arrs, dtype, causal, scale, split=False):
         B, H, N, d = q.shape
         dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
         ws = torch.empty(attn.attn_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device="cuda")
-        attn.attn_bwd_prep(o, do, ws, causal)
-        attn.attn_bwd_main(q, k, v, o, lse, do, dq, dk, dv, ws, causal, scale)
+        attn.attn_bwd_prep(o, do, lse, ws)
+        attn.attn_bwd_main(q, k, v, do, dq, dk, dv, ws, causal, scale)
     else:
         dq, dk, dv = attn.backward(q, k, v, o, lse, do, causal, scale)
     torch.cuda.synchronize()
