@@ -34,8 +34,9 @@
 //                         The last CTA of a head to finish converts that head's
 //                         dQ to the output type.
 //
-// Roles (192 threads): warps 0-3 compute (thread t = TMEM lane t), warp 4
-// TMA producer, warp 5 MMA issuer and TMEM owner.
+// Roles (320 threads): warps 0-7 compute (warp w reads TMEM lanes 32 (w % 4)
+// .. + 31 and the query-column half w / 4 of each tile), warp 8 TMA producer,
+// warp 9 MMA issuer and TMEM owner.
 // Tensor memory (512 columns): S^T/P^T at 0, dP^T at 128, dV at 256, dK at
 // 256 + D.  For D = 128 the dQ tile is formed transposed, dQ^T = K^T dS^T
 // (lane = feature, column = query), in the dP^T columns once dS^T has been
@@ -138,17 +139,19 @@ struct BwdCfg {
                          B_PTF = B_DPF + 1, B_DVD = B_PTF + 1, B_DSF = B_DVD + 1,
                          B_DQF = B_DSF + 1, B_DQE = B_DQF + 1, B_FIN = B_DQE + 1,
                          B_DR = B_FIN + 1, B_ENDA = B_DR + 1, B_ENDB = B_ENDA + 1,
-                         NBAR = B_ENDB + 1;
+                         B_SRD = B_ENDB + 1, NBAR = B_SRD + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
     static constexpr uint32_t COL_DQ = D == 128 ? COL_DP : 384;
-    static constexpr int NTHREADS = 192;
+    static constexpr int NCOMPUTE = 256;             // 8 compute warps
+    static constexpr int NTHREADS = NCOMPUTE + 64;   // + TMA warp + MMA warp
+    static constexpr int WARP_TMA = NCOMPUTE / 32, WARP_MMA = WARP_TMA + 1;
 };
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV,
@@ -186,20 +189,21 @@ __global__ void __launch_bounds__(192, 1)
         }
         mbar_init(BAR(C::B_SF), 1);
         mbar_init(BAR(C::B_DPF), 1);
-        mbar_init(BAR(C::B_PTF), 128);
+        mbar_init(BAR(C::B_PTF), C::NCOMPUTE);
         mbar_init(BAR(C::B_DVD), 1);
-        mbar_init(BAR(C::B_DSF), 128);
+        mbar_init(BAR(C::B_DSF), C::NCOMPUTE);
         mbar_init(BAR(C::B_DQF), 1);
-        mbar_init(BAR(C::B_DQE), 128);
+        mbar_init(BAR(C::B_DQE), C::NCOMPUTE);
         mbar_init(BAR(C::B_FIN), 1);
         mbar_init(BAR(C::B_DR), 1);
-        mbar_init(BAR(C::B_ENDA), 128);
+        mbar_init(BAR(C::B_ENDA), C::NCOMPUTE);
         mbar_init(BAR(C::B_ENDB), 1);
+        mbar_init(BAR(C::B_SRD), C::NCOMPUTE / 2);
         *abort_flag = 0u;
         *last_flag = 0u;
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == C::WARP_MMA) {
         tmem_alloc(base + C::OFF_MISC, C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -208,7 +212,7 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp == C::WARP_TMA) {
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
@@ -255,7 +259,7 @@ __global__ void __launch_bounds__(192, 1)
                     if (do_issued[s] > 0) wait_drain(BAR(C::B_DOF + s), (do_issued[s] - 1) & 1);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == C::WARP_MMA) {
         // ------------------------------------------------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t ID_SS = idesc_f16(BF16, 128, 128, false, false);
@@ -339,20 +343,25 @@ __global__ void __launch_bounds__(192, 1)
         __syncwarp();
     } else {
         // ---------------------------------------------------------- compute
-        const int r = threadIdx.x;  // TMEM lane
-        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        // Warp w owns TMEM lanes 32 (w % 4) .. + 31 (a warp may only touch its
+        // lane quarter) and column half h = w / 4 of every 128-wide tile.
+        const int quarter = warp & 3, half = warp >> 2;
+        const int r = quarter * 32 + lane;  // TMEM lane
+        const int tid = threadIdx.x;        // 0 .. NCOMPUTE-1
+        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
         const int key = j * 128 + r;
         const bool key_valid = key < p.N;
         const float sl = p.scale_log2;
         const size_t head_row0 = static_cast<size_t>(bh) * p.N;
         const uint32_t sDST = base + C::OFF_DST;
+        const int c0 = half * 64;  // first query column of this thread's half
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
             const int i = i_begin + it;
             const int q0 = i * 128;
             const uint32_t ph = it & 1;
-            const float* L = sLD + (it % C::QST) * 256;
-            const float* Dd = L + 128;
+            const float4* L4 = reinterpret_cast<const float4*>(sLD + (it % C::QST) * 256 + c0);
+            const float4* D4 = reinterpret_cast<const float4*>(sLD + (it % C::QST) * 256 + 128 + c0);
 
             // ---- P^T = exp2(S^T scale log2e - L2), into tensor memory over S^T
             // (wait on the load barrier too: it makes the bulk-copied L2/D visible)
@@ -361,29 +370,49 @@ __global__ void __launch_bounds__(192, 1)
             if (ok) ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SF), ph, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            float pv[128];
+            float pv[64];
             {
-                uint32_t sv[4][32];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + C::COL_S + c * 32u, sv[c]);
+                uint32_t sv[2][32];
+                tmem_ld32(lane_addr + C::COL_S + c0, sv[0]);
+                tmem_ld32(lane_addr + C::COL_S + c0 + 32u, sv[1]);
                 tmem_ld_wait();
-#pragma unroll
-                for (int c = 0; c < 4; ++c) reg_fence32(sv[c]);
-                // causal: on the diagonal tile query q0 + c sees key j*128 + r iff c >= r
-                const int lo = (p.causal && i == j) ? r : 0;
-                const int hi = key_valid ? 128 : 0;
-#pragma unroll
-                for (int c = 0; c < 128; ++c) {
-                    const float e = ex2(fmaf(__uint_as_float(sv[c >> 5][c & 31]), sl, -L[c]));
-                    pv[c] = (c < lo || c >= hi) ? 0.f : e;
+                reg_fence32(sv[0]);
+                reg_fence32(sv[1]);
+                if (half == 0) {  // half 1 writes P^T over columns half 0 reads
+                    tc_fence_before();
+                    mbar_arrive(BAR(C::B_SRD));
                 }
-                uint32_t ph2[2][32];
 #pragma unroll
-                for (int c = 0; c < 64; ++c) ph2[c >> 5][c & 31] = pack2<BF16>(pv[2 * c], pv[2 * c + 1]);
-                tmem_st32(lane_addr + C::COL_S, ph2[0]);
-                tmem_st32(lane_addr + C::COL_S + 32u, ph2[1]);
-                tmem_st_wait();
+                for (int g = 0; g < 16; ++g) {
+                    const float4 l4 = L4[g];
+                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int c = 4 * g + e;
+                        pv[c] = ex2(fmaf(__uint_as_float(sv[c >> 5][c & 31]), sl, -lv[e]));
+                    }
+                }
+                // causal diagonal tile: query q0 + c sees key j*128 + r iff c >= r;
+                // key rows past N see nothing
+                if (!key_valid || (p.causal && i == j)) {
+                    const int lo = key_valid ? r - c0 : 64;
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        if (c < lo) pv[c] = 0.f;
+                }
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) pk[c] = pack2<BF16>(pv[2 * c], pv[2 * c + 1]);
+                if (half == 1) {
+                    ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SRD), ph, abort_flag));
+                    tc_fence_after();
+                }
+                if (ok) {
+                    tmem_st32(lane_addr + C::COL_S + half * 32u, pk);
+                    tmem_st_wait();
+                }
             }
+            if (!ok) break;
             tc_fence_before();
             mbar_arrive(BAR(C::B_PTF));
 
@@ -392,18 +421,24 @@ __global__ void __launch_bounds__(192, 1)
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
+            for (int c4 = 0; c4 < 2; ++c4) {
                 uint32_t dpv[32];
-                tmem_ld32(lane_addr + C::COL_DP + c4 * 32u, dpv);
+                tmem_ld32(lane_addr + C::COL_DP + c0 + c4 * 32u, dpv);
                 tmem_ld_wait();
                 reg_fence32(dpv);
                 float dsv[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    dsv[e] = pv[c4 * 32 + e] * (__uint_as_float(dpv[e]) - Dd[c4 * 32 + e]);
+                for (int g = 0; g < 8; ++g) {
+                    const float4 d4 = D4[c4 * 8 + g];
+                    const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dsv[4 * g + e] =
+                            pv[c4 * 32 + 4 * g + e] * (__uint_as_float(dpv[4 * g + e]) - dd[e]);
+                }
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
-                    const int c = c4 * 4 + g;  // 16-byte chunk index (8 columns)
+                    const int c = half * 8 + c4 * 4 + g;  // 16-byte chunk index (8 columns)
                     st_shared_v4(sDST + (c >> 3) * 16384u + sw128_off(r, c & 7),
                                  pack2<BF16>(dsv[8 * g + 0], dsv[8 * g + 1]),
                                  pack2<BF16>(dsv[8 * g + 2], dsv[8 * g + 3]),
@@ -420,57 +455,54 @@ __global__ void __launch_bounds__(192, 1)
             if (!ok) break;
             tc_fence_after();
             if constexpr (D == 128) {
-                // lane r holds feature r of dQ for the tile's 128 queries
+                // lane r holds feature r of dQ; this half covers queries c0 .. c0+63
                 float* col = p.dqacc + head_row0 * D + r;
                 const int nq = min(128, p.N - q0);
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
+                for (int c4 = 0; c4 < 2; ++c4) {
                     uint32_t v[32];
-                    tmem_ld32(lane_addr + C::COL_DQ + c4 * 32u, v);
+                    tmem_ld32(lane_addr + C::COL_DQ + c0 + c4 * 32u, v);
                     tmem_ld_wait();
                     reg_fence32(v);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
-                        const int qc = c4 * 32 + e;
+                        const int qc = c0 + c4 * 32 + e;
                         if (qc < nq)
                             red_add_f32(col + static_cast<size_t>(q0 + qc) * D,
                                         __uint_as_float(v[e]) * p.scale);
                     }
                 }
             } else {
-                // lane r holds query row q0 + r of dQ (64 features)
+                // lane r holds query row q0 + r of dQ; this half covers features 32h .. 32h+31
                 const int qr = q0 + r;
-                float* row = p.dqacc + (head_row0 + qr) * D;
+                float* row = p.dqacc + (head_row0 + qr) * D + half * 32;
+                uint32_t v[32];
+                tmem_ld32(lane_addr + C::COL_DQ + half * 32u, v);
+                tmem_ld_wait();
+                reg_fence32(v);
+                if (qr < p.N) {
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t v[32];
-                    tmem_ld32(lane_addr + C::COL_DQ + c * 32u, v);
-                    tmem_ld_wait();
-                    reg_fence32(v);
-                    if (qr < p.N) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            red_add_v4_f32(row + c * 32 + 4 * e, __uint_as_float(v[4 * e]) * p.scale,
-                                           __uint_as_float(v[4 * e + 1]) * p.scale,
-                                           __uint_as_float(v[4 * e + 2]) * p.scale,
-                                           __uint_as_float(v[4 * e + 3]) * p.scale);
-                    }
+                    for (int e = 0; e < 8; ++e)
+                        red_add_v4_f32(row + 4 * e, __uint_as_float(v[4 * e]) * p.scale,
+                                       __uint_as_float(v[4 * e + 1]) * p.scale,
+                                       __uint_as_float(v[4 * e + 2]) * p.scale,
+                                       __uint_as_float(v[4 * e + 3]) * p.scale);
                 }
             }
             tc_fence_before();
             mbar_arrive(BAR(C::B_DQE));
         }
         if (ok) ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_FIN), 0, abort_flag));
-        if (ok) {  // dK_j, dV_j rows: thread r holds key row j*128 + r
+        if (ok) {  // dK_j, dV_j rows: lane r holds key row j*128 + r; this half, D/2 features
             tc_fence_after();
-            const size_t rowoff = (head_row0 + key) * (D * 2);
+            const size_t rowoff = (head_row0 + key) * (D * 2) + half * D;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
                 uint8_t* out = static_cast<uint8_t*>(which ? p.dv : p.dk) + rowoff;
-                const uint32_t col = which ? C::COL_DV : C::COL_DK;
+                const uint32_t col = (which ? C::COL_DV : C::COL_DK) + half * (D / 2);
                 const float mul = which ? 1.f : p.scale;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = 0; c < D / 64; ++c) {
                     uint32_t v[32];
                     tmem_ld32(lane_addr + col + c * 32u, v);
                     tmem_ld_wait();
@@ -494,7 +526,7 @@ __global__ void __launch_bounds__(192, 1)
             // cannot leave the others waiting for ever.
             __threadfence();
             mbar_arrive(BAR(C::B_ENDA));
-            if (r == 0) {
+            if (tid == 0) {
                 if (wait_bounded(BAR(C::B_ENDA), 0, abort_flag)) {
                     const int done = atomicAdd(p.counters + bh, 1);
                     *last_flag = (done == p.n_ktiles - 1) ? 1u : 0u;
@@ -507,7 +539,7 @@ __global__ void __launch_bounds__(192, 1)
                 const float4* src = reinterpret_cast<const float4*>(p.dqacc + head_row0 * D);
                 uint2* out = reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.dq) + head_row0 * D * 2);
                 const long long n4 = static_cast<long long>(p.N) * D / 4;
-                for (long long e = r; e < n4; e += 128) {
+                for (long long e = tid; e < n4; e += C::NCOMPUTE) {
                     const float4 x = __ldcg(src + e);
                     out[e] = make_uint2(pack2<BF16>(x.x, x.y), pack2<BF16>(x.z, x.w));
                 }
@@ -517,7 +549,7 @@ __global__ void __launch_bounds__(192, 1)
 #undef BAR
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == C::WARP_MMA) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
