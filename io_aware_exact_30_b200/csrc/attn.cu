@@ -14,6 +14,7 @@
 #include "ptx.cuh"
 #include "fwd_sm100.cuh"
 #include "bwd_sm100.cuh"
+#include "bwd128_sm100.cuh"
 
 namespace {
 
@@ -72,6 +73,7 @@ int check_device(int* dev_out) {
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                FwdCfg<128>::SMEM_BYTES) == cudaSuccess;
     ok &= attn::bwd_set_attributes();
+    ok &= attn::bwd128_set_attributes();
     if (!ok) {
         cudaGetLastError();
         g_dev_state[dev] = -1;
@@ -104,14 +106,15 @@ int check_shape(int B, int H, int N, int d, int dtype, float scale) {
     return ATTN_OK;
 }
 
-// 3-D view (d, N, B*H) of a contiguous (B, H, N, d) half tensor; box 64 x 128 x 1,
+// 3-D view (d, N, B*H) of a contiguous (B, H, N, d) half tensor; box 64 x rows x 1,
 // 128-byte swizzle, out-of-range rows read as zero.
-bool make_map(CUtensorMap* m, const void* ptr, int dtype, int BH, int N, int d) {
+bool make_map(CUtensorMap* m, const void* ptr, int dtype, int BH, int N, int d,
+              unsigned rows = 128) {
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                           static_cast<cuuint64_t>(BH)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                              static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
-    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t box[3] = {64, rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = encode_fn()(
         m, dtype == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
@@ -251,10 +254,14 @@ int bwd_main_dispatch(const void* q, const void* k, const void* v, const void* d
                                                     N, c, scale, st)
                   : attn::bwd_main_launch<64, false>(mq, mk, mv, mdo, dq, dk, dv, workspace, B, H,
                                                      N, c, scale, st);
-    return bf ? attn::bwd_main_launch<128, true>(mq, mk, mv, mdo, dq, dk, dv, workspace, B, H, N,
-                                                 c, scale, st)
-              : attn::bwd_main_launch<128, false>(mq, mk, mv, mdo, dq, dk, dv, workspace, B, H, N,
-                                                  c, scale, st);
+    // d = 128: 64-query inner tiles
+    CUtensorMap mq64, mdo64;
+    if (!make_map(&mq64, q, dtype, BH, N, d, 64) || !make_map(&mdo64, dout, dtype, BH, N, d, 64))
+        return ATTN_ERR_LAUNCH;
+    return bf ? attn::bwd_main128_launch<true>(mq64, mk, mv, mdo64, dq, dk, dv, workspace, B, H, N,
+                                               c, scale, st)
+              : attn::bwd_main128_launch<false>(mq64, mk, mv, mdo64, dq, dk, dv, workspace, B, H,
+                                                N, c, scale, st);
 }
 }  // namespace
 

@@ -1,0 +1,533 @@
+// Backward main kernel for head dimension 128: the same recompute backward as
+// attn_bwd_main_kernel (see bwd_sm100.cuh for the method and its sources),
+// with 64-query inner tiles so that every accumulator of the tile loop has
+// tensor memory of its own and no stage waits for another to be drained.
+//
+// One CTA per (head, 128-key tile j); K_j, V_j stay in shared memory, 64-query
+// tiles of Q, dO (and their L2, D statistics) stream through a 3-stage
+// pipeline.  Per query tile i:
+//   S^T  = K_j Q_i^T                     tensor memory, double-buffered
+//   P^T  = exp2(S^T scale log2e - L2_i)  written back over S^T as half
+//   dP^T = V_j dO_i^T                    tensor memory
+//   dV  += P^T dO_i                      A operand read from tensor memory
+//   dS^T = P^T (dP^T - D_i)              shared memory, half
+//   dK  += dS^T Q_i
+//   dQ^T = K_j^T dS^T                    tensor memory, drained by dQ warps
+//                                        into a shared fp32 tile that one bulk
+//                                        reduction adds into the accumulator
+// Tensor memory (512 columns): S^T buffers at 0 and 64, dP^T at 128, dQ^T at
+// 192, dV at 256, dK at 384.
+//
+// Roles (448 threads): warps 0-7 compute P^T and dS^T (warp w reads TMEM
+// lanes 32 (w % 4) .. + 31 and query-column half w / 4 of the 64-wide tile),
+// warps 8-11 drain dQ^T (lane = feature) through the shared staging tile into
+// the fp32 accumulator, warp 12 TMA producer, warp 13 MMA issuer and TMEM owner.
+#pragma once
+
+#include "bwd_sm100.cuh"
+#include "ptx.cuh"
+
+namespace attn {
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+
+struct Bwd128Cfg {
+    static constexpr int D = 128;
+    static constexpr int QT = 64;                     // query rows per inner tile
+    static constexpr uint32_t KTILE = 128u * D * 2u;  // 32 KB: K or V tile
+    static constexpr uint32_t QTILE = 64u * D * 2u;   // 16 KB: Q or dO tile
+    static constexpr int ST = 3;                      // Q / dO / statistics stages
+    static constexpr uint32_t OFF_K = 0;
+    static constexpr uint32_t OFF_V = OFF_K + KTILE;
+    static constexpr uint32_t OFF_Q = OFF_V + KTILE;
+    static constexpr uint32_t OFF_DO = OFF_Q + ST * QTILE;
+    static constexpr uint32_t OFF_DST = OFF_DO + ST * QTILE;  // 128 keys x 64 queries half
+    static constexpr uint32_t OFF_STG = OFF_DST + 16384u;     // dQ tile, 64 x 128 fp32 rows
+    static constexpr uint32_t OFF_LD = OFF_STG + 32768u;      // ST x (64 L2 + 64 D) fp32
+    static constexpr uint32_t OFF_BAR = OFF_LD + ST * 512u;
+    static constexpr int B_KV = 0, B_QF = 1, B_QE = B_QF + ST, B_DOF = B_QE + ST,
+                         B_DOE = B_DOF + ST, B_SF = B_DOE + ST, B_DPF = B_SF + 2,
+                         B_PTF = B_DPF + 1, B_DVD = B_PTF + 1, B_DSF = B_DVD + 2,
+                         B_DQF = B_DSF + 1, B_DQE = B_DQF + 1, B_FIN = B_DQE + 1,
+                         B_DR = B_FIN + 1, B_ENDA = B_DR + 1, B_ENDB = B_ENDA + 1,
+                         B_SRD = B_ENDB + 1, B_STGF = B_SRD + 1, B_STGE = B_STGF + 1,
+                         NBAR = B_STGE + 1;
+    static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 192, COL_DV = 256, COL_DK = 384;
+    static constexpr int NCOMPUTE = 256, NDQ = 128;
+    static constexpr int NTHREADS = NCOMPUTE + NDQ + 64;
+    static constexpr int WARP_DQ0 = NCOMPUTE / 32;
+    static constexpr int WARP_TMA = WARP_DQ0 + NDQ / 32, WARP_MMA = WARP_TMA + 1;
+};
+
+template <bool BF16>
+__global__ void __launch_bounds__(448, 1)
+    attn_bwd_main128_kernel(const __grid_constant__ CUtensorMap tmQ,
+                            const __grid_constant__ CUtensorMap tmK,
+                            const __grid_constant__ CUtensorMap tmV,
+                            const __grid_constant__ CUtensorMap tmDO, const BwdParams p) {
+    using C = Bwd128Cfg;
+    constexpr int D = C::D;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // Work item: head-major, the heaviest key tile (j = 0 under the causal mask) first.
+    const int bh = static_cast<int>(blockIdx.x) / p.n_ktiles;
+    const int j = static_cast<int>(blockIdx.x) % p.n_ktiles;
+    const int n_q64 = (p.N + 63) / 64;
+    const int i_begin = p.causal ? 2 * j : 0;
+    const int n_it = n_q64 - i_begin;
+
+    const uint32_t bar0 = base + C::OFF_BAR;
+#define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + C::OFF_MISC);
+    volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(gbase + C::OFF_MISC + 4);
+    volatile uint32_t* last_flag = reinterpret_cast<volatile uint32_t*>(gbase + C::OFF_MISC + 8);
+    const float* sLD = reinterpret_cast<const float*>(gbase + C::OFF_LD);
+
+    if (threadIdx.x == 0) {
+        mbar_init(BAR(C::B_KV), 1);
+        for (int s = 0; s < C::ST; ++s) {
+            mbar_init(BAR(C::B_QF + s), 1);
+            mbar_init(BAR(C::B_QE + s), 1);
+            mbar_init(BAR(C::B_DOF + s), 1);
+            mbar_init(BAR(C::B_DOE + s), 1);
+        }
+        mbar_init(BAR(C::B_SF), 1);
+        mbar_init(BAR(C::B_SF + 1), 1);
+        mbar_init(BAR(C::B_DPF), 1);
+        mbar_init(BAR(C::B_PTF), C::NCOMPUTE);
+        mbar_init(BAR(C::B_DVD), 1);
+        mbar_init(BAR(C::B_DVD + 1), 1);
+        mbar_init(BAR(C::B_DSF), C::NCOMPUTE);
+        mbar_init(BAR(C::B_DQF), 1);
+        mbar_init(BAR(C::B_DQE), C::NDQ);
+        mbar_init(BAR(C::B_FIN), 1);
+        mbar_init(BAR(C::B_DR), 1);
+        mbar_init(BAR(C::B_ENDA), C::NCOMPUTE + C::NDQ);
+        mbar_init(BAR(C::B_ENDB), 1);
+        mbar_init(BAR(C::B_SRD), C::NCOMPUTE / 2);
+        mbar_init(BAR(C::B_STGF), C::NDQ);
+        mbar_init(BAR(C::B_STGE), 1);
+        *abort_flag = 0u;
+        *last_flag = 0u;
+        fence_mbar_init();
+    }
+    if (warp == C::WARP_MMA) {
+        tmem_alloc(base + C::OFF_MISC, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == C::WARP_TMA) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            tma_prefetch_desc(&tmDO);
+            mbar_arrive_expect_tx(BAR(C::B_KV), 2 * C::KTILE);
+#pragma unroll
+            for (int kb = 0; kb < 2; ++kb) {
+                tma_load_3d(base + C::OFF_K + kb * 16384u, &tmK, BAR(C::B_KV), kb * 64, j * 128, bh);
+                tma_load_3d(base + C::OFF_V + kb * 16384u, &tmV, BAR(C::B_KV), kb * 64, j * 128, bh);
+            }
+            int q_issued[C::ST], do_issued[C::ST];
+            for (int s = 0; s < C::ST; ++s) q_issued[s] = do_issued[s] = 0;
+            const size_t ld_row0 = static_cast<size_t>(bh) * p.Np;
+            for (int it = 0; it < n_it; ++it) {
+                const int i = i_begin + it;
+                const int s = it % C::ST, n = it / C::ST;
+                if (!wait_bounded(BAR(C::B_QE + s), (n & 1) ^ 1, abort_flag)) break;
+                const uint32_t sq = base + C::OFF_Q + s * C::QTILE;
+                const uint32_t sld = base + C::OFF_LD + s * 512u;
+                mbar_arrive_expect_tx(BAR(C::B_QF + s), C::QTILE + 512u);
+                tma_load_3d(sq, &tmQ, BAR(C::B_QF + s), 0, i * 64, bh);
+                tma_load_3d(sq + 8192u, &tmQ, BAR(C::B_QF + s), 64, i * 64, bh);
+                bulk_load(sld, p.l2pad + ld_row0 + i * 64, 256u, BAR(C::B_QF + s));
+                bulk_load(sld + 256u, p.dpad + ld_row0 + i * 64, 256u, BAR(C::B_QF + s));
+                q_issued[s] = n + 1;
+                if (!wait_bounded(BAR(C::B_DOE + s), (n & 1) ^ 1, abort_flag)) break;
+                const uint32_t sdo = base + C::OFF_DO + s * C::QTILE;
+                mbar_arrive_expect_tx(BAR(C::B_DOF + s), C::QTILE);
+                tma_load_3d(sdo, &tmDO, BAR(C::B_DOF + s), 0, i * 64, bh);
+                tma_load_3d(sdo + 8192u, &tmDO, BAR(C::B_DOF + s), 64, i * 64, bh);
+                do_issued[s] = n + 1;
+            }
+            if (*abort_flag) {
+                wait_drain(BAR(C::B_KV), 0);
+                for (int s = 0; s < C::ST; ++s) {
+                    if (q_issued[s] > 0) wait_drain(BAR(C::B_QF + s), (q_issued[s] - 1) & 1);
+                    if (do_issued[s] > 0) wait_drain(BAR(C::B_DOF + s), (do_issued[s] - 1) & 1);
+                }
+            }
+        }
+    } else if (warp == C::WARP_MMA) {
+        // ------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t ID_S = idesc_f16(BF16, 128, 64, false, false);   // S^T, dP^T
+            constexpr uint32_t ID_KV = idesc_f16(BF16, 128, 128, false, true);  // dV, dK
+            constexpr uint32_t ID_DQT = idesc_f16(BF16, 128, 64, true, true);   // dQ^T
+            const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sDST = base + C::OFF_DST;
+            bool ok = wait_bounded(BAR(C::B_KV), 0, abort_flag);
+            // S^T(t) = K Q_t^T into S buffer t & 1
+            auto issue_s = [&](int t) -> bool {
+                const int s = t % C::ST;
+                if (!wait_bounded(BAR(C::B_QF + s), (t / C::ST) & 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t sQ = base + C::OFF_Q + s * C::QTILE;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * 8192u + (kk & 3) * 32u;
+                    const uint32_t offk = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                    mma_ss(tmem + C::COL_S + (t & 1) * 64u, sdesc_sw128(sK + offk, 16, 1024),
+                           sdesc_sw128(sQ + off, 16, 1024), ID_S, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(BAR(C::B_SF + (t & 1)));
+                return true;
+            };
+            // Issue order per tile: dP^T(it), dV(it), S^T(it+1), dK(it) + dQ^T(it).
+            // Every wait below is for the newest phase its barrier can have
+            // reached, so no waiter can fall two phases behind.
+            if (ok && n_it > 0) ok = issue_s(0);
+            for (int it = 0; ok && it < n_it; ++it) {
+                const uint32_t ph = it & 1;
+                const int s = it % C::ST, n = it / C::ST;
+                const uint32_t sQ = base + C::OFF_Q + s * C::QTILE;
+                const uint32_t sDO = base + C::OFF_DO + s * C::QTILE;
+                // dP^T(it) = V dO^T: the compute warps have read dP^T(it-1)
+                if (!(ok = wait_bounded(BAR(C::B_DOF + s), n & 1, abort_flag))) break;
+                if (it >= 1 && !(ok = wait_bounded(BAR(C::B_DSF), ph ^ 1, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * 8192u + (kk & 3) * 32u;
+                    const uint32_t offk = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                    mma_ss(tmem + C::COL_DP, sdesc_sw128(sV + offk, 16, 1024),
+                           sdesc_sw128(sDO + off, 16, 1024), ID_S, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(BAR(C::B_DPF));
+                // dV += P^T dO (P^T from tensor memory)
+                if (!(ok = wait_bounded(BAR(C::B_PTF), ph, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ts(tmem + C::COL_DV, tmem + C::COL_S + (it & 1) * 64u + kk * 8u,
+                           sdesc_sw128(sDO + kk * 2048u, 8192, 1024), ID_KV,
+                           (it > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(BAR(C::B_DVD + (it & 1)));
+                mma_commit(BAR(C::B_DOE + s));
+                // S^T(it+1): its buffer held P^T(it-1), read by dV(it-1)
+                if (it + 1 < n_it) {
+                    if (it >= 1 && !(ok = wait_bounded(BAR(C::B_DVD + ((it - 1) & 1)),
+                                                       ((it - 1) >> 1) & 1, abort_flag)))
+                        break;
+                    if (!(ok = issue_s(it + 1))) break;
+                }
+                // dK += dS^T Q ; dQ^T = K^T dS^T (its columns drained for it-1)
+                if (!(ok = wait_bounded(BAR(C::B_DSF), ph, abort_flag))) break;
+                if (it >= 1 && !(ok = wait_bounded(BAR(C::B_DQE), ph ^ 1, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ss(tmem + C::COL_DK, sdesc_sw128(sDST + kk * 32u, 16, 1024),
+                           sdesc_sw128(sQ + kk * 2048u, 8192, 1024), ID_KV,
+                           (it > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(tmem + C::COL_DQ, sdesc_sw128(sK + kk * 2048u, 16384, 1024),
+                           sdesc_sw128(sDST + kk * 2048u, 8192, 1024), ID_DQT, kk > 0 ? 1u : 0u);
+                mma_commit(BAR(C::B_QE + s));
+                mma_commit(BAR(C::B_DQF));
+            }
+            if (ok) mma_commit(BAR(C::B_FIN));
+            if (*abort_flag) {
+                mma_commit(BAR(C::B_DR));
+                wait_drain(BAR(C::B_DR), 0);
+            }
+        }
+        __syncwarp();
+    } else if (warp >= C::WARP_DQ0) {
+        // --------------------------------------------------------- dQ warps
+        // Each tile's dQ^T leaves tensor memory at once (freeing its columns),
+        // is scaled and written as row-major fp32 rows into a shared staging
+        // tile (lane = feature: one 128-byte row segment per warp store), and
+        // one thread adds the whole tile into the fp32 accumulator with a
+        // single asynchronous bulk reduction.
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;  // TMEM lane = feature of dQ
+        const bool issuer = warp == C::WARP_DQ0 && lane == 0;
+        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        const uint32_t stg = base + C::OFF_STG + r * 4u;
+        float* acc_head = p.dqacc + static_cast<size_t>(bh) * p.N * D;
+        bool dq_ok = true;
+        for (int it = 0; it < n_it; ++it) {
+            const int q0 = (i_begin + it) * 64;
+            if (!(dq_ok = __all_sync(0xffffffffu,
+                                     wait_bounded(BAR(C::B_DQF), it & 1, abort_flag))))
+                break;
+            tc_fence_after();
+            uint32_t v[2][32];
+            tmem_ld32(lane_addr + C::COL_DQ, v[0]);
+            tmem_ld32(lane_addr + C::COL_DQ + 32u, v[1]);
+            tmem_ld_wait();
+            reg_fence32(v[0]);
+            reg_fence32(v[1]);
+            tc_fence_before();
+            mbar_arrive(BAR(C::B_DQE));  // the values are in registers: columns free
+            // the previous tile's bulk reduction has finished reading the staging tile
+            if (it >= 1 && !(dq_ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_STGE),
+                                                                         (it - 1) & 1, abort_flag))))
+                break;
+#pragma unroll
+            for (int e = 0; e < 64; ++e)
+                st_shared_f32(stg + e * 512u, __uint_as_float(v[e >> 5][e & 31]) * p.scale);
+            fence_proxy_async_smem();
+            mbar_arrive(BAR(C::B_STGF));
+            if (issuer) {
+                if (!wait_bounded(BAR(C::B_STGF), it & 1, abort_flag)) {
+                    dq_ok = false;
+                } else {
+                    const int nq = min(64, p.N - q0);
+                    bulk_reduce_add_f32(acc_head + static_cast<size_t>(q0) * D,
+                                        base + C::OFF_STG, static_cast<uint32_t>(nq) * 512u);
+                    bulk_commit();
+                    bulk_wait_read_all();
+                    mbar_arrive(BAR(C::B_STGE));
+                }
+            }
+            dq_ok = __all_sync(0xffffffffu, dq_ok);
+            if (!dq_ok) break;
+        }
+        if (issuer) {
+            // every reduction complete and visible before the completion count
+            bulk_wait_all();
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            __threadfence();
+        }
+    } else {
+        // ---------------------------------------------------------- compute
+        const int quarter = warp & 3, half = warp >> 2;
+        const int r = quarter * 32 + lane;  // TMEM lane = key row of the tile
+        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        const int key = j * 128 + r;
+        const bool key_valid = key < p.N;
+        const float sl = p.scale_log2;
+        const size_t head_row0 = static_cast<size_t>(bh) * p.N;
+        const uint32_t sDST = base + C::OFF_DST;
+        const int c0 = half * 32;  // first query column of this thread's half
+        bool ok = true;
+        for (int it = 0; it < n_it; ++it) {
+            const int i = i_begin + it;
+            const int q0 = i * 64;
+            const uint32_t ph = it & 1;
+            const int s = it % C::ST;
+            const float4* L4 = reinterpret_cast<const float4*>(sLD + s * 128 + c0);
+            const float4* D4 = reinterpret_cast<const float4*>(sLD + s * 128 + 64 + c0);
+            const uint32_t colS = C::COL_S + (it & 1) * 64u;
+
+            // ---- P^T = exp2(S^T scale log2e - L2), written back over S^T
+            ok = __all_sync(0xffffffffu,
+                            wait_bounded(BAR(C::B_QF + s), (it / C::ST) & 1, abort_flag));
+            if (ok)
+                ok = __all_sync(0xffffffffu,
+                                wait_bounded(BAR(C::B_SF + (it & 1)), (it >> 1) & 1, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            float pv[32];
+            {
+                uint32_t sv[32];
+                tmem_ld32(lane_addr + colS + c0, sv);
+                tmem_ld_wait();
+                reg_fence32(sv);
+                if (half == 0) {  // half 1 writes P^T over columns half 0 reads
+                    tc_fence_before();
+                    mbar_arrive(BAR(C::B_SRD));
+                }
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    const float4 l4 = L4[g];
+                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        pv[4 * g + e] = ex2(fmaf(__uint_as_float(sv[4 * g + e]), sl, -lv[e]));
+                }
+                // query q0 + c0 + c sees key j*128 + r iff q0 + c0 + c >= key
+                if (!key_valid || (p.causal && q0 < (j + 1) * 128)) {
+                    const int lo = key_valid ? key - q0 - c0 : 32;
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        if (c < lo) pv[c] = 0.f;
+                }
+                uint32_t pk[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c) pk[c] = pack2<BF16>(pv[2 * c], pv[2 * c + 1]);
+                if (half == 1) {
+                    ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SRD), ph, abort_flag));
+                    tc_fence_after();
+                }
+                if (ok) {
+                    tmem_st16(lane_addr + colS + half * 16u, pk);
+                    tmem_st_wait();
+                }
+            }
+            if (!ok) break;
+            tc_fence_before();
+            mbar_arrive(BAR(C::B_PTF));
+
+            // ---- dS^T = P^T (dP^T - D), half, into shared memory
+            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_DPF), ph, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            {
+                uint32_t dpv[32];
+                tmem_ld32(lane_addr + C::COL_DP + c0, dpv);
+                tmem_ld_wait();
+                reg_fence32(dpv);
+                tc_fence_before();
+                float dsv[32];
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    const float4 d4 = D4[g];
+                    const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dsv[4 * g + e] = pv[4 * g + e] * (__uint_as_float(dpv[4 * g + e]) - dd[e]);
+                }
+#pragma unroll
+                for (int g = 0; g < 4; ++g)  // 16-byte chunks 4 half + g of the 128-byte key row
+                    st_shared_v4(sDST + sw128_off(r, half * 4 + g),
+                                 pack2<BF16>(dsv[8 * g + 0], dsv[8 * g + 1]),
+                                 pack2<BF16>(dsv[8 * g + 2], dsv[8 * g + 3]),
+                                 pack2<BF16>(dsv[8 * g + 4], dsv[8 * g + 5]),
+                                 pack2<BF16>(dsv[8 * g + 6], dsv[8 * g + 7]));
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(BAR(C::B_DSF));
+        }
+        if (ok) ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_FIN), 0, abort_flag));
+        if (ok) {  // dK_j, dV_j rows: lane r holds key row j*128 + r; this half, 64 features
+            tc_fence_after();
+            const size_t rowoff = (head_row0 + key) * (D * 2) + half * D;
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                uint8_t* out = static_cast<uint8_t*>(which ? p.dv : p.dk) + rowoff;
+                const uint32_t colA = (which ? C::COL_DV : C::COL_DK) + half * 64u;
+                const float mul = which ? 1.f : p.scale;
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(lane_addr + colA + c * 32u, v);
+                    tmem_ld_wait();
+                    reg_fence32(v);
+                    uint32_t h[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        h[e] = pack2<BF16>(__uint_as_float(v[2 * e]) * mul,
+                                           __uint_as_float(v[2 * e + 1]) * mul);
+                    if (key_valid) {
+                        uint4* d4 = reinterpret_cast<uint4*>(out + c * 64);
+                        d4[0] = make_uint4(h[0], h[1], h[2], h[3]);
+                        d4[1] = make_uint4(h[4], h[5], h[6], h[7]);
+                        d4[2] = make_uint4(h[8], h[9], h[10], h[11]);
+                        d4[3] = make_uint4(h[12], h[13], h[14], h[15]);
+                    }
+                }
+            }
+        }
+    }
+    if (warp < C::WARP_TMA) {
+        // The last CTA of this head to finish converts the head's dQ.  Bounded
+        // mbarrier syncs (not bar.sync): a warp that gave up cannot leave the
+        // others waiting for ever.
+        const int tid = threadIdx.x;  // 0 .. NCOMPUTE + NDQ - 1
+        bool ok = __all_sync(0xffffffffu, *abort_flag == 0u);
+        if (ok) {
+            __threadfence();
+            mbar_arrive(BAR(C::B_ENDA));
+            if (tid == 0) {
+                if (wait_bounded(BAR(C::B_ENDA), 0, abort_flag)) {
+                    const int done = atomicAdd(p.counters + bh, 1);
+                    *last_flag = (done == p.n_ktiles - 1) ? 1u : 0u;
+                }
+                mbar_arrive(BAR(C::B_ENDB));
+            }
+            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_ENDB), 0, abort_flag));
+        }
+        if (ok && *last_flag) {
+            __threadfence();
+            const size_t head_row0 = static_cast<size_t>(bh) * p.N;
+            const float4* src = reinterpret_cast<const float4*>(p.dqacc + head_row0 * D);
+            uint2* out = reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.dq) + head_row0 * D * 2);
+            const long long n4 = static_cast<long long>(p.N) * D / 4;
+            for (long long e = tid; e < n4; e += C::NCOMPUTE + C::NDQ) {
+                const float4 x = __ldcg(src + e);
+                out[e] = make_uint2(pack2<BF16>(x.x, x.y), pack2<BF16>(x.z, x.w));
+            }
+        }
+    }
+#undef BAR
+    tc_fence_before();
+    __syncthreads();
+    if (warp == C::WARP_MMA) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+inline bool bwd128_set_attributes() {
+    return cudaFuncSetAttribute(attn_bwd_main128_kernel<true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Bwd128Cfg::SMEM_BYTES) == cudaSuccess &&
+           cudaFuncSetAttribute(attn_bwd_main128_kernel<false>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Bwd128Cfg::SMEM_BYTES) == cudaSuccess;
+}
+
+// mq, mdo must be tensor maps with 64-row boxes; mk, mv with 128-row boxes.
+template <bool BF16>
+int bwd_main128_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                       const CUtensorMap& mdo, void* dq, void* dk, void* dv, void* ws, int B,
+                       int H, int N, int causal, float scale, cudaStream_t st) {
+    BwdParams p;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    p.l2pad = reinterpret_cast<const float*>(w);
+    p.dpad = reinterpret_cast<const float*>(w + bwd_ws_off_d(B, H, N));
+    p.dqacc = reinterpret_cast<float*>(w + bwd_ws_off_dq(B, H, N));
+    p.counters = reinterpret_cast<int*>(w + bwd_ws_off_cnt(B, H, N, 128));
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    p.BH = B * H;
+    p.N = N;
+    p.Np = static_cast<int>(bwd_np(N));
+    p.n_qtiles = (N + 63) / 64;
+    p.n_ktiles = (N + 127) / 128;
+    p.causal = causal;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    const long long nblocks = 1LL * p.n_ktiles * p.BH;
+    if (nblocks >= (1LL << 31)) return -2;
+    attn_bwd_main128_kernel<BF16><<<static_cast<unsigned>(nblocks), Bwd128Cfg::NTHREADS,
+                                    Bwd128Cfg::SMEM_BYTES, st>>>(mq, mk, mv, mdo, p);
+    return cudaGetLastError() == cudaSuccess ? 0 : -7;
+}
+
+}  // namespace attn
