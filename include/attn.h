@@ -172,6 +172,10 @@ int attn_last_device_status(void* stream);
  */
 int attn_selftest_wait_timeout(unsigned timeout_us, void* stream);
 
+/* Text of the last CUDA runtime error this library reported (on this host
+ * thread) as ATTN_ERR_LAUNCH or ATTN_ERR_DEVICE; "no error" if none. */
+const char* attn_last_cuda_error_string(void);
+
 /* Static description of a status code. */
 const char* attn_strerror(int status);
 

@@ -32,7 +32,7 @@ BWD_LAUNCHES = 2
 # Every symbol include/attn.h declares.
 EXPORTS = ("attn_fwd", "attn_bwd", "attn_bwd_prep", "attn_bwd_main", "attn_bwd_workspace_bytes",
            "attn_bwd_noalloc", "attn_last_device_status", "attn_selftest_wait_timeout",
-           "attn_strerror", "attn_version")
+           "attn_last_cuda_error_string", "attn_strerror", "attn_version")
 
 # Size of the built-in scratch attn_bwd_noalloc uses (bytes, per device).
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -41,7 +41,10 @@ NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 class AttnError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {STATUS.get(status, status)} ({strerror(status)})")
+        extra = ""
+        if status in (-6, -7):
+            extra = f"; CUDA: {lib().attn_last_cuda_error_string().decode()}"
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({strerror(status)}{extra})")
 
 
 _lib = None
@@ -73,6 +76,8 @@ def lib() -> ctypes.CDLL:
         L.attn_selftest_wait_timeout.restype = ci
         L.attn_strerror.argtypes = [ci]
         L.attn_strerror.restype = ctypes.c_char_p
+        L.attn_last_cuda_error_string.argtypes = []
+        L.attn_last_cuda_error_string.restype = ctypes.c_char_p
         L.attn_version.argtypes = []
         L.attn_version.restype = ctypes.c_char_p
         _lib = L

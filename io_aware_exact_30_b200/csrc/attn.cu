@@ -20,6 +20,15 @@ namespace {
 
 using attn::FwdCfg;
 
+// Last CUDA runtime error this library turned into ATTN_ERR_LAUNCH/DEVICE.
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+bool launch_ok() {
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) g_last_cuda_error = e;
+    return e == cudaSuccess;
+}
+
 constexpr int kMaxDevices = 64;
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -75,10 +84,11 @@ int check_device(int* dev_out) {
     ok &= attn::bwd_set_attributes();
     ok &= attn::bwd128_set_attributes();
     if (!ok) {
-        cudaGetLastError();
+        g_last_cuda_error = cudaGetLastError();
         g_dev_state[dev] = -1;
         return ATTN_ERR_DEVICE;
     }
+    attn::bwd_error_hook() = [](cudaError_t e) { g_last_cuda_error = e; };
     g_dev_state[dev] = 1;
     return ATTN_OK;
 }
@@ -127,11 +137,11 @@ bool make_map(CUtensorMap* m, const void* ptr, int dtype, int BH, int N, int d,
 template <int D, bool BF16>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const attn::FwdParams& p, cudaStream_t st) {
-    const long long nblocks = 1LL * p.n_qtiles * p.BH;
+    const long long nblocks = 1LL * p.n_pairs * p.BH;
     if (nblocks >= (1LL << 31)) return ATTN_ERR_SHAPE;
     attn::attn_fwd_kernel<D, BF16><<<static_cast<unsigned>(nblocks), FwdCfg<D>::NTHREADS,
                                      FwdCfg<D>::SMEM_BYTES, st>>>(mq, mk, mv, p);
-    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+    return launch_ok() ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
 __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
@@ -200,6 +210,7 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
     p.BH = BH;
     p.N = N;
     p.n_qtiles = (N + 127) / 128;
+    p.n_pairs = (p.n_qtiles + 1) / 2;
     p.causal = causal ? 1 : 0;
     p.scale_log2 = scale * 1.4426950408889634f;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -348,7 +359,7 @@ int attn_selftest_wait_timeout(unsigned timeout_us, void* stream) {
     if (rc) return rc;
     selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<unsigned long long>(timeout_us) * 1000ull);
-    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+    return launch_ok() ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
 const char* attn_strerror(int status) {
@@ -369,5 +380,7 @@ const char* attn_strerror(int status) {
 }
 
 const char* attn_version(void) { return "0.1.0"; }
+
+const char* attn_last_cuda_error_string(void) { return cudaGetErrorString(g_last_cuda_error); }
 
 }  // extern "C"

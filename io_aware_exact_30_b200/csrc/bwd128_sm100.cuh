@@ -29,16 +29,6 @@
 
 namespace attn {
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-        "r"(r[15])
-        : "memory");
-}
-
 struct Bwd128Cfg {
     static constexpr int D = 128;
     static constexpr int QT = 64;                     // query rows per inner tile
@@ -527,7 +517,9 @@ int bwd_main128_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     if (nblocks >= (1LL << 31)) return -2;
     attn_bwd_main128_kernel<BF16><<<static_cast<unsigned>(nblocks), Bwd128Cfg::NTHREADS,
                                     Bwd128Cfg::SMEM_BYTES, st>>>(mq, mk, mv, mdo, p);
-    return cudaGetLastError() == cudaSuccess ? 0 : -7;
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) bwd_record_error(e);
+    return e == cudaSuccess ? 0 : -7;
 }
 
 }  // namespace attn

@@ -48,6 +48,15 @@
 
 namespace attn {
 
+// Hook the host side installs to keep the last CUDA error of a launch.
+inline void (*&bwd_error_hook())(cudaError_t) {
+    static void (*hook)(cudaError_t) = nullptr;
+    return hook;
+}
+inline void bwd_record_error(cudaError_t e) {
+    if (bwd_error_hook()) bwd_error_hook()(e);
+}
+
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Workspace: L2 (BH*Np fp32) | D (BH*Np fp32) | dQ accumulator (BH*N*d fp32) |
@@ -586,7 +595,9 @@ int bwd_prep_launch(const void* o, const void* dout, const float* lse, void* ws,
         reinterpret_cast<float*>(w), reinterpret_cast<float*>(w + bwd_ws_off_d(B, H, N)),
         reinterpret_cast<float4*>(w + bwd_ws_off_dq(B, H, N)),
         reinterpret_cast<int*>(w + bwd_ws_off_cnt(B, H, N, D)), N, Np, rows_padded, B * H);
-    return cudaGetLastError() == cudaSuccess ? 0 : -7;
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) bwd_record_error(e);
+    return e == cudaSuccess ? 0 : -7;
 }
 
 template <int D, bool BF16>
@@ -614,7 +625,9 @@ int bwd_main_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensor
     if (nblocks >= (1LL << 31)) return -2;
     attn_bwd_main_kernel<D, BF16><<<static_cast<unsigned>(nblocks), BwdCfg<D>::NTHREADS,
                                     BwdCfg<D>::SMEM_BYTES, st>>>(mq, mk, mv, mdo, p);
-    return cudaGetLastError() == cudaSuccess ? 0 : -7;
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) bwd_record_error(e);
+    return e == cudaSuccess ? 0 : -7;
 }
 
 }  // namespace attn

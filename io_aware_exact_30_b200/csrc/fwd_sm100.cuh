@@ -1,30 +1,43 @@
-// Forward kernel: exact attention, one 128-row query tile per CTA, streaming
-// 128-key tiles of K and V through a TMA pipeline, scores and output
-// accumulated in tensor memory by tcgen05 MMAs, softmax statistics kept per
-// row in registers with the online (running max / running sum) recurrence.
+// Forward kernel: exact attention, two 128-row query tiles per CTA sharing
+// each 128-key tile of K and V streamed through a TMA pipeline; scores and
+// outputs accumulate in tensor memory through tcgen05 MMAs; softmax
+// statistics live per row in registers and follow the online (running max /
+// running sum) recurrence.
 //
 // Method: "Is a full day of context better than ten minutes? FlashAttention
 // and the sequence-length question" (marketmaker.cc), sections "Flash
 // Attention algorithm" (tiles of Q, K, V staged on chip, S_ij and P_ij never
 // leave it), "online softmax recurrence" (the accumulator is rescaled by
-// exp(m_old - m_new) whenever the running max grows), "FA2: parallelism"
+// exp(m_old - m_new) when the running max grows), "FA2: parallelism"
 // (normalise by the running sum once, after the last tile; parallel over
-// query tiles; one thread owns one query row so no cross-warp reduction),
-// "FA3: Hopper" (asynchronous producer/consumer warps, the score MMA of one
-// block overlapping the softmax of the previous one) and "causal masking"
-// (key tiles wholly in the future of the query tile are neither loaded nor
-// computed; only the diagonal tile is masked element-wise).  The statistic
-// written out is the log-sum-exp — "Performance optimisation with
+// query tiles; one thread owns one query row so there is no cross-warp
+// reduction), "FA3: Hopper" (asynchronous producer and consumer warps; the
+// matmul of one block overlaps the softmax of another) and "causal masking"
+// (key tiles wholly in the future of a query tile are neither loaded for it
+// nor computed; only diagonal tiles are masked element-wise).  The row
+// statistic written out is the log-sum-exp — "Performance optimisation with
 // Flash-Attention 2" (Medium), section "Flash Attention 2".
 //
-// Roles (192 threads):
-//   warps 0-3  softmax: thread t owns query row t = TMEM lane t
-//   warp 4     TMA producer (one lane)
-//   warp 5     TMEM allocator and tcgen05 MMA issuer (one lane)
-// Tensor memory (512 columns): S double buffer at columns 0 and 128 (fp32,
-// 128 x 128 each), O accumulator at column 256 (fp32, 128 x D).
-// Shared memory: Q tile, STAGES x (K tile, V tile), P tile (bf16/fp16,
-// 128 x 128), all in the 128-byte-swizzled K-major layout TMA writes.
+// B200 form:
+//  - Two query tiles (2p, 2p+1) per CTA, each with its own softmax warpgroup;
+//    while one group exponentiates its tile, the tensor core computes the
+//    other tile's S = Q K^T or P V, so MMA and MUFU work overlap.
+//  - P is written back into tensor memory over its S (half precision, two
+//    values per 32-bit column) and is the A operand of O += P V, so P never
+//    touches shared memory.
+//  - The max used for the exponent is only moved (and O rescaled) when the
+//    row max grows by more than 2^8; otherwise the stale max is kept.  Every
+//    exponent and the final normaliser use the same max, so the result is
+//    the same softmax; values stay below 2^8 times their normalised size.
+//  - The per-element arithmetic uses the packed fp32x2 instructions; the
+//    exponentials stay on the multi-function unit (measured: moving a share
+//    of them to a polynomial on the FMA pipe costs more issue slots than it
+//    saves here).
+//
+// Roles (320 threads): warps 0-3 softmax of tile 0, warps 4-7 softmax of tile
+// 1 (thread t of a group owns query row t = TMEM lane t), warp 8 TMA
+// producer, warp 9 TMEM owner and MMA issuer.
+// Tensor memory: S/P of tile i at column 128 i, O of tile i at 256 + D i.
 #pragma once
 
 #include "ptx.cuh"
@@ -37,6 +50,7 @@ struct FwdParams {
     int BH;
     int N;
     int n_qtiles;
+    int n_pairs;
     int causal;
     float scale_log2;  // scale * log2(e)
 };
@@ -45,33 +59,28 @@ template <int D>
 struct FwdCfg {
     static constexpr int KB = D / 64;                 // 64-column swizzle blocks per row
     static constexpr uint32_t TILE = 128u * D * 2u;   // bytes of a 128 x D half tile
-    static constexpr int STAGES = 2;
-    static constexpr uint32_t P_BYTES = 128u * 128u * 2u;
-    static constexpr uint32_t OFF_Q = 0;
-    static constexpr uint32_t OFF_K = OFF_Q + TILE;
+    static constexpr int STAGES = D == 64 ? 4 : 2;
+    static constexpr uint32_t OFF_Q = 0;              // two query tiles
+    static constexpr uint32_t OFF_K = OFF_Q + 2 * TILE;
     static constexpr uint32_t OFF_V = OFF_K + STAGES * TILE;
-    static constexpr uint32_t OFF_P = OFF_V + STAGES * TILE;
-    static constexpr uint32_t OFF_BAR = OFF_P + P_BYTES;
-    // barrier indices
-    static constexpr int B_Q = 0;
-    static constexpr int B_KF = 1;
-    static constexpr int B_VF = B_KF + STAGES;
-    static constexpr int B_KE = B_VF + STAGES;
-    static constexpr int B_SF = B_KE + STAGES;
-    static constexpr int B_SE = B_SF + 2;
-    static constexpr int B_PF = B_SE + 2;
-    static constexpr int B_OD = B_PF + 1;
-    static constexpr int B_DR = B_OD + 1;
-    static constexpr int NBAR = B_DR + 1;
+    static constexpr uint32_t OFF_BAR = OFF_V + STAGES * TILE;
+    static constexpr int B_Q = 0, B_KF = 1, B_VF = B_KF + STAGES, B_KE = B_VF + STAGES,
+                         B_SF = B_KE + STAGES, B_PF = B_SF + 2, B_OD = B_PF + 2, B_DR = B_OD + 2,
+                         NBAR = B_DR + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_O = 256;
-    static constexpr int NTHREADS = 192;
+    static constexpr int NTHREADS = 320;
+    static constexpr int WARP_TMA = 8, WARP_MMA = 9;
 };
 
+// Move the running max (and rescale O) only when the row max grows by more
+// than this many binary orders of magnitude.
+constexpr float kRescaleThreshold = 8.f;
+
 template <int D, bool BF16>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
     using C = FwdCfg<D>;
@@ -82,13 +91,15 @@ __global__ void __launch_bounds__(192, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Work item: head-major, so the CTAs resident at one time share a few
-    // heads' K/V in L2; within a head the heaviest query tile (largest index
-    // under the causal mask) goes first.
-    const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x) % p.n_qtiles;
-    const int bh = static_cast<int>(blockIdx.x) / p.n_qtiles;
+    // Work item: head-major; within a head the heaviest pair of query tiles first.
+    const int pair = p.n_pairs - 1 - static_cast<int>(blockIdx.x) % p.n_pairs;
+    const int bh = static_cast<int>(blockIdx.x) / p.n_pairs;
     const int n_kv_all = (p.N + 127) >> 7;
-    const int nkv = p.causal ? min(n_kv_all, qt + 1) : n_kv_all;
+    const bool has1 = 2 * pair + 1 < p.n_qtiles;
+    int nkv_t[2];
+    nkv_t[0] = p.causal ? min(n_kv_all, 2 * pair + 1) : n_kv_all;
+    nkv_t[1] = has1 ? (p.causal ? min(n_kv_all, 2 * pair + 2) : n_kv_all) : 0;
+    const int nkv = max(nkv_t[0], nkv_t[1]);
 
     const uint32_t bar0 = base + C::OFF_BAR;
 #define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
@@ -102,17 +113,16 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(BAR(C::B_VF + s), 1);
             mbar_init(BAR(C::B_KE + s), 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(BAR(C::B_SF + b), 1);
-            mbar_init(BAR(C::B_SE + b), 128);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(BAR(C::B_SF + t), 1);
+            mbar_init(BAR(C::B_PF + t), 128);
+            mbar_init(BAR(C::B_OD + t), 1);
         }
-        mbar_init(BAR(C::B_PF), 128);
-        mbar_init(BAR(C::B_OD), 1);
         mbar_init(BAR(C::B_DR), 1);
         *abort_flag = 0u;
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == C::WARP_MMA) {
         tmem_alloc(base + C::OFF_MISC, C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -121,16 +131,18 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp == C::WARP_TMA) {
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
-            mbar_arrive_expect_tx(BAR(C::B_Q), C::TILE);
+            mbar_arrive_expect_tx(BAR(C::B_Q), has1 ? 2 * C::TILE : C::TILE);
+            for (int t = 0; t < (has1 ? 2 : 1); ++t)
 #pragma unroll
-            for (int kb = 0; kb < C::KB; ++kb)
-                tma_load_3d(base + C::OFF_Q + kb * 16384u, &tmQ, BAR(C::B_Q), kb * 64, qt * 128, bh);
+                for (int kb = 0; kb < C::KB; ++kb)
+                    tma_load_3d(base + C::OFF_Q + t * C::TILE + kb * 16384u, &tmQ, BAR(C::B_Q),
+                                kb * 64, (2 * pair + t) * 128, bh);
             int issued[C::STAGES];
 #pragma unroll
             for (int s = 0; s < C::STAGES; ++s) issued[s] = 0;
@@ -158,44 +170,67 @@ __global__ void __launch_bounds__(192, 1)
                     }
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == C::WARP_MMA) {
         // ------------------------------------------------------- MMA issuer
+        // Order per key tile j: O_0 += P_0 V_j, S_0 = Q_0 K_{j+1}^T,
+        // O_1 += P_1 V_j, S_1 = Q_1 K_{j+1}^T; each S is issued once the P V
+        // that reads the same tensor-memory columns has completed, without
+        // waiting for the other tile's softmax.
         if (lane == 0) {
             constexpr uint32_t ID_S = idesc_f16(BF16, 128, 128, false, false);
             constexpr uint32_t ID_O = idesc_f16(BF16, 128, D, false, true);
             bool ok = wait_bounded(BAR(C::B_Q), 0, abort_flag);
-            tc_fence_after();
-            for (int j = 0; ok && j <= nkv; ++j) {
-                if (j < nkv) {  // S(j) = Q K_j^T into S buffer j & 1
-                    const int s = j % C::STAGES, n = j / C::STAGES, b = j & 1, nb = j >> 1;
-                    if (!wait_bounded(BAR(C::B_KF + s), n & 1, abort_flag)) break;
-                    if (!wait_bounded(BAR(C::B_SE + b), (nb & 1) ^ 1, abort_flag)) break;
-                    tc_fence_after();
-                    const uint32_t sq = base + C::OFF_Q, sk = base + C::OFF_K + s * C::TILE;
+            auto issue_s = [&](int t, int j) {
+                const uint32_t sq = base + C::OFF_Q + t * C::TILE;
+                const uint32_t sk = base + C::OFF_K + (j % C::STAGES) * C::TILE;
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                        mma_ss(tmem + b * 128u, sdesc_sw128(sq + off, 16, 1024),
-                               sdesc_sw128(sk + off, 16, 1024), ID_S, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(BAR(C::B_SF + b));
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                    mma_ss(tmem + t * 128u, sdesc_sw128(sq + off, 16, 1024),
+                           sdesc_sw128(sk + off, 16, 1024), ID_S, kk > 0 ? 1u : 0u);
                 }
-                if (j >= 1) {  // O += P(j-1) V_{j-1}
-                    const int jp = j - 1, sp = jp % C::STAGES, np = jp / C::STAGES;
-                    if (!wait_bounded(BAR(C::B_PF), jp & 1, abort_flag)) break;
-                    if (!wait_bounded(BAR(C::B_VF + sp), np & 1, abort_flag)) break;
+                mma_commit(BAR(C::B_SF + t));
+            };
+            if (ok && nkv > 0) {
+                ok = wait_bounded(BAR(C::B_KF), 0, abort_flag);
+                if (ok) {
                     tc_fence_after();
-                    const uint32_t sP = base + C::OFF_P, sv = base + C::OFF_V + sp * C::TILE;
+                    for (int t = 0; t < 2; ++t)
+                        if (nkv_t[t] > 0) issue_s(t, 0);
+                }
+            }
+            for (int j = 0; ok && j < nkv; ++j) {
+                const int s = j % C::STAGES, n = j / C::STAGES;
+                if (!(ok = wait_bounded(BAR(C::B_VF + s), n & 1, abort_flag))) break;
+                const uint32_t sv = base + C::OFF_V + s * C::TILE;
+                bool k_next = false;  // K_{j+1} has landed
+                for (int t = 0; ok && t < 2; ++t) {
+                    if (j >= nkv_t[t]) continue;
+                    if (!(ok = wait_bounded(BAR(C::B_PF + t), j & 1, abort_flag))) break;
+                    tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        mma_ss(tmem + C::COL_O,
-                               sdesc_sw128(sP + (kk >> 2) * 16384u + (kk & 3) * 32u, 16, 1024),
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(tmem + C::COL_O + t * D, tmem + t * 128u + kk * 8u,
                                sdesc_sw128(sv + kk * 2048u, 16384, 1024), ID_O,
-                               (jp > 0 || kk > 0) ? 1u : 0u);
+                               (j > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(BAR(C::B_OD + t));
+                    // This tile's next S as soon as its P V has read P (the other
+                    // tile's softmax is not waited for).
+                    if (j + 1 < nkv_t[t]) {
+                        if (!k_next) {
+                            const int s1 = (j + 1) % C::STAGES;
+                            if (!(ok = wait_bounded(BAR(C::B_KF + s1), ((j + 1) / C::STAGES) & 1,
+                                                    abort_flag)))
+                                break;
+                            k_next = true;
+                        }
+                        if (!(ok = wait_bounded(BAR(C::B_OD + t), j & 1, abort_flag))) break;
+                        tc_fence_after();
+                        issue_s(t, j + 1);
                     }
-                    mma_commit(BAR(C::B_KE + sp));
-                    mma_commit(BAR(C::B_OD));
                 }
+                if (!ok) break;
+                mma_commit(BAR(C::B_KE + s));
             }
             if (*abort_flag) {  // every issued MMA must finish before TMEM is freed
                 mma_commit(BAR(C::B_DR));
@@ -205,89 +240,127 @@ __global__ void __launch_bounds__(192, 1)
         __syncwarp();
     } else {
         // ---------------------------------------------------------- softmax
-        const int r = threadIdx.x;  // row of the tile == TMEM lane
-        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-        const int qrow = qt * 128 + r;
+        const int t = warp >> 2;          // query tile of this warpgroup
+        const int r = threadIdx.x & 127;  // row of the tile == TMEM lane
+        const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        const uint32_t colS = t * 128u, colO = C::COL_O + t * D;
+        const int qrow = (2 * pair + t) * 128 + r;
+        const int my_nkv = nkv_t[t];
         const float sl = p.scale_log2;
         float m = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int j = 0; j < nkv; ++j) {
-            const int b = j & 1, nb = j >> 1;
-            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SF + b), nb & 1, abort_flag));
+        for (int j = 0; j < my_nkv; ++j) {
+            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SF + t), j & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            uint32_t sr[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + b * 128u + c * 32u, sr[c]);
-            tmem_ld_wait();
-#pragma unroll
-            for (int c = 0; c < 4; ++c) reg_fence32(sr[c]);
-            tc_fence_before();
-            mbar_arrive(BAR(C::B_SE + b));
-
-            float s[128];
-#pragma unroll
-            for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
             // keys at or past N, and (causal) keys after this query, are masked
             const int key0 = j * 128;
             int limit = p.N - key0;
             if (p.causal) limit = min(limit, qrow - key0 + 1);
-            if (limit < 128) {
+            // pass 1: row max over the 128 scores (two chunks of 64 in flight);
+            // tiles without masked columns (all but diagonal and tail tiles)
+            // take the unmasked path
+            const bool full = __all_sync(0xffffffffu, limit >= 128);
+            float mx = -INFINITY;
 #pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    if (c >= limit) s[c] = -INFINITY;
+            for (int h = 0; h < 2; ++h) {
+                uint32_t a[32], b[32];
+                tmem_ld32(lane_addr + colS + h * 64u, a);
+                tmem_ld32(lane_addr + colS + h * 64u + 32u, b);
+                tmem_ld_wait();
+                reg_fence32(a);
+                reg_fence32(b);
+                if (full) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        mx = max3(mx, __uint_as_float(a[e]), __uint_as_float(a[e + 1]));
+                        mx = max3(mx, __uint_as_float(b[e]), __uint_as_float(b[e + 1]));
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int ca = h * 64 + e, cb = ca + 32;
+                        if (ca < limit) mx = fmaxf(mx, __uint_as_float(a[e]));
+                        if (cb < limit) mx = fmaxf(mx, __uint_as_float(b[e]));
+                    }
+                }
             }
-            float mx = s[0];
-#pragma unroll
-            for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
-            const float m_new = fmaxf(m, mx * sl);
-            const float alpha = ex2(m - m_new);
-            float sum = 0.f;
-#pragma unroll
-            for (int c = 0; c < 128; ++c) {
-                s[c] = ex2(fmaf(s[c], sl, -m_new));
-                sum += s[c];
-            }
-            l = fmaf(l, alpha, sum);
-            m = m_new;
-
-            if (j >= 1) {  // PV(j-1) must be done: O is rescaled and P's buffer reused
-                ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_OD), (j - 1) & 1, abort_flag));
-                if (!ok) break;
-                tc_fence_after();
-                if (__any_sync(0xffffffffu, alpha != 1.f)) {
+            const float m_tile = mx * sl;
+            // Move the max only when it grows past the threshold (the first
+            // tile always sets it); rescaling O needs O(j-1) complete.
+            const bool move = m_tile > m + kRescaleThreshold;
+            if (__any_sync(0xffffffffu, move)) {
+                const float m_new = move ? m_tile : m;
+                const float alpha = ex2(m - m_new);  // 0 on the first tile, 1 if not moved
+                if (j > 0) {
+                    ok = __all_sync(0xffffffffu,
+                                    wait_bounded(BAR(C::B_OD + t), (j - 1) & 1, abort_flag));
+                    if (!ok) break;
+                    tc_fence_after();
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t o[32];
-                        tmem_ld32(lane_addr + C::COL_O + c * 32u, o);
+                        tmem_ld32(lane_addr + colO + c * 32u, o);
                         tmem_ld_wait();
                         reg_fence32(o);
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
                             o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tmem_st32(lane_addr + C::COL_O + c * 32u, o);
+                        tmem_st32(lane_addr + colO + c * 32u, o);
                     }
                     tmem_st_wait();
                 }
+                l *= alpha;
+                m = m_new;
             }
-            // P (rounded to the input type) into the swizzled K-major tile
-            const uint32_t sP = base + C::OFF_P;
+            // pass 2: P = 2^(s scale log2e - m) chunk by chunk, written back as
+            // half over columns pass 2 has already read (P chunk c -> 16c..16c+15)
+            uint64_t sum2 = f2(0.f, 0.f);
+            const uint64_t sl2 = f2(sl, sl), negm2 = f2(-m, -m);
+            uint32_t cur[32];
+            tmem_ld32(lane_addr + colS, cur);
+            tmem_ld_wait();
+            reg_fence32(cur);
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const uint32_t addr = sP + (c >> 3) * 16384u + sw128_off(r, c & 7);
-                st_shared_v4(addr, pack2<BF16>(s[8 * c + 0], s[8 * c + 1]),
-                             pack2<BF16>(s[8 * c + 2], s[8 * c + 3]),
-                             pack2<BF16>(s[8 * c + 4], s[8 * c + 5]),
-                             pack2<BF16>(s[8 * c + 6], s[8 * c + 7]));
+            for (int c = 0; c < 4; ++c) {
+                uint32_t nxt[32];
+                if (c < 3) tmem_ld32(lane_addr + colS + (c + 1) * 32u, nxt);
+                uint32_t pk[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    uint64_t x = fma2(f2(__uint_as_float(cur[2 * q]), __uint_as_float(cur[2 * q + 1])),
+                                      sl2, negm2);
+                    if (!full) {
+                        float2 xv = unf2(x);
+                        if (c * 32 + 2 * q >= limit) xv.x = -INFINITY;
+                        if (c * 32 + 2 * q + 1 >= limit) xv.y = -INFINITY;
+                        x = f2(xv.x, xv.y);
+                    }
+                    const float2 xv = unf2(x);
+                    const uint64_t pp = f2(ex2(xv.x), ex2(xv.y));
+                    sum2 = add2(sum2, pp);
+                    const float2 pv = unf2(pp);
+                    pk[q] = pack2<BF16>(pv.x, pv.y);
+                }
+                tmem_st16(lane_addr + colS + c * 16u, pk);
+                if (c < 3) {
+                    tmem_ld_wait();
+                    reg_fence32(nxt);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) cur[e] = nxt[e];
+                }
             }
-            fence_proxy_async_smem();
+            const float2 sv2 = unf2(sum2);
+            const float sum = sv2.x + sv2.y;
+            l += sum;
+            tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(BAR(C::B_PF));
+            mbar_arrive(BAR(C::B_PF + t));
         }
-        if (ok) {
-            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_OD), (nkv - 1) & 1, abort_flag));
-        }
-        if (ok) {
+        if (ok && my_nkv > 0)
+            ok = __all_sync(0xffffffffu,
+                            wait_bounded(BAR(C::B_OD + t), (my_nkv - 1) & 1, abort_flag));
+        if (ok && my_nkv > 0) {
             tc_fence_after();
             const float inv_l = 1.f / l;
             uint8_t* orow = static_cast<uint8_t*>(p.o) +
@@ -295,7 +368,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
-                tmem_ld32(lane_addr + C::COL_O + c * 32u, o);
+                tmem_ld32(lane_addr + colO + c * 32u, o);
                 tmem_ld_wait();
                 reg_fence32(o);
                 uint32_t h[16];
@@ -318,7 +391,7 @@ __global__ void __launch_bounds__(192, 1)
 #undef BAR
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == C::WARP_MMA) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }

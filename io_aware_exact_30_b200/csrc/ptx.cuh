@@ -223,6 +223,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         "r"(r[29]), "r"(r[30]), "r"(r[31])
         : "memory");
 }
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -262,6 +272,73 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x on the FMA pipe: x = j + f with j = round(x), f in [-1/2, 1/2]
+// (Cody-Waite style reduction); 2^f by a degree-3 polynomial with p(0) = 1
+// whose coefficients minimise the maximum relative error (about 1.0e-4) on
+// [-1/2, 1/2]; 2^j added to the exponent field.  x is clamped at -127, which
+// yields exactly 0, so x = -inf gives 0 as ex2 does.  The coefficients and the
+// error bound come from exp2_fit.py beside this file.
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -127.f);
+    const float t = x + 12582912.f;  // 1.5 * 2^23: the low mantissa bits of t hold round(x)
+    const float f = x - (t - 12582912.f);
+    float p = fmaf(0.0550089068710804f, f, 0.2422109991312027f);
+    p = fmaf(p, f, 0.693282961845398f);
+    p = fmaf(p, f, 1.f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// ---- packed fp32 pairs (sm_100 f32x2 arithmetic): two lanes per instruction
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 unf2(uint64_t v) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+// exp2_poly on a pair: the same reduction and polynomial, with the
+// floating-point steps done two lanes per instruction.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
+    float2 v = unf2(x);
+    v.x = fmaxf(v.x, -127.f);
+    v.y = fmaxf(v.y, -127.f);
+    const uint64_t xc = f2(v.x, v.y);
+    const uint64_t magic = f2(12582912.f, 12582912.f);
+    const uint64_t t = add2(xc, magic);
+    const uint64_t r = add2(t, f2(-12582912.f, -12582912.f));
+    const uint64_t f = fma2(r, f2(-1.f, -1.f), xc);
+    uint64_t p = fma2(f2(0.0550089068710804f, 0.0550089068710804f), f,
+                      f2(0.2422109991312027f, 0.2422109991312027f));
+    p = fma2(p, f, f2(0.693282961845398f, 0.693282961845398f));
+    p = fma2(p, f, f2(1.f, 1.f));
+    const float2 pv = unf2(p), tv = unf2(t);
+    return f2(__int_as_float(__float_as_int(pv.x) + (__float_as_int(tv.x) << 23)),
+              __int_as_float(__float_as_int(pv.y) + (__float_as_int(tv.y) << 23)));
 }
 
 template <bool BF16>
