@@ -64,6 +64,26 @@ def flops(B, H, N, d, causal):
     return f, 2.5 * f  # forward, backward
 
 
+def kernel_traffic(kernel):
+    """DRAM bytes per launch for `kernel` from profiles/traffic.json, or None when
+    the kernel's sources have changed since those counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        entry = json.load(f).get(kernel)
+    if not entry:
+        return None
+    m = hashlib.sha1()
+    for src in entry["sources"]:
+        with open(os.path.join(ROOT, src), "rb") as f:
+            m.update(f.read())
+    if m.hexdigest() != entry["source_sha1"]:
+        return None
+    return entry["dram_bytes_read"] + entry["dram_bytes_write"]
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -292,9 +312,10 @@ def run_ours(args, rank, world, local_rank):
     value = job_tflops(f_step, world, ms_step)
     burst, sustained, hbm, src = peaks()
     if passes == "fwdbwd":
-        dom = ("attn_bwd_main", f_bwd, main_ms)
+        dom = ("attn_bwd_main128_kernel" if d == 128 else "attn_bwd_main_kernel", f_bwd, main_ms)
     else:
-        dom = ("attn_fwd", f_fwd, fwd_ms)
+        dom = ("attn_fwd_kernel", f_fwd, fwd_ms)
+    traffic = kernel_traffic(dom[0]) if args.workload == "large_head" else None
     achieved = dom[1] / (dom[2] * 1e-3) / 1e12
     line = {
         "metric": METRIC,
@@ -331,7 +352,8 @@ def run_ours(args, rank, world, local_rank):
             "peak_kind": f"bf16_tflops_sustained ({src})",
             "unit": "TFLOP/s",
             "frac": round(achieved / sustained, 4),
-            "traffic": None,
+            "traffic": traffic,
+            "traffic_unit": "bytes per launch (ncu dram read+write; profiles/traffic.json)",
         },
         "e2e": {"value": round(job_tflops(f_step, world, e2e_ms), 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
