@@ -217,7 +217,7 @@ def run_ours(args, rank, world, local_rank):
         flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
 
     stream = torch.cuda.current_stream(dev)
-    n_launch = {"fwd": 1, "fwdbwd": 1 + attn.BWD_LAUNCHES}[passes]
+    n_launch = {"fwd": 1, "fwdbwd": 1 + attn.bwd_launches(d)}[passes]
 
     def step(evs=None):
         if flush is not None:

@@ -26,8 +26,10 @@ STATUS = {
     -8: "ATTN_ERR_TIMEOUT", -9: "ATTN_ERR_ARG", -10: "ATTN_ERR_SCRATCH",
 }
 
-# Kernel launches one attn_bwd call makes (D preprocess, main backward).
-BWD_LAUNCHES = 2
+# Kernel launches one attn_bwd call makes: the preprocess, then the main
+# backward (d = 64), or the main backward and the dQ conversion (d = 128).
+def bwd_launches(d: int) -> int:
+    return 2 if d == 64 else 3
 
 # Every symbol include/attn.h declares.
 EXPORTS = ("attn_fwd", "attn_bwd", "attn_bwd_prep", "attn_bwd_main", "attn_bwd_workspace_bytes",

@@ -49,6 +49,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // Per-device state: sm_100 check and the opt-in shared-memory size, done once.
 std::mutex g_dev_mu;
 int g_dev_state[kMaxDevices];  // 0 unknown, 1 ready, -1 unsupported
+int g_sm_count[kMaxDevices];   // multiprocessors: the persistent kernels' grid size
 
 int check_device(int* dev_out) {
     int dev = -1;
@@ -63,7 +64,8 @@ int check_device(int* dev_out) {
     int maj = 0, mnr = 0;
     cudaDeviceGetAttribute(&maj, cudaDevAttrComputeCapabilityMajor, dev);
     cudaDeviceGetAttribute(&mnr, cudaDevAttrComputeCapabilityMinor, dev);
-    if (maj != 10 || mnr != 0 || encode_fn() == nullptr) {
+    cudaDeviceGetAttribute(&g_sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (maj != 10 || mnr != 0 || encode_fn() == nullptr || g_sm_count[dev] < 1) {
         cudaGetLastError();
         g_dev_state[dev] = -1;
         return ATTN_ERR_DEVICE;
@@ -136,9 +138,10 @@ bool make_map(CUtensorMap* m, const void* ptr, int dtype, int BH, int N, int d,
 
 template <int D, bool BF16>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-               const attn::FwdParams& p, cudaStream_t st) {
-    const long long nblocks = 1LL * p.n_pairs * p.BH;
-    if (nblocks >= (1LL << 31)) return ATTN_ERR_SHAPE;
+               const attn::FwdParams& p, int sm_count, cudaStream_t st) {
+    const long long items = 1LL * p.n_pairs * p.BH;
+    if (items >= (1LL << 31)) return ATTN_ERR_SHAPE;
+    const int nblocks = static_cast<int>(items < sm_count ? items : sm_count);
     attn::attn_fwd_kernel<D, BF16><<<static_cast<unsigned>(nblocks), FwdCfg<D>::NTHREADS,
                                      FwdCfg<D>::SMEM_BYTES, st>>>(mq, mk, mv, p);
     return launch_ok() ? ATTN_OK : ATTN_ERR_LAUNCH;
@@ -211,12 +214,22 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
     p.N = N;
     p.n_qtiles = (N + 127) / 128;
     p.n_pairs = (p.n_qtiles + 1) / 2;
+    {
+        // heads whose K and V together take at most about 48 MB of L2
+        const long long kv_head = 2LL * N * d * 2;
+        const long long g = (48LL << 20) / (kv_head > 0 ? kv_head : 1);
+        p.group = static_cast<int>(g < 1 ? 1 : (g > BH ? BH : g));
+    }
     p.causal = causal ? 1 : 0;
     p.scale_log2 = scale * 1.4426950408889634f;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool bf = dtype == ATTN_BF16;
-    if (d == 64) return bf ? launch_fwd<64, true>(mq, mk, mv, p, st) : launch_fwd<64, false>(mq, mk, mv, p, st);
-    return bf ? launch_fwd<128, true>(mq, mk, mv, p, st) : launch_fwd<128, false>(mq, mk, mv, p, st);
+    const int sms = g_sm_count[dev];
+    if (d == 64)
+        return bf ? launch_fwd<64, true>(mq, mk, mv, p, sms, st)
+                  : launch_fwd<64, false>(mq, mk, mv, p, sms, st);
+    return bf ? launch_fwd<128, true>(mq, mk, mv, p, sms, st)
+              : launch_fwd<128, false>(mq, mk, mv, p, sms, st);
 }
 
 size_t attn_bwd_workspace_bytes(int B, int H, int N, int d) {
@@ -269,10 +282,13 @@ int bwd_main_dispatch(const void* q, const void* k, const void* v, const void* d
     CUtensorMap mq64, mdo64;
     if (!make_map(&mq64, q, dtype, BH, N, d, 64) || !make_map(&mdo64, dout, dtype, BH, N, d, 64))
         return ATTN_ERR_LAUNCH;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const int sms = g_sm_count[dev];
     return bf ? attn::bwd_main128_launch<true>(mq64, mk, mv, mdo64, dq, dk, dv, workspace, B, H, N,
-                                               c, scale, st)
+                                               c, scale, sms, st)
               : attn::bwd_main128_launch<false>(mq64, mk, mv, mdo64, dq, dk, dv, workspace, B, H,
-                                                N, c, scale, st);
+                                                N, c, scale, sms, st);
 }
 }  // namespace
 

@@ -3,9 +3,10 @@
 // with 64-query inner tiles so that every accumulator of the tile loop has
 // tensor memory of its own and no stage waits for another to be drained.
 //
-// One CTA per (head, 128-key tile j); K_j, V_j stay in shared memory, 64-query
-// tiles of Q, dO (and their L2, D statistics) stream through a 3-stage
-// pipeline.  Per query tile i:
+// Persistent: one CTA per multiprocessor walks a list of (head, 128-key tile
+// j) work items (see BwdItems).  For each, K_j and V_j are loaded into shared
+// memory and 64-query tiles of Q, dO (and their L2, D statistics) stream
+// through a 3-stage pipeline that runs on across items.  Per query tile i:
 //   S^T  = K_j Q_i^T                     tensor memory, double-buffered
 //   P^T  = exp2(S^T scale log2e - L2_i)  written back over S^T as half
 //   dP^T = V_j dO_i^T                    tensor memory
@@ -15,6 +16,8 @@
 //   dQ^T = K_j^T dS^T                    tensor memory, drained by dQ warps
 //                                        into a shared fp32 tile that one bulk
 //                                        reduction adds into the accumulator
+// A separate small kernel converts the fp32 dQ accumulator to the output type
+// after the main kernel.
 // Tensor memory (512 columns): S^T buffers at 0 and 64, dP^T at 128, dQ^T at
 // 192, dV at 256, dK at 384.
 //
@@ -47,8 +50,8 @@ struct Bwd128Cfg {
                          B_DOE = B_DOF + ST, B_SF = B_DOE + ST, B_DPF = B_SF + 2,
                          B_PTF = B_DPF + 1, B_DVD = B_PTF + 1, B_DSF = B_DVD + 2,
                          B_DQF = B_DSF + 1, B_DQE = B_DQF + 1, B_FIN = B_DQE + 1,
-                         B_DR = B_FIN + 1, B_ENDA = B_DR + 1, B_ENDB = B_ENDA + 1,
-                         B_SRD = B_ENDB + 1, B_STGF = B_SRD + 1, B_STGE = B_STGF + 1,
+                         B_DR = B_FIN + 1, B_KVE = B_DR + 1, B_ACCE = B_KVE + 1,
+                         B_SRD = B_ACCE + 1, B_STGF = B_SRD + 1, B_STGE = B_STGF + 1,
                          NBAR = B_STGE + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
@@ -58,6 +61,36 @@ struct Bwd128Cfg {
     static constexpr int NTHREADS = NCOMPUTE + NDQ + 64;
     static constexpr int WARP_DQ0 = NCOMPUTE / 32;
     static constexpr int WARP_TMA = WARP_DQ0 + NDQ / 32, WARP_MMA = WARP_TMA + 1;
+};
+
+// Persistent schedule.  A work item is (head, 128-key tile j); under the
+// causal mask it costs n_q64 - 2j query tiles, otherwise n_q64.  Heads are
+// taken in groups whose K, V, Q and dO fit in L2 together; within a group
+// the items are listed heaviest first (j ascending, heads in order within a
+// j) when causal, head-major otherwise, and the list is dealt to the CTAs in
+// snake order (round r: item r*G + c to CTA c for even r, to CTA G - 1 - c
+// for odd r), which balances the CTAs' totals.
+struct BwdItems {
+    int round;
+    __device__ BwdItems() : round(0) {}
+    __device__ bool next(const BwdParams& p, int& bh, int& j) {
+        const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+        const long long k = 1LL * round * G + ((round & 1) ? (G - 1 - c) : c);
+        if (k >= 1LL * p.BH * p.n_ktiles) return false;
+        ++round;
+        const int ki = static_cast<int>(k);
+        if (p.causal) {
+            const int per_group = p.group * p.n_ktiles;
+            const int g = ki / per_group, i = ki % per_group;
+            const int heads = min(p.group, p.BH - g * p.group);
+            j = i / heads;
+            bh = g * p.group + i % heads;
+        } else {
+            bh = ki / p.n_ktiles;
+            j = ki % p.n_ktiles;
+        }
+        return true;
+    }
 };
 
 template <bool BF16>
@@ -74,23 +107,18 @@ __global__ void __launch_bounds__(448, 1)
     uint8_t* gbase = smem_raw + (base - raw);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-
-    // Work item: head-major, the heaviest key tile (j = 0 under the causal mask) first.
-    const int bh = static_cast<int>(blockIdx.x) / p.n_ktiles;
-    const int j = static_cast<int>(blockIdx.x) % p.n_ktiles;
     const int n_q64 = (p.N + 63) / 64;
-    const int i_begin = p.causal ? 2 * j : 0;
-    const int n_it = n_q64 - i_begin;
 
     const uint32_t bar0 = base + C::OFF_BAR;
 #define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + C::OFF_MISC);
     volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(gbase + C::OFF_MISC + 4);
-    volatile uint32_t* last_flag = reinterpret_cast<volatile uint32_t*>(gbase + C::OFF_MISC + 8);
     const float* sLD = reinterpret_cast<const float*>(gbase + C::OFF_LD);
 
     if (threadIdx.x == 0) {
         mbar_init(BAR(C::B_KV), 1);
+        mbar_init(BAR(C::B_KVE), 1);
+        mbar_init(BAR(C::B_ACCE), C::NCOMPUTE);
         for (int s = 0; s < C::ST; ++s) {
             mbar_init(BAR(C::B_QF + s), 1);
             mbar_init(BAR(C::B_QE + s), 1);
@@ -108,13 +136,10 @@ __global__ void __launch_bounds__(448, 1)
         mbar_init(BAR(C::B_DQE), C::NDQ);
         mbar_init(BAR(C::B_FIN), 1);
         mbar_init(BAR(C::B_DR), 1);
-        mbar_init(BAR(C::B_ENDA), C::NCOMPUTE + C::NDQ);
-        mbar_init(BAR(C::B_ENDB), 1);
         mbar_init(BAR(C::B_SRD), C::NCOMPUTE / 2);
         mbar_init(BAR(C::B_STGF), C::NDQ);
         mbar_init(BAR(C::B_STGE), 1);
         *abort_flag = 0u;
-        *last_flag = 0u;
         fence_mbar_init();
     }
     if (warp == C::WARP_MMA) {
@@ -133,19 +158,16 @@ __global__ void __launch_bounds__(448, 1)
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
             tma_prefetch_desc(&tmDO);
-            mbar_arrive_expect_tx(BAR(C::B_KV), 2 * C::KTILE);
-#pragma unroll
-            for (int kb = 0; kb < 2; ++kb) {
-                tma_load_3d(base + C::OFF_K + kb * 16384u, &tmK, BAR(C::B_KV), kb * 64, j * 128, bh);
-                tma_load_3d(base + C::OFF_V + kb * 16384u, &tmV, BAR(C::B_KV), kb * 64, j * 128, bh);
-            }
             int q_issued[C::ST], do_issued[C::ST];
             for (int s = 0; s < C::ST; ++s) q_issued[s] = do_issued[s] = 0;
-            const size_t ld_row0 = static_cast<size_t>(bh) * p.Np;
-            for (int it = 0; it < n_it; ++it) {
-                const int i = i_begin + it;
-                const int s = it % C::ST, n = it / C::ST;
-                if (!wait_bounded(BAR(C::B_QE + s), (n & 1) ^ 1, abort_flag)) break;
+            int g = 0, items = 0, bh = 0, j = 0;
+            bool ok = true;
+            BwdItems iter;
+            // query tile i of head bh into ring slot g % ST
+            auto load_tile = [&](int i) -> bool {
+                const int s = g % C::ST, n = g / C::ST;
+                const size_t ld_row0 = static_cast<size_t>(bh) * p.Np;
+                if (!wait_bounded(BAR(C::B_QE + s), (n & 1) ^ 1, abort_flag)) return false;
                 const uint32_t sq = base + C::OFF_Q + s * C::QTILE;
                 const uint32_t sld = base + C::OFF_LD + s * 512u;
                 mbar_arrive_expect_tx(BAR(C::B_QF + s), C::QTILE + 512u);
@@ -154,15 +176,38 @@ __global__ void __launch_bounds__(448, 1)
                 bulk_load(sld, p.l2pad + ld_row0 + i * 64, 256u, BAR(C::B_QF + s));
                 bulk_load(sld + 256u, p.dpad + ld_row0 + i * 64, 256u, BAR(C::B_QF + s));
                 q_issued[s] = n + 1;
-                if (!wait_bounded(BAR(C::B_DOE + s), (n & 1) ^ 1, abort_flag)) break;
+                if (!wait_bounded(BAR(C::B_DOE + s), (n & 1) ^ 1, abort_flag)) return false;
                 const uint32_t sdo = base + C::OFF_DO + s * C::QTILE;
                 mbar_arrive_expect_tx(BAR(C::B_DOF + s), C::QTILE);
                 tma_load_3d(sdo, &tmDO, BAR(C::B_DOF + s), 0, i * 64, bh);
                 tma_load_3d(sdo + 8192u, &tmDO, BAR(C::B_DOF + s), 64, i * 64, bh);
                 do_issued[s] = n + 1;
+                ++g;
+                return true;
+            };
+            while (ok && iter.next(p, bh, j)) {
+                const int i_begin = p.causal ? 2 * j : 0;
+                const int n_it = n_q64 - i_begin;
+                const int pre = min(C::ST, n_it);
+                // The item's first query tiles go ahead of its K/V, which wait
+                // until the previous item's MMAs are done with K and V.
+                for (int it = 0; ok && it < pre; ++it) ok = load_tile(i_begin + it);
+                if (!ok) break;
+                if (items > 0 && !(ok = wait_bounded(BAR(C::B_KVE), (items - 1) & 1, abort_flag)))
+                    break;
+                mbar_arrive_expect_tx(BAR(C::B_KV), 2 * C::KTILE);
+#pragma unroll
+                for (int kb = 0; kb < 2; ++kb) {
+                    tma_load_3d(base + C::OFF_K + kb * 16384u, &tmK, BAR(C::B_KV), kb * 64, j * 128,
+                                bh);
+                    tma_load_3d(base + C::OFF_V + kb * 16384u, &tmV, BAR(C::B_KV), kb * 64, j * 128,
+                                bh);
+                }
+                ++items;
+                for (int it = pre; ok && it < n_it; ++it) ok = load_tile(i_begin + it);
             }
-            if (*abort_flag) {
-                wait_drain(BAR(C::B_KV), 0);
+            if (*abort_flag) {  // let every copy in flight land before the CTA exits
+                if (items > 0) wait_drain(BAR(C::B_KV), (items - 1) & 1);
                 for (int s = 0; s < C::ST; ++s) {
                     if (q_issued[s] > 0) wait_drain(BAR(C::B_QF + s), (q_issued[s] - 1) & 1);
                     if (do_issued[s] > 0) wait_drain(BAR(C::B_DOF + s), (do_issued[s] - 1) & 1);
@@ -176,79 +221,93 @@ __global__ void __launch_bounds__(448, 1)
             constexpr uint32_t ID_KV = idesc_f16(BF16, 128, 128, false, true);  // dV, dK
             constexpr uint32_t ID_DQT = idesc_f16(BF16, 128, 64, true, true);   // dQ^T
             const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sDST = base + C::OFF_DST;
-            bool ok = wait_bounded(BAR(C::B_KV), 0, abort_flag);
-            // S^T(t) = K Q_t^T into S buffer t & 1
-            auto issue_s = [&](int t) -> bool {
-                const int s = t % C::ST;
-                if (!wait_bounded(BAR(C::B_QF + s), (t / C::ST) & 1, abort_flag)) return false;
+            // S^T(g) = K Q_g^T into S buffer g & 1; that buffer held P^T(g-2),
+            // which dV(g-2) read (the newest phase of its barrier).
+            auto issue_s = [&](int g) -> bool {
+                const int s = g % C::ST;
+                if (g >= 2 &&
+                    !wait_bounded(BAR(C::B_DVD + (g & 1)), ((g - 2) >> 1) & 1, abort_flag))
+                    return false;
+                if (!wait_bounded(BAR(C::B_QF + s), (g / C::ST) & 1, abort_flag)) return false;
                 tc_fence_after();
                 const uint32_t sQ = base + C::OFF_Q + s * C::QTILE;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * 8192u + (kk & 3) * 32u;
                     const uint32_t offk = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                    mma_ss(tmem + C::COL_S + (t & 1) * 64u, sdesc_sw128(sK + offk, 16, 1024),
+                    mma_ss(tmem + C::COL_S + (g & 1) * 64u, sdesc_sw128(sK + offk, 16, 1024),
                            sdesc_sw128(sQ + off, 16, 1024), ID_S, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(BAR(C::B_SF + (t & 1)));
+                mma_commit(BAR(C::B_SF + (g & 1)));
                 return true;
             };
-            // Issue order per tile: dP^T(it), dV(it), S^T(it+1), dK(it) + dQ^T(it).
+            // Issue order per tile g: dP^T(g), dV(g), S^T(g+1), dK(g) + dQ^T(g).
             // Every wait below is for the newest phase its barrier can have
-            // reached, so no waiter can fall two phases behind.
-            if (ok && n_it > 0) ok = issue_s(0);
-            for (int it = 0; ok && it < n_it; ++it) {
-                const uint32_t ph = it & 1;
-                const int s = it % C::ST, n = it / C::ST;
-                const uint32_t sQ = base + C::OFF_Q + s * C::QTILE;
-                const uint32_t sDO = base + C::OFF_DO + s * C::QTILE;
-                // dP^T(it) = V dO^T: the compute warps have read dP^T(it-1)
-                if (!(ok = wait_bounded(BAR(C::B_DOF + s), n & 1, abort_flag))) break;
-                if (it >= 1 && !(ok = wait_bounded(BAR(C::B_DSF), ph ^ 1, abort_flag))) break;
-                tc_fence_after();
+            // reached, so no waiter can fall two phases behind.  Phase
+            // parities run on the tile count g across work items.
+            int g = 0, items = 0, bh = 0, j = 0;
+            bool ok = true;
+            BwdItems iter;
+            while (ok && iter.next(p, bh, j)) {
+                const int n_it = n_q64 - (p.causal ? 2 * j : 0);
+                if (!(ok = wait_bounded(BAR(C::B_KV), items & 1, abort_flag))) break;
+                if (!(ok = issue_s(g))) break;
+                for (int it = 0; ok && it < n_it; ++it, ++g) {
+                    const uint32_t ph = g & 1;
+                    const int s = g % C::ST, n = g / C::ST;
+                    const uint32_t sQ = base + C::OFF_Q + s * C::QTILE;
+                    const uint32_t sDO = base + C::OFF_DO + s * C::QTILE;
+                    // dP^T(g) = V dO^T: the compute warps have read dP^T(g-1)
+                    if (!(ok = wait_bounded(BAR(C::B_DOF + s), n & 1, abort_flag))) break;
+                    if (g >= 1 && !(ok = wait_bounded(BAR(C::B_DSF), ph ^ 1, abort_flag))) break;
+                    tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * 8192u + (kk & 3) * 32u;
-                    const uint32_t offk = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                    mma_ss(tmem + C::COL_DP, sdesc_sw128(sV + offk, 16, 1024),
-                           sdesc_sw128(sDO + off, 16, 1024), ID_S, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(BAR(C::B_DPF));
-                // dV += P^T dO (P^T from tensor memory)
-                if (!(ok = wait_bounded(BAR(C::B_PTF), ph, abort_flag))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(tmem + C::COL_DV, tmem + C::COL_S + (it & 1) * 64u + kk * 8u,
-                           sdesc_sw128(sDO + kk * 2048u, 8192, 1024), ID_KV,
-                           (it > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(BAR(C::B_DVD + (it & 1)));
-                mma_commit(BAR(C::B_DOE + s));
-                // S^T(it+1): its buffer held P^T(it-1), read by dV(it-1)
-                if (it + 1 < n_it) {
-                    if (it >= 1 && !(ok = wait_bounded(BAR(C::B_DVD + ((it - 1) & 1)),
-                                                       ((it - 1) >> 1) & 1, abort_flag)))
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t off = (kk >> 2) * 8192u + (kk & 3) * 32u;
+                        const uint32_t offk = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                        mma_ss(tmem + C::COL_DP, sdesc_sw128(sV + offk, 16, 1024),
+                               sdesc_sw128(sDO + off, 16, 1024), ID_S, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(BAR(C::B_DPF));
+                    // dV += P^T dO (P^T from tensor memory).  The item's first
+                    // dV and dK overwrite accumulators that the previous item's
+                    // epilogue must have read.
+                    if (!(ok = wait_bounded(BAR(C::B_PTF), ph, abort_flag))) break;
+                    if (it == 0 && items > 0 &&
+                        !(ok = wait_bounded(BAR(C::B_ACCE), (items - 1) & 1, abort_flag)))
                         break;
-                    if (!(ok = issue_s(it + 1))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ts(tmem + C::COL_DV, tmem + C::COL_S + (g & 1) * 64u + kk * 8u,
+                               sdesc_sw128(sDO + kk * 2048u, 8192, 1024), ID_KV,
+                               (it > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(BAR(C::B_DVD + (g & 1)));
+                    mma_commit(BAR(C::B_DOE + s));
+                    if (it + 1 < n_it && !(ok = issue_s(g + 1))) break;
+                    // dK += dS^T Q ; dQ^T = K^T dS^T (its columns drained for g-1)
+                    if (!(ok = wait_bounded(BAR(C::B_DSF), ph, abort_flag))) break;
+                    if (g >= 1 && !(ok = wait_bounded(BAR(C::B_DQE), ph ^ 1, abort_flag))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss(tmem + C::COL_DK, sdesc_sw128(sDST + kk * 32u, 16, 1024),
+                               sdesc_sw128(sQ + kk * 2048u, 8192, 1024), ID_KV,
+                               (it > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ss(tmem + C::COL_DQ, sdesc_sw128(sK + kk * 2048u, 16384, 1024),
+                               sdesc_sw128(sDST + kk * 2048u, 8192, 1024), ID_DQT,
+                               kk > 0 ? 1u : 0u);
+                    mma_commit(BAR(C::B_QE + s));
+                    mma_commit(BAR(C::B_DQF));
                 }
-                // dK += dS^T Q ; dQ^T = K^T dS^T (its columns drained for it-1)
-                if (!(ok = wait_bounded(BAR(C::B_DSF), ph, abort_flag))) break;
-                if (it >= 1 && !(ok = wait_bounded(BAR(C::B_DQE), ph ^ 1, abort_flag))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ss(tmem + C::COL_DK, sdesc_sw128(sDST + kk * 32u, 16, 1024),
-                           sdesc_sw128(sQ + kk * 2048u, 8192, 1024), ID_KV,
-                           (it > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tmem + C::COL_DQ, sdesc_sw128(sK + kk * 2048u, 16384, 1024),
-                           sdesc_sw128(sDST + kk * 2048u, 8192, 1024), ID_DQT, kk > 0 ? 1u : 0u);
-                mma_commit(BAR(C::B_QE + s));
-                mma_commit(BAR(C::B_DQF));
+                if (!ok) break;
+                mma_commit(BAR(C::B_FIN));  // dK, dV of this item complete
+                mma_commit(BAR(C::B_KVE));  // K, V no longer read
+                ++items;
             }
-            if (ok) mma_commit(BAR(C::B_FIN));
-            if (*abort_flag) {
+            if (*abort_flag) {  // every issued MMA must finish before TMEM is freed
                 mma_commit(BAR(C::B_DR));
                 wait_drain(BAR(C::B_DR), 0);
             }
@@ -266,154 +325,164 @@ __global__ void __launch_bounds__(448, 1)
         const bool issuer = warp == C::WARP_DQ0 && lane == 0;
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
         const uint32_t stg = base + C::OFF_STG + r * 4u;
-        float* acc_head = p.dqacc + static_cast<size_t>(bh) * p.N * D;
+        int g = 0, bh = 0, j = 0;
         bool dq_ok = true;
-        for (int it = 0; it < n_it; ++it) {
-            const int q0 = (i_begin + it) * 64;
-            if (!(dq_ok = __all_sync(0xffffffffu,
-                                     wait_bounded(BAR(C::B_DQF), it & 1, abort_flag))))
-                break;
-            tc_fence_after();
-            uint32_t v[2][32];
-            tmem_ld32(lane_addr + C::COL_DQ, v[0]);
-            tmem_ld32(lane_addr + C::COL_DQ + 32u, v[1]);
-            tmem_ld_wait();
-            reg_fence32(v[0]);
-            reg_fence32(v[1]);
-            tc_fence_before();
-            mbar_arrive(BAR(C::B_DQE));  // the values are in registers: columns free
-            // the previous tile's bulk reduction has finished reading the staging tile
-            if (it >= 1 && !(dq_ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_STGE),
-                                                                         (it - 1) & 1, abort_flag))))
-                break;
+        BwdItems iter;
+        while (dq_ok && iter.next(p, bh, j)) {
+            const int i_begin = p.causal ? 2 * j : 0;
+            const int n_it = n_q64 - i_begin;
+            float* acc_head = p.dqacc + static_cast<size_t>(bh) * p.N * D;
+            for (int it = 0; it < n_it; ++it, ++g) {
+                const int q0 = (i_begin + it) * 64;
+                if (!(dq_ok = __all_sync(0xffffffffu,
+                                         wait_bounded(BAR(C::B_DQF), g & 1, abort_flag))))
+                    break;
+                tc_fence_after();
+                uint32_t v[2][32];
+                tmem_ld32(lane_addr + C::COL_DQ, v[0]);
+                tmem_ld32(lane_addr + C::COL_DQ + 32u, v[1]);
+                tmem_ld_wait();
+                reg_fence32(v[0]);
+                reg_fence32(v[1]);
+                tc_fence_before();
+                mbar_arrive(BAR(C::B_DQE));  // the values are in registers: columns free
+                // the previous tile's bulk reduction has finished reading the staging tile
+                if (g >= 1 && !(dq_ok = __all_sync(0xffffffffu,
+                                                   wait_bounded(BAR(C::B_STGE), (g - 1) & 1,
+                                                                abort_flag))))
+                    break;
 #pragma unroll
-            for (int e = 0; e < 64; ++e)
-                st_shared_f32(stg + e * 512u, __uint_as_float(v[e >> 5][e & 31]) * p.scale);
-            fence_proxy_async_smem();
-            mbar_arrive(BAR(C::B_STGF));
-            if (issuer) {
-                if (!wait_bounded(BAR(C::B_STGF), it & 1, abort_flag)) {
-                    dq_ok = false;
-                } else {
-                    const int nq = min(64, p.N - q0);
-                    bulk_reduce_add_f32(acc_head + static_cast<size_t>(q0) * D,
-                                        base + C::OFF_STG, static_cast<uint32_t>(nq) * 512u);
-                    bulk_commit();
-                    bulk_wait_read_all();
-                    mbar_arrive(BAR(C::B_STGE));
+                for (int e = 0; e < 64; ++e)
+                    st_shared_f32(stg + e * 512u, __uint_as_float(v[e >> 5][e & 31]) * p.scale);
+                fence_proxy_async_smem();
+                mbar_arrive(BAR(C::B_STGF));
+                if (issuer) {
+                    if (!wait_bounded(BAR(C::B_STGF), g & 1, abort_flag)) {
+                        dq_ok = false;
+                    } else {
+                        const int nq = min(64, p.N - q0);
+                        bulk_reduce_add_f32(acc_head + static_cast<size_t>(q0) * D,
+                                            base + C::OFF_STG, static_cast<uint32_t>(nq) * 512u);
+                        bulk_commit();
+                        bulk_wait_read_all();
+                        mbar_arrive(BAR(C::B_STGE));
+                    }
                 }
+                dq_ok = __all_sync(0xffffffffu, dq_ok);
+                if (!dq_ok) break;
             }
-            dq_ok = __all_sync(0xffffffffu, dq_ok);
-            if (!dq_ok) break;
         }
-        if (issuer) {
-            // every reduction complete and visible before the completion count
-            bulk_wait_all();
-            asm volatile("fence.proxy.async.global;" ::: "memory");
-            __threadfence();
-        }
+        if (issuer) bulk_wait_all();  // every reduction complete before the CTA exits
     } else {
         // ---------------------------------------------------------- compute
         const int quarter = warp & 3, half = warp >> 2;
         const int r = quarter * 32 + lane;  // TMEM lane = key row of the tile
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-        const int key = j * 128 + r;
-        const bool key_valid = key < p.N;
         const float sl = p.scale_log2;
-        const size_t head_row0 = static_cast<size_t>(bh) * p.N;
         const uint32_t sDST = base + C::OFF_DST;
         const int c0 = half * 32;  // first query column of this thread's half
+        int g = 0, items = 0, bh = 0, j = 0;
         bool ok = true;
-        for (int it = 0; it < n_it; ++it) {
-            const int i = i_begin + it;
-            const int q0 = i * 64;
-            const uint32_t ph = it & 1;
-            const int s = it % C::ST;
-            const float4* L4 = reinterpret_cast<const float4*>(sLD + s * 128 + c0);
-            const float4* D4 = reinterpret_cast<const float4*>(sLD + s * 128 + 64 + c0);
-            const uint32_t colS = C::COL_S + (it & 1) * 64u;
+        BwdItems iter;
+        while (ok && iter.next(p, bh, j)) {
+            const int i_begin = p.causal ? 2 * j : 0;
+            const int n_it = n_q64 - i_begin;
+            const int key = j * 128 + r;
+            const bool key_valid = key < p.N;
+            const size_t head_row0 = static_cast<size_t>(bh) * p.N;
+            for (int it = 0; it < n_it; ++it, ++g) {
+                const int q0 = (i_begin + it) * 64;
+                const uint32_t ph = g & 1;
+                const int s = g % C::ST;
+                const float4* L4 = reinterpret_cast<const float4*>(sLD + s * 128 + c0);
+                const float4* D4 = reinterpret_cast<const float4*>(sLD + s * 128 + 64 + c0);
+                const uint32_t colS = C::COL_S + (g & 1) * 64u;
 
-            // ---- P^T = exp2(S^T scale log2e - L2), written back over S^T
-            ok = __all_sync(0xffffffffu,
-                            wait_bounded(BAR(C::B_QF + s), (it / C::ST) & 1, abort_flag));
-            if (ok)
+                // ---- P^T = exp2(S^T scale log2e - L2), written back over S^T
+                // (wait on the load barrier too: it makes the bulk-copied L2/D visible)
                 ok = __all_sync(0xffffffffu,
-                                wait_bounded(BAR(C::B_SF + (it & 1)), (it >> 1) & 1, abort_flag));
-            if (!ok) break;
-            tc_fence_after();
-            float pv[32];
-            {
-                uint32_t sv[32];
-                tmem_ld32(lane_addr + colS + c0, sv);
-                tmem_ld_wait();
-                reg_fence32(sv);
-                if (half == 0) {  // half 1 writes P^T over columns half 0 reads
-                    tc_fence_before();
-                    mbar_arrive(BAR(C::B_SRD));
-                }
+                                wait_bounded(BAR(C::B_QF + s), (g / C::ST) & 1, abort_flag));
+                if (ok)
+                    ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SF + (g & 1)), (g >> 1) & 1,
+                                                              abort_flag));
+                if (!ok) break;
+                tc_fence_after();
+                float pv[32];
+                {
+                    uint32_t sv[32];
+                    tmem_ld32(lane_addr + colS + c0, sv);
+                    tmem_ld_wait();
+                    reg_fence32(sv);
+                    if (half == 0) {  // half 1 writes P^T over columns half 0 reads
+                        tc_fence_before();
+                        mbar_arrive(BAR(C::B_SRD));
+                    }
 #pragma unroll
-                for (int g = 0; g < 8; ++g) {
-                    const float4 l4 = L4[g];
-                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                    for (int e4 = 0; e4 < 8; ++e4) {
+                        const float4 l4 = L4[e4];
+                        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        pv[4 * g + e] = ex2(fmaf(__uint_as_float(sv[4 * g + e]), sl, -lv[e]));
-                }
-                // query q0 + c0 + c sees key j*128 + r iff q0 + c0 + c >= key
-                if (!key_valid || (p.causal && q0 < (j + 1) * 128)) {
-                    const int lo = key_valid ? key - q0 - c0 : 32;
+                        for (int e = 0; e < 4; ++e)
+                            pv[4 * e4 + e] =
+                                ex2(fmaf(__uint_as_float(sv[4 * e4 + e]), sl, -lv[e]));
+                    }
+                    // query q0 + c0 + c sees key j*128 + r iff q0 + c0 + c >= key
+                    if (!key_valid || (p.causal && q0 < (j + 1) * 128)) {
+                        const int lo = key_valid ? key - q0 - c0 : 32;
 #pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        if (c < lo) pv[c] = 0.f;
-                }
-                uint32_t pk[16];
+                        for (int c = 0; c < 32; ++c)
+                            if (c < lo) pv[c] = 0.f;
+                    }
+                    uint32_t pk[16];
 #pragma unroll
-                for (int c = 0; c < 16; ++c) pk[c] = pack2<BF16>(pv[2 * c], pv[2 * c + 1]);
-                if (half == 1) {
-                    ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SRD), ph, abort_flag));
-                    tc_fence_after();
+                    for (int c = 0; c < 16; ++c) pk[c] = pack2<BF16>(pv[2 * c], pv[2 * c + 1]);
+                    if (half == 1) {
+                        ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SRD), ph, abort_flag));
+                        tc_fence_after();
+                    }
+                    if (ok) {
+                        tmem_st16(lane_addr + colS + half * 16u, pk);
+                        tmem_st_wait();
+                    }
                 }
-                if (ok) {
-                    tmem_st16(lane_addr + colS + half * 16u, pk);
-                    tmem_st_wait();
-                }
-            }
-            if (!ok) break;
-            tc_fence_before();
-            mbar_arrive(BAR(C::B_PTF));
-
-            // ---- dS^T = P^T (dP^T - D), half, into shared memory
-            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_DPF), ph, abort_flag));
-            if (!ok) break;
-            tc_fence_after();
-            {
-                uint32_t dpv[32];
-                tmem_ld32(lane_addr + C::COL_DP + c0, dpv);
-                tmem_ld_wait();
-                reg_fence32(dpv);
+                if (!ok) break;
                 tc_fence_before();
-                float dsv[32];
+                mbar_arrive(BAR(C::B_PTF));
+
+                // ---- dS^T = P^T (dP^T - D), half, into shared memory
+                ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_DPF), ph, abort_flag));
+                if (!ok) break;
+                tc_fence_after();
+                {
+                    uint32_t dpv[32];
+                    tmem_ld32(lane_addr + C::COL_DP + c0, dpv);
+                    tmem_ld_wait();
+                    reg_fence32(dpv);
+                    tc_fence_before();
+                    float dsv[32];
 #pragma unroll
-                for (int g = 0; g < 8; ++g) {
-                    const float4 d4 = D4[g];
-                    const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+                    for (int e4 = 0; e4 < 8; ++e4) {
+                        const float4 d4 = D4[e4];
+                        const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        dsv[4 * g + e] = pv[4 * g + e] * (__uint_as_float(dpv[4 * g + e]) - dd[e]);
+                        for (int e = 0; e < 4; ++e)
+                            dsv[4 * e4 + e] =
+                                pv[4 * e4 + e] * (__uint_as_float(dpv[4 * e4 + e]) - dd[e]);
+                    }
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)  // 16-byte chunks 4 half + c of the 128-byte key row
+                        st_shared_v4(sDST + sw128_off(r, half * 4 + c),
+                                     pack2<BF16>(dsv[8 * c + 0], dsv[8 * c + 1]),
+                                     pack2<BF16>(dsv[8 * c + 2], dsv[8 * c + 3]),
+                                     pack2<BF16>(dsv[8 * c + 4], dsv[8 * c + 5]),
+                                     pack2<BF16>(dsv[8 * c + 6], dsv[8 * c + 7]));
                 }
-#pragma unroll
-                for (int g = 0; g < 4; ++g)  // 16-byte chunks 4 half + g of the 128-byte key row
-                    st_shared_v4(sDST + sw128_off(r, half * 4 + g),
-                                 pack2<BF16>(dsv[8 * g + 0], dsv[8 * g + 1]),
-                                 pack2<BF16>(dsv[8 * g + 2], dsv[8 * g + 3]),
-                                 pack2<BF16>(dsv[8 * g + 4], dsv[8 * g + 5]),
-                                 pack2<BF16>(dsv[8 * g + 6], dsv[8 * g + 7]));
+                fence_proxy_async_smem();
+                mbar_arrive(BAR(C::B_DSF));
             }
-            fence_proxy_async_smem();
-            mbar_arrive(BAR(C::B_DSF));
-        }
-        if (ok) ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_FIN), 0, abort_flag));
-        if (ok) {  // dK_j, dV_j rows: lane r holds key row j*128 + r; this half, 64 features
+            if (ok) ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_FIN), items & 1, abort_flag));
+            if (!ok) break;
+            // dK_j, dV_j rows: lane r holds key row j*128 + r; this half, 64 features
             tc_fence_after();
             const size_t rowoff = (head_row0 + key) * (D * 2) + half * D;
 #pragma unroll
@@ -441,36 +510,10 @@ __global__ void __launch_bounds__(448, 1)
                     }
                 }
             }
-        }
-    }
-    if (warp < C::WARP_TMA) {
-        // The last CTA of this head to finish converts the head's dQ.  Bounded
-        // mbarrier syncs (not bar.sync): a warp that gave up cannot leave the
-        // others waiting for ever.
-        const int tid = threadIdx.x;  // 0 .. NCOMPUTE + NDQ - 1
-        bool ok = __all_sync(0xffffffffu, *abort_flag == 0u);
-        if (ok) {
-            __threadfence();
-            mbar_arrive(BAR(C::B_ENDA));
-            if (tid == 0) {
-                if (wait_bounded(BAR(C::B_ENDA), 0, abort_flag)) {
-                    const int done = atomicAdd(p.counters + bh, 1);
-                    *last_flag = (done == p.n_ktiles - 1) ? 1u : 0u;
-                }
-                mbar_arrive(BAR(C::B_ENDB));
-            }
-            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_ENDB), 0, abort_flag));
-        }
-        if (ok && *last_flag) {
-            __threadfence();
-            const size_t head_row0 = static_cast<size_t>(bh) * p.N;
-            const float4* src = reinterpret_cast<const float4*>(p.dqacc + head_row0 * D);
-            uint2* out = reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.dq) + head_row0 * D * 2);
-            const long long n4 = static_cast<long long>(p.N) * D / 4;
-            for (long long e = tid; e < n4; e += C::NCOMPUTE + C::NDQ) {
-                const float4 x = __ldcg(src + e);
-                out[e] = make_uint2(pack2<BF16>(x.x, x.y), pack2<BF16>(x.z, x.w));
-            }
+            // dK and dV have been read: the next item may overwrite them
+            tc_fence_before();
+            mbar_arrive(BAR(C::B_ACCE));
+            ++items;
         }
     }
 #undef BAR
@@ -479,6 +522,18 @@ __global__ void __launch_bounds__(448, 1)
     if (warp == C::WARP_MMA) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// dq = dQ accumulator (fp32, scale already applied) rounded to the output type.
+template <bool BF16>
+__global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float4* __restrict__ acc,
+                                                                  uint2* __restrict__ dq,
+                                                                  long long n4) {
+    for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < n4;
+         e += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const float4 x = acc[e];
+        dq[e] = make_uint2(pack2<BF16>(x.x, x.y), pack2<BF16>(x.z, x.w));
     }
 }
 
@@ -492,10 +547,12 @@ inline bool bwd128_set_attributes() {
 }
 
 // mq, mdo must be tensor maps with 64-row boxes; mk, mv with 128-row boxes.
+// Launches the persistent main kernel on min(#SMs, #items) CTAs, then the dQ
+// conversion.
 template <bool BF16>
 int bwd_main128_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                        const CUtensorMap& mdo, void* dq, void* dk, void* dv, void* ws, int B,
-                       int H, int N, int causal, float scale, cudaStream_t st) {
+                       int H, int N, int causal, float scale, int sm_count, cudaStream_t st) {
     BwdParams p;
     uint8_t* w = static_cast<uint8_t*>(ws);
     p.l2pad = reinterpret_cast<const float*>(w);
@@ -513,11 +570,28 @@ int bwd_main128_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     p.causal = causal;
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
-    const long long nblocks = 1LL * p.n_ktiles * p.BH;
-    if (nblocks >= (1LL << 31)) return -2;
+    {
+        // heads whose K, V, Q and dO together take at most about 48 MB of L2
+        const long long per_head = 4LL * N * 128 * 2;
+        const long long g = (48LL << 20) / per_head;
+        p.group = static_cast<int>(g < 1 ? 1 : (g > p.BH ? p.BH : g));
+    }
+    const long long items = 1LL * p.n_ktiles * p.BH;
+    if (items >= (1LL << 31)) return -2;
+    const int nblocks = static_cast<int>(items < sm_count ? items : sm_count);
     attn_bwd_main128_kernel<BF16><<<static_cast<unsigned>(nblocks), Bwd128Cfg::NTHREADS,
                                     Bwd128Cfg::SMEM_BYTES, st>>>(mq, mk, mv, mdo, p);
-    const cudaError_t e = cudaGetLastError();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        bwd_record_error(e);
+        return -7;
+    }
+    const long long n4 = 1LL * p.BH * N * 128 / 4;
+    const long long want = (n4 + 255) / 256;
+    const int cblocks = static_cast<int>(want < 4LL * sm_count ? want : 4LL * sm_count);
+    attn_bwd_dq_convert_kernel<BF16><<<cblocks, 256, 0, st>>>(
+        reinterpret_cast<const float4*>(p.dqacc), static_cast<uint2*>(dq), n4);
+    e = cudaGetLastError();
     if (e != cudaSuccess) bwd_record_error(e);
     return e == cudaSuccess ? 0 : -7;
 }

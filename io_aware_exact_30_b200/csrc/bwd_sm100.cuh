@@ -125,6 +125,7 @@ struct BwdParams {
     int Np;
     int n_qtiles;
     int n_ktiles;
+    int group;  // persistent kernels: heads per scheduling group
     int causal;
     float scale;
     float scale_log2;

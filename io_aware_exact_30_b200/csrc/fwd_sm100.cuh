@@ -50,9 +50,55 @@ struct FwdParams {
     int BH;
     int N;
     int n_qtiles;
-    int n_pairs;
+    int n_pairs;         // query-tile pairs per head
+    int group;           // heads per scheduling group (their K/V fit in L2)
     int causal;
-    float scale_log2;  // scale * log2(e)
+    float scale_log2;    // scale * log2(e)
+};
+
+// Persistent schedule.  A work item is (head, pair of query tiles); there are
+// BH * n_pairs of them.  Heads are taken in groups of `group` heads whose K/V
+// fit comfortably in L2 together; within a group the items are listed
+// heaviest first — under the causal mask pair p costs 4p + 3 key-tile steps,
+// so the group's list runs from the last pair down, heads in order within a
+// pair; without the mask all items cost the same and the list is head-major.
+// The list is dealt to the CTAs in snake order: round r gives item r*G + c to
+// CTA c when r is even and to CTA G - 1 - c when r is odd (G = grid size),
+// which balances the CTAs' totals to within about one small item.
+struct FwdItems {
+    int round;
+    __device__ FwdItems() : round(0) {}
+    __device__ bool next(const FwdParams& p, int& bh, int& pair) {
+        const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+        const long long k = 1LL * round * G + ((round & 1) ? (G - 1 - c) : c);
+        if (k >= 1LL * p.BH * p.n_pairs) return false;
+        ++round;
+        const int ki = static_cast<int>(k);
+        if (p.causal) {
+            const int per_group = p.group * p.n_pairs;
+            const int g = ki / per_group, i = ki % per_group;
+            const int heads = min(p.group, p.BH - g * p.group);
+            pair = p.n_pairs - 1 - i / heads;
+            bh = g * p.group + i % heads;
+        } else {
+            bh = ki / p.n_pairs;
+            pair = ki % p.n_pairs;
+        }
+        return true;
+    }
+};
+
+struct FwdItemShape {
+    bool has1;
+    int nkv_t[2];
+    int nkv;
+    __device__ FwdItemShape(const FwdParams& p, int pair) {
+        const int n_kv_all = (p.N + 127) >> 7;
+        has1 = 2 * pair + 1 < p.n_qtiles;
+        nkv_t[0] = p.causal ? min(n_kv_all, 2 * pair + 1) : n_kv_all;
+        nkv_t[1] = has1 ? (p.causal ? min(n_kv_all, 2 * pair + 2) : n_kv_all) : 0;
+        nkv = max(nkv_t[0], nkv_t[1]);
+    }
 };
 
 template <int D>
@@ -66,7 +112,7 @@ struct FwdCfg {
     static constexpr uint32_t OFF_BAR = OFF_V + STAGES * TILE;
     static constexpr int B_Q = 0, B_KF = 1, B_VF = B_KF + STAGES, B_KE = B_VF + STAGES,
                          B_SF = B_KE + STAGES, B_PF = B_SF + 2, B_OD = B_PF + 2, B_DR = B_OD + 2,
-                         NBAR = B_DR + 1;
+                         B_QE = B_DR + 1, B_OE = B_QE + 1, NBAR = B_OE + 2;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
     static constexpr uint32_t TMEM_COLS = 512;
@@ -91,16 +137,6 @@ __global__ void __launch_bounds__(320, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Work item: head-major; within a head the heaviest pair of query tiles first.
-    const int pair = p.n_pairs - 1 - static_cast<int>(blockIdx.x) % p.n_pairs;
-    const int bh = static_cast<int>(blockIdx.x) / p.n_pairs;
-    const int n_kv_all = (p.N + 127) >> 7;
-    const bool has1 = 2 * pair + 1 < p.n_qtiles;
-    int nkv_t[2];
-    nkv_t[0] = p.causal ? min(n_kv_all, 2 * pair + 1) : n_kv_all;
-    nkv_t[1] = has1 ? (p.causal ? min(n_kv_all, 2 * pair + 2) : n_kv_all) : 0;
-    const int nkv = max(nkv_t[0], nkv_t[1]);
-
     const uint32_t bar0 = base + C::OFF_BAR;
 #define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + C::OFF_MISC);
@@ -108,6 +144,7 @@ __global__ void __launch_bounds__(320, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(BAR(C::B_Q), 1);
+        mbar_init(BAR(C::B_QE), 1);
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(BAR(C::B_KF + s), 1);
             mbar_init(BAR(C::B_VF + s), 1);
@@ -117,6 +154,7 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(BAR(C::B_SF + t), 1);
             mbar_init(BAR(C::B_PF + t), 128);
             mbar_init(BAR(C::B_OD + t), 1);
+            mbar_init(BAR(C::B_OE + t), 128);
         }
         mbar_init(BAR(C::B_DR), 1);
         *abort_flag = 0u;
@@ -137,32 +175,42 @@ __global__ void __launch_bounds__(320, 1)
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
-            mbar_arrive_expect_tx(BAR(C::B_Q), has1 ? 2 * C::TILE : C::TILE);
-            for (int t = 0; t < (has1 ? 2 : 1); ++t)
-#pragma unroll
-                for (int kb = 0; kb < C::KB; ++kb)
-                    tma_load_3d(base + C::OFF_Q + t * C::TILE + kb * 16384u, &tmQ, BAR(C::B_Q),
-                                kb * 64, (2 * pair + t) * 128, bh);
             int issued[C::STAGES];
 #pragma unroll
             for (int s = 0; s < C::STAGES; ++s) issued[s] = 0;
-            for (int j = 0; j < nkv; ++j) {
-                const int s = j % C::STAGES, n = j / C::STAGES;
-                if (!wait_bounded(BAR(C::B_KE + s), (n & 1) ^ 1, abort_flag)) break;
-                const uint32_t sk = base + C::OFF_K + s * C::TILE;
-                const uint32_t sv = base + C::OFF_V + s * C::TILE;
-                mbar_arrive_expect_tx(BAR(C::B_KF + s), C::TILE);
+            int kv = 0, items = 0, bh, pair;
+            FwdItems iter;
+            bool ok = true;
+            while (ok && iter.next(p, bh, pair)) {
+                const FwdItemShape sh(p, pair);
+                // the previous item's S MMAs are done reading the query tiles
+                if (items > 0 && !(ok = wait_bounded(BAR(C::B_QE), (items - 1) & 1, abort_flag)))
+                    break;
+                mbar_arrive_expect_tx(BAR(C::B_Q), sh.has1 ? 2 * C::TILE : C::TILE);
+                for (int t = 0; t < (sh.has1 ? 2 : 1); ++t)
 #pragma unroll
-                for (int kb = 0; kb < C::KB; ++kb)
-                    tma_load_3d(sk + kb * 16384u, &tmK, BAR(C::B_KF + s), kb * 64, j * 128, bh);
-                mbar_arrive_expect_tx(BAR(C::B_VF + s), C::TILE);
+                    for (int kb = 0; kb < C::KB; ++kb)
+                        tma_load_3d(base + C::OFF_Q + t * C::TILE + kb * 16384u, &tmQ, BAR(C::B_Q),
+                                    kb * 64, (2 * pair + t) * 128, bh);
+                ++items;
+                for (int j = 0; j < sh.nkv; ++j, ++kv) {
+                    const int s = kv % C::STAGES, n = kv / C::STAGES;
+                    if (!(ok = wait_bounded(BAR(C::B_KE + s), (n & 1) ^ 1, abort_flag))) break;
+                    const uint32_t sk = base + C::OFF_K + s * C::TILE;
+                    const uint32_t sv = base + C::OFF_V + s * C::TILE;
+                    mbar_arrive_expect_tx(BAR(C::B_KF + s), C::TILE);
 #pragma unroll
-                for (int kb = 0; kb < C::KB; ++kb)
-                    tma_load_3d(sv + kb * 16384u, &tmV, BAR(C::B_VF + s), kb * 64, j * 128, bh);
-                issued[s] = n + 1;
+                    for (int kb = 0; kb < C::KB; ++kb)
+                        tma_load_3d(sk + kb * 16384u, &tmK, BAR(C::B_KF + s), kb * 64, j * 128, bh);
+                    mbar_arrive_expect_tx(BAR(C::B_VF + s), C::TILE);
+#pragma unroll
+                    for (int kb = 0; kb < C::KB; ++kb)
+                        tma_load_3d(sv + kb * 16384u, &tmV, BAR(C::B_VF + s), kb * 64, j * 128, bh);
+                    issued[s] = n + 1;
+                }
             }
             if (*abort_flag) {  // let every copy in flight land before the CTA exits
-                wait_drain(BAR(C::B_Q), 0);
+                if (items > 0) wait_drain(BAR(C::B_Q), (items - 1) & 1);
                 for (int s = 0; s < C::STAGES; ++s)
                     if (issued[s] > 0) {
                         wait_drain(BAR(C::B_KF + s), (issued[s] - 1) & 1);
@@ -175,14 +223,14 @@ __global__ void __launch_bounds__(320, 1)
         // Order per key tile j: O_0 += P_0 V_j, S_0 = Q_0 K_{j+1}^T,
         // O_1 += P_1 V_j, S_1 = Q_1 K_{j+1}^T; each S is issued once the P V
         // that reads the same tensor-memory columns has completed, without
-        // waiting for the other tile's softmax.
+        // waiting for the other tile's softmax.  Phase parities come from
+        // running counts across the CTA's work items.
         if (lane == 0) {
             constexpr uint32_t ID_S = idesc_f16(BF16, 128, 128, false, false);
             constexpr uint32_t ID_O = idesc_f16(BF16, 128, D, false, true);
-            bool ok = wait_bounded(BAR(C::B_Q), 0, abort_flag);
-            auto issue_s = [&](int t, int j) {
+            auto issue_s = [&](int t, int kvi) {
                 const uint32_t sq = base + C::OFF_Q + t * C::TILE;
-                const uint32_t sk = base + C::OFF_K + (j % C::STAGES) * C::TILE;
+                const uint32_t sk = base + C::OFF_K + (kvi % C::STAGES) * C::TILE;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
@@ -191,46 +239,70 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 mma_commit(BAR(C::B_SF + t));
             };
-            if (ok && nkv > 0) {
-                ok = wait_bounded(BAR(C::B_KF), 0, abort_flag);
-                if (ok) {
-                    tc_fence_after();
-                    for (int t = 0; t < 2; ++t)
-                        if (nkv_t[t] > 0) issue_s(t, 0);
-                }
-            }
-            for (int j = 0; ok && j < nkv; ++j) {
-                const int s = j % C::STAGES, n = j / C::STAGES;
-                if (!(ok = wait_bounded(BAR(C::B_VF + s), n & 1, abort_flag))) break;
-                const uint32_t sv = base + C::OFF_V + s * C::TILE;
-                bool k_next = false;  // K_{j+1} has landed
+            int kv = 0, items = 0, n_pv[2] = {0, 0}, n_done[2] = {0, 0}, bh, pair;
+            FwdItems iter;
+            bool ok = true;
+            while (ok && iter.next(p, bh, pair)) {
+                const FwdItemShape sh(p, pair);
+                if (!(ok = wait_bounded(BAR(C::B_Q), items & 1, abort_flag))) break;
+                if (!(ok = wait_bounded(BAR(C::B_KF + kv % C::STAGES), (kv / C::STAGES) & 1,
+                                        abort_flag)))
+                    break;
                 for (int t = 0; ok && t < 2; ++t) {
-                    if (j >= nkv_t[t]) continue;
-                    if (!(ok = wait_bounded(BAR(C::B_PF + t), j & 1, abort_flag))) break;
+                    if (sh.nkv_t[t] == 0) continue;
+                    // S_t's columns held P_t of the previous item: its last P V is done
+                    if (n_pv[t] > 0 &&
+                        !(ok = wait_bounded(BAR(C::B_OD + t), (n_pv[t] - 1) & 1, abort_flag)))
+                        break;
                     tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ts(tmem + C::COL_O + t * D, tmem + t * 128u + kk * 8u,
-                               sdesc_sw128(sv + kk * 2048u, 16384, 1024), ID_O,
-                               (j > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(BAR(C::B_OD + t));
-                    // This tile's next S as soon as its P V has read P (the other
-                    // tile's softmax is not waited for).
-                    if (j + 1 < nkv_t[t]) {
-                        if (!k_next) {
-                            const int s1 = (j + 1) % C::STAGES;
-                            if (!(ok = wait_bounded(BAR(C::B_KF + s1), ((j + 1) / C::STAGES) & 1,
-                                                    abort_flag)))
-                                break;
-                            k_next = true;
-                        }
-                        if (!(ok = wait_bounded(BAR(C::B_OD + t), j & 1, abort_flag))) break;
+                    issue_s(t, kv);
+                }
+                for (int j = 0; ok && j < sh.nkv; ++j) {
+                    const int kvj = kv + j;
+                    const int s = kvj % C::STAGES, n = kvj / C::STAGES;
+                    if (!(ok = wait_bounded(BAR(C::B_VF + s), n & 1, abort_flag))) break;
+                    const uint32_t sv = base + C::OFF_V + s * C::TILE;
+                    bool k_next = false;  // K_{j+1} has landed
+                    for (int t = 0; ok && t < 2; ++t) {
+                        if (j >= sh.nkv_t[t]) continue;
+                        if (!(ok = wait_bounded(BAR(C::B_PF + t), n_pv[t] & 1, abort_flag))) break;
+                        // the first P V of an item overwrites O_t: the previous
+                        // item's epilogue must have read it
+                        if (j == 0 && n_done[t] > 0 &&
+                            !(ok = wait_bounded(BAR(C::B_OE + t), (n_done[t] - 1) & 1, abort_flag)))
+                            break;
                         tc_fence_after();
-                        issue_s(t, j + 1);
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_ts(tmem + C::COL_O + t * D, tmem + t * 128u + kk * 8u,
+                                   sdesc_sw128(sv + kk * 2048u, 16384, 1024), ID_O,
+                                   (j > 0 || kk > 0) ? 1u : 0u);
+                        mma_commit(BAR(C::B_OD + t));
+                        ++n_pv[t];
+                        if (j + 1 < sh.nkv_t[t]) {
+                            if (!k_next) {
+                                const int k1 = kvj + 1;
+                                if (!(ok = wait_bounded(BAR(C::B_KF + k1 % C::STAGES),
+                                                        (k1 / C::STAGES) & 1, abort_flag)))
+                                    break;
+                                k_next = true;
+                            }
+                            // O_t += P_t V_j has read P_t: its columns may take the next S
+                            if (!(ok = wait_bounded(BAR(C::B_OD + t), (n_pv[t] - 1) & 1, abort_flag)))
+                                break;
+                            tc_fence_after();
+                            issue_s(t, kvj + 1);
+                        }
                     }
+                    if (!ok) break;
+                    mma_commit(BAR(C::B_KE + s));
                 }
                 if (!ok) break;
-                mma_commit(BAR(C::B_KE + s));
+                mma_commit(BAR(C::B_QE));  // every S of this item is issued
+                kv += sh.nkv;
+                ++items;
+                for (int t = 0; t < 2; ++t)
+                    if (sh.nkv_t[t] > 0) ++n_done[t];
             }
             if (*abort_flag) {  // every issued MMA must finish before TMEM is freed
                 mma_commit(BAR(C::B_DR));
@@ -244,123 +316,129 @@ __global__ void __launch_bounds__(320, 1)
         const int r = threadIdx.x & 127;  // row of the tile == TMEM lane
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         const uint32_t colS = t * 128u, colO = C::COL_O + t * D;
-        const int qrow = (2 * pair + t) * 128 + r;
-        const int my_nkv = nkv_t[t];
         const float sl = p.scale_log2;
-        float m = -INFINITY, l = 0.f;
+        int n_s = 0, bh, pair;  // S tiles of this query-tile slot seen so far
+        FwdItems iter;
         bool ok = true;
-        for (int j = 0; j < my_nkv; ++j) {
-            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SF + t), j & 1, abort_flag));
-            if (!ok) break;
-            tc_fence_after();
-            // keys at or past N, and (causal) keys after this query, are masked
-            const int key0 = j * 128;
-            int limit = p.N - key0;
-            if (p.causal) limit = min(limit, qrow - key0 + 1);
-            // pass 1: row max over the 128 scores (two chunks of 64 in flight);
-            // tiles without masked columns (all but diagonal and tail tiles)
-            // take the unmasked path
-            const bool full = __all_sync(0xffffffffu, limit >= 128);
-            float mx = -INFINITY;
+        while (ok && iter.next(p, bh, pair)) {
+            const FwdItemShape sh(p, pair);
+            const int my_nkv = sh.nkv_t[t];
+            if (my_nkv == 0) continue;
+            const int qrow = (2 * pair + t) * 128 + r;
+            float m = -INFINITY, l = 0.f;
+            for (int j = 0; j < my_nkv; ++j) {
+                ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SF + t), n_s & 1, abort_flag));
+                if (!ok) break;
+                ++n_s;
+                tc_fence_after();
+                // keys at or past N, and (causal) keys after this query, are masked
+                const int key0 = j * 128;
+                int limit = p.N - key0;
+                if (p.causal) limit = min(limit, qrow - key0 + 1);
+                // pass 1: row max over the 128 scores (two chunks of 64 in flight);
+                // tiles without masked columns (all but diagonal and tail tiles)
+                // take the unmasked path
+                const bool full = __all_sync(0xffffffffu, limit >= 128);
+                float mx = -INFINITY;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t a[32], b[32];
-                tmem_ld32(lane_addr + colS + h * 64u, a);
-                tmem_ld32(lane_addr + colS + h * 64u + 32u, b);
-                tmem_ld_wait();
-                reg_fence32(a);
-                reg_fence32(b);
-                if (full) {
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        mx = max3(mx, __uint_as_float(a[e]), __uint_as_float(a[e + 1]));
-                        mx = max3(mx, __uint_as_float(b[e]), __uint_as_float(b[e + 1]));
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int ca = h * 64 + e, cb = ca + 32;
-                        if (ca < limit) mx = fmaxf(mx, __uint_as_float(a[e]));
-                        if (cb < limit) mx = fmaxf(mx, __uint_as_float(b[e]));
-                    }
-                }
-            }
-            const float m_tile = mx * sl;
-            // Move the max only when it grows past the threshold (the first
-            // tile always sets it); rescaling O needs O(j-1) complete.
-            const bool move = m_tile > m + kRescaleThreshold;
-            if (__any_sync(0xffffffffu, move)) {
-                const float m_new = move ? m_tile : m;
-                const float alpha = ex2(m - m_new);  // 0 on the first tile, 1 if not moved
-                if (j > 0) {
-                    ok = __all_sync(0xffffffffu,
-                                    wait_bounded(BAR(C::B_OD + t), (j - 1) & 1, abort_flag));
-                    if (!ok) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(lane_addr + colO + c * 32u, o);
-                        tmem_ld_wait();
-                        reg_fence32(o);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tmem_st32(lane_addr + colO + c * 32u, o);
-                    }
-                    tmem_st_wait();
-                }
-                l *= alpha;
-                m = m_new;
-            }
-            // pass 2: P = 2^(s scale log2e - m) chunk by chunk, written back as
-            // half over columns pass 2 has already read (P chunk c -> 16c..16c+15)
-            uint64_t sum2 = f2(0.f, 0.f);
-            const uint64_t sl2 = f2(sl, sl), negm2 = f2(-m, -m);
-            uint32_t cur[32];
-            tmem_ld32(lane_addr + colS, cur);
-            tmem_ld_wait();
-            reg_fence32(cur);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t nxt[32];
-                if (c < 3) tmem_ld32(lane_addr + colS + (c + 1) * 32u, nxt);
-                uint32_t pk[16];
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    uint64_t x = fma2(f2(__uint_as_float(cur[2 * q]), __uint_as_float(cur[2 * q + 1])),
-                                      sl2, negm2);
-                    if (!full) {
-                        float2 xv = unf2(x);
-                        if (c * 32 + 2 * q >= limit) xv.x = -INFINITY;
-                        if (c * 32 + 2 * q + 1 >= limit) xv.y = -INFINITY;
-                        x = f2(xv.x, xv.y);
-                    }
-                    const float2 xv = unf2(x);
-                    const uint64_t pp = f2(ex2(xv.x), ex2(xv.y));
-                    sum2 = add2(sum2, pp);
-                    const float2 pv = unf2(pp);
-                    pk[q] = pack2<BF16>(pv.x, pv.y);
-                }
-                tmem_st16(lane_addr + colS + c * 16u, pk);
-                if (c < 3) {
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t a[32], b[32];
+                    tmem_ld32(lane_addr + colS + h * 64u, a);
+                    tmem_ld32(lane_addr + colS + h * 64u + 32u, b);
                     tmem_ld_wait();
-                    reg_fence32(nxt);
+                    reg_fence32(a);
+                    reg_fence32(b);
+                    if (full) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) cur[e] = nxt[e];
+                        for (int e = 0; e < 32; e += 2) {
+                            mx = max3(mx, __uint_as_float(a[e]), __uint_as_float(a[e + 1]));
+                            mx = max3(mx, __uint_as_float(b[e]), __uint_as_float(b[e + 1]));
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int ca = h * 64 + e, cb = ca + 32;
+                            if (ca < limit) mx = fmaxf(mx, __uint_as_float(a[e]));
+                            if (cb < limit) mx = fmaxf(mx, __uint_as_float(b[e]));
+                        }
+                    }
                 }
+                const float m_tile = mx * sl;
+                // Move the max only when it grows past the threshold (the first
+                // tile always sets it); rescaling O needs O(j-1) complete.
+                const bool move = m_tile > m + kRescaleThreshold;
+                if (__any_sync(0xffffffffu, move)) {
+                    const float m_new = move ? m_tile : m;
+                    const float alpha = ex2(m - m_new);  // 0 on the first tile, 1 if not moved
+                    if (j > 0) {
+                        ok = __all_sync(0xffffffffu,
+                                        wait_bounded(BAR(C::B_OD + t), (n_s - 2) & 1, abort_flag));
+                        if (!ok) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t o[32];
+                            tmem_ld32(lane_addr + colO + c * 32u, o);
+                            tmem_ld_wait();
+                            reg_fence32(o);
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                            tmem_st32(lane_addr + colO + c * 32u, o);
+                        }
+                        tmem_st_wait();
+                    }
+                    l *= alpha;
+                    m = m_new;
+                }
+                // pass 2: P = 2^(s scale log2e - m) chunk by chunk, written back as
+                // half over columns pass 2 has already read (P chunk c -> 16c..16c+15)
+                uint64_t sum2 = f2(0.f, 0.f);
+                const uint64_t sl2 = f2(sl, sl), negm2 = f2(-m, -m);
+                uint32_t cur[32];
+                tmem_ld32(lane_addr + colS, cur);
+                tmem_ld_wait();
+                reg_fence32(cur);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t nxt[32];
+                    if (c < 3) tmem_ld32(lane_addr + colS + (c + 1) * 32u, nxt);
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        uint64_t x = fma2(f2(__uint_as_float(cur[2 * q]), __uint_as_float(cur[2 * q + 1])),
+                                          sl2, negm2);
+                        if (!full) {
+                            float2 xv = unf2(x);
+                            if (c * 32 + 2 * q >= limit) xv.x = -INFINITY;
+                            if (c * 32 + 2 * q + 1 >= limit) xv.y = -INFINITY;
+                            x = f2(xv.x, xv.y);
+                        }
+                        const float2 xv = unf2(x);
+                        const uint64_t pp = f2(ex2(xv.x), ex2(xv.y));
+                        sum2 = add2(sum2, pp);
+                        const float2 pv = unf2(pp);
+                        pk[q] = pack2<BF16>(pv.x, pv.y);
+                    }
+                    tmem_st16(lane_addr + colS + c * 16u, pk);
+                    if (c < 3) {
+                        tmem_ld_wait();
+                        reg_fence32(nxt);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) cur[e] = nxt[e];
+                    }
+                }
+                const float2 sv2 = unf2(sum2);
+                const float sum = sv2.x + sv2.y;
+                l += sum;
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(BAR(C::B_PF + t));
             }
-            const float2 sv2 = unf2(sum2);
-            const float sum = sv2.x + sv2.y;
-            l += sum;
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(BAR(C::B_PF + t));
-        }
-        if (ok && my_nkv > 0)
-            ok = __all_sync(0xffffffffu,
-                            wait_bounded(BAR(C::B_OD + t), (my_nkv - 1) & 1, abort_flag));
-        if (ok && my_nkv > 0) {
+            if (ok)
+                ok = __all_sync(0xffffffffu,
+                                wait_bounded(BAR(C::B_OD + t), (n_s - 1) & 1, abort_flag));
+            if (!ok) break;
             tc_fence_after();
             const float inv_l = 1.f / l;
             uint8_t* orow = static_cast<uint8_t*>(p.o) +
@@ -384,6 +462,8 @@ __global__ void __launch_bounds__(320, 1)
                     dst[3] = make_uint4(h[12], h[13], h[14], h[15]);
                 }
             }
+            tc_fence_before();
+            mbar_arrive(BAR(C::B_OE + t));  // O_t has been read: the next item may overwrite it
             if (qrow < p.N)
                 p.lse[static_cast<size_t>(bh) * p.N + qrow] = m * 0.69314718055994531f + logf(l);
         }
