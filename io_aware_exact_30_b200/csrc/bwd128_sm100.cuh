@@ -46,8 +46,7 @@ struct Bwd128Cfg {
     static constexpr uint32_t OFF_STG = OFF_DST + 16384u;     // dQ tile, 64 x 128 fp32 rows
     static constexpr uint32_t OFF_LD = OFF_STG + 32768u;      // ST x (64 L2 + 64 D) fp32
     static constexpr uint32_t OFF_BAR = OFF_LD + ST * 512u;
-    static constexpr int B_KV = 0, B_QF = 1, B_QE = B_QF + ST, B_DOF = B_QE + ST,
-                         B_DOE = B_DOF + ST, B_SF = B_DOE + ST, B_DPF = B_SF + 2,
+    static constexpr int B_KV = 0, B_QF = 1, B_QE = B_QF + ST, B_SF = B_QE + ST, B_DPF = B_SF + 2,
                          B_PTF = B_DPF + 1, B_DVD = B_PTF + 1, B_DSF = B_DVD + 2,
                          B_DQF = B_DSF + 1, B_DQE = B_DQF + 1, B_FIN = B_DQE + 1,
                          B_DR = B_FIN + 1, B_KVE = B_DR + 1, B_ACCE = B_KVE + 1,
@@ -122,8 +121,6 @@ __global__ void __launch_bounds__(448, 1)
         for (int s = 0; s < C::ST; ++s) {
             mbar_init(BAR(C::B_QF + s), 1);
             mbar_init(BAR(C::B_QE + s), 1);
-            mbar_init(BAR(C::B_DOF + s), 1);
-            mbar_init(BAR(C::B_DOE + s), 1);
         }
         mbar_init(BAR(C::B_SF), 1);
         mbar_init(BAR(C::B_SF + 1), 1);
@@ -158,30 +155,27 @@ __global__ void __launch_bounds__(448, 1)
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
             tma_prefetch_desc(&tmDO);
-            int q_issued[C::ST], do_issued[C::ST];
-            for (int s = 0; s < C::ST; ++s) q_issued[s] = do_issued[s] = 0;
+            int issued[C::ST];
+            for (int s = 0; s < C::ST; ++s) issued[s] = 0;
             int g = 0, items = 0, bh = 0, j = 0;
             bool ok = true;
             BwdItems iter;
-            // query tile i of head bh into ring slot g % ST
+            // query tile i of head bh (Q, dO and their L2, D rows) into ring slot g % ST
             auto load_tile = [&](int i) -> bool {
                 const int s = g % C::ST, n = g / C::ST;
                 const size_t ld_row0 = static_cast<size_t>(bh) * p.Np;
                 if (!wait_bounded(BAR(C::B_QE + s), (n & 1) ^ 1, abort_flag)) return false;
                 const uint32_t sq = base + C::OFF_Q + s * C::QTILE;
+                const uint32_t sdo = base + C::OFF_DO + s * C::QTILE;
                 const uint32_t sld = base + C::OFF_LD + s * 512u;
-                mbar_arrive_expect_tx(BAR(C::B_QF + s), C::QTILE + 512u);
+                mbar_arrive_expect_tx(BAR(C::B_QF + s), 2 * C::QTILE + 512u);
                 tma_load_3d(sq, &tmQ, BAR(C::B_QF + s), 0, i * 64, bh);
                 tma_load_3d(sq + 8192u, &tmQ, BAR(C::B_QF + s), 64, i * 64, bh);
+                tma_load_3d(sdo, &tmDO, BAR(C::B_QF + s), 0, i * 64, bh);
+                tma_load_3d(sdo + 8192u, &tmDO, BAR(C::B_QF + s), 64, i * 64, bh);
                 bulk_load(sld, p.l2pad + ld_row0 + i * 64, 256u, BAR(C::B_QF + s));
                 bulk_load(sld + 256u, p.dpad + ld_row0 + i * 64, 256u, BAR(C::B_QF + s));
-                q_issued[s] = n + 1;
-                if (!wait_bounded(BAR(C::B_DOE + s), (n & 1) ^ 1, abort_flag)) return false;
-                const uint32_t sdo = base + C::OFF_DO + s * C::QTILE;
-                mbar_arrive_expect_tx(BAR(C::B_DOF + s), C::QTILE);
-                tma_load_3d(sdo, &tmDO, BAR(C::B_DOF + s), 0, i * 64, bh);
-                tma_load_3d(sdo + 8192u, &tmDO, BAR(C::B_DOF + s), 64, i * 64, bh);
-                do_issued[s] = n + 1;
+                issued[s] = n + 1;
                 ++g;
                 return true;
             };
@@ -208,10 +202,8 @@ __global__ void __launch_bounds__(448, 1)
             }
             if (*abort_flag) {  // let every copy in flight land before the CTA exits
                 if (items > 0) wait_drain(BAR(C::B_KV), (items - 1) & 1);
-                for (int s = 0; s < C::ST; ++s) {
-                    if (q_issued[s] > 0) wait_drain(BAR(C::B_QF + s), (q_issued[s] - 1) & 1);
-                    if (do_issued[s] > 0) wait_drain(BAR(C::B_DOF + s), (do_issued[s] - 1) & 1);
-                }
+                for (int s = 0; s < C::ST; ++s)
+                    if (issued[s] > 0) wait_drain(BAR(C::B_QF + s), (issued[s] - 1) & 1);
             }
         }
     } else if (warp == C::WARP_MMA) {
@@ -221,16 +213,10 @@ __global__ void __launch_bounds__(448, 1)
             constexpr uint32_t ID_KV = idesc_f16(BF16, 128, 128, false, true);  // dV, dK
             constexpr uint32_t ID_DQT = idesc_f16(BF16, 128, 64, true, true);   // dQ^T
             const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sDST = base + C::OFF_DST;
-            // S^T(g) = K Q_g^T into S buffer g & 1; that buffer held P^T(g-2),
-            // which dV(g-2) read (the newest phase of its barrier).
-            auto issue_s = [&](int g) -> bool {
-                const int s = g % C::ST;
-                if (g >= 2 &&
-                    !wait_bounded(BAR(C::B_DVD + (g & 1)), ((g - 2) >> 1) & 1, abort_flag))
-                    return false;
-                if (!wait_bounded(BAR(C::B_QF + s), (g / C::ST) & 1, abort_flag)) return false;
-                tc_fence_after();
-                const uint32_t sQ = base + C::OFF_Q + s * C::QTILE;
+            // S^T(g) = K Q_g^T into S buffer g & 1 (the caller has waited for Q_g
+            // and for dV(g-2), the last reader of that buffer)
+            auto issue_s = [&](int g) {
+                const uint32_t sQ = base + C::OFF_Q + (g % C::ST) * C::QTILE;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * 8192u + (kk & 3) * 32u;
@@ -239,28 +225,35 @@ __global__ void __launch_bounds__(448, 1)
                            sdesc_sw128(sQ + off, 16, 1024), ID_S, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(BAR(C::B_SF + (g & 1)));
-                return true;
             };
-            // Issue order per tile g: dP^T(g), dV(g), S^T(g+1), dK(g) + dQ^T(g).
-            // Every wait below is for the newest phase its barrier can have
-            // reached, so no waiter can fall two phases behind.  Phase
+            // Issue order per tile g: dP^T(g), dV(g), S^T(g+1), dK(g) + dQ^T(g),
+            // with two waits per tile, each testing all its barriers at once (a
+            // dependent wait stalls the issue of queued MMAs).  dP^T(g) needs no
+            // wait of its own: dO_g landed with Q_g (waited before S^T(g)), and
+            // the compute warps released dP^T(g-1) before the DSF(g-1) wait that
+            // preceded dK(g-1).  Every wait is for the newest phase its barrier
+            // can have reached, so no waiter can fall two phases behind; phase
             // parities run on the tile count g across work items.
             int g = 0, items = 0, bh = 0, j = 0;
             bool ok = true;
             BwdItems iter;
             while (ok && iter.next(p, bh, j)) {
                 const int n_it = n_q64 - (p.causal ? 2 * j : 0);
-                if (!(ok = wait_bounded(BAR(C::B_KV), items & 1, abort_flag))) break;
-                if (!(ok = issue_s(g))) break;
+                if (!(ok = wait3(BAR(C::B_KV), items & 1, true, BAR(C::B_QF + g % C::ST),
+                                 (g / C::ST) & 1, true, BAR(C::B_DVD + (g & 1)), ((g - 2) >> 1) & 1,
+                                 g >= 2, abort_flag)))
+                    break;
+                tc_fence_after();
+                issue_s(g);
+                // the item's first dV and dK overwrite accumulators that the
+                // previous item's epilogue must have read
+                if (items > 0 && !(ok = wait_bounded(BAR(C::B_ACCE), (items - 1) & 1, abort_flag)))
+                    break;
                 for (int it = 0; ok && it < n_it; ++it, ++g) {
                     const uint32_t ph = g & 1;
-                    const int s = g % C::ST, n = g / C::ST;
+                    const int s = g % C::ST;
                     const uint32_t sQ = base + C::OFF_Q + s * C::QTILE;
                     const uint32_t sDO = base + C::OFF_DO + s * C::QTILE;
-                    // dP^T(g) = V dO^T: the compute warps have read dP^T(g-1)
-                    if (!(ok = wait_bounded(BAR(C::B_DOF + s), n & 1, abort_flag))) break;
-                    if (g >= 1 && !(ok = wait_bounded(BAR(C::B_DSF), ph ^ 1, abort_flag))) break;
-                    tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t off = (kk >> 2) * 8192u + (kk & 3) * 32u;
@@ -269,12 +262,13 @@ __global__ void __launch_bounds__(448, 1)
                                sdesc_sw128(sDO + off, 16, 1024), ID_S, kk > 0 ? 1u : 0u);
                     }
                     mma_commit(BAR(C::B_DPF));
-                    // dV += P^T dO (P^T from tensor memory).  The item's first
-                    // dV and dK overwrite accumulators that the previous item's
-                    // epilogue must have read.
-                    if (!(ok = wait_bounded(BAR(C::B_PTF), ph, abort_flag))) break;
-                    if (it == 0 && items > 0 &&
-                        !(ok = wait_bounded(BAR(C::B_ACCE), (items - 1) & 1, abort_flag)))
+                    // dV += P^T dO (P^T from tensor memory); then S^T(g+1), whose
+                    // buffer dV(g-1) read
+                    const bool more = it + 1 < n_it;
+                    const int g1 = g + 1;
+                    if (!(ok = wait3(BAR(C::B_PTF), ph, true, BAR(C::B_QF + g1 % C::ST),
+                                     (g1 / C::ST) & 1, more, BAR(C::B_DVD + (g1 & 1)),
+                                     ((g1 - 2) >> 1) & 1, more && g1 >= 2, abort_flag)))
                         break;
                     tc_fence_after();
 #pragma unroll
@@ -283,11 +277,11 @@ __global__ void __launch_bounds__(448, 1)
                                sdesc_sw128(sDO + kk * 2048u, 8192, 1024), ID_KV,
                                (it > 0 || kk > 0) ? 1u : 0u);
                     mma_commit(BAR(C::B_DVD + (g & 1)));
-                    mma_commit(BAR(C::B_DOE + s));
-                    if (it + 1 < n_it && !(ok = issue_s(g + 1))) break;
+                    if (more) issue_s(g1);
                     // dK += dS^T Q ; dQ^T = K^T dS^T (its columns drained for g-1)
-                    if (!(ok = wait_bounded(BAR(C::B_DSF), ph, abort_flag))) break;
-                    if (g >= 1 && !(ok = wait_bounded(BAR(C::B_DQE), ph ^ 1, abort_flag))) break;
+                    if (!(ok = wait3(BAR(C::B_DSF), ph, true, BAR(C::B_DQE), ph ^ 1, g >= 1, 0u, 0u,
+                                     false, abort_flag)))
+                        break;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
@@ -299,7 +293,7 @@ __global__ void __launch_bounds__(448, 1)
                         mma_ss(tmem + C::COL_DQ, sdesc_sw128(sK + kk * 2048u, 16384, 1024),
                                sdesc_sw128(sDST + kk * 2048u, 8192, 1024), ID_DQT,
                                kk > 0 ? 1u : 0u);
-                    mma_commit(BAR(C::B_QE + s));
+                    mma_commit(BAR(C::B_QE + s));  // Q_g, dO_g no longer read
                     mma_commit(BAR(C::B_DQF));
                 }
                 if (!ok) break;

@@ -244,33 +244,35 @@ __global__ void __launch_bounds__(320, 1)
             bool ok = true;
             while (ok && iter.next(p, bh, pair)) {
                 const FwdItemShape sh(p, pair);
-                if (!(ok = wait_bounded(BAR(C::B_Q), items & 1, abort_flag))) break;
-                if (!(ok = wait_bounded(BAR(C::B_KF + kv % C::STAGES), (kv / C::STAGES) & 1,
-                                        abort_flag)))
+                // Q of this item, K_0, and for each tile t the previous item's
+                // last P_t V, which read the columns S_t is about to take.
+                // Waits test all their barriers at once: a dependent wait stalls
+                // the issue of queued MMAs, so one stall per group.
+                const bool w0 = sh.nkv_t[0] > 0 && n_pv[0] > 0, w1 = sh.nkv_t[1] > 0 && n_pv[1] > 0;
+                if (!(ok = wait3(BAR(C::B_Q), items & 1, true, BAR(C::B_KF + kv % C::STAGES),
+                                 (kv / C::STAGES) & 1, true, BAR(C::B_OD), (n_pv[0] - 1) & 1, w0,
+                                 abort_flag)))
                     break;
-                for (int t = 0; ok && t < 2; ++t) {
-                    if (sh.nkv_t[t] == 0) continue;
-                    // S_t's columns held P_t of the previous item: its last P V is done
-                    if (n_pv[t] > 0 &&
-                        !(ok = wait_bounded(BAR(C::B_OD + t), (n_pv[t] - 1) & 1, abort_flag)))
-                        break;
-                    tc_fence_after();
-                    issue_s(t, kv);
-                }
+                if (w1 && !(ok = wait_bounded(BAR(C::B_OD + 1), (n_pv[1] - 1) & 1, abort_flag)))
+                    break;
+                tc_fence_after();
+                for (int t = 0; t < 2; ++t)
+                    if (sh.nkv_t[t] > 0) issue_s(t, kv);
                 for (int j = 0; ok && j < sh.nkv; ++j) {
                     const int kvj = kv + j;
                     const int s = kvj % C::STAGES, n = kvj / C::STAGES;
-                    if (!(ok = wait_bounded(BAR(C::B_VF + s), n & 1, abort_flag))) break;
                     const uint32_t sv = base + C::OFF_V + s * C::TILE;
+                    const int k1 = kvj + 1;
                     bool k_next = false;  // K_{j+1} has landed
                     for (int t = 0; ok && t < 2; ++t) {
-                        if (j >= sh.nkv_t[t]) continue;
-                        if (!(ok = wait_bounded(BAR(C::B_PF + t), n_pv[t] & 1, abort_flag))) break;
-                        // the first P V of an item overwrites O_t: the previous
-                        // item's epilogue must have read it
-                        if (j == 0 && n_done[t] > 0 &&
-                            !(ok = wait_bounded(BAR(C::B_OE + t), (n_done[t] - 1) & 1, abort_flag)))
+                        const bool act = j < sh.nkv_t[t];
+                        // V_j (first tile only), P_t, and at an item's first j the
+                        // previous epilogue's read of O_t, which P_t V overwrites
+                        if (!(ok = wait3(BAR(C::B_VF + s), n & 1, t == 0, BAR(C::B_PF + t),
+                                         n_pv[t] & 1, act, BAR(C::B_OE + t), (n_done[t] - 1) & 1,
+                                         act && j == 0 && n_done[t] > 0, abort_flag)))
                             break;
+                        if (!act) continue;
                         tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
@@ -280,18 +282,14 @@ __global__ void __launch_bounds__(320, 1)
                         mma_commit(BAR(C::B_OD + t));
                         ++n_pv[t];
                         if (j + 1 < sh.nkv_t[t]) {
-                            if (!k_next) {
-                                const int k1 = kvj + 1;
-                                if (!(ok = wait_bounded(BAR(C::B_KF + k1 % C::STAGES),
-                                                        (k1 / C::STAGES) & 1, abort_flag)))
-                                    break;
-                                k_next = true;
-                            }
                             // O_t += P_t V_j has read P_t: its columns may take the next S
-                            if (!(ok = wait_bounded(BAR(C::B_OD + t), (n_pv[t] - 1) & 1, abort_flag)))
+                            if (!(ok = wait3(BAR(C::B_OD + t), (n_pv[t] - 1) & 1, true,
+                                             BAR(C::B_KF + k1 % C::STAGES), (k1 / C::STAGES) & 1,
+                                             !k_next, 0u, 0u, false, abort_flag)))
                                 break;
+                            k_next = true;
                             tc_fence_after();
-                            issue_s(t, kvj + 1);
+                            issue_s(t, k1);
                         }
                     }
                     if (!ok) break;

@@ -77,6 +77,35 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
+// Non-blocking test of a phase's completion.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits for up to three phases (entries with en == false are skipped).  All
+// tests are issued before any result is used: a thread with tensor-core work
+// queued stalls for each dependent shared-memory access until that work has
+// been handed to the tensor core, so one stall per group instead of one per
+// barrier.  Falls back to wait_bounded for whatever has not completed.
+__device__ __forceinline__ bool wait3(uint32_t b0, uint32_t p0, bool e0, uint32_t b1, uint32_t p1,
+                                      bool e1, uint32_t b2, uint32_t p2, bool e2,
+                                      volatile uint32_t* abort_flag) {
+    const bool r0 = !e0 || mbar_test_wait(b0, p0);
+    const bool r1 = !e1 || mbar_test_wait(b1, p1);
+    const bool r2 = !e2 || mbar_test_wait(b2, p2);
+    if (r0 && r1 && r2) return true;
+    return (r0 || wait_bounded(b0, p0, abort_flag)) && (r1 || wait_bounded(b1, p1, abort_flag)) &&
+           (r2 || wait_bounded(b2, p2, abort_flag));
+}
+
 // Bounded wait used only while draining after an abort: ignores the abort flag.
 __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
     uint32_t never = 0;
