@@ -49,7 +49,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // Per-device state: sm_100 check and the opt-in shared-memory size, done once.
 std::mutex g_dev_mu;
 int g_dev_state[kMaxDevices];  // 0 unknown, 1 ready, -1 unsupported
-int g_sm_count[kMaxDevices];   // multiprocessors: the persistent kernels' grid size
+int g_sm_count[kMaxDevices];   // multiprocessors: grid size of the static schedules
 
 int check_device(int* dev_out) {
     int dev = -1;
@@ -139,9 +139,11 @@ bool make_map(CUtensorMap* m, const void* ptr, int dtype, int BH, int N, int d,
 template <int D, bool BF16>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const attn::FwdParams& p, int sm_count, cudaStream_t st) {
+    // causal: one CTA per work item, running CTAs take pending CTAs' items;
+    // otherwise one CTA per multiprocessor
     const long long items = 1LL * p.n_pairs * p.BH;
     if (items >= (1LL << 31)) return ATTN_ERR_SHAPE;
-    const int nblocks = static_cast<int>(items < sm_count ? items : sm_count);
+    const int nblocks = static_cast<int>(p.causal || items < sm_count ? items : sm_count);
     attn::attn_fwd_kernel<D, BF16><<<static_cast<unsigned>(nblocks), FwdCfg<D>::NTHREADS,
                                      FwdCfg<D>::SMEM_BYTES, st>>>(mq, mk, mv, p);
     return launch_ok() ? ATTN_OK : ATTN_ERR_LAUNCH;
@@ -224,12 +226,11 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
     p.scale_log2 = scale * 1.4426950408889634f;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool bf = dtype == ATTN_BF16;
-    const int sms = g_sm_count[dev];
     if (d == 64)
-        return bf ? launch_fwd<64, true>(mq, mk, mv, p, sms, st)
-                  : launch_fwd<64, false>(mq, mk, mv, p, sms, st);
-    return bf ? launch_fwd<128, true>(mq, mk, mv, p, sms, st)
-              : launch_fwd<128, false>(mq, mk, mv, p, sms, st);
+        return bf ? launch_fwd<64, true>(mq, mk, mv, p, g_sm_count[dev], st)
+                  : launch_fwd<64, false>(mq, mk, mv, p, g_sm_count[dev], st);
+    return bf ? launch_fwd<128, true>(mq, mk, mv, p, g_sm_count[dev], st)
+              : launch_fwd<128, false>(mq, mk, mv, p, g_sm_count[dev], st);
 }
 
 size_t attn_bwd_workspace_bytes(int B, int H, int N, int d) {

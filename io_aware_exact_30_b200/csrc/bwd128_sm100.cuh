@@ -3,8 +3,9 @@
 // with 64-query inner tiles so that every accumulator of the tile loop has
 // tensor memory of its own and no stage waits for another to be drained.
 //
-// Persistent: one CTA per multiprocessor walks a list of (head, 128-key tile
-// j) work items (see BwdItems).  For each, K_j and V_j are loaded into shared
+// Persistent: CTAs take (head, 128-key tile j) work items through an
+// ItemStream (see bwd_item): dynamically under the causal mask, in static
+// snake order otherwise.  For each, K_j and V_j are loaded into shared
 // memory and 64-query tiles of Q, dO (and their L2, D statistics) stream
 // through a 3-stage pipeline that runs on across items.  Per query tile i:
 //   S^T  = K_j Q_i^T                     tensor memory, double-buffered
@@ -51,46 +52,37 @@ struct Bwd128Cfg {
                          B_DQF = B_DSF + 1, B_DQE = B_DQF + 1, B_FIN = B_DQE + 1,
                          B_DR = B_FIN + 1, B_KVE = B_DR + 1, B_ACCE = B_KVE + 1,
                          B_SRD = B_ACCE + 1, B_STGF = B_SRD + 1, B_STGE = B_STGF + 1,
-                         NBAR = B_STGE + 1;
+                         B_CLCF = B_STGE + 1, B_CLCE = B_CLCF + 2, NBAR = B_CLCE + 2;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
-    static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
+    static constexpr uint32_t OFF_CLC = (OFF_MISC + 16 + 15) & ~15u;  // 2 x 16-byte responses
+    static constexpr uint32_t SMEM_BYTES = OFF_CLC + 32 + 1024;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 192, COL_DV = 256, COL_DK = 384;
     static constexpr int NCOMPUTE = 256, NDQ = 128;
+    // arrivals that free a work-item response: producer, MMA, 8 compute and 4 dQ warps
+    static constexpr int CLC_CONSUMERS = 2 + NCOMPUTE / 32 + NDQ / 32;
     static constexpr int NTHREADS = NCOMPUTE + NDQ + 64;
     static constexpr int WARP_DQ0 = NCOMPUTE / 32;
     static constexpr int WARP_TMA = WARP_DQ0 + NDQ / 32, WARP_MMA = WARP_TMA + 1;
 };
 
-// Persistent schedule.  A work item is (head, 128-key tile j); under the
-// causal mask it costs n_q64 - 2j query tiles, otherwise n_q64.  Heads are
-// taken in groups whose K, V, Q and dO fit in L2 together; within a group
-// the items are listed heaviest first (j ascending, heads in order within a
-// j) when causal, head-major otherwise, and the list is dealt to the CTAs in
-// snake order (round r: item r*G + c to CTA c for even r, to CTA G - 1 - c
-// for odd r), which balances the CTAs' totals.
-struct BwdItems {
-    int round;
-    __device__ BwdItems() : round(0) {}
-    __device__ bool next(const BwdParams& p, int& bh, int& j) {
-        const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
-        const long long k = 1LL * round * G + ((round & 1) ? (G - 1 - c) : c);
-        if (k >= 1LL * p.BH * p.n_ktiles) return false;
-        ++round;
-        const int ki = static_cast<int>(k);
-        if (p.causal) {
-            const int per_group = p.group * p.n_ktiles;
-            const int g = ki / per_group, i = ki % per_group;
-            const int heads = min(p.group, p.BH - g * p.group);
-            j = i / heads;
-            bh = g * p.group + i % heads;
-        } else {
-            bh = ki / p.n_ktiles;
-            j = ki % p.n_ktiles;
-        }
-        return true;
+// Work item k of the list: (head bh, 128-key tile j).  Under the causal mask
+// item (bh, j) costs n_q64 - 2j query tiles, otherwise n_q64.  Heads are taken
+// in groups whose K, V, Q and dO fit in L2 together; within a group the items
+// are listed heaviest first (j ascending, heads in order within a j) when
+// causal, head-major otherwise.
+__device__ __forceinline__ void bwd_item(const BwdParams& p, int k, int& bh, int& j) {
+    if (p.causal) {
+        const int per_group = p.group * p.n_ktiles;
+        const int g = k / per_group, i = k % per_group;
+        const int heads = min(p.group, p.BH - g * p.group);
+        j = i / heads;
+        bh = g * p.group + i % heads;
+    } else {
+        bh = k / p.n_ktiles;
+        j = k % p.n_ktiles;
     }
-};
+}
 
 template <bool BF16>
 __global__ void __launch_bounds__(448, 1)
@@ -136,6 +128,10 @@ __global__ void __launch_bounds__(448, 1)
         mbar_init(BAR(C::B_SRD), C::NCOMPUTE / 2);
         mbar_init(BAR(C::B_STGF), C::NDQ);
         mbar_init(BAR(C::B_STGE), 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(BAR(C::B_CLCF + i), 1);
+            mbar_init(BAR(C::B_CLCE + i), C::CLC_CONSUMERS);
+        }
         *abort_flag = 0u;
         fence_mbar_init();
     }
@@ -147,6 +143,8 @@ __global__ void __launch_bounds__(448, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    ItemStream cs(p.causal != 0, p.BH * p.n_ktiles, base + C::OFF_CLC, BAR(C::B_CLCF),
+                  BAR(C::B_CLCE));
 
     if (warp == C::WARP_TMA) {
         // ------------------------------------------------------ TMA producer
@@ -159,7 +157,6 @@ __global__ void __launch_bounds__(448, 1)
             for (int s = 0; s < C::ST; ++s) issued[s] = 0;
             int g = 0, items = 0, bh = 0, j = 0;
             bool ok = true;
-            BwdItems iter;
             // query tile i of head bh (Q, dO and their L2, D rows) into ring slot g % ST
             auto load_tile = [&](int i) -> bool {
                 const int s = g % C::ST, n = g / C::ST;
@@ -179,7 +176,8 @@ __global__ void __launch_bounds__(448, 1)
                 ++g;
                 return true;
             };
-            while (ok && iter.next(p, bh, j)) {
+            while (ok && cs.cur >= 0) {
+                bwd_item(p, cs.cur, bh, j);
                 const int i_begin = p.causal ? 2 * j : 0;
                 const int n_it = n_q64 - i_begin;
                 const int pre = min(C::ST, n_it);
@@ -199,8 +197,11 @@ __global__ void __launch_bounds__(448, 1)
                 }
                 ++items;
                 for (int it = pre; ok && it < n_it; ++it) ok = load_tile(i_begin + it);
+                // once an item's loads are issued, ask for the next item
+                if (ok) ok = cs.request(abort_flag) && cs.advance(abort_flag, false);
             }
             if (*abort_flag) {  // let every copy in flight land before the CTA exits
+                cs.drain();
                 if (items > 0) wait_drain(BAR(C::B_KV), (items - 1) & 1);
                 for (int s = 0; s < C::ST; ++s)
                     if (issued[s] > 0) wait_drain(BAR(C::B_QF + s), (issued[s] - 1) & 1);
@@ -236,8 +237,8 @@ __global__ void __launch_bounds__(448, 1)
             // parities run on the tile count g across work items.
             int g = 0, items = 0, bh = 0, j = 0;
             bool ok = true;
-            BwdItems iter;
-            while (ok && iter.next(p, bh, j)) {
+            while (ok && cs.cur >= 0) {
+                bwd_item(p, cs.cur, bh, j);
                 const int n_it = n_q64 - (p.causal ? 2 * j : 0);
                 if (!(ok = wait3(BAR(C::B_KV), items & 1, true, BAR(C::B_QF + g % C::ST),
                                  (g / C::ST) & 1, true, BAR(C::B_DVD + (g & 1)), ((g - 2) >> 1) & 1,
@@ -300,6 +301,7 @@ __global__ void __launch_bounds__(448, 1)
                 mma_commit(BAR(C::B_FIN));  // dK, dV of this item complete
                 mma_commit(BAR(C::B_KVE));  // K, V no longer read
                 ++items;
+                ok = cs.advance(abort_flag, false);
             }
             if (*abort_flag) {  // every issued MMA must finish before TMEM is freed
                 mma_commit(BAR(C::B_DR));
@@ -321,8 +323,8 @@ __global__ void __launch_bounds__(448, 1)
         const uint32_t stg = base + C::OFF_STG + r * 4u;
         int g = 0, bh = 0, j = 0;
         bool dq_ok = true;
-        BwdItems iter;
-        while (dq_ok && iter.next(p, bh, j)) {
+        while (dq_ok && cs.cur >= 0) {
+            bwd_item(p, cs.cur, bh, j);
             const int i_begin = p.causal ? 2 * j : 0;
             const int n_it = n_q64 - i_begin;
             float* acc_head = p.dqacc + static_cast<size_t>(bh) * p.N * D;
@@ -365,6 +367,7 @@ __global__ void __launch_bounds__(448, 1)
                 dq_ok = __all_sync(0xffffffffu, dq_ok);
                 if (!dq_ok) break;
             }
+            if (dq_ok) dq_ok = cs.advance(abort_flag, true);
         }
         if (issuer) bulk_wait_all();  // every reduction complete before the CTA exits
     } else {
@@ -377,8 +380,8 @@ __global__ void __launch_bounds__(448, 1)
         const int c0 = half * 32;  // first query column of this thread's half
         int g = 0, items = 0, bh = 0, j = 0;
         bool ok = true;
-        BwdItems iter;
-        while (ok && iter.next(p, bh, j)) {
+        while (ok && cs.cur >= 0) {
+            bwd_item(p, cs.cur, bh, j);
             const int i_begin = p.causal ? 2 * j : 0;
             const int n_it = n_q64 - i_begin;
             const int key = j * 128 + r;
@@ -508,6 +511,7 @@ __global__ void __launch_bounds__(448, 1)
             tc_fence_before();
             mbar_arrive(BAR(C::B_ACCE));
             ++items;
+            ok = cs.advance(abort_flag, true);
         }
     }
 #undef BAR
@@ -541,8 +545,9 @@ inline bool bwd128_set_attributes() {
 }
 
 // mq, mdo must be tensor maps with 64-row boxes; mk, mv with 128-row boxes.
-// Launches the persistent main kernel on min(#SMs, #items) CTAs, then the dQ
-// conversion.
+// Launches the persistent main kernel, then the dQ conversion.  Causal: one CTA
+// per work item, running CTAs take pending CTAs' items; otherwise one CTA per
+// multiprocessor.
 template <bool BF16>
 int bwd_main128_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                        const CUtensorMap& mdo, void* dq, void* dk, void* dv, void* ws, int B,
@@ -572,7 +577,7 @@ int bwd_main128_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     }
     const long long items = 1LL * p.n_ktiles * p.BH;
     if (items >= (1LL << 31)) return -2;
-    const int nblocks = static_cast<int>(items < sm_count ? items : sm_count);
+    const int nblocks = static_cast<int>(causal || items < sm_count ? items : sm_count);
     attn_bwd_main128_kernel<BF16><<<static_cast<unsigned>(nblocks), Bwd128Cfg::NTHREADS,
                                     Bwd128Cfg::SMEM_BYTES, st>>>(mq, mk, mv, mdo, p);
     cudaError_t e = cudaGetLastError();

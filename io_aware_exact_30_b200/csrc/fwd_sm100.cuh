@@ -57,36 +57,25 @@ struct FwdParams {
 };
 
 // Persistent schedule.  A work item is (head, pair of query tiles); there are
-// BH * n_pairs of them.  Heads are taken in groups of `group` heads whose K/V
-// fit comfortably in L2 together; within a group the items are listed
-// heaviest first — under the causal mask pair p costs 4p + 3 key-tile steps,
-// so the group's list runs from the last pair down, heads in order within a
-// pair; without the mask all items cost the same and the list is head-major.
-// The list is dealt to the CTAs in snake order: round r gives item r*G + c to
-// CTA c when r is even and to CTA G - 1 - c when r is odd (G = grid size),
-// which balances the CTAs' totals to within about one small item.
-struct FwdItems {
-    int round;
-    __device__ FwdItems() : round(0) {}
-    __device__ bool next(const FwdParams& p, int& bh, int& pair) {
-        const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
-        const long long k = 1LL * round * G + ((round & 1) ? (G - 1 - c) : c);
-        if (k >= 1LL * p.BH * p.n_pairs) return false;
-        ++round;
-        const int ki = static_cast<int>(k);
-        if (p.causal) {
-            const int per_group = p.group * p.n_pairs;
-            const int g = ki / per_group, i = ki % per_group;
-            const int heads = min(p.group, p.BH - g * p.group);
-            pair = p.n_pairs - 1 - i / heads;
-            bh = g * p.group + i % heads;
-        } else {
-            bh = ki / p.n_pairs;
-            pair = ki % p.n_pairs;
-        }
-        return true;
+// BH * n_pairs of them, taken through an ItemStream: dynamically under the
+// causal mask (unequal costs), in static snake order otherwise.  Heads are taken in groups of
+// `group` heads whose K/V fit comfortably in L2 together; within a group the
+// items are listed heaviest first — under the causal mask pair p costs 4p + 3
+// key-tile steps, so the group's list runs from the last pair down, heads in
+// order within a pair; without the mask all items cost the same and the list
+// is head-major.
+__device__ __forceinline__ void fwd_item(const FwdParams& p, int k, int& bh, int& pair) {
+    if (p.causal) {
+        const int per_group = p.group * p.n_pairs;
+        const int g = k / per_group, i = k % per_group;
+        const int heads = min(p.group, p.BH - g * p.group);
+        pair = p.n_pairs - 1 - i / heads;
+        bh = g * p.group + i % heads;
+    } else {
+        bh = k / p.n_pairs;
+        pair = k % p.n_pairs;
     }
-};
+}
 
 struct FwdItemShape {
     bool has1;
@@ -112,9 +101,13 @@ struct FwdCfg {
     static constexpr uint32_t OFF_BAR = OFF_V + STAGES * TILE;
     static constexpr int B_Q = 0, B_KF = 1, B_VF = B_KF + STAGES, B_KE = B_VF + STAGES,
                          B_SF = B_KE + STAGES, B_PF = B_SF + 2, B_OD = B_PF + 2, B_DR = B_OD + 2,
-                         B_QE = B_DR + 1, B_OE = B_QE + 1, NBAR = B_OE + 2;
+                         B_QE = B_DR + 1, B_OE = B_QE + 1, B_CLCF = B_OE + 2, B_CLCE = B_CLCF + 2,
+                         NBAR = B_CLCE + 2;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
-    static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+    static constexpr uint32_t OFF_CLC = (OFF_MISC + 16 + 15) & ~15u;  // 2 x 16-byte responses
+    static constexpr uint32_t SMEM_BYTES = OFF_CLC + 32 + 1024;  // + alignment slack
+    // arrivals that free a work-item response: producer, MMA and 8 softmax warps
+    static constexpr int CLC_CONSUMERS = 10;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_O = 256;
     static constexpr int NTHREADS = 320;
@@ -157,6 +150,10 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(BAR(C::B_OE + t), 128);
         }
         mbar_init(BAR(C::B_DR), 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(BAR(C::B_CLCF + i), 1);
+            mbar_init(BAR(C::B_CLCE + i), C::CLC_CONSUMERS);
+        }
         *abort_flag = 0u;
         fence_mbar_init();
     }
@@ -168,6 +165,8 @@ __global__ void __launch_bounds__(320, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    ItemStream cs(p.causal != 0, p.BH * p.n_pairs, base + C::OFF_CLC, BAR(C::B_CLCF),
+                  BAR(C::B_CLCE));
 
     if (warp == C::WARP_TMA) {
         // ------------------------------------------------------ TMA producer
@@ -179,9 +178,11 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int s = 0; s < C::STAGES; ++s) issued[s] = 0;
             int kv = 0, items = 0, bh, pair;
-            FwdItems iter;
             bool ok = true;
-            while (ok && iter.next(p, bh, pair)) {
+            // once an item's loads are issued, ask for the next item
+            for (; ok && cs.cur >= 0;
+                 ok = ok && cs.request(abort_flag) && cs.advance(abort_flag, false)) {
+                fwd_item(p, cs.cur, bh, pair);
                 const FwdItemShape sh(p, pair);
                 // the previous item's S MMAs are done reading the query tiles
                 if (items > 0 && !(ok = wait_bounded(BAR(C::B_QE), (items - 1) & 1, abort_flag)))
@@ -210,6 +211,7 @@ __global__ void __launch_bounds__(320, 1)
                 }
             }
             if (*abort_flag) {  // let every copy in flight land before the CTA exits
+                cs.drain();
                 if (items > 0) wait_drain(BAR(C::B_Q), (items - 1) & 1);
                 for (int s = 0; s < C::STAGES; ++s)
                     if (issued[s] > 0) {
@@ -240,9 +242,9 @@ __global__ void __launch_bounds__(320, 1)
                 mma_commit(BAR(C::B_SF + t));
             };
             int kv = 0, items = 0, n_pv[2] = {0, 0}, n_done[2] = {0, 0}, bh, pair;
-            FwdItems iter;
             bool ok = true;
-            while (ok && iter.next(p, bh, pair)) {
+            for (; ok && cs.cur >= 0; ok = ok && cs.advance(abort_flag, false)) {
+                fwd_item(p, cs.cur, bh, pair);
                 const FwdItemShape sh(p, pair);
                 // Q of this item, K_0, and for each tile t the previous item's
                 // last P_t V, which read the columns S_t is about to take.
@@ -316,9 +318,9 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t colS = t * 128u, colO = C::COL_O + t * D;
         const float sl = p.scale_log2;
         int n_s = 0, bh, pair;  // S tiles of this query-tile slot seen so far
-        FwdItems iter;
         bool ok = true;
-        while (ok && iter.next(p, bh, pair)) {
+        for (; ok && cs.cur >= 0; ok = ok && cs.advance(abort_flag, true)) {
+            fwd_item(p, cs.cur, bh, pair);
             const FwdItemShape sh(p, pair);
             const int my_nkv = sh.nkv_t[t];
             if (my_nkv == 0) continue;

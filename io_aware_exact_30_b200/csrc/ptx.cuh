@@ -106,6 +106,33 @@ __device__ __forceinline__ bool wait3(uint32_t b0, uint32_t p0, bool e0, uint32_
            (r2 || wait_bounded(b2, p2, abort_flag));
 }
 
+// ---------------------------------------------------- cluster launch control --
+// Asks the scheduler to cancel the launch of a not-yet-running CTA of this
+// grid; a 16-byte response lands at `resp` and completes 16 transaction bytes
+// on `bar`.  No request may follow one whose response reported failure.
+__device__ __forceinline__ void clc_try_cancel(uint32_t resp, uint32_t bar) {
+    asm volatile(
+        "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 "
+        "[%0], [%1];" ::"r"(resp),
+        "r"(bar)
+        : "memory");
+}
+// Decodes a response: the cancelled CTA's x index, or -1 if nothing was cancelled.
+__device__ __forceinline__ int clc_result(uint32_t resp) {
+    uint64_t lo, hi;
+    asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];" : "=l"(lo), "=l"(hi) : "r"(resp) : "memory");
+    uint32_t ok, x;
+    asm volatile(
+        "{\n\t.reg .b128 r;\n\t.reg .pred p;\n\t"
+        "mov.b128 r, {%2, %3};\n\t"
+        "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t"
+        "clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, r;\n\t}"
+        : "=r"(ok), "=r"(x)
+        : "l"(lo), "l"(hi));
+    return ok ? static_cast<int>(x) : -1;
+}
+
 // Bounded wait used only while draining after an abort: ignores the abort flag.
 __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
     uint32_t never = 0;
@@ -404,5 +431,67 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                  "r"(d)
                  : "memory");
 }
+
+// Work items of a persistent kernel.  Items are listed in the order they
+// should start; each CTA begins with the item of its own index.
+//  - Dynamic (items of unequal cost): the grid has one CTA per item, and when
+//    a CTA's producer has issued its current item's loads it asks, through
+//    cluster launch control, to cancel a pending CTA's launch and takes that
+//    CTA's item: items go to whichever CTA frees up first.  Every role reads
+//    the response when it finishes its current item.  Responses alternate
+//    between two 16-byte slots; `full` barriers (count 1 + 16 tx bytes) signal
+//    a response, `empty` barriers (one arrival per consuming thread or warp)
+//    free its slot.
+//  - Static (items of equal cost): the grid has at most one CTA per
+//    multiprocessor and the list is dealt in snake order (round r gives item
+//    r*G + c to CTA c when r is even and to CTA G - 1 - c when r is odd).
+struct ItemStream {
+    uint32_t resp, full, empty;  // shared addresses: 2 x 16 B, 2 x 8 B, 2 x 8 B
+    int total;                   // items in the list
+    int cur;                     // current item, -1 once none is left
+    int t;                       // items finished so far
+    bool dynamic;
+    bool pending;                // producer only: a request is in flight
+    __device__ ItemStream(bool dynamic_, int total_, uint32_t resp_, uint32_t full_,
+                          uint32_t empty_)
+        : resp(resp_), full(full_), empty(empty_), total(total_),
+          cur(static_cast<int>(blockIdx.x)), t(0), dynamic(dynamic_), pending(false) {}
+    // Producer (one thread), once its current item is issued: request the next.
+    __device__ bool request(volatile uint32_t* abort_flag) {
+        if (!dynamic) return true;
+        const int k = t + 1, slot = k & 1, u = (k - 1) >> 1;
+        if (u >= 1 && !wait_bounded(empty + 8u * slot, (u - 1) & 1, abort_flag)) return false;
+        mbar_arrive_expect_tx(full + 8u * slot, 16u);
+        clc_try_cancel(resp + 16u * slot, full + 8u * slot);
+        pending = true;
+        return true;
+    }
+    // Every role after finishing the current item: moves to the next one.  A
+    // role with a whole warp in the loop passes warp = true (all lanes read the
+    // response, lane 0 arrives); a single-thread role passes false.
+    __device__ bool advance(volatile uint32_t* abort_flag, bool warp) {
+        if (!dynamic) {
+            ++t;
+            const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+            const long long k = 1LL * t * G + ((t & 1) ? (G - 1 - c) : c);
+            cur = k < total ? static_cast<int>(k) : -1;
+            return true;
+        }
+        const int k = t + 1, slot = k & 1, u = (k - 1) >> 1;
+        bool ok = wait_bounded(full + 8u * slot, u & 1, abort_flag);
+        if (warp) ok = __all_sync(0xffffffffu, ok);
+        if (!ok) return false;
+        cur = clc_result(resp + 16u * slot);
+        if (warp) __syncwarp();
+        if (!warp || (threadIdx.x & 31) == 0) mbar_arrive(empty + 8u * slot);
+        pending = false;
+        ++t;
+        return true;
+    }
+    // Producer after an abort: let an outstanding response land before exit.
+    __device__ void drain() {
+        if (pending) wait_drain(full + 8u * ((t + 1) & 1), (t >> 1) & 1);
+    }
+};
 
 }  // namespace attn
