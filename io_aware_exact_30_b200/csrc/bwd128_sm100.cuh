@@ -22,10 +22,15 @@
 // Tensor memory (512 columns): S^T buffers at 0 and 64, dP^T at 128, dQ^T at
 // 192, dV at 256, dK at 384.
 //
-// Roles (448 threads): warps 0-7 compute P^T and dS^T (warp w reads TMEM
+// Roles (480 threads): warps 0-7 compute P^T and dS^T (warp w reads TMEM
 // lanes 32 (w % 4) .. + 31 and query-column half w / 4 of the 64-wide tile),
 // warps 8-11 drain dQ^T (lane = feature) through the shared staging tile into
-// the fp32 accumulator, warp 12 TMA producer, warp 13 MMA issuer and TMEM owner.
+// the fp32 accumulator, warp 12 TMA producer, warp 13 issues S^T and dP^T (and
+// owns the tensor memory), warp 14 issues dV, dK and dQ^T.  A thread that
+// issues MMAs stalls at each dependent shared-memory access (a barrier test)
+// until its queued MMAs have been handed to the tensor core; with two issuers
+// on different SM sub-partitions one keeps the tensor core fed while the other
+// waits.
 #pragma once
 
 #include "bwd_sm100.cuh"
@@ -48,22 +53,25 @@ struct Bwd128Cfg {
     static constexpr uint32_t OFF_LD = OFF_STG + 32768u;      // ST x (64 L2 + 64 D) fp32
     static constexpr uint32_t OFF_BAR = OFF_LD + ST * 512u;
     static constexpr int B_KV = 0, B_QF = 1, B_QE = B_QF + ST, B_SF = B_QE + ST, B_DPF = B_SF + 2,
-                         B_PTF = B_DPF + 1, B_DVD = B_PTF + 1, B_DSF = B_DVD + 2,
-                         B_DQF = B_DSF + 1, B_DQE = B_DQF + 1, B_FIN = B_DQE + 1,
-                         B_DR = B_FIN + 1, B_KVE = B_DR + 1, B_ACCE = B_KVE + 1,
-                         B_SRD = B_ACCE + 1, B_STGF = B_SRD + 1, B_STGE = B_STGF + 1,
-                         B_CLCF = B_STGE + 1, B_CLCE = B_CLCF + 2, NBAR = B_CLCE + 2;
+                         B_PTF = B_DPF + 1, B_DVD = B_PTF + 2, B_DSF = B_DVD + 2,
+                         B_DSTE = B_DSF + 1, B_DQF = B_DSTE + 1, B_DQE = B_DQF + 1,
+                         B_FIN = B_DQE + 1, B_DR = B_FIN + 1, B_KVE = B_DR + 2, B_ACCE = B_KVE + 1,
+                         B_SRD = B_ACCE + 1, B_STGF = B_SRD + 2, B_STGE = B_STGF + 1,
+                         B_CLCF = B_STGE + 1, B_CLCE = B_CLCF + 2, B_DPE = B_CLCE + 2,
+                         NBAR = B_DPE + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr uint32_t OFF_CLC = (OFF_MISC + 16 + 15) & ~15u;  // 2 x 16-byte responses
     static constexpr uint32_t SMEM_BYTES = OFF_CLC + 32 + 1024;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 192, COL_DV = 256, COL_DK = 384;
     static constexpr int NCOMPUTE = 256, NDQ = 128;
-    // arrivals that free a work-item response: producer, MMA, 8 compute and 4 dQ warps
-    static constexpr int CLC_CONSUMERS = 2 + NCOMPUTE / 32 + NDQ / 32;
-    static constexpr int NTHREADS = NCOMPUTE + NDQ + 64;
+    // arrivals that free a work-item response: producer, 2 MMA issuers, 8 compute
+    // and 4 dQ warps
+    static constexpr int CLC_CONSUMERS = 3 + NCOMPUTE / 32 + NDQ / 32;
+    static constexpr int NTHREADS = NCOMPUTE + NDQ + 96;
     static constexpr int WARP_DQ0 = NCOMPUTE / 32;
-    static constexpr int WARP_TMA = WARP_DQ0 + NDQ / 32, WARP_MMA = WARP_TMA + 1;
+    static constexpr int WARP_TMA = WARP_DQ0 + NDQ / 32, WARP_MMA = WARP_TMA + 1,
+                         WARP_MMB = WARP_MMA + 1;
 };
 
 // Work item k of the list: (head bh, 128-key tile j).  Under the causal mask
@@ -85,7 +93,7 @@ __device__ __forceinline__ void bwd_item(const BwdParams& p, int k, int& bh, int
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(448, 1)
+__global__ void __launch_bounds__(480, 1)
     attn_bwd_main128_kernel(const __grid_constant__ CUtensorMap tmQ,
                             const __grid_constant__ CUtensorMap tmK,
                             const __grid_constant__ CUtensorMap tmV,
@@ -108,24 +116,27 @@ __global__ void __launch_bounds__(448, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(BAR(C::B_KV), 1);
-        mbar_init(BAR(C::B_KVE), 1);
+        mbar_init(BAR(C::B_KVE), 2);  // one commit from each issuer
         mbar_init(BAR(C::B_ACCE), C::NCOMPUTE);
         for (int s = 0; s < C::ST; ++s) {
             mbar_init(BAR(C::B_QF + s), 1);
-            mbar_init(BAR(C::B_QE + s), 1);
+            mbar_init(BAR(C::B_QE + s), 2);  // one commit from each issuer
         }
-        mbar_init(BAR(C::B_SF), 1);
-        mbar_init(BAR(C::B_SF + 1), 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(BAR(C::B_SF + i), 1);
+            mbar_init(BAR(C::B_PTF + i), C::NCOMPUTE);
+            mbar_init(BAR(C::B_DVD + i), 1);
+            mbar_init(BAR(C::B_DR + i), 1);
+        }
         mbar_init(BAR(C::B_DPF), 1);
-        mbar_init(BAR(C::B_PTF), C::NCOMPUTE);
-        mbar_init(BAR(C::B_DVD), 1);
-        mbar_init(BAR(C::B_DVD + 1), 1);
         mbar_init(BAR(C::B_DSF), C::NCOMPUTE);
+        mbar_init(BAR(C::B_DSTE), 1);
+        mbar_init(BAR(C::B_DPE), C::NCOMPUTE);
         mbar_init(BAR(C::B_DQF), 1);
         mbar_init(BAR(C::B_DQE), C::NDQ);
         mbar_init(BAR(C::B_FIN), 1);
-        mbar_init(BAR(C::B_DR), 1);
         mbar_init(BAR(C::B_SRD), C::NCOMPUTE / 2);
+        mbar_init(BAR(C::B_SRD + 1), C::NCOMPUTE / 2);
         mbar_init(BAR(C::B_STGF), C::NDQ);
         mbar_init(BAR(C::B_STGE), 1);
         for (int i = 0; i < 2; ++i) {
@@ -207,15 +218,24 @@ __global__ void __launch_bounds__(448, 1)
                     if (issued[s] > 0) wait_drain(BAR(C::B_QF + s), (issued[s] - 1) & 1);
             }
         }
-    } else if (warp == C::WARP_MMA) {
-        // ------------------------------------------------------- MMA issuer
+    } else if (warp == C::WARP_MMA || warp == C::WARP_MMB) {
+        // ------------------------------------------------------ MMA issuers
+        // Issuer A (warp 13): S^T(g) and dP^T(g).  Issuer B (warp 14): dV(g),
+        // dK(g) and dQ^T(g).  Each waits once per group of MMAs, testing all
+        // the group's barriers at once.  Every wait is for the newest phase its
+        // barrier can have reached before the waiter's own next commit, so no
+        // waiter can fall two phases behind; phase parities run on the tile
+        // count g across work items.  Q_g / dO_g and K / V are released by one
+        // commit from each issuer.
         if (lane == 0) {
             constexpr uint32_t ID_S = idesc_f16(BF16, 128, 64, false, false);   // S^T, dP^T
             constexpr uint32_t ID_KV = idesc_f16(BF16, 128, 128, false, true);  // dV, dK
             constexpr uint32_t ID_DQT = idesc_f16(BF16, 128, 64, true, true);   // dQ^T
             const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sDST = base + C::OFF_DST;
-            // S^T(g) = K Q_g^T into S buffer g & 1 (the caller has waited for Q_g
-            // and for dV(g-2), the last reader of that buffer)
+            const bool is_a = warp == C::WARP_MMA;
+            int g = 0, items = 0, bh = 0, j = 0;
+            bool ok = true;
+            // S^T(g) = K Q_g^T into S buffer g & 1
             auto issue_s = [&](int g) {
                 const uint32_t sQ = base + C::OFF_Q + (g % C::ST) * C::QTILE;
 #pragma unroll
@@ -227,85 +247,94 @@ __global__ void __launch_bounds__(448, 1)
                 }
                 mma_commit(BAR(C::B_SF + (g & 1)));
             };
-            // Issue order per tile g: dP^T(g), dV(g), S^T(g+1), dK(g) + dQ^T(g),
-            // with two waits per tile, each testing all its barriers at once (a
-            // dependent wait stalls the issue of queued MMAs).  dP^T(g) needs no
-            // wait of its own: dO_g landed with Q_g (waited before S^T(g)), and
-            // the compute warps released dP^T(g-1) before the DSF(g-1) wait that
-            // preceded dK(g-1).  Every wait is for the newest phase its barrier
-            // can have reached, so no waiter can fall two phases behind; phase
-            // parities run on the tile count g across work items.
-            int g = 0, items = 0, bh = 0, j = 0;
-            bool ok = true;
             while (ok && cs.cur >= 0) {
                 bwd_item(p, cs.cur, bh, j);
                 const int n_it = n_q64 - (p.causal ? 2 * j : 0);
-                if (!(ok = wait3(BAR(C::B_KV), items & 1, true, BAR(C::B_QF + g % C::ST),
-                                 (g / C::ST) & 1, true, BAR(C::B_DVD + (g & 1)), ((g - 2) >> 1) & 1,
-                                 g >= 2, abort_flag)))
-                    break;
-                tc_fence_after();
-                issue_s(g);
-                // the item's first dV and dK overwrite accumulators that the
-                // previous item's epilogue must have read
-                if (items > 0 && !(ok = wait_bounded(BAR(C::B_ACCE), (items - 1) & 1, abort_flag)))
-                    break;
-                for (int it = 0; ok && it < n_it; ++it, ++g) {
-                    const uint32_t ph = g & 1;
-                    const int s = g % C::ST;
-                    const uint32_t sQ = base + C::OFF_Q + s * C::QTILE;
-                    const uint32_t sDO = base + C::OFF_DO + s * C::QTILE;
+                if (is_a) {
+                    // the item's K, V; Q_g; dV(g-2), the last reader of S buffer g & 1
+                    if (!(ok = wait3(BAR(C::B_KV), items & 1, true, BAR(C::B_QF + g % C::ST),
+                                     (g / C::ST) & 1, true, BAR(C::B_DVD + (g & 1)),
+                                     ((g - 2) >> 1) & 1, g >= 2, abort_flag)))
+                        break;
+                    tc_fence_after();
+                    issue_s(g);
+                    for (int it = 0; ok && it < n_it; ++it, ++g) {
+                        const int s = g % C::ST, g1 = g + 1;
+                        const bool more = it + 1 < n_it;
+                        const uint32_t sDO = base + C::OFF_DO + s * C::QTILE;
+                        // dP^T(g) overwrites dP^T(g-1), which the compute warps have
+                        // loaded (DPE) before they compute dS^T(g-1); S^T(g+1) needs
+                        // Q_{g+1} and dV(g-1) done with S buffer (g+1) & 1
+                        if (!(ok = wait3(BAR(C::B_DPE), (g - 1) & 1, g >= 1,
+                                         BAR(C::B_QF + g1 % C::ST), (g1 / C::ST) & 1, more,
+                                         BAR(C::B_DVD + (g1 & 1)), ((g1 - 2) >> 1) & 1,
+                                         more && g1 >= 2, abort_flag)))
+                            break;
+                        tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t off = (kk >> 2) * 8192u + (kk & 3) * 32u;
-                        const uint32_t offk = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                        mma_ss(tmem + C::COL_DP, sdesc_sw128(sV + offk, 16, 1024),
-                               sdesc_sw128(sDO + off, 16, 1024), ID_S, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint32_t off = (kk >> 2) * 8192u + (kk & 3) * 32u;
+                            const uint32_t offk = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                            mma_ss(tmem + C::COL_DP, sdesc_sw128(sV + offk, 16, 1024),
+                                   sdesc_sw128(sDO + off, 16, 1024), ID_S, kk > 0 ? 1u : 0u);
+                        }
+                        mma_commit(BAR(C::B_DPF));
+                        mma_commit(BAR(C::B_QE + s));  // A's reads of Q_g, dO_g
+                        if (more) issue_s(g1);
                     }
-                    mma_commit(BAR(C::B_DPF));
-                    // dV += P^T dO (P^T from tensor memory); then S^T(g+1), whose
-                    // buffer dV(g-1) read
-                    const bool more = it + 1 < n_it;
-                    const int g1 = g + 1;
-                    if (!(ok = wait3(BAR(C::B_PTF), ph, true, BAR(C::B_QF + g1 % C::ST),
-                                     (g1 / C::ST) & 1, more, BAR(C::B_DVD + (g1 & 1)),
-                                     ((g1 - 2) >> 1) & 1, more && g1 >= 2, abort_flag)))
-                        break;
-                    tc_fence_after();
+                    if (!ok) break;
+                    mma_commit(BAR(C::B_KVE));  // A's reads of K, V
+                } else {
+                    for (int it = 0; ok && it < n_it; ++it, ++g) {
+                        const uint32_t ph = g & 1;
+                        const int s = g % C::ST;
+                        const uint32_t sQ = base + C::OFF_Q + s * C::QTILE;
+                        const uint32_t sDO = base + C::OFF_DO + s * C::QTILE;
+                        // dV += P^T dO: P^T(g) in tensor memory, dO_g landed; the item's
+                        // first dV (then dK) overwrites accumulators that the previous
+                        // item's epilogue must have read
+                        if (!(ok = wait3(BAR(C::B_PTF + (g & 1)), (g >> 1) & 1, true,
+                                         BAR(C::B_QF + s), (g / C::ST) & 1, true, BAR(C::B_ACCE),
+                                         (items - 1) & 1, it == 0 && items > 0, abort_flag)))
+                            break;
+                        tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_ts(tmem + C::COL_DV, tmem + C::COL_S + (g & 1) * 64u + kk * 8u,
-                               sdesc_sw128(sDO + kk * 2048u, 8192, 1024), ID_KV,
-                               (it > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(BAR(C::B_DVD + (g & 1)));
-                    if (more) issue_s(g1);
-                    // dK += dS^T Q ; dQ^T = K^T dS^T (its columns drained for g-1)
-                    if (!(ok = wait3(BAR(C::B_DSF), ph, true, BAR(C::B_DQE), ph ^ 1, g >= 1, 0u, 0u,
-                                     false, abort_flag)))
-                        break;
-                    tc_fence_after();
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_ts(tmem + C::COL_DV, tmem + C::COL_S + (g & 1) * 64u + kk * 8u,
+                                   sdesc_sw128(sDO + kk * 2048u, 8192, 1024), ID_KV,
+                                   (it > 0 || kk > 0) ? 1u : 0u);
+                        mma_commit(BAR(C::B_DVD + (g & 1)));
+                        // dK += dS^T Q ; dQ^T = K^T dS^T: dS^T(g) stored, dQ^T(g-1)
+                        // drained, the item's K landed
+                        if (!(ok = wait3(BAR(C::B_DSF), ph, true, BAR(C::B_DQE), ph ^ 1, g >= 1,
+                                         BAR(C::B_KV), items & 1, it == 0, abort_flag)))
+                            break;
+                        tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_ss(tmem + C::COL_DK, sdesc_sw128(sDST + kk * 32u, 16, 1024),
-                               sdesc_sw128(sQ + kk * 2048u, 8192, 1024), ID_KV,
-                               (it > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_ss(tmem + C::COL_DK, sdesc_sw128(sDST + kk * 32u, 16, 1024),
+                                   sdesc_sw128(sQ + kk * 2048u, 8192, 1024), ID_KV,
+                                   (it > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ss(tmem + C::COL_DQ, sdesc_sw128(sK + kk * 2048u, 16384, 1024),
-                               sdesc_sw128(sDST + kk * 2048u, 8192, 1024), ID_DQT,
-                               kk > 0 ? 1u : 0u);
-                    mma_commit(BAR(C::B_QE + s));  // Q_g, dO_g no longer read
-                    mma_commit(BAR(C::B_DQF));
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_ss(tmem + C::COL_DQ, sdesc_sw128(sK + kk * 2048u, 16384, 1024),
+                                   sdesc_sw128(sDST + kk * 2048u, 8192, 1024), ID_DQT,
+                                   kk > 0 ? 1u : 0u);
+                        mma_commit(BAR(C::B_QE + s));  // B's reads of Q_g, dO_g
+                        mma_commit(BAR(C::B_DQF));
+                        mma_commit(BAR(C::B_DSTE));    // dS^T(g) no longer read
+                    }
+                    if (!ok) break;
+                    mma_commit(BAR(C::B_FIN));  // dK, dV of this item complete
+                    mma_commit(BAR(C::B_KVE));  // B's reads of K
                 }
-                if (!ok) break;
-                mma_commit(BAR(C::B_FIN));  // dK, dV of this item complete
-                mma_commit(BAR(C::B_KVE));  // K, V no longer read
                 ++items;
                 ok = cs.advance(abort_flag, false);
             }
             if (*abort_flag) {  // every issued MMA must finish before TMEM is freed
-                mma_commit(BAR(C::B_DR));
-                wait_drain(BAR(C::B_DR), 0);
+                const uint32_t dr = BAR(C::B_DR + (is_a ? 0 : 1));
+                mma_commit(dr);
+                wait_drain(dr, 0);
             }
         }
         __syncwarp();
@@ -410,9 +439,12 @@ __global__ void __launch_bounds__(448, 1)
                     tmem_ld32(lane_addr + colS + c0, sv);
                     tmem_ld_wait();
                     reg_fence32(sv);
-                    if (half == 0) {  // half 1 writes P^T over columns half 0 reads
+                    // half 1 writes P^T over columns half 0 reads.  One barrier per
+                    // S buffer: half 0 cannot arrive for tile g + 2 before S^T(g+2),
+                    // which waits for dV(g), which waits for half 1's P^T(g).
+                    if (half == 0) {
                         tc_fence_before();
-                        mbar_arrive(BAR(C::B_SRD));
+                        mbar_arrive(BAR(C::B_SRD + (g & 1)));
                     }
 #pragma unroll
                     for (int e4 = 0; e4 < 8; ++e4) {
@@ -434,7 +466,8 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
                     for (int c = 0; c < 16; ++c) pk[c] = pack2<BF16>(pv[2 * c], pv[2 * c + 1]);
                     if (half == 1) {
-                        ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SRD), ph, abort_flag));
+                        ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SRD + (g & 1)),
+                                                                  (g >> 1) & 1, abort_flag));
                         tc_fence_after();
                     }
                     if (ok) {
@@ -444,10 +477,12 @@ __global__ void __launch_bounds__(448, 1)
                 }
                 if (!ok) break;
                 tc_fence_before();
-                mbar_arrive(BAR(C::B_PTF));
+                mbar_arrive(BAR(C::B_PTF + (g & 1)));
 
-                // ---- dS^T = P^T (dP^T - D), half, into shared memory
-                ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_DPF), ph, abort_flag));
+                // ---- dS^T = P^T (dP^T - D), half, into shared memory once dK(g-1)
+                // and dQ^T(g-1) are done reading the previous dS^T
+                ok = __all_sync(0xffffffffu, wait3(BAR(C::B_DPF), ph, true, BAR(C::B_DSTE), ph ^ 1,
+                                                   g >= 1, 0u, 0u, false, abort_flag));
                 if (!ok) break;
                 tc_fence_after();
                 {
@@ -456,6 +491,7 @@ __global__ void __launch_bounds__(448, 1)
                     tmem_ld_wait();
                     reg_fence32(dpv);
                     tc_fence_before();
+                    mbar_arrive(BAR(C::B_DPE));  // dP^T(g) is in registers: dP^T(g+1) may go
                     float dsv[32];
 #pragma unroll
                     for (int e4 = 0; e4 < 8; ++e4) {
