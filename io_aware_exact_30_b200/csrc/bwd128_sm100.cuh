@@ -12,7 +12,7 @@
 //   P^T  = exp2(S^T scale log2e - L2_i)  written back over S^T as half
 //   dP^T = V_j dO_i^T                    tensor memory
 //   dV  += P^T dO_i                      A operand read from tensor memory
-//   dS^T = P^T (dP^T - D_i)              shared memory, half
+//   dS^T = P^T (dP^T - D_i)              shared memory, half, double-buffered
 //   dK  += dS^T Q_i
 //   dQ^T = K_j^T dS^T                    tensor memory, drained by dQ warps
 //                                        into a shared fp32 tile that one bulk
@@ -48,13 +48,14 @@ struct Bwd128Cfg {
     static constexpr uint32_t OFF_V = OFF_K + KTILE;
     static constexpr uint32_t OFF_Q = OFF_V + KTILE;
     static constexpr uint32_t OFF_DO = OFF_Q + ST * QTILE;
-    static constexpr uint32_t OFF_DST = OFF_DO + ST * QTILE;  // 128 keys x 64 queries half
-    static constexpr uint32_t OFF_STG = OFF_DST + 16384u;     // dQ tile, 64 x 128 fp32 rows
+    static constexpr uint32_t DSTILE = 16384u;                // dS^T: 128 keys x 64 queries half
+    static constexpr uint32_t OFF_DST = OFF_DO + ST * QTILE;  // two dS^T buffers
+    static constexpr uint32_t OFF_STG = OFF_DST + 2 * DSTILE; // dQ tile, 64 x 128 fp32 rows
     static constexpr uint32_t OFF_LD = OFF_STG + 32768u;      // ST x (64 L2 + 64 D) fp32
     static constexpr uint32_t OFF_BAR = OFF_LD + ST * 512u;
     static constexpr int B_KV = 0, B_QF = 1, B_QE = B_QF + ST, B_SF = B_QE + ST, B_DPF = B_SF + 2,
                          B_PTF = B_DPF + 1, B_DVD = B_PTF + 2, B_DSF = B_DVD + 2,
-                         B_DSTE = B_DSF + 1, B_DQF = B_DSTE + 1, B_DQE = B_DQF + 1,
+                         B_DSTE = B_DSF + 2, B_DQF = B_DSTE + 2, B_DQE = B_DQF + 1,
                          B_FIN = B_DQE + 1, B_DR = B_FIN + 1, B_KVE = B_DR + 2, B_ACCE = B_KVE + 1,
                          B_SRD = B_ACCE + 1, B_STGF = B_SRD + 2, B_STGE = B_STGF + 1,
                          B_CLCF = B_STGE + 1, B_CLCE = B_CLCF + 2, B_DPE = B_CLCE + 2,
@@ -62,6 +63,7 @@ struct Bwd128Cfg {
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr uint32_t OFF_CLC = (OFF_MISC + 16 + 15) & ~15u;  // 2 x 16-byte responses
     static constexpr uint32_t SMEM_BYTES = OFF_CLC + 32 + 1024;
+    static_assert(SMEM_BYTES <= 232448u, "dynamic shared memory above the sm_100 per-block limit");
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 192, COL_DV = 256, COL_DK = 384;
     static constexpr int NCOMPUTE = 256, NDQ = 128;
@@ -130,7 +132,9 @@ __global__ void __launch_bounds__(480, 1)
         }
         mbar_init(BAR(C::B_DPF), 1);
         mbar_init(BAR(C::B_DSF), C::NCOMPUTE);
+        mbar_init(BAR(C::B_DSF + 1), C::NCOMPUTE);
         mbar_init(BAR(C::B_DSTE), 1);
+        mbar_init(BAR(C::B_DSTE + 1), 1);
         mbar_init(BAR(C::B_DPE), C::NCOMPUTE);
         mbar_init(BAR(C::B_DQF), 1);
         mbar_init(BAR(C::B_DQE), C::NDQ);
@@ -290,6 +294,7 @@ __global__ void __launch_bounds__(480, 1)
                         const int s = g % C::ST;
                         const uint32_t sQ = base + C::OFF_Q + s * C::QTILE;
                         const uint32_t sDO = base + C::OFF_DO + s * C::QTILE;
+                        const uint32_t sDS = sDST + (g & 1) * C::DSTILE;
                         // dV += P^T dO: P^T(g) in tensor memory, dO_g landed; the item's
                         // first dV (then dK) overwrites accumulators that the previous
                         // item's epilogue must have read
@@ -306,23 +311,24 @@ __global__ void __launch_bounds__(480, 1)
                         mma_commit(BAR(C::B_DVD + (g & 1)));
                         // dK += dS^T Q ; dQ^T = K^T dS^T: dS^T(g) stored, dQ^T(g-1)
                         // drained, the item's K landed
-                        if (!(ok = wait3(BAR(C::B_DSF), ph, true, BAR(C::B_DQE), ph ^ 1, g >= 1,
+                        if (!(ok = wait3(BAR(C::B_DSF + (g & 1)), (g >> 1) & 1, true, BAR(C::B_DQE),
+                                         ph ^ 1, g >= 1,
                                          BAR(C::B_KV), items & 1, it == 0, abort_flag)))
                             break;
                         tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            mma_ss(tmem + C::COL_DK, sdesc_sw128(sDST + kk * 32u, 16, 1024),
+                            mma_ss(tmem + C::COL_DK, sdesc_sw128(sDS + kk * 32u, 16, 1024),
                                    sdesc_sw128(sQ + kk * 2048u, 8192, 1024), ID_KV,
                                    (it > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
                             mma_ss(tmem + C::COL_DQ, sdesc_sw128(sK + kk * 2048u, 16384, 1024),
-                                   sdesc_sw128(sDST + kk * 2048u, 8192, 1024), ID_DQT,
+                                   sdesc_sw128(sDS + kk * 2048u, 8192, 1024), ID_DQT,
                                    kk > 0 ? 1u : 0u);
                         mma_commit(BAR(C::B_QE + s));  // B's reads of Q_g, dO_g
                         mma_commit(BAR(C::B_DQF));
-                        mma_commit(BAR(C::B_DSTE));    // dS^T(g) no longer read
+                        mma_commit(BAR(C::B_DSTE + (g & 1)));  // dS^T(g) no longer read
                     }
                     if (!ok) break;
                     mma_commit(BAR(C::B_FIN));  // dK, dV of this item complete
@@ -479,10 +485,11 @@ __global__ void __launch_bounds__(480, 1)
                 tc_fence_before();
                 mbar_arrive(BAR(C::B_PTF + (g & 1)));
 
-                // ---- dS^T = P^T (dP^T - D), half, into shared memory once dK(g-1)
-                // and dQ^T(g-1) are done reading the previous dS^T
-                ok = __all_sync(0xffffffffu, wait3(BAR(C::B_DPF), ph, true, BAR(C::B_DSTE), ph ^ 1,
-                                                   g >= 1, 0u, 0u, false, abort_flag));
+                // ---- dS^T = P^T (dP^T - D), half, into shared-memory buffer g & 1
+                // once dK(g-2) and dQ^T(g-2) are done reading it
+                ok = __all_sync(0xffffffffu,
+                                wait3(BAR(C::B_DPF), ph, true, BAR(C::B_DSTE + (g & 1)),
+                                      ((g - 2) >> 1) & 1, g >= 2, 0u, 0u, false, abort_flag));
                 if (!ok) break;
                 tc_fence_after();
                 {
@@ -504,14 +511,16 @@ __global__ void __launch_bounds__(480, 1)
                     }
 #pragma unroll
                     for (int c = 0; c < 4; ++c)  // 16-byte chunks 4 half + c of the 128-byte key row
-                        st_shared_v4(sDST + sw128_off(r, half * 4 + c),
+                        st_shared_v4(sDST + (g & 1) * C::DSTILE + sw128_off(r, half * 4 + c),
                                      pack2<BF16>(dsv[8 * c + 0], dsv[8 * c + 1]),
                                      pack2<BF16>(dsv[8 * c + 2], dsv[8 * c + 3]),
                                      pack2<BF16>(dsv[8 * c + 4], dsv[8 * c + 5]),
                                      pack2<BF16>(dsv[8 * c + 6], dsv[8 * c + 7]));
                 }
                 fence_proxy_async_smem();
-                mbar_arrive(BAR(C::B_DSF));
+                // one barrier per dS^T buffer: the arrival for tile g + 2 needs
+                // dK(g) and dQ^T(g), which issuer B starts only after seeing tile g's
+                mbar_arrive(BAR(C::B_DSF + (g & 1)));
             }
             if (ok) ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_FIN), items & 1, abort_flag));
             if (!ok) break;
