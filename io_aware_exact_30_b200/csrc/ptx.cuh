@@ -330,22 +330,6 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// 2^x on the FMA pipe: x = j + f with j = round(x), f in [-1/2, 1/2]
-// (Cody-Waite style reduction); 2^f by a degree-3 polynomial with p(0) = 1
-// whose coefficients minimise the maximum relative error (about 1.0e-4) on
-// [-1/2, 1/2]; 2^j added to the exponent field.  x is clamped at -127, which
-// yields exactly 0, so x = -inf gives 0 as ex2 does.  The coefficients and the
-// error bound come from exp2_fit.py beside this file.
-__device__ __forceinline__ float exp2_poly(float x) {
-    x = fmaxf(x, -127.f);
-    const float t = x + 12582912.f;  // 1.5 * 2^23: the low mantissa bits of t hold round(x)
-    const float f = x - (t - 12582912.f);
-    float p = fmaf(0.0550089068710804f, f, 0.2422109991312027f);
-    p = fmaf(p, f, 0.693282961845398f);
-    p = fmaf(p, f, 1.f);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 // ---- packed fp32 pairs (sm_100 f32x2 arithmetic): two lanes per instruction
 __device__ __forceinline__ uint64_t f2(float lo, float hi) {
     uint64_t r;
@@ -377,26 +361,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
 }
-// exp2_poly on a pair: the same reduction and polynomial, with the
-// floating-point steps done two lanes per instruction.
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
-    float2 v = unf2(x);
-    v.x = fmaxf(v.x, -127.f);
-    v.y = fmaxf(v.y, -127.f);
-    const uint64_t xc = f2(v.x, v.y);
-    const uint64_t magic = f2(12582912.f, 12582912.f);
-    const uint64_t t = add2(xc, magic);
-    const uint64_t r = add2(t, f2(-12582912.f, -12582912.f));
-    const uint64_t f = fma2(r, f2(-1.f, -1.f), xc);
-    uint64_t p = fma2(f2(0.0550089068710804f, 0.0550089068710804f), f,
-                      f2(0.2422109991312027f, 0.2422109991312027f));
-    p = fma2(p, f, f2(0.693282961845398f, 0.693282961845398f));
-    p = fma2(p, f, f2(1.f, 1.f));
-    const float2 pv = unf2(p), tv = unf2(t);
-    return f2(__int_as_float(__float_as_int(pv.x) + (__float_as_int(tv.x) << 23)),
-              __int_as_float(__float_as_int(pv.y) + (__float_as_int(tv.y) << 23)));
-}
-
 template <bool BF16>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     if constexpr (BF16) {
