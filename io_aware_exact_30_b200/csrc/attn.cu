@@ -280,16 +280,18 @@ int bwd_main_dispatch(const void* q, const void* k, const void* v, const void* d
                   : attn::bwd_main_launch<64, false>(mq, mk, mv, mdo, dq, dk, dv, workspace, B, H,
                                                      N, c, scale, st);
     // d = 128: 64-query inner tiles
-    CUtensorMap mq64, mdo64;
-    if (!make_map(&mq64, q, dtype, BH, N, d, 64) || !make_map(&mdo64, dout, dtype, BH, N, d, 64))
+    // (dK and dV leave through TMA stores)
+    CUtensorMap mq64, mdo64, mdk, mdv;
+    if (!make_map(&mq64, q, dtype, BH, N, d, 64) || !make_map(&mdo64, dout, dtype, BH, N, d, 64) ||
+        !make_map(&mdk, dk, dtype, BH, N, d) || !make_map(&mdv, dv, dtype, BH, N, d))
         return ATTN_ERR_LAUNCH;
     int dev = 0;
     cudaGetDevice(&dev);
     const int sms = g_sm_count[dev];
-    return bf ? attn::bwd_main128_launch<true>(mq64, mk, mv, mdo64, dq, dk, dv, workspace, B, H, N,
-                                               c, scale, sms, st)
-              : attn::bwd_main128_launch<false>(mq64, mk, mv, mdo64, dq, dk, dv, workspace, B, H,
-                                                N, c, scale, sms, st);
+    return bf ? attn::bwd_main128_launch<true>(mq64, mk, mv, mdo64, mdk, mdv, dq, dk, dv,
+                                               workspace, B, H, N, c, scale, sms, st)
+              : attn::bwd_main128_launch<false>(mq64, mk, mv, mdo64, mdk, mdv, dq, dk, dv,
+                                                workspace, B, H, N, c, scale, sms, st);
 }
 }  // namespace
 

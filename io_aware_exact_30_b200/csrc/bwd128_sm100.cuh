@@ -59,7 +59,8 @@ struct Bwd128Cfg {
                          B_FIN = B_DQE + 1, B_DR = B_FIN + 1, B_KVE = B_DR + 2, B_ACCE = B_KVE + 1,
                          B_SRD = B_ACCE + 1, B_STGF = B_SRD + 2, B_STGE = B_STGF + 1,
                          B_CLCF = B_STGE + 1, B_CLCE = B_CLCF + 2, B_DPE = B_CLCE + 2,
-                         NBAR = B_DPE + 1;
+                         B_EPS = B_DPE + 1, B_EPF = B_EPS + 1, B_DQD = B_EPF + 1,
+                         NBAR = B_DQD + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr uint32_t OFF_CLC = (OFF_MISC + 16 + 15) & ~15u;  // 2 x 16-byte responses
     static constexpr uint32_t SMEM_BYTES = OFF_CLC + 32 + 1024;
@@ -99,7 +100,9 @@ __global__ void __launch_bounds__(480, 1)
     attn_bwd_main128_kernel(const __grid_constant__ CUtensorMap tmQ,
                             const __grid_constant__ CUtensorMap tmK,
                             const __grid_constant__ CUtensorMap tmV,
-                            const __grid_constant__ CUtensorMap tmDO, const BwdParams p) {
+                            const __grid_constant__ CUtensorMap tmDO,
+                            const __grid_constant__ CUtensorMap tmDK,
+                            const __grid_constant__ CUtensorMap tmDV, const BwdParams p) {
     using C = Bwd128Cfg;
     constexpr int D = C::D;
     extern __shared__ uint8_t smem_raw[];
@@ -136,6 +139,9 @@ __global__ void __launch_bounds__(480, 1)
         mbar_init(BAR(C::B_DSTE), 1);
         mbar_init(BAR(C::B_DSTE + 1), 1);
         mbar_init(BAR(C::B_DPE), C::NCOMPUTE);
+        mbar_init(BAR(C::B_EPS), C::NCOMPUTE);
+        mbar_init(BAR(C::B_EPF), 1);
+        mbar_init(BAR(C::B_DQD), 1);
         mbar_init(BAR(C::B_DQF), 1);
         mbar_init(BAR(C::B_DQE), C::NDQ);
         mbar_init(BAR(C::B_FIN), 1);
@@ -212,8 +218,19 @@ __global__ void __launch_bounds__(480, 1)
                 }
                 ++items;
                 for (int it = pre; ok && it < n_it; ++it) ok = load_tile(i_begin + it);
-                // once an item's loads are issued, ask for the next item
+                // once an item's loads are issued, ask for the next item, and start
+                // its K and V on their way into L2 (they are loaded into shared
+                // memory only when this item's MMAs release K and V)
                 if (ok) ok = cs.request(abort_flag) && cs.advance(abort_flag, false);
+                if (ok && cs.cur >= 0) {
+                    int nbh, nj;
+                    bwd_item(p, cs.cur, nbh, nj);
+#pragma unroll
+                    for (int kb = 0; kb < 2; ++kb) {
+                        tma_prefetch_l2_3d(&tmK, kb * 64, nj * 128, nbh);
+                        tma_prefetch_l2_3d(&tmV, kb * 64, nj * 128, nbh);
+                    }
+                }
             }
             if (*abort_flag) {  // let every copy in flight land before the CTA exits
                 cs.drain();
@@ -397,6 +414,7 @@ __global__ void __launch_bounds__(480, 1)
                         bulk_commit();
                         bulk_wait_read_all();
                         mbar_arrive(BAR(C::B_STGE));
+                        if (it + 1 == n_it) mbar_arrive(BAR(C::B_DQD));  // item's staging done
                     }
                 }
                 dq_ok = __all_sync(0xffffffffu, dq_ok);
@@ -421,7 +439,6 @@ __global__ void __launch_bounds__(480, 1)
             const int n_it = n_q64 - i_begin;
             const int key = j * 128 + r;
             const bool key_valid = key < p.N;
-            const size_t head_row0 = static_cast<size_t>(bh) * p.N;
             for (int it = 0; it < n_it; ++it, ++g) {
                 const int q0 = (i_begin + it) * 64;
                 const uint32_t ph = g & 1;
@@ -524,40 +541,70 @@ __global__ void __launch_bounds__(480, 1)
             }
             if (ok) ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_FIN), items & 1, abort_flag));
             if (!ok) break;
-            // dK_j, dV_j rows: lane r holds key row j*128 + r; this half, 64 features
+            // dK_j, dV_j: lane r holds key row j*128 + r, this half's 64 features.
+            // TMEM -> registers (rounded), then tensor memory is released.  The rows
+            // go through 128-byte-swizzled shared boxes, dK into the two dS^T
+            // buffers (all MMAs are done with them) and dV into the dQ staging tile
+            // once its last reduction has read it, and leave by TMA tensor stores,
+            // which skip rows at or past N.
             tc_fence_after();
-            const size_t rowoff = (head_row0 + key) * (D * 2) + half * D;
+            uint32_t hk[32], hv[32];
 #pragma unroll
-            for (int which = 0; which < 2; ++which) {
-                uint8_t* out = static_cast<uint8_t*>(which ? p.dv : p.dk) + rowoff;
-                const uint32_t colA = (which ? C::COL_DV : C::COL_DK) + half * 64u;
-                const float mul = which ? 1.f : p.scale;
+            for (int c = 0; c < 2; ++c) {
+                uint32_t v[32];
+                tmem_ld32(lane_addr + C::COL_DK + half * 64u + c * 32u, v);
+                tmem_ld_wait();
+                reg_fence32(v);
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t v[32];
-                    tmem_ld32(lane_addr + colA + c * 32u, v);
-                    tmem_ld_wait();
-                    reg_fence32(v);
-                    uint32_t h[16];
+                for (int e = 0; e < 16; ++e)
+                    hk[16 * c + e] = pack2<BF16>(__uint_as_float(v[2 * e]) * p.scale,
+                                                 __uint_as_float(v[2 * e + 1]) * p.scale);
+                tmem_ld32(lane_addr + C::COL_DV + half * 64u + c * 32u, v);
+                tmem_ld_wait();
+                reg_fence32(v);
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        h[e] = pack2<BF16>(__uint_as_float(v[2 * e]) * mul,
-                                           __uint_as_float(v[2 * e + 1]) * mul);
-                    if (key_valid) {
-                        uint4* d4 = reinterpret_cast<uint4*>(out + c * 64);
-                        d4[0] = make_uint4(h[0], h[1], h[2], h[3]);
-                        d4[1] = make_uint4(h[4], h[5], h[6], h[7]);
-                        d4[2] = make_uint4(h[8], h[9], h[10], h[11]);
-                        d4[3] = make_uint4(h[12], h[13], h[14], h[15]);
-                    }
-                }
+                for (int e = 0; e < 16; ++e)
+                    hv[16 * c + e] =
+                        pack2<BF16>(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
             }
             // dK and dV have been read: the next item may overwrite them
             tc_fence_before();
             mbar_arrive(BAR(C::B_ACCE));
+            // The item's last dQ reduction has read the staging tile.  (A parity
+            // wait is only valid for a phase whose predecessor has completed; the
+            // dQ warps may be two tiles behind here, so the per-tile barrier
+            // cannot be used and the per-item one, waited in order, is.)
+            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_DQD), items & 1, abort_flag));
+            if (!ok) break;
+            {
+                const uint32_t boxk = base + C::OFF_DST + half * C::DSTILE;
+                const uint32_t boxv = base + C::OFF_STG + half * 16384u;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    st_shared_v4(boxk + sw128_off(r, c), hk[4 * c], hk[4 * c + 1], hk[4 * c + 2],
+                                 hk[4 * c + 3]);
+                    st_shared_v4(boxv + sw128_off(r, c), hv[4 * c], hv[4 * c + 1], hv[4 * c + 2],
+                                 hv[4 * c + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(BAR(C::B_EPS));
+            if (threadIdx.x == 0 && wait_bounded(BAR(C::B_EPS), items & 1, abort_flag)) {
+#pragma unroll
+                for (int kb = 0; kb < 2; ++kb) {
+                    tma_store_3d(&tmDK, base + C::OFF_DST + kb * C::DSTILE, kb * 64, j * 128, bh);
+                    tma_store_3d(&tmDV, base + C::OFF_STG + kb * 16384u, kb * 64, j * 128, bh);
+                }
+                bulk_commit();
+                bulk_wait_read_all();  // the shared boxes may be reused
+                mbar_arrive(BAR(C::B_EPF));
+            }
+            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_EPF), items & 1, abort_flag));
+            if (!ok) break;
             ++items;
             ok = cs.advance(abort_flag, true);
         }
+        if (threadIdx.x == 0) bulk_wait_all();  // every dK/dV store complete before the CTA exits
     }
 #undef BAR
     tc_fence_before();
@@ -589,14 +636,15 @@ inline bool bwd128_set_attributes() {
                                 Bwd128Cfg::SMEM_BYTES) == cudaSuccess;
 }
 
-// mq, mdo must be tensor maps with 64-row boxes; mk, mv with 128-row boxes.
+// mq, mdo must be tensor maps with 64-row boxes; mk, mv, mdk, mdv with 128-row boxes.
 // Launches the persistent main kernel, then the dQ conversion.  Causal: one CTA
 // per work item, running CTAs take pending CTAs' items; otherwise one CTA per
 // multiprocessor.
 template <bool BF16>
 int bwd_main128_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                       const CUtensorMap& mdo, void* dq, void* dk, void* dv, void* ws, int B,
-                       int H, int N, int causal, float scale, int sm_count, cudaStream_t st) {
+                       const CUtensorMap& mdo, const CUtensorMap& mdk, const CUtensorMap& mdv,
+                       void* dq, void* dk, void* dv, void* ws, int B, int H, int N, int causal,
+                       float scale, int sm_count, cudaStream_t st) {
     BwdParams p;
     uint8_t* w = static_cast<uint8_t*>(ws);
     p.l2pad = reinterpret_cast<const float*>(w);
@@ -624,7 +672,7 @@ int bwd_main128_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     if (items >= (1LL << 31)) return -2;
     const int nblocks = static_cast<int>(causal || items < sm_count ? items : sm_count);
     attn_bwd_main128_kernel<BF16><<<static_cast<unsigned>(nblocks), Bwd128Cfg::NTHREADS,
-                                    Bwd128Cfg::SMEM_BYTES, st>>>(mq, mk, mv, mdo, p);
+                                    Bwd128Cfg::SMEM_BYTES, st>>>(mq, mk, mv, mdo, mdk, mdv, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
         bwd_record_error(e);
