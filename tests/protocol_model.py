@@ -1,0 +1,367 @@
+"""A model of the mbarrier protocol of the d = 128 backward main kernel
+(io_aware_exact_30_b200/csrc/bwd128_sm100.cuh), for checking it on the CPU
+under many random schedules.  Test infrastructure only.
+
+Each role of the kernel is a generator that yields the same sequence of
+barrier operations, with the same barriers, arrival counts and phase indices,
+as the kernel's code; asynchronous work (TMA loads, MMAs and their commits,
+the bulk stores) is queued and completed at random later points, MMAs in issue
+order per issuing thread.  Buffers carry a version tag: every read states the
+version it must see, every write sets one.
+
+Groups of threads that run the same code are modelled by a few agents each
+(two per column half of the compute warps, two dQ warps), so the barriers'
+arrival counts are the number of modelled agents, not of threads.
+
+The checker reports:
+  * a barrier test for phase k while the barrier is not in phase k or k + 1
+    (the parity test would return a wrong answer: ahead, it succeeds on phase
+    k - 2; two behind, it waits for a phase that needs the waiter itself),
+  * an arrival that does not land in the phase it is meant for,
+  * a read that sees another version than the one it needs,
+  * a schedule in which nothing can move before every role has finished.
+
+`Variant` switches reproduce protocol mistakes that were made while building
+the kernel, so the tests can show that the checker catches each of them.
+"""
+
+import random
+from dataclasses import dataclass, field
+
+
+class ProtocolError(AssertionError):
+    pass
+
+
+@dataclass
+class Variant:
+    single_srd: bool = False      # one barrier (not one per S buffer) for the shared S^T read
+    single_dsf: bool = False      # one barrier (not one per dS^T buffer) for dS^T ready
+    epilogue_tile_wait: bool = False  # epilogue waits the per-tile staging barrier, not DQD
+    no_dpe: bool = False          # dP^T(g) waits for dS^T(g-1) instead of the dP^T release
+
+
+class Barrier:
+    def __init__(self, name, count):
+        self.name, self.count, self.pending, self.completed = name, count, 0, 0
+
+    def arrive(self, use):
+        if self.completed != use:
+            raise ProtocolError(f"{self.name}: arrival for phase {use} while in phase "
+                                f"{self.completed}")
+        self.pending += 1
+        if self.pending == self.count:
+            self.pending = 0
+            self.completed += 1
+
+    def test(self, k):
+        """The hardware's parity test for phase k, checked against its meaning."""
+        if self.completed not in (k, k + 1):
+            raise ProtocolError(f"{self.name}: test for phase {k} while in phase "
+                                f"{self.completed}")
+        return self.completed == k + 1
+
+
+@dataclass
+class World:
+    bars: dict = field(default_factory=dict)
+    buf: dict = field(default_factory=dict)
+
+    def bar(self, name, count=1):
+        if name not in self.bars:
+            self.bars[name] = Barrier(name, count)
+        return self.bars[name]
+
+    def read(self, key, want):
+        have = self.buf.get(key)
+        if have != want:
+            raise ProtocolError(f"read of {key}: wants {want}, holds {have}")
+
+    def write(self, key, value):
+        self.buf[key] = value
+
+
+ST = 3          # Q / dO / statistics stages
+NCOMP = 4       # compute agents: (half, quarter) for half in 0,1 and quarter in 0,1
+NDQ = 2         # dQ agents; agent 0 holds the reduction issuer
+
+
+# ---------------------------------------------------------------------------
+# Roles.  Operations yielded:
+#   ("wait", [(bar, k), ...])          all tests must pass (tested together)
+#   ("arrive", bar, use)
+#   ("async", queue, fn)               fn() runs when the queue delivers it
+# Reads and writes between two yields happen when the role moves on from the
+# first of them.  `plan` lists the number of 64-query tiles of each work item
+# of one CTA, in the order the CTA takes them.
+# ---------------------------------------------------------------------------
+
+def producer(plan, v):
+    g = 0
+    for item, n_it in enumerate(plan):
+        def load_tile(g):
+            s, n = g % ST, g // ST
+            yield ("wait", [(f"QE{s}", n - 1)])
+
+            def land(g=g, s=s, n=n):
+                W.write(("Q", s), g)
+                W.write(("DO", s), g)
+                W.write(("LD", s), g)
+                W.bar(f"QF{s}").arrive(n)
+            yield ("async", "tma", land)
+        pre = min(ST, n_it)
+        for _ in range(pre):
+            yield from load_tile(g)
+            g += 1
+        if item > 0:
+            yield ("wait", [("KVE", item - 1)])
+
+        def land_kv(item=item):
+            W.write("K", item)
+            W.write("V", item)
+            W.bar("KV").arrive(item)
+        yield ("async", "tma", land_kv)
+        for _ in range(pre, n_it):
+            yield from load_tile(g)
+            g += 1
+
+
+def issuer_a(plan, v):
+    g = 0
+    for item, n_it in enumerate(plan):
+        waits = [("KV", item), (f"QF{g % ST}", g // ST)]
+        if g >= 2:
+            waits.append((f"DVD{g & 1}", (g - 2) >> 1))
+        yield ("wait", waits)
+        yield from mma_s(g, item)
+        for it in range(n_it):
+            s, g1, more = g % ST, g + 1, it + 1 < n_it
+            waits = []
+            if g >= 1:
+                waits.append(("DSF0" if v.single_dsf else f"DSF{(g - 1) & 1}",
+                              (g - 1) if v.single_dsf else (g - 1) >> 1) if v.no_dpe
+                             else ("DPE", g - 1))
+            if more:
+                waits.append((f"QF{g1 % ST}", g1 // ST))
+                if g1 >= 2:
+                    waits.append((f"DVD{g1 & 1}", (g1 - 2) >> 1))
+            yield ("wait", waits)
+
+            def dp(g=g, s=s, item=item):
+                W.read("V", item)
+                W.read(("DO", s), g)
+                W.write("DP", g)
+            yield ("async", "A", dp)
+            yield ("async", "A", lambda g=g: W.bar("DPF").arrive(g))
+            yield ("async", "A", lambda s=s, g=g: W.bar(f"QE{s}", 2).arrive(g // ST))
+            if more:
+                yield from mma_s(g1, item)
+            g += 1
+        yield ("async", "A", lambda item=item: W.bar("KVE", 2).arrive(item))
+
+
+def mma_s(g, item):
+    s = g % ST
+
+    def run(g=g, s=s, item=item):
+        W.read("K", item)
+        W.read(("Q", s), g)
+        for q in range(2):
+            for r in ("R0", "R1", "R2"):
+                W.write(("S", g & 1, q, r), ("S", g))
+    yield ("async", "A", run)
+    yield ("async", "A", lambda g=g: W.bar(f"SF{g & 1}").arrive(g >> 1))
+
+
+def issuer_b(plan, v):
+    g = 0
+    for item, n_it in enumerate(plan):
+        for it in range(n_it):
+            s = g % ST
+            waits = [(f"PTF{g & 1}", g >> 1), (f"QF{s}", g // ST)]
+            if it == 0 and item > 0:
+                waits.append(("ACCE", item - 1))
+            yield ("wait", waits)
+
+            def dv(g=g, s=s, item=item, it=it):
+                for q in range(2):
+                    W.read(("S", g & 1, q, "R0"), ("P", g))
+                    W.read(("S", g & 1, q, "R1"), ("P", g))
+                W.read(("DO", s), g)
+                W.write("DVACC", (item, it + 1))
+            yield ("async", "B", dv)
+            yield ("async", "B", lambda g=g: W.bar(f"DVD{g & 1}").arrive(g >> 1))
+            dsf = ("DSF0", g) if v.single_dsf else (f"DSF{g & 1}", g >> 1)
+            waits = [dsf]
+            if g >= 1:
+                waits.append(("DQE", g - 1))
+            if it == 0:
+                waits.append(("KV", item))
+            yield ("wait", waits)
+
+            def dkdq(g=g, s=s, item=item, it=it):
+                b = g & 1
+                for h in range(2):
+                    W.read(("DS", b, h), g)
+                W.read(("Q", s), g)
+                W.read("K", item)
+                W.write("DKACC", (item, it + 1))
+                W.write("DQ", g)
+            yield ("async", "B", dkdq)
+            yield ("async", "B", lambda s=s, g=g: W.bar(f"QE{s}", 2).arrive(g // ST))
+            yield ("async", "B", lambda g=g: W.bar("DQF").arrive(g))
+            yield ("async", "B", lambda g=g: W.bar(f"DSTE{g & 1}").arrive(g >> 1))
+            g += 1
+        yield ("async", "B", lambda item=item: W.bar("FIN").arrive(item))
+        yield ("async", "B", lambda item=item: W.bar("KVE", 2).arrive(item))
+
+
+def compute(agent, plan, v):
+    half, q = agent // 2, agent % 2
+    g = 0
+    for item, n_it in enumerate(plan):
+        for it in range(n_it):
+            s, b = g % ST, g & 1
+            yield ("wait", [(f"QF{s}", g // ST)])
+            yield ("wait", [(f"SF{b}", g >> 1)])
+            W.read(("LD", s), g)
+            srd = ("SRD0", g) if v.single_srd else (f"SRD{b}", g >> 1)
+            if half == 0:
+                W.read(("S", b, q, "R0"), ("S", g))
+                W.read(("S", b, q, "R1"), ("S", g))
+                yield ("arrive", srd[0], srd[1])
+                W.write(("S", b, q, "R0"), ("P", g))
+            else:
+                W.read(("S", b, q, "R2"), ("S", g))
+                yield ("wait", [srd])
+                W.write(("S", b, q, "R1"), ("P", g))
+            yield ("arrive", f"PTF{b}", g >> 1)
+            waits = [("DPF", g)]
+            if g >= 2:
+                waits.append((f"DSTE{b}", (g - 2) >> 1))
+            yield ("wait", waits)
+            W.read("DP", g)
+            W.read(("LD", s), g)
+            if not v.no_dpe:
+                yield ("arrive", "DPE", g)
+            W.write(("DS", b, half), g)
+            dsf = ("DSF0", g) if v.single_dsf else (f"DSF{b}", g >> 1)
+            yield ("arrive", dsf[0], dsf[1])
+            g += 1
+        # epilogue
+        yield ("wait", [("FIN", item)])
+        W.read("DVACC", (item, n_it))
+        W.read("DKACC", (item, n_it))
+        yield ("arrive", "ACCE", item)
+        if v.epilogue_tile_wait:
+            yield ("wait", [("STGE", g - 1)])
+        else:
+            yield ("wait", [("DQD", item)])
+        # half h stages its 64 columns: dV into the staging tile's h-th 16 KB,
+        # dK into dS^T buffer h (both column halves of the tile loop's layout)
+        W.write(("STG", half), ("dV", item))
+        W.write(("DS", half, 0), ("dK", item))
+        W.write(("DS", half, 1), ("dK", item))
+        yield ("arrive", "EPS", item)
+        if agent == 0:
+            yield ("wait", [("EPS", item)])
+
+            def store(item=item):
+                for h in range(2):
+                    W.read(("STG", h), ("dV", item))
+                    W.read(("DS", h, 0), ("dK", item))
+                    W.read(("DS", h, 1), ("dK", item))
+                W.bar("EPF").arrive(item)
+            yield ("async", "store", store)
+        yield ("wait", [("EPF", item)])
+
+
+def dq_role(agent, plan, v):
+    g = 0
+    for item, n_it in enumerate(plan):
+        for it in range(n_it):
+            yield ("wait", [("DQF", g)])
+            W.read("DQ", g)
+            yield ("arrive", "DQE", g)
+            if g >= 1:
+                yield ("wait", [("STGE", g - 1)])
+            # each dQ warp writes its feature columns in both 16 KB halves
+            for h in range(2):
+                W.write(("STG", h), ("dQ", g))
+            yield ("arrive", "STGF", g)
+            if agent == 0:
+                yield ("wait", [("STGF", g)])
+                for h in range(2):
+                    W.read(("STG", h), ("dQ", g))
+                yield ("arrive", "STGE", g)
+                if it + 1 == n_it:
+                    yield ("arrive", "DQD", item)
+            g += 1
+
+
+W = None  # the world of the schedule being run (the roles read it as a global)
+
+
+def run_schedule(plan, seed, variant=None, max_steps=200000):
+    """Runs one random schedule of one CTA working through `plan`; raises
+    ProtocolError on a violation or a deadlock."""
+    global W
+    v = variant or Variant()
+    W = World()
+    counts = {"KVE": 2, "ACCE": NCOMP, "PTF0": NCOMP, "PTF1": NCOMP, "DSF0": NCOMP,
+              "DSF1": NCOMP, "DPE": NCOMP, "SRD0": NCOMP // 2, "SRD1": NCOMP // 2,
+              "EPS": NCOMP, "DQE": NDQ, "STGF": NDQ}
+    for s in range(ST):
+        counts[f"QE{s}"] = 2
+    if v.single_dsf:
+        counts["DSF0"] = NCOMP
+    for name, c in counts.items():
+        W.bar(name, c)
+    rng = random.Random(seed)
+    roles = {"prod": producer(plan, v), "A": issuer_a(plan, v), "B": issuer_b(plan, v)}
+    for a in range(NCOMP):
+        roles[f"comp{a}"] = compute(a, plan, v)
+    for a in range(NDQ):
+        roles[f"dq{a}"] = dq_role(a, plan, v)
+    nxt = {name: None for name in roles}       # pending operation of each role
+    queues = {"tma": [], "A": [], "B": [], "store": []}
+    done = set()
+
+    def advance(name):
+        try:
+            nxt[name] = next(roles[name])
+        except StopIteration:
+            nxt[name] = None
+            done.add(name)
+
+    for name in roles:
+        advance(name)
+    for _ in range(max_steps):
+        if len(done) == len(roles) and not any(queues.values()):
+            return
+        choices = []
+        for name, op in nxt.items():
+            if op is None:
+                continue
+            if op[0] == "wait":
+                # the kernel tests all barriers of a group; each test is checked
+                if all(W.bar(b).test(k) for b, k in op[1]):
+                    choices.append(("role", name))
+            else:
+                choices.append(("role", name))
+        for qn, q in queues.items():
+            if q:
+                choices.append(("queue", qn))
+        if not choices:
+            raise ProtocolError(f"deadlock: pending {[(n, o[0], o[1] if o[0] == 'wait' else '') for n, o in nxt.items() if o]}")
+        kind, name = rng.choice(choices)
+        if kind == "queue":
+            queues[name].pop(0)()
+            continue
+        op = nxt[name]
+        if op[0] == "arrive":
+            W.bar(op[1]).arrive(op[2])
+        elif op[0] == "async":
+            queues[op[1]].append(op[2])
+        advance(name)
+    raise ProtocolError("schedule did not finish")
