@@ -112,11 +112,14 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
  * multiple of 128 rows), and clears the fp32 dQ accumulator and the per-head
  * completion counters.
  *
- * attn_bwd_main: for every 128-key tile, recomputes S and P per 128-query tile
- * from q, k and the statistics attn_bwd_prep staged (never storing P), forms
- * dV, dK in tensor memory and adds the dQ contributions into the workspace
- * accumulator; the last tile of each head to finish converts that head's dQ
- * into dq.  Requires the workspace as attn_bwd_prep left it.
+ * attn_bwd_main: for every 128-key tile, recomputes S and P per query tile
+ * (128 rows for d = 64, 64 rows for d = 128) from q, k and the statistics
+ * attn_bwd_prep staged (never storing P), forms dV, dK in tensor memory and
+ * adds the dQ contributions into the workspace accumulator.  dq is the
+ * accumulator rounded to the dtype: for d = 64 the last key tile of each head
+ * to finish converts that head, found through the completion counters; for
+ * d = 128 a second kernel, launched by the same call on the same stream,
+ * converts all of it.  Requires the workspace as attn_bwd_prep left it.
  */
 int attn_bwd_prep(const void* o, const void* dout, const float* lse, void* workspace, int B,
                   int H, int N, int d, attn_dtype_t dtype, void* stream);
