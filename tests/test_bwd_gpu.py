@@ -90,3 +90,34 @@ def test_bwd_workspace_contents_do_not_matter():
     torch.cuda.synchronize()
     ref = oracle.bwd(*f64, True, default_scale(d))
     check_grads([t.double().cpu().numpy() for t in (dq, dk, dv)], ref, "garbage workspace")
+
+
+# Shapes whose work items outnumber the multiprocessors (several items per
+# persistent CTA, taken dynamically under the causal mask and in static snake
+# order without it), with ragged key and query tails, and one with long items.
+MANY_ITEMS = [
+    (2, 40, 1000, 128, True),
+    (3, 20, 777, 128, False),
+    (1, 2, 5000, 128, True),
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,causal", MANY_ITEMS)
+def test_fwd_bwd_many_items_per_cta(B, H, N, d, causal):
+    arrs, f64 = inputs(B, H, N, d, seed=2, with_dout=True)
+    scale = default_scale(d)
+    q, k, v, do = (to_device(a, "bf16") for a in arrs)
+    o, lse = attn.forward(q, k, v, causal, scale)
+    dq, dk, dv = attn.backward(q, k, v, o, lse, do, causal, scale)
+    torch.cuda.synchronize()
+    assert attn.attn_last_device_status() == 0
+    got = [t.double().cpu().numpy() for t in (o, lse, dq, dk, dv)]
+    for bh in (0, B * H - 1):
+        b, h = divmod(bh, H)
+        sel = [x[b:b + 1, h:h + 1] for x in f64]
+        o_ref, lse_ref = oracle.fwd(*sel[:3], causal, scale)
+        o_err = float(np.abs(got[0][b:b + 1, h:h + 1] - o_ref).max())
+        l_err = float(np.abs(got[1][b:b + 1, h:h + 1] - lse_ref).max())
+        assert o_err <= 1e-2 and l_err <= 1e-3, (bh, o_err, l_err)
+        ref = oracle.bwd(*sel, causal, scale)
+        check_grads([x[b:b + 1, h:h + 1] for x in got[2:]], ref, f"{(B, H, N, d, causal)} head {bh}")
