@@ -1,0 +1,219 @@
+"""A model of the mbarrier protocol of the forward kernel
+(io_aware_exact_30_b200/csrc/fwd_sm100.cuh), checked on the CPU under random
+schedules with the same rules as protocol_model.py (the d = 128 backward).
+Test infrastructure only.
+
+Roles: the TMA producer, the single MMA issuer (order per key tile j:
+O_0 += P_0 V_j, S_0(j+1), O_1 += P_1 V_j, S_1(j+1)) and, per query tile, the
+softmax warps, modelled as two agents each.  Whether a softmax step moves the
+kept max (and rescales O, which needs the previous P V complete) depends on
+the data in the kernel; the model decides it at random.
+
+A work item is given by (nkv_0, nkv_1), the key-tile steps of its two query
+tiles: equal without the mask; under the causal mask tile 1 has one more, and
+the last pair of an odd tile count has nkv_1 = 0.
+"""
+
+import random
+
+from protocol_model import Barrier, ProtocolError, World
+
+ST = 2      # K/V stages (d = 128)
+NSM = 2     # softmax agents per query tile
+
+
+class Variant:
+    def __init__(self, ke_before_pv=False, epilogue_no_od_wait=False):
+        # release the K/V stage before the tile-1 P V of the step is issued
+        self.ke_before_pv = ke_before_pv
+        # the epilogue reads O without waiting for the last P V
+        self.epilogue_no_od_wait = epilogue_no_od_wait
+
+
+W = None
+
+
+def producer(plan, v):
+    kv = 0
+    for item, (n0, n1) in enumerate(plan):
+        nkv = max(n0, n1)
+        if item > 0:
+            yield ("wait", [("QE", item - 1)])
+
+        def land_q(item=item):
+            W.write("Q", item)
+            W.bar("Q").arrive(item)
+        yield ("async", "tma", land_q)
+        for j in range(nkv):
+            kvj = kv + j
+            s, n = kvj % ST, kvj // ST
+            yield ("wait", [(f"KE{s}", n - 1)])
+
+            def land_k(kvj=kvj, s=s, n=n):
+                W.write(("K", s), kvj)
+                W.bar(f"KF{s}").arrive(n)
+
+            def land_v(kvj=kvj, s=s, n=n):
+                W.write(("V", s), kvj)
+                W.bar(f"VF{s}").arrive(n)
+            yield ("async", "tma", land_k)
+            yield ("async", "tma", land_v)
+        kv += nkv
+
+
+def issuer(plan, v):
+    kv = 0
+    n_pv, n_s, n_done = [0, 0], [0, 0], [0, 0]
+
+    def issue_s(t, kvi, item):
+        s = kvi % ST
+
+        def run(t=t, kvi=kvi, s=s, item=item):
+            W.read("Q", item)
+            W.read(("K", s), kvi)
+            for a in range(NSM):
+                W.write(("S", t, a), ("S", kvi))
+        yield ("async", "mma", run)
+        k = n_s[t]
+        n_s[t] += 1
+        yield ("async", "mma", lambda t=t, k=k: W.bar(f"SF{t}").arrive(k))
+
+    for item, (n0, n1) in enumerate(plan):
+        nkv_t = (n0, n1)
+        nkv = max(n0, n1)
+        waits = [("Q", item), (f"KF{kv % ST}", kv // ST)]
+        if n0 > 0 and n_pv[0] > 0:
+            waits.append(("OD0", n_pv[0] - 1))
+        yield ("wait", waits)
+        if n1 > 0 and n_pv[1] > 0:
+            yield ("wait", [("OD1", n_pv[1] - 1)])
+        for t in range(2):
+            if nkv_t[t] > 0:
+                yield from issue_s(t, kv, item)
+        for j in range(nkv):
+            kvj = kv + j
+            s, n = kvj % ST, kvj // ST
+            k1 = kvj + 1
+            k_next = False
+            for t in range(2):
+                act = j < nkv_t[t]
+                waits = []
+                if t == 0:
+                    waits.append((f"VF{s}", n))
+                if act:
+                    waits.append((f"PF{t}", n_pv[t]))
+                    if j == 0 and n_done[t] > 0:
+                        waits.append((f"OE{t}", n_done[t] - 1))
+                if waits:
+                    yield ("wait", waits)
+                if t == 1 and v.ke_before_pv:
+                    yield ("async", "mma", lambda s=s, n=n: W.bar(f"KE{s}").arrive(n))
+                if not act:
+                    continue
+
+                def pv(t=t, kvj=kvj, s=s, item=item, j=j):
+                    for a in range(NSM):
+                        W.read(("S", t, a), ("P", kvj))
+                    W.read(("V", s), kvj)
+                    W.write(("O", t), (item, j + 1))
+                yield ("async", "mma", pv)
+                k = n_pv[t]
+                n_pv[t] += 1
+                yield ("async", "mma", lambda t=t, k=k: W.bar(f"OD{t}").arrive(k))
+                if j + 1 < nkv_t[t]:
+                    waits = [(f"OD{t}", n_pv[t] - 1)]
+                    if not k_next:
+                        waits.append((f"KF{k1 % ST}", k1 // ST))
+                    yield ("wait", waits)
+                    k_next = True
+                    yield from issue_s(t, k1, item)
+            if not v.ke_before_pv:
+                yield ("async", "mma", lambda s=s, n=n: W.bar(f"KE{s}").arrive(n))
+        yield ("async", "mma", lambda item=item: W.bar("QE").arrive(item))
+        kv += nkv
+        for t in range(2):
+            if nkv_t[t] > 0:
+                n_done[t] += 1
+
+
+def softmax(t, agent, plan, v, rng):
+    kv = 0
+    n_s = 0
+    done = 0
+    for item, nk in enumerate(plan):
+        my = nk[t]
+        nkv = max(nk)
+        if my == 0:
+            kv += nkv
+            continue
+        for j in range(my):
+            yield ("wait", [(f"SF{t}", n_s)])
+            n_s += 1
+            W.read(("S", t, agent), ("S", kv + j))
+            if j > 0 and rng.random() < 0.3:
+                # the kept max moves: O is rescaled, which needs P V(j-1)
+                yield ("wait", [(f"OD{t}", n_s - 2)])
+                W.read(("O", t), (item, j))
+            W.write(("S", t, agent), ("P", kv + j))
+            yield ("arrive", f"PF{t}", n_s - 1)
+        if not v.epilogue_no_od_wait:
+            yield ("wait", [(f"OD{t}", n_s - 1)])
+        W.read(("O", t), (item, my))
+        yield ("arrive", f"OE{t}", done)
+        done += 1
+        kv += nkv
+
+
+def run_schedule(plan, seed, variant=None, max_steps=200000):
+    global W
+    v = variant or Variant()
+    W = World()
+    for t in range(2):
+        W.bar(f"PF{t}", NSM)
+        W.bar(f"OE{t}", NSM)
+    rng = random.Random(seed)
+    roles = {"prod": producer(plan, v), "mma": issuer(plan, v)}
+    for t in range(2):
+        for a in range(NSM):
+            roles[f"sm{t}{a}"] = softmax(t, a, plan, v, random.Random(seed * 7 + 2 * t + a))
+    nxt = {n: None for n in roles}
+    queues = {"tma": [], "mma": []}
+    done = set()
+
+    def advance(name):
+        try:
+            nxt[name] = next(roles[name])
+        except StopIteration:
+            nxt[name] = None
+            done.add(name)
+
+    for name in roles:
+        advance(name)
+    for _ in range(max_steps):
+        if len(done) == len(roles) and not any(queues.values()):
+            return
+        choices = []
+        for name, op in nxt.items():
+            if op is None:
+                continue
+            if op[0] == "wait":
+                if all(W.bar(b).test(k) for b, k in op[1]):
+                    choices.append(("role", name))
+            else:
+                choices.append(("role", name))
+        for qn, q in queues.items():
+            if q:
+                choices.append(("queue", qn))
+        if not choices:
+            raise ProtocolError("deadlock: " + str([(n, o) for n, o in nxt.items() if o]))
+        kind, name = rng.choice(choices)
+        if kind == "queue":
+            queues[name].pop(0)()
+            continue
+        op = nxt[name]
+        if op[0] == "arrive":
+            W.bar(op[1]).arrive(op[2])
+        elif op[0] == "async":
+            queues[op[1]].append(op[2])
+        advance(name)
+    raise ProtocolError("schedule did not finish")

@@ -1,0 +1,32 @@
+"""The forward kernel's mbarrier protocol, checked on the CPU under random
+schedules (tests/protocol_model_fwd.py mirrors the kernel's roles): barrier
+tests in the phase they are for or the next, arrivals in their phase, reads of
+the versions they need, no deadlock; and protocol mistakes are rejected."""
+
+import pytest
+
+import protocol_model_fwd as pf
+
+PLANS = {
+    "noncausal": [(3, 3), (3, 3), (1, 1)],
+    "causal": [(1, 2), (3, 4), (5, 0)],
+    "causal-repeat": [(2, 3), (2, 3), (2, 3), (4, 5)],
+    "single-step": [(1, 0), (1, 2), (1, 1)],
+}
+
+
+@pytest.mark.parametrize("name", sorted(PLANS))
+def test_forward_protocol_holds_under_random_schedules(name):
+    for seed in range(150):
+        pf.run_schedule(PLANS[name], seed)
+
+
+@pytest.mark.parametrize("mistake", ["ke_before_pv", "epilogue_no_od_wait"])
+def test_checker_rejects_forward_mistakes(mistake):
+    caught = 0
+    for seed in range(300):
+        try:
+            pf.run_schedule([(1, 2), (3, 4), (5, 0), (2, 2)], seed, pf.Variant(**{mistake: True}))
+        except pf.ProtocolError:
+            caught += 1
+    assert caught > 0, f"{mistake} was never caught"
