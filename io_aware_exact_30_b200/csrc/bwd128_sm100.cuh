@@ -17,8 +17,10 @@
 //   dQ^T = K_j^T dS^T                    tensor memory, drained by dQ warps
 //                                        into a shared fp32 tile that one bulk
 //                                        reduction adds into the accumulator
-// A separate small kernel converts the fp32 dQ accumulator to the output type
-// after the main kernel.
+// At the end of an item dK and dV leave tensor memory through 128-byte-swizzled
+// shared boxes (the two dS^T buffers and the dQ staging tile) and TMA tensor
+// stores.  A separate small kernel converts the fp32 dQ accumulator to the
+// output type after the main kernel.
 // Tensor memory (512 columns): S^T buffers at 0 and 64, dP^T at 128, dQ^T at
 // 192, dV at 256, dK at 384.
 //
@@ -51,6 +53,7 @@ struct Bwd128Cfg {
     static constexpr uint32_t DSTILE = 16384u;                // dS^T: 128 keys x 64 queries half
     static constexpr uint32_t OFF_DST = OFF_DO + ST * QTILE;  // two dS^T buffers
     static constexpr uint32_t OFF_STG = OFF_DST + 2 * DSTILE; // dQ tile, 64 x 128 fp32 rows
+                                                              // (also the dV boxes at item end)
     static constexpr uint32_t OFF_LD = OFF_STG + 32768u;      // ST x (64 L2 + 64 D) fp32
     static constexpr uint32_t OFF_BAR = OFF_LD + ST * 512u;
     static constexpr int B_KV = 0, B_QF = 1, B_QE = B_QF + ST, B_SF = B_QE + ST, B_DPF = B_SF + 2,
