@@ -39,6 +39,7 @@ class Variant:
     single_dsf: bool = False      # one barrier (not one per dS^T buffer) for dS^T ready
     epilogue_tile_wait: bool = False  # epilogue waits the per-tile staging barrier, not DQD
     no_dpe: bool = False          # dP^T(g) waits for dS^T(g-1) instead of the dP^T release
+    own_region_p: bool = False    # each half writes P^T over its own S^T columns, no SRD
 
 
 class Barrier:
@@ -167,7 +168,7 @@ def mma_s(g, item):
         W.read("K", item)
         W.read(("Q", s), g)
         for q in range(2):
-            for r in ("R0", "R1", "R2"):
+            for r in ("R0", "R1", "R2", "R3"):   # S^T columns 0-15, 16-31, 32-47, 48-63
                 W.write(("S", g & 1, q, r), ("S", g))
     yield ("async", "A", run)
     yield ("async", "A", lambda g=g: W.bar(f"SF{g & 1}").arrive(g >> 1))
@@ -186,7 +187,7 @@ def issuer_b(plan, v):
             def dv(g=g, s=s, item=item, it=it):
                 for q in range(2):
                     W.read(("S", g & 1, q, "R0"), ("P", g))
-                    W.read(("S", g & 1, q, "R1"), ("P", g))
+                    W.read(("S", g & 1, q, "R2" if v.own_region_p else "R1"), ("P", g))
                 W.read(("DO", s), g)
                 W.write("DVACC", (item, it + 1))
             yield ("async", "B", dv)
@@ -229,12 +230,17 @@ def compute(agent, plan, v):
             if half == 0:
                 W.read(("S", b, q, "R0"), ("S", g))
                 W.read(("S", b, q, "R1"), ("S", g))
-                yield ("arrive", srd[0], srd[1])
+                if not v.own_region_p:
+                    yield ("arrive", srd[0], srd[1])
                 W.write(("S", b, q, "R0"), ("P", g))
             else:
                 W.read(("S", b, q, "R2"), ("S", g))
-                yield ("wait", [srd])
-                W.write(("S", b, q, "R1"), ("P", g))
+                W.read(("S", b, q, "R3"), ("S", g))
+                if v.own_region_p:
+                    W.write(("S", b, q, "R2"), ("P", g))
+                else:
+                    yield ("wait", [srd])
+                    W.write(("S", b, q, "R1"), ("P", g))
             yield ("arrive", f"PTF{b}", g >> 1)
             waits = [("DPF", g)]
             if g >= 2:

@@ -26,6 +26,12 @@ def test_earlier_correct_design_also_holds():
         pm.run_schedule([3, 2, 4, 1], seed, pm.Variant(no_dpe=True))
 
 
+def test_own_region_p_layout_needs_no_shared_read_barrier():
+    # each half writing P^T over its own S^T columns (dV reading them there)
+    for seed in range(120):
+        pm.run_schedule([3, 2, 4, 1], seed, pm.Variant(own_region_p=True))
+
+
 @pytest.mark.parametrize("mistake", ["single_srd", "single_dsf", "epilogue_tile_wait"])
 def test_checker_rejects_known_mistakes(mistake):
     caught = 0
