@@ -23,11 +23,20 @@ NSM = 2     # softmax agents per query tile
 
 
 class Variant:
-    def __init__(self, ke_before_pv=False, epilogue_no_od_wait=False):
+    def __init__(self, ke_before_pv=False, epilogue_no_od_wait=False, split=False,
+                 split_no_exchange_wait=False):
         # release the K/V stage before the tile-1 P V of the step is issued
         self.ke_before_pv = ke_before_pv
         # the epilogue reads O without waiting for the last P V
         self.epilogue_no_od_wait = epilogue_no_od_wait
+        # design variant: each tile's softmax split over two column halves (each
+        # writing P over its own S columns), the row max exchanged through
+        # shared memory per key tile (one barrier and one slot per step parity)
+        # and the row sum per item
+        self.split = split
+        # mistake for the split design: read the other half's max without
+        # waiting for the exchange barrier
+        self.split_no_exchange_wait = split_no_exchange_wait
 
 
 W = None
@@ -71,7 +80,7 @@ def issuer(plan, v):
         def run(t=t, kvi=kvi, s=s, item=item):
             W.read("Q", item)
             W.read(("K", s), kvi)
-            for a in range(NSM):
+            for a in range(nagents(v)):
                 W.write(("S", t, a), ("S", kvi))
         yield ("async", "mma", run)
         k = n_s[t]
@@ -112,10 +121,11 @@ def issuer(plan, v):
                     continue
 
                 def pv(t=t, kvj=kvj, s=s, item=item, j=j):
-                    for a in range(NSM):
+                    for a in range(nagents(v)):
                         W.read(("S", t, a), ("P", kvj))
                     W.read(("V", s), kvj)
-                    W.write(("O", t), (item, j + 1))
+                    for hh in range(2 if v.split else 1):
+                        W.write(("O", t, hh), (item, j + 1))
                 yield ("async", "mma", pv)
                 k = n_pv[t]
                 n_pv[t] += 1
@@ -153,12 +163,53 @@ def softmax(t, agent, plan, v, rng):
             if j > 0 and rng.random() < 0.3:
                 # the kept max moves: O is rescaled, which needs P V(j-1)
                 yield ("wait", [(f"OD{t}", n_s - 2)])
-                W.read(("O", t), (item, j))
+                W.read(("O", t, 0), (item, j))
             W.write(("S", t, agent), ("P", kv + j))
             yield ("arrive", f"PF{t}", n_s - 1)
         if not v.epilogue_no_od_wait:
             yield ("wait", [(f"OD{t}", n_s - 1)])
-        W.read(("O", t), (item, my))
+        W.read(("O", t, 0), (item, my))
+        yield ("arrive", f"OE{t}", done)
+        done += 1
+        kv += nkv
+
+
+def nagents(v):
+    return 2 * NSM if v.split else NSM
+
+
+def softmax_split(t, h, qq, plan, v, seed):
+    """Half h (key columns 64 h ..) of row quarter qq of tile t."""
+    agent = h * NSM + qq
+    kv = n_s = done = 0
+    for item, nk in enumerate(plan):
+        my, nkv = nk[t], max(nk)
+        if my == 0:
+            kv += nkv
+            continue
+        for j in range(my):
+            yield ("wait", [(f"SF{t}", n_s)])
+            slot = n_s & 1
+            n_s += 1
+            W.read(("S", t, agent), ("S", kv + j))
+            W.write(("PMAX", t, slot, h, qq), kv + j)
+            mx = f"MX{t}{qq}{n_s - 1 & 1}"
+            yield ("arrive", mx, (n_s - 1) >> 1)
+            if not v.split_no_exchange_wait:
+                yield ("wait", [(mx, (n_s - 1) >> 1)])
+            W.read(("PMAX", t, slot, 1 - h, qq), kv + j)
+            # both halves see the same row max, so they take the same decision
+            if j > 0 and random.Random(seed * 1009 + t * 97 + qq * 13 + n_s).random() < 0.3:
+                yield ("wait", [(f"OD{t}", n_s - 2)])
+                W.read(("O", t, h), (item, j))
+            W.write(("S", t, agent), ("P", kv + j))
+            yield ("arrive", f"PF{t}", n_s - 1)
+        yield ("wait", [(f"OD{t}", n_s - 1)])
+        W.write(("PSUM", t, h, qq), item)
+        yield ("arrive", f"LX{t}{qq}", done)
+        yield ("wait", [(f"LX{t}{qq}", done)])
+        W.read(("PSUM", t, 1 - h, qq), item)
+        W.read(("O", t, h), (item, my))
         yield ("arrive", f"OE{t}", done)
         done += 1
         kv += nkv
@@ -169,13 +220,22 @@ def run_schedule(plan, seed, variant=None, max_steps=200000):
     v = variant or Variant()
     W = World()
     for t in range(2):
-        W.bar(f"PF{t}", NSM)
-        W.bar(f"OE{t}", NSM)
+        W.bar(f"PF{t}", nagents(v))
+        W.bar(f"OE{t}", nagents(v))
+        for qq in range(NSM):
+            W.bar(f"LX{t}{qq}", 2)
+            for sl in range(2):
+                W.bar(f"MX{t}{qq}{sl}", 2)
     rng = random.Random(seed)
     roles = {"prod": producer(plan, v), "mma": issuer(plan, v)}
     for t in range(2):
-        for a in range(NSM):
-            roles[f"sm{t}{a}"] = softmax(t, a, plan, v, random.Random(seed * 7 + 2 * t + a))
+        if v.split:
+            for h in range(2):
+                for qq in range(NSM):
+                    roles[f"sm{t}{h}{qq}"] = softmax_split(t, h, qq, plan, v, seed)
+        else:
+            for a in range(NSM):
+                roles[f"sm{t}{a}"] = softmax(t, a, plan, v, random.Random(seed * 7 + 2 * t + a))
     nxt = {n: None for n in roles}
     queues = {"tma": [], "mma": []}
     done = set()

@@ -21,12 +21,22 @@ def test_forward_protocol_holds_under_random_schedules(name):
         pf.run_schedule(PLANS[name], seed)
 
 
-@pytest.mark.parametrize("mistake", ["ke_before_pv", "epilogue_no_od_wait"])
+@pytest.mark.parametrize("name", sorted(PLANS))
+def test_split_softmax_design_holds(name):
+    # next-step design: each tile's softmax over two column halves, exchanging
+    # the row max per key tile and the row sum per item
+    for seed in range(100):
+        pf.run_schedule(PLANS[name], seed, pf.Variant(split=True))
+
+
+@pytest.mark.parametrize("mistake", ["ke_before_pv", "epilogue_no_od_wait",
+                                     "split_no_exchange_wait"])
 def test_checker_rejects_forward_mistakes(mistake):
     caught = 0
     for seed in range(300):
         try:
-            pf.run_schedule([(1, 2), (3, 4), (5, 0), (2, 2)], seed, pf.Variant(**{mistake: True}))
+            kw = {mistake: True, "split": mistake.startswith("split")}
+            pf.run_schedule([(1, 2), (3, 4), (5, 0), (2, 2)], seed, pf.Variant(**kw))
         except pf.ProtocolError:
             caught += 1
     assert caught > 0, f"{mistake} was never caught"
