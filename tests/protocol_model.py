@@ -40,6 +40,13 @@ class Variant:
     epilogue_tile_wait: bool = False  # epilogue waits the per-tile staging barrier, not DQD
     no_dpe: bool = False          # dP^T(g) waits for dS^T(g-1) instead of the dP^T release
     own_region_p: bool = False    # each half writes P^T over its own S^T columns, no SRD
+    # design variant: P^T and dS^T computed by two warp groups in a pipeline (the
+    # P group writes P^T of tile g+1 while the dS group forms dS^T of tile g,
+    # reading P^T back from tensor memory).  No new barrier: the dS group
+    # releases dP^T (DPE) only after it has read P^T too, and S^T(g+2) is issued
+    # after issuer A's wait for DPE(g).
+    pd_split: bool = False
+    pd_split_early_dpe: bool = False  # mistake: DPE before the dS group reads P^T
 
 
 class Barrier:
@@ -92,8 +99,10 @@ NDQ = 2         # dQ agents; agent 0 holds the reduction issuer
 #   ("wait", [(bar, k), ...])          all tests must pass (tested together)
 #   ("arrive", bar, use)
 #   ("async", queue, fn)               fn() runs when the queue delivers it
-# Reads and writes between two yields happen when the role moves on from the
-# first of them.  `plan` lists the number of 64-query tiles of each work item
+#   ("read", key, version) / ("write", key, version)   a role's own access
+# Every operation of a role is a step of its own, so any other step can fall
+# between two of them; the effects of an MMA or a copy happen at once when it
+# completes.  `plan` lists the number of 64-query tiles of each work item
 # of one CTA, in the order the CTA takes them.
 # ---------------------------------------------------------------------------
 
@@ -225,39 +234,39 @@ def compute(agent, plan, v):
             s, b = g % ST, g & 1
             yield ("wait", [(f"QF{s}", g // ST)])
             yield ("wait", [(f"SF{b}", g >> 1)])
-            W.read(("LD", s), g)
+            yield ("read", ("LD", s), g)
             srd = ("SRD0", g) if v.single_srd else (f"SRD{b}", g >> 1)
             if half == 0:
-                W.read(("S", b, q, "R0"), ("S", g))
-                W.read(("S", b, q, "R1"), ("S", g))
+                yield ("read", ("S", b, q, "R0"), ("S", g))
+                yield ("read", ("S", b, q, "R1"), ("S", g))
                 if not v.own_region_p:
                     yield ("arrive", srd[0], srd[1])
-                W.write(("S", b, q, "R0"), ("P", g))
+                yield ("write", ("S", b, q, "R0"), ("P", g))
             else:
-                W.read(("S", b, q, "R2"), ("S", g))
-                W.read(("S", b, q, "R3"), ("S", g))
+                yield ("read", ("S", b, q, "R2"), ("S", g))
+                yield ("read", ("S", b, q, "R3"), ("S", g))
                 if v.own_region_p:
-                    W.write(("S", b, q, "R2"), ("P", g))
+                    yield ("write", ("S", b, q, "R2"), ("P", g))
                 else:
                     yield ("wait", [srd])
-                    W.write(("S", b, q, "R1"), ("P", g))
+                    yield ("write", ("S", b, q, "R1"), ("P", g))
             yield ("arrive", f"PTF{b}", g >> 1)
             waits = [("DPF", g)]
             if g >= 2:
                 waits.append((f"DSTE{b}", (g - 2) >> 1))
             yield ("wait", waits)
-            W.read("DP", g)
-            W.read(("LD", s), g)
+            yield ("read", "DP", g)
+            yield ("read", ("LD", s), g)
             if not v.no_dpe:
                 yield ("arrive", "DPE", g)
-            W.write(("DS", b, half), g)
+            yield ("write", ("DS", b, half), g)
             dsf = ("DSF0", g) if v.single_dsf else (f"DSF{b}", g >> 1)
             yield ("arrive", dsf[0], dsf[1])
             g += 1
         # epilogue
         yield ("wait", [("FIN", item)])
-        W.read("DVACC", (item, n_it))
-        W.read("DKACC", (item, n_it))
+        yield ("read", "DVACC", (item, n_it))
+        yield ("read", "DKACC", (item, n_it))
         yield ("arrive", "ACCE", item)
         if v.epilogue_tile_wait:
             yield ("wait", [("STGE", g - 1)])
@@ -265,9 +274,9 @@ def compute(agent, plan, v):
             yield ("wait", [("DQD", item)])
         # half h stages its 64 columns: dV into the staging tile's h-th 16 KB,
         # dK into dS^T buffer h (both column halves of the tile loop's layout)
-        W.write(("STG", half), ("dV", item))
-        W.write(("DS", half, 0), ("dK", item))
-        W.write(("DS", half, 1), ("dK", item))
+        yield ("write", ("STG", half), ("dV", item))
+        yield ("write", ("DS", half, 0), ("dK", item))
+        yield ("write", ("DS", half, 1), ("dK", item))
         yield ("arrive", "EPS", item)
         if agent == 0:
             yield ("wait", [("EPS", item)])
@@ -282,23 +291,93 @@ def compute(agent, plan, v):
         yield ("wait", [("EPF", item)])
 
 
+def compute_p(q, plan, v):
+    """pd_split: P^T of every tile for the key rows of quarter q, and the dV
+    part of the epilogue."""
+    g = 0
+    for item, n_it in enumerate(plan):
+        for it in range(n_it):
+            s, b = g % ST, g & 1
+            yield ("wait", [(f"QF{s}", g // ST)])
+            yield ("wait", [(f"SF{b}", g >> 1)])
+            yield ("read", ("LD", s), g)
+            for r in ("R0", "R1", "R2", "R3"):
+                yield ("read", ("S", b, q, r), ("S", g))
+            yield ("write", ("S", b, q, "R0"), ("P", g))
+            yield ("write", ("S", b, q, "R1"), ("P", g))
+            yield ("arrive", f"PTF{b}", g >> 1)
+            g += 1
+        yield ("wait", [("FIN", item)])
+        yield ("read", "DVACC", (item, n_it))
+        yield ("arrive", "ACCE", item)
+        yield ("wait", [("DQD", item)])
+        yield ("write", ("STG", 0), ("dV", item))
+        yield ("write", ("STG", 1), ("dV", item))
+        yield ("arrive", "EPS", item)
+        if q == 0:
+            yield ("wait", [("EPS", item)])
+
+            def store(item=item):
+                for h in range(2):
+                    W.read(("STG", h), ("dV", item))
+                    W.read(("DS", h, 0), ("dK", item))
+                    W.read(("DS", h, 1), ("dK", item))
+                W.bar("EPF").arrive(item)
+            yield ("async", "store", store)
+        yield ("wait", [("EPF", item)])
+
+
+def compute_ds(q, plan, v):
+    """pd_split: dS^T of every tile for the key rows of quarter q (P^T read back
+    from tensor memory), and the dK part of the epilogue."""
+    g = 0
+    for item, n_it in enumerate(plan):
+        for it in range(n_it):
+            s, b = g % ST, g & 1
+            waits = [(f"QF{s}", g // ST), (f"PTF{b}", g >> 1), ("DPF", g)]
+            if g >= 2:
+                waits.append((f"DSTE{b}", (g - 2) >> 1))
+            yield ("wait", waits)
+            yield ("read", ("LD", s), g)
+            yield ("read", "DP", g)
+            if v.pd_split_early_dpe:
+                yield ("arrive", "DPE", g)
+            yield ("read", ("S", b, q, "R0"), ("P", g))
+            yield ("read", ("S", b, q, "R1"), ("P", g))
+            if not v.pd_split_early_dpe:
+                yield ("arrive", "DPE", g)
+            yield ("write", ("DS", b, 0), g)
+            yield ("write", ("DS", b, 1), g)
+            yield ("arrive", f"DSF{b}", g >> 1)
+            g += 1
+        yield ("wait", [("FIN", item)])
+        yield ("read", "DKACC", (item, n_it))
+        yield ("arrive", "ACCE", item)
+        yield ("write", ("DS", 0, 0), ("dK", item))
+        yield ("write", ("DS", 0, 1), ("dK", item))
+        yield ("write", ("DS", 1, 0), ("dK", item))
+        yield ("write", ("DS", 1, 1), ("dK", item))
+        yield ("arrive", "EPS", item)
+        yield ("wait", [("EPF", item)])
+
+
 def dq_role(agent, plan, v):
     g = 0
     for item, n_it in enumerate(plan):
         for it in range(n_it):
             yield ("wait", [("DQF", g)])
-            W.read("DQ", g)
+            yield ("read", "DQ", g)
             yield ("arrive", "DQE", g)
             if g >= 1:
                 yield ("wait", [("STGE", g - 1)])
             # each dQ warp writes its feature columns in both 16 KB halves
             for h in range(2):
-                W.write(("STG", h), ("dQ", g))
+                yield ("write", ("STG", h), ("dQ", g))
             yield ("arrive", "STGF", g)
             if agent == 0:
                 yield ("wait", [("STGF", g)])
                 for h in range(2):
-                    W.read(("STG", h), ("dQ", g))
+                    yield ("read", ("STG", h), ("dQ", g))
                 yield ("arrive", "STGE", g)
                 if it + 1 == n_it:
                     yield ("arrive", "DQD", item)
@@ -321,12 +400,21 @@ def run_schedule(plan, seed, variant=None, max_steps=200000):
         counts[f"QE{s}"] = 2
     if v.single_dsf:
         counts["DSF0"] = NCOMP
+    if v.pd_split:
+        half = NCOMP // 2      # 2 P agents, 2 dS agents
+        counts.update({"PTF0": half, "PTF1": half, "DPE": half,
+                       "DSF0": half, "DSF1": half, "ACCE": NCOMP, "EPS": NCOMP})
     for name, c in counts.items():
         W.bar(name, c)
     rng = random.Random(seed)
     roles = {"prod": producer(plan, v), "A": issuer_a(plan, v), "B": issuer_b(plan, v)}
-    for a in range(NCOMP):
-        roles[f"comp{a}"] = compute(a, plan, v)
+    if v.pd_split:
+        for q in range(NCOMP // 2):
+            roles[f"p{q}"] = compute_p(q, plan, v)
+            roles[f"d{q}"] = compute_ds(q, plan, v)
+    else:
+        for a in range(NCOMP):
+            roles[f"comp{a}"] = compute(a, plan, v)
     for a in range(NDQ):
         roles[f"dq{a}"] = dq_role(a, plan, v)
     nxt = {name: None for name in roles}       # pending operation of each role
@@ -369,5 +457,9 @@ def run_schedule(plan, seed, variant=None, max_steps=200000):
             W.bar(op[1]).arrive(op[2])
         elif op[0] == "async":
             queues[op[1]].append(op[2])
+        elif op[0] == "read":
+            W.read(op[1], op[2])
+        elif op[0] == "write":
+            W.write(op[1], op[2])
         advance(name)
     raise ProtocolError("schedule did not finish")

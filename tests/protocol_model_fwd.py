@@ -9,6 +9,10 @@ softmax warps, modelled as two agents each.  Whether a softmax step moves the
 kept max (and rescales O, which needs the previous P V complete) depends on
 the data in the kernel; the model decides it at random.
 
+Every operation of a role (barrier tests and arrivals, its own reads and
+writes) is a step of its own; the effects of an MMA or a copy happen at once
+when it completes.
+
 A work item is given by (nkv_0, nkv_1), the key-tile steps of its two query
 tiles: equal without the mask; under the causal mask tile 1 has one more, and
 the last pair of an odd tile count has nkv_1 = 0.
@@ -159,16 +163,16 @@ def softmax(t, agent, plan, v, rng):
         for j in range(my):
             yield ("wait", [(f"SF{t}", n_s)])
             n_s += 1
-            W.read(("S", t, agent), ("S", kv + j))
+            yield ("read", ("S", t, agent), ("S", kv + j))
             if j > 0 and rng.random() < 0.3:
                 # the kept max moves: O is rescaled, which needs P V(j-1)
                 yield ("wait", [(f"OD{t}", n_s - 2)])
-                W.read(("O", t, 0), (item, j))
-            W.write(("S", t, agent), ("P", kv + j))
+                yield ("read", ("O", t, 0), (item, j))
+            yield ("write", ("S", t, agent), ("P", kv + j))
             yield ("arrive", f"PF{t}", n_s - 1)
         if not v.epilogue_no_od_wait:
             yield ("wait", [(f"OD{t}", n_s - 1)])
-        W.read(("O", t, 0), (item, my))
+        yield ("read", ("O", t, 0), (item, my))
         yield ("arrive", f"OE{t}", done)
         done += 1
         kv += nkv
@@ -191,25 +195,25 @@ def softmax_split(t, h, qq, plan, v, seed):
             yield ("wait", [(f"SF{t}", n_s)])
             slot = n_s & 1
             n_s += 1
-            W.read(("S", t, agent), ("S", kv + j))
-            W.write(("PMAX", t, slot, h, qq), kv + j)
+            yield ("read", ("S", t, agent), ("S", kv + j))
+            yield ("write", ("PMAX", t, slot, h, qq), kv + j)
             mx = f"MX{t}{qq}{n_s - 1 & 1}"
             yield ("arrive", mx, (n_s - 1) >> 1)
             if not v.split_no_exchange_wait:
                 yield ("wait", [(mx, (n_s - 1) >> 1)])
-            W.read(("PMAX", t, slot, 1 - h, qq), kv + j)
+            yield ("read", ("PMAX", t, slot, 1 - h, qq), kv + j)
             # both halves see the same row max, so they take the same decision
             if j > 0 and random.Random(seed * 1009 + t * 97 + qq * 13 + n_s).random() < 0.3:
                 yield ("wait", [(f"OD{t}", n_s - 2)])
-                W.read(("O", t, h), (item, j))
-            W.write(("S", t, agent), ("P", kv + j))
+                yield ("read", ("O", t, h), (item, j))
+            yield ("write", ("S", t, agent), ("P", kv + j))
             yield ("arrive", f"PF{t}", n_s - 1)
         yield ("wait", [(f"OD{t}", n_s - 1)])
-        W.write(("PSUM", t, h, qq), item)
+        yield ("write", ("PSUM", t, h, qq), item)
         yield ("arrive", f"LX{t}{qq}", done)
         yield ("wait", [(f"LX{t}{qq}", done)])
-        W.read(("PSUM", t, 1 - h, qq), item)
-        W.read(("O", t, h), (item, my))
+        yield ("read", ("PSUM", t, 1 - h, qq), item)
+        yield ("read", ("O", t, h), (item, my))
         yield ("arrive", f"OE{t}", done)
         done += 1
         kv += nkv
@@ -275,5 +279,9 @@ def run_schedule(plan, seed, variant=None, max_steps=200000):
             W.bar(op[1]).arrive(op[2])
         elif op[0] == "async":
             queues[op[1]].append(op[2])
+        elif op[0] == "read":
+            W.read(op[1], op[2])
+        elif op[0] == "write":
+            W.write(op[1], op[2])
         advance(name)
     raise ProtocolError("schedule did not finish")

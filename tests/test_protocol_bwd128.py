@@ -32,12 +32,21 @@ def test_own_region_p_layout_needs_no_shared_read_barrier():
         pm.run_schedule([3, 2, 4, 1], seed, pm.Variant(own_region_p=True))
 
 
-@pytest.mark.parametrize("mistake", ["single_srd", "single_dsf", "epilogue_tile_wait"])
+@pytest.mark.parametrize("plan", PLANS, ids=lambda p: "-".join(map(str, p)))
+def test_pipelined_p_ds_groups_design_holds(plan):
+    # next-step design: P^T and dS^T in two warp groups working on consecutive tiles
+    for seed in range(80):
+        pm.run_schedule(plan, seed, pm.Variant(pd_split=True))
+
+
+@pytest.mark.parametrize("mistake", ["single_srd", "single_dsf", "epilogue_tile_wait",
+                                     "pd_split_early_dpe"])
 def test_checker_rejects_known_mistakes(mistake):
     caught = 0
     for seed in range(400):
         try:
-            pm.run_schedule([3, 2, 4, 1], seed, pm.Variant(**{mistake: True}))
+            kw = {mistake: True, "pd_split": mistake.startswith("pd_split")}
+            pm.run_schedule([3, 2, 4, 1], seed, pm.Variant(**kw))
         except pm.ProtocolError:
             caught += 1
     assert caught > 0, f"{mistake} was never caught"
