@@ -138,28 +138,37 @@ class ClockSampler:
             self.proc.kill()
         self.file.flush()
         self.file.seek(0)
-        mhz, mx, reasons, all_mhz = [], None, set(), []
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for line in self.file.read().splitlines():
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 10:
-                continue
-            try:
-                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
-                sm, smx = float(parts[2]), float(parts[3])
-            except ValueError:
-                continue
-            all_mhz.append(sm)
-            mx = smx
-            if self.t0 is not None and self.t0 - 1 <= ts <= self.t1 + 1:
-                mhz.append(sm)
-                for n, v in zip(names, parts[6:10]):
-                    if v.lower() == "active":
-                        reasons.add(n)
+        text = self.file.read()
         os.unlink(self.file.name)
-        src = mhz or all_mhz
-        return {"sm_mhz": statistics.median(src) if src else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(mhz)}
+        return parse_clock_samples(text, self.t0, self.t1)
+
+
+def parse_clock_samples(text, t0, t1):
+    """Summary of `nvidia-smi --query-gpu=<ClockSampler.FIELDS>` csv lines: the
+    median SM clock over the samples taken within a second of [t0, t1] (all
+    samples if none is), the max clock, and every throttle reason seen active
+    in that window."""
+    mhz, mx, reasons, all_mhz = [], None, set(), []
+    names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    for line in text.splitlines():
+        parts = [x.strip() for x in line.split(",")]
+        if len(parts) < 10:
+            continue
+        try:
+            ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+            sm, smx = float(parts[2]), float(parts[3])
+        except ValueError:
+            continue
+        all_mhz.append(sm)
+        mx = smx
+        if t0 is not None and t1 is not None and t0 - 1 <= ts <= t1 + 1:
+            mhz.append(sm)
+            for n, v in zip(names, parts[6:10]):
+                if v.lower() == "active":
+                    reasons.add(n)
+    src = mhz or all_mhz
+    return {"sm_mhz": statistics.median(src) if src else None, "sm_max_mhz": mx,
+            "reasons": sorted(reasons), "samples": len(mhz)}
 
 
 def rank_seed(seed: int, rank: int) -> int:

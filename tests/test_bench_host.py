@@ -1,0 +1,90 @@
+"""Host-side logic of bench.py, on the CPU: the FLOP convention against the
+survey's per-config table, the traffic lookup and its invalidation when a
+kernel source changes, clock-sample parsing, and the weak-scaling helpers."""
+
+import json
+import os
+import shutil
+import sys
+import time
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+# (B, H, N, d, causal, forward GFLOP, fwd+bwd GFLOP or None), from the measurement
+# table of the survey (4 B H N^2 d forward, x 3.5 with the backward, halved causal)
+TABLE = [
+    (1, 2, 256, 64, False, 0.0336, None),
+    (8, 16, 512, 64, False, 8.59, None),
+    (8, 12, 1024, 64, True, 12.9, 45.1),
+    (1, 12, 23400, 64, True, 841.0, None),
+    (4, 16, 4096, 128, True, 275.0, 962.0),
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,causal,gf,gfb", TABLE)
+def test_flops_match_the_table(B, H, N, d, causal, gf, gfb):
+    f, fb = bench.flops(B, H, N, d, causal)
+    assert f / 1e9 == pytest.approx(gf, rel=2e-3)
+    if gfb is not None:
+        assert (f + fb) / 1e9 == pytest.approx(gfb, rel=2e-3)
+
+
+def test_workloads_cover_the_five_configs():
+    shapes = {(w[0], w[1], w[2], w[3], w[4]) for w in bench.WORKLOADS.values()}
+    for B, H, N, d, causal, _, _ in TABLE:
+        assert (B, H, N, d, causal) in shapes
+
+
+def _copy_tree(dst):
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        table = json.load(f)
+    os.makedirs(os.path.join(dst, "profiles"))
+    shutil.copy(os.path.join(ROOT, "profiles", "traffic.json"), os.path.join(dst, "profiles"))
+    for entry in table.values():
+        if isinstance(entry, dict):
+            for src in entry["sources"]:
+                os.makedirs(os.path.dirname(os.path.join(dst, src)), exist_ok=True)
+                shutil.copy(os.path.join(ROOT, src), os.path.join(dst, src))
+    return table
+
+
+def test_traffic_is_summed_and_dropped_when_a_source_changes(tmp_path, monkeypatch):
+    table = _copy_tree(str(tmp_path))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    names = [k for k in table if not k.startswith("_")]
+    want = sum(table[k]["dram_bytes_read"] + table[k]["dram_bytes_write"] for k in names)
+    assert bench.kernel_traffic(names) == want
+    assert bench.kernel_traffic(names + ["no_such_kernel"]) is None
+    src = os.path.join(str(tmp_path), table[names[0]]["sources"][-1])
+    with open(src, "a") as f:
+        f.write("\n// changed\n")
+    assert bench.kernel_traffic(names[:1]) is None
+
+
+def test_clock_samples_window_median_and_reasons():
+    t0 = time.mktime(time.strptime("2026/01/01 10:00:10", "%Y/%m/%d %H:%M:%S"))
+    t1 = t0 + 5
+
+    def line(sec, mhz, cap="Not Active", therm="Not Active"):
+        return (f"2026/01/01 10:00:{sec:02d}.123, 0, {mhz}, 1965, 900.0, 0x4, "
+                f"Not Active, Not Active, {therm}, {cap}")
+    text = "\n".join([
+        line(2, 500, therm="Active"),         # before the window: ignored
+        line(10, 1965), line(12, 1900, cap="Active"), line(14, 1950),
+        line(30, 300, therm="Active"),        # after the window: ignored
+        "garbage line",
+    ])
+    got = bench.parse_clock_samples(text, t0, t1)
+    assert got["sm_mhz"] == 1950 and got["sm_max_mhz"] == 1965
+    assert got["reasons"] == ["sw_power_cap"] and got["samples"] == 3
+    assert bench.parse_clock_samples("", t0, t1)["sm_mhz"] is None
+
+
+def test_weak_scaling_helpers():
+    # whole-job TFLOP/s: every rank's FLOPs over the slowest rank's time
+    assert bench.job_tflops(1e12, 4, 2.0) == pytest.approx(2000.0)
+    assert len({bench.rank_seed(7, r) for r in range(8)}) == 8
