@@ -3,7 +3,11 @@
 on the CPU under random schedules with the rules of protocol_model.py.  Test
 infrastructure only.
 
-One CTA works on one 128-key tile: the producer loads K/V once and streams
+One CTA works on one 128-key tile (or, in the `persistent` design variant,
+on a list of them, taking each K/V pair once the previous item's MMAs have
+released the last: KVE, with the tile rings and barrier phases running on
+across items and the accumulators reused after the epilogue read them: ACCE):
+the producer loads K/V and streams
 128-query tiles of Q (with the row statistics) and dO through two stages each;
 one thread issues, per tile, S^T, dP^T, dV, then dK and dQ (in that order,
 each group after its barriers); the compute warps (two column halves x row
@@ -22,133 +26,159 @@ NCOMP = 4    # (half, quarter) agents
 
 
 class Variant:
-    def __init__(self, no_srd=False, no_dsf_wait=False):
+    def __init__(self, no_srd=False, no_dsf_wait=False, no_acce=False):
         self.no_srd = no_srd              # mistake: half 1 writes P^T without the SRD wait
         self.no_dsf_wait = no_dsf_wait    # mistake: dK / dQ issued without waiting for dS^T
+        # persistent: the next item's first dV without the accumulator-release
+        # wait.  Not a mistake: the compute warps read dV/dK in the epilogue
+        # before they write the next item's P^T, which that dV waits for, so
+        # the wait only guards the order.
+        self.no_acce = no_acce
 
 
 W = None
 
 
-def producer(n_it, v):
-    def land_kv():
-        W.write("K", 0)
-        W.write("V", 0)
-        W.bar("KV").arrive(0)
-    yield ("async", "tma", land_kv)
-    for it in range(n_it):
-        qs, qn, ds, dn = it % QST, it // QST, it % DOST, it // DOST
-        yield ("wait", [(f"QE{qs}", qn - 1)])
+def producer(plan, v):
+    g = 0
+    for item, n_it in enumerate(plan):
+        if item > 0:
+            yield ("wait", [("KVE", item - 1)])
 
-        def land_q(it=it, qs=qs, qn=qn):
-            W.write(("Q", qs), it)
-            W.write(("LD", qs), it)
-            W.bar(f"QF{qs}").arrive(qn)
-        yield ("async", "tma", land_q)
-        yield ("wait", [(f"DOE{ds}", dn - 1)])
+        def land_kv(item=item):
+            W.write("K", item)
+            W.write("V", item)
+            W.bar("KV").arrive(item)
+        yield ("async", "tma", land_kv)
+        for _ in range(n_it):
+            qs, qn, ds, dn = g % QST, g // QST, g % DOST, g // DOST
+            yield ("wait", [(f"QE{qs}", qn - 1)])
 
-        def land_do(it=it, ds=ds, dn=dn):
-            W.write(("DO", ds), it)
-            W.bar(f"DOF{ds}").arrive(dn)
-        yield ("async", "tma", land_do)
+            def land_q(g=g, qs=qs, qn=qn):
+                W.write(("Q", qs), g)
+                W.write(("LD", qs), g)
+                W.bar(f"QF{qs}").arrive(qn)
+            yield ("async", "tma", land_q)
+            yield ("wait", [(f"DOE{ds}", dn - 1)])
+
+            def land_do(g=g, ds=ds, dn=dn):
+                W.write(("DO", ds), g)
+                W.bar(f"DOF{ds}").arrive(dn)
+            yield ("async", "tma", land_do)
+            g += 1
 
 
-def issuer(n_it, v):
-    yield ("wait", [("KV", 0)])
-    for it in range(n_it):
-        qs, qn, ds, dn = it % QST, it // QST, it % DOST, it // DOST
-        waits = [(f"QF{qs}", qn)]
-        if it > 0:
-            waits.append(("DVD", it - 1))
-        yield ("wait", waits)
-
-        def s_mma(it=it, qs=qs):
-            W.read("K", 0)
-            W.read(("Q", qs), it)
-            for q in range(2):
-                for r in ("R0", "R1", "R2", "R3"):
-                    W.write(("S", q, r), ("S", it))
-        yield ("async", "mma", s_mma)
-        yield ("async", "mma", lambda it=it: W.bar("SF").arrive(it))
-        yield ("wait", [(f"DOF{ds}", dn)])
-
-        def dp_mma(it=it, ds=ds):
-            W.read("V", 0)
-            W.read(("DO", ds), it)
-            W.write("DP", it)
-        yield ("async", "mma", dp_mma)
-        yield ("async", "mma", lambda it=it: W.bar("DPF").arrive(it))
-        yield ("wait", [("PTF", it)])
-
-        def dv_mma(it=it, ds=ds):
-            for q in range(2):
-                W.read(("S", q, "R0"), ("P", it))
-                W.read(("S", q, "R1"), ("P", it))
-            W.read(("DO", ds), it)
-            W.write("DVACC", it + 1)
-        yield ("async", "mma", dv_mma)
-        yield ("async", "mma", lambda it=it: W.bar("DVD").arrive(it))
-        yield ("async", "mma", lambda ds=ds, dn=dn: W.bar(f"DOE{ds}").arrive(dn))
-        waits = [] if v.no_dsf_wait else [("DSF", it)]
-        if it > 0:
-            waits.append(("DQE", it - 1))
-        if waits:
+def issuer(plan, v):
+    g = 0
+    for item, n_it in enumerate(plan):
+        yield ("wait", [("KV", item)])
+        for it in range(n_it):
+            qs, qn, ds, dn = g % QST, g // QST, g % DOST, g // DOST
+            waits = [(f"QF{qs}", qn)]
+            if g > 0:
+                waits.append(("DVD", g - 1))
             yield ("wait", waits)
 
-        def dkdq_mma(it=it, qs=qs):
-            for h in range(2):
-                W.read(("DS", h), it)
-            W.read(("Q", qs), it)
-            W.read("K", 0)
-            W.write("DKACC", it + 1)
-            W.write("DQ", it)
-        yield ("async", "mma", dkdq_mma)
-        yield ("async", "mma", lambda qs=qs, qn=qn: W.bar(f"QE{qs}").arrive(qn))
-        yield ("async", "mma", lambda it=it: W.bar("DQF").arrive(it))
-    yield ("async", "mma", lambda: W.bar("FIN").arrive(0))
+            def s_mma(g=g, qs=qs, item=item):
+                W.read("K", item)
+                W.read(("Q", qs), g)
+                for q in range(2):
+                    for r in ("R0", "R1", "R2", "R3"):
+                        W.write(("S", q, r), ("S", g))
+            yield ("async", "mma", s_mma)
+            yield ("async", "mma", lambda g=g: W.bar("SF").arrive(g))
+            yield ("wait", [(f"DOF{ds}", dn)])
+
+            def dp_mma(g=g, ds=ds, item=item):
+                W.read("V", item)
+                W.read(("DO", ds), g)
+                W.write("DP", g)
+            yield ("async", "mma", dp_mma)
+            yield ("async", "mma", lambda g=g: W.bar("DPF").arrive(g))
+            waits = [("PTF", g)]
+            if it == 0 and item > 0 and not v.no_acce:
+                waits.append(("ACCE", item - 1))
+            yield ("wait", waits)
+
+            def dv_mma(g=g, ds=ds, item=item, it=it):
+                for q in range(2):
+                    W.read(("S", q, "R0"), ("P", g))
+                    W.read(("S", q, "R1"), ("P", g))
+                W.read(("DO", ds), g)
+                W.write("DVACC", (item, it + 1))
+            yield ("async", "mma", dv_mma)
+            yield ("async", "mma", lambda g=g: W.bar("DVD").arrive(g))
+            yield ("async", "mma", lambda ds=ds, dn=dn: W.bar(f"DOE{ds}").arrive(dn))
+            waits = [] if v.no_dsf_wait else [("DSF", g)]
+            if g > 0:
+                waits.append(("DQE", g - 1))
+            if waits:
+                yield ("wait", waits)
+
+            def dkdq_mma(g=g, qs=qs, item=item, it=it):
+                for h in range(2):
+                    W.read(("DS", h), g)
+                W.read(("Q", qs), g)
+                W.read("K", item)
+                W.write("DKACC", (item, it + 1))
+                W.write("DQ", g)
+            yield ("async", "mma", dkdq_mma)
+            yield ("async", "mma", lambda qs=qs, qn=qn: W.bar(f"QE{qs}").arrive(qn))
+            yield ("async", "mma", lambda g=g: W.bar("DQF").arrive(g))
+            g += 1
+        yield ("async", "mma", lambda item=item: W.bar("FIN").arrive(item))
+        yield ("async", "mma", lambda item=item: W.bar("KVE").arrive(item))
 
 
-def compute(agent, n_it, v):
+def compute(agent, plan, v):
     half, q = agent // 2, agent % 2
-    for it in range(n_it):
-        qs, qn = it % QST, it // QST
-        yield ("wait", [(f"QF{qs}", qn)])
-        yield ("wait", [("SF", it)])
-        for r in (("R0", "R1") if half == 0 else ("R2", "R3")):
-            yield ("read", ("S", q, r), ("S", it))
-        yield ("read", ("LD", qs), it)
-        if half == 0:
-            if not v.no_srd:
-                yield ("arrive", "SRD", it)
-            yield ("write", ("S", q, "R0"), ("P", it))
-        else:
-            if not v.no_srd:
-                yield ("wait", [("SRD", it)])
-            yield ("write", ("S", q, "R1"), ("P", it))
-        yield ("arrive", "PTF", it)
-        yield ("wait", [("DPF", it)])
-        yield ("read", "DP", it)
-        yield ("read", ("LD", qs), it)
-        yield ("write", ("DS", half), it)
-        yield ("arrive", "DSF", it)
-        yield ("wait", [("DQF", it)])
-        yield ("read", "DQ", it)
-        yield ("arrive", "DQE", it)
-    yield ("wait", [("FIN", 0)])
-    yield ("read", "DVACC", n_it)
-    yield ("read", "DKACC", n_it)
+    g = 0
+    for item, n_it in enumerate(plan):
+        for it in range(n_it):
+            qs, qn = g % QST, g // QST
+            yield ("wait", [(f"QF{qs}", qn)])
+            yield ("wait", [("SF", g)])
+            for r in (("R0", "R1") if half == 0 else ("R2", "R3")):
+                yield ("read", ("S", q, r), ("S", g))
+            yield ("read", ("LD", qs), g)
+            if half == 0:
+                if not v.no_srd:
+                    yield ("arrive", "SRD", g)
+                yield ("write", ("S", q, "R0"), ("P", g))
+            else:
+                if not v.no_srd:
+                    yield ("wait", [("SRD", g)])
+                yield ("write", ("S", q, "R1"), ("P", g))
+            yield ("arrive", "PTF", g)
+            yield ("wait", [("DPF", g)])
+            yield ("read", "DP", g)
+            yield ("read", ("LD", qs), g)
+            yield ("write", ("DS", half), g)
+            yield ("arrive", "DSF", g)
+            yield ("wait", [("DQF", g)])
+            yield ("read", "DQ", g)
+            yield ("arrive", "DQE", g)
+            g += 1
+        yield ("wait", [("FIN", item)])
+        yield ("read", "DVACC", (item, n_it))
+        yield ("read", "DKACC", (item, n_it))
+        yield ("arrive", "ACCE", item)
 
 
-def run_schedule(n_it, seed, variant=None, max_steps=200000):
+def run_schedule(plan, seed, variant=None, max_steps=200000):
+    """plan: the number of 128-query tiles of one work item (an int: the kernel
+    as it is, one item per CTA), or of each item a persistent CTA takes."""
     global W
     v = variant or Variant()
+    plan = [plan] if isinstance(plan, int) else list(plan)
     W = World()
-    for name, c in {"PTF": NCOMP, "DSF": NCOMP, "DQE": NCOMP, "SRD": NCOMP // 2}.items():
+    for name, c in {"PTF": NCOMP, "DSF": NCOMP, "DQE": NCOMP, "SRD": NCOMP // 2,
+                    "ACCE": NCOMP}.items():
         W.bar(name, c)
     rng = random.Random(seed)
-    roles = {"prod": producer(n_it, v), "mma": issuer(n_it, v)}
+    roles = {"prod": producer(plan, v), "mma": issuer(plan, v)}
     for a in range(NCOMP):
-        roles[f"comp{a}"] = compute(a, n_it, v)
+        roles[f"comp{a}"] = compute(a, plan, v)
     nxt = {n: None for n in roles}
     queues = {"tma": [], "mma": []}
     done = set()

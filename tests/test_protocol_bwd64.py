@@ -1,6 +1,7 @@
 """The d = 64 backward kernel's mbarrier protocol on the CPU under random
-schedules (tests/protocol_model_bwd64.py mirrors the kernel's roles), and the
-checker rejecting two mistakes in it."""
+schedules (tests/protocol_model_bwd64.py mirrors the kernel's roles): the
+kernel as it is (one work item per CTA), the persistent design for it, and the
+checker rejecting two mistakes."""
 
 import pytest
 
@@ -13,12 +14,25 @@ def test_d64_protocol_holds_under_random_schedules(n_it):
         pm.run_schedule(n_it, seed)
 
 
+@pytest.mark.parametrize("plan", [[3, 1, 4], [1, 1, 1, 1], [2, 5, 2], [8, 1]],
+                         ids=lambda p: "-".join(map(str, p)))
+def test_persistent_d64_design_holds(plan):
+    for seed in range(100):
+        pm.run_schedule(plan, seed)
+
+
+def test_accumulator_release_is_implied_by_the_role_order():
+    for seed in range(150):
+        pm.run_schedule([3, 2, 4, 1], seed, pm.Variant(no_acce=True))
+
+
 @pytest.mark.parametrize("mistake", ["no_srd", "no_dsf_wait"])
-def test_checker_rejects_d64_mistakes(mistake):
+@pytest.mark.parametrize("plan", [5, [3, 2, 4, 1]], ids=["one-item", "persistent"])
+def test_checker_rejects_d64_mistakes(mistake, plan):
     caught = 0
     for seed in range(300):
         try:
-            pm.run_schedule(5, seed, pm.Variant(**{mistake: True}))
+            pm.run_schedule(plan, seed, pm.Variant(**{mistake: True}))
         except pm.ProtocolError:
             caught += 1
     assert caught > 0
