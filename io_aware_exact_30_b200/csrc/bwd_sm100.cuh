@@ -19,7 +19,9 @@
 //                         both fp32 in a per-head array padded to a multiple of
 //                         128 rows (padding: D = 0, L2 = +inf so P = 0); zeroes
 //                         the fp32 dQ accumulator and the per-head counters.
-//   attn_bwd_main_kernel  one CTA per (head, 128-key tile j); K_j, V_j stay in
+//   attn_bwd_main_kernel  (head dimension 64; 128 has its own kernel in
+//                         bwd128_sm100.cuh)
+//                         one CTA per (head, 128-key tile j); K_j, V_j stay in
 //                         shared memory while the 128-query tiles i stream
 //                         through (Q double-buffered).  Per query tile:
 //                           S^T  = K_j Q_i^T          (tensor memory)
@@ -136,7 +138,8 @@ struct BwdCfg {
     static constexpr int KB = D / 64;
     static constexpr uint32_t TILE = 128u * D * 2u;
     static constexpr int QST = 2;
-    static constexpr int DOST = D == 128 ? 1 : 2;
+    static_assert(D == 64, "head dimension 128 has its own kernel (bwd128_sm100.cuh)");
+    static constexpr int DOST = 2;
     static constexpr uint32_t OFF_K = 0;
     static constexpr uint32_t OFF_V = OFF_K + TILE;
     static constexpr uint32_t OFF_Q = OFF_V + TILE;
@@ -154,7 +157,7 @@ struct BwdCfg {
     static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
-    static constexpr uint32_t COL_DQ = D == 128 ? COL_DP : 384;
+    static constexpr uint32_t COL_DQ = 384;
     static constexpr int NCOMPUTE = 256;             // 8 compute warps
     static constexpr int NTHREADS = NCOMPUTE + 64;   // + TMA warp + MMA warp
     static constexpr int WARP_TMA = NCOMPUTE / 32, WARP_MMA = WARP_TMA + 1;
@@ -274,7 +277,6 @@ __global__ void __launch_bounds__(320, 1)
         if (lane == 0) {
             constexpr uint32_t ID_SS = idesc_f16(BF16, 128, 128, false, false);
             constexpr uint32_t ID_KV = idesc_f16(BF16, 128, D, false, true);
-            constexpr uint32_t ID_DQT = idesc_f16(BF16, 128, 128, true, true);  // D == 128
             constexpr uint32_t ID_DQ = idesc_f16(BF16, 128, D, true, true);     // D == 64
             const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sDST = base + C::OFF_DST;
             bool ok = wait_bounded(BAR(C::B_KV), 0, abort_flag);
@@ -295,10 +297,8 @@ __global__ void __launch_bounds__(320, 1)
                            sdesc_sw128(sQ + off, 16, 1024), ID_SS, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(BAR(C::B_SF));
-                // dP^T = V dO^T; for D = 128 the columns hold dQ^T(it-1) until drained
+                // dP^T = V dO^T
                 if (!(ok = wait_bounded(BAR(C::B_DOF + ds), dn & 1, abort_flag))) break;
-                if (D == 128 && it > 0 && !(ok = wait_bounded(BAR(C::B_DQE), ph ^ 1, abort_flag)))
-                    break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -319,8 +319,7 @@ __global__ void __launch_bounds__(320, 1)
                 mma_commit(BAR(C::B_DOE + ds));
                 // dK += dS^T Q ; dQ partial
                 if (!(ok = wait_bounded(BAR(C::B_DSF), ph, abort_flag))) break;
-                if (D == 64 && it > 0 && !(ok = wait_bounded(BAR(C::B_DQE), ph ^ 1, abort_flag)))
-                    break;
+                if (it > 0 && !(ok = wait_bounded(BAR(C::B_DQE), ph ^ 1, abort_flag))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
@@ -328,19 +327,11 @@ __global__ void __launch_bounds__(320, 1)
                            sdesc_sw128(sDST + (kk >> 2) * 16384u + (kk & 3) * 32u, 16, 1024),
                            sdesc_sw128(sQ + kk * 2048u, 16384, 1024), ID_KV,
                            (it > 0 || kk > 0) ? 1u : 0u);
-                if constexpr (D == 128) {
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)  // dQ^T = K^T dS^T: A = K (MN-major), B = dS^T (MN-major)
-                        mma_ss(tmem + C::COL_DQ, sdesc_sw128(sK + kk * 2048u, 16384, 1024),
-                               sdesc_sw128(sDST + kk * 2048u, 16384, 1024), ID_DQT,
-                               kk > 0 ? 1u : 0u);
-                } else {
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)  // dQ = dS K: A = dS^T read MN-major, B = K MN-major
-                        mma_ss(tmem + C::COL_DQ, sdesc_sw128(sDST + kk * 2048u, 16384, 1024),
-                               sdesc_sw128(sK + kk * 2048u, 16384, 1024), ID_DQ,
-                               kk > 0 ? 1u : 0u);
-                }
+                for (int kk = 0; kk < 8; ++kk)  // dQ = dS K: A = dS^T read MN-major, B = K MN-major
+                    mma_ss(tmem + C::COL_DQ, sdesc_sw128(sDST + kk * 2048u, 16384, 1024),
+                           sdesc_sw128(sK + kk * 2048u, 16384, 1024), ID_DQ,
+                           kk > 0 ? 1u : 0u);
                 mma_commit(BAR(C::B_QE + qs));
                 mma_commit(BAR(C::B_DQF));
             }
@@ -464,40 +455,20 @@ __global__ void __launch_bounds__(320, 1)
             ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_DQF), ph, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            if constexpr (D == 128) {
-                // lane r holds feature r of dQ; this half covers queries c0 .. c0+63
-                float* col = p.dqacc + head_row0 * D + r;
-                const int nq = min(128, p.N - q0);
+            // lane r holds query row q0 + r of dQ; this half covers features 32h .. 32h+31
+            const int qr = q0 + r;
+            float* row = p.dqacc + (head_row0 + qr) * D + half * 32;
+            uint32_t v[32];
+            tmem_ld32(lane_addr + C::COL_DQ + half * 32u, v);
+            tmem_ld_wait();
+            reg_fence32(v);
+            if (qr < p.N) {
 #pragma unroll
-                for (int c4 = 0; c4 < 2; ++c4) {
-                    uint32_t v[32];
-                    tmem_ld32(lane_addr + C::COL_DQ + c0 + c4 * 32u, v);
-                    tmem_ld_wait();
-                    reg_fence32(v);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int qc = c0 + c4 * 32 + e;
-                        if (qc < nq)
-                            red_add_f32(col + static_cast<size_t>(q0 + qc) * D,
-                                        __uint_as_float(v[e]) * p.scale);
-                    }
-                }
-            } else {
-                // lane r holds query row q0 + r of dQ; this half covers features 32h .. 32h+31
-                const int qr = q0 + r;
-                float* row = p.dqacc + (head_row0 + qr) * D + half * 32;
-                uint32_t v[32];
-                tmem_ld32(lane_addr + C::COL_DQ + half * 32u, v);
-                tmem_ld_wait();
-                reg_fence32(v);
-                if (qr < p.N) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        red_add_v4_f32(row + 4 * e, __uint_as_float(v[4 * e]) * p.scale,
-                                       __uint_as_float(v[4 * e + 1]) * p.scale,
-                                       __uint_as_float(v[4 * e + 2]) * p.scale,
-                                       __uint_as_float(v[4 * e + 3]) * p.scale);
-                }
+                for (int e = 0; e < 8; ++e)
+                    red_add_v4_f32(row + 4 * e, __uint_as_float(v[4 * e]) * p.scale,
+                                   __uint_as_float(v[4 * e + 1]) * p.scale,
+                                   __uint_as_float(v[4 * e + 2]) * p.scale,
+                                   __uint_as_float(v[4 * e + 3]) * p.scale);
             }
             tc_fence_before();
             mbar_arrive(BAR(C::B_DQE));
@@ -573,12 +544,6 @@ inline bool bwd_set_attributes() {
     ok &= cudaFuncSetAttribute(attn_bwd_main_kernel<64, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                BwdCfg<64>::SMEM_BYTES) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(attn_bwd_main_kernel<128, true>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               BwdCfg<128>::SMEM_BYTES) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(attn_bwd_main_kernel<128, false>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               BwdCfg<128>::SMEM_BYTES) == cudaSuccess;
     return ok;
 }
 
