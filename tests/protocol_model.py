@@ -5,9 +5,11 @@ under many random schedules.  Test infrastructure only.
 Each role of the kernel is a generator that yields the same sequence of
 barrier operations, with the same barriers, arrival counts and phase indices,
 as the kernel's code; asynchronous work (TMA loads, MMAs and their commits,
-the bulk stores) is queued and completed at random later points, MMAs in issue
-order per issuing thread.  Buffers carry a version tag: every read states the
-version it must see, every write sets one.
+the bulk stores) is queued and completed at random later points, in any order
+the hardware allows (`AsyncWork`): a commit after everything its thread issued
+before it, an MMA after the earlier MMAs of its thread on the same
+accumulator, a copy at any time.  Buffers carry a version tag: every read
+states the version it must see, every write sets one.
 
 Groups of threads that run the same code are modelled by a few agents each
 (two per column half of the compute warps, two dQ warps), so the barriers'
@@ -89,6 +91,59 @@ class World:
         self.buf[key] = value
 
 
+class AsyncWork:
+    """Asynchronous operations in flight, per issuing unit (a TMA producer, an
+    MMA-issuing thread, the bulk-store unit), completed in an order the
+    hardware allows.  Each operation carries a tag:
+      * "commit" (the default): a tcgen05.commit, or a bulk-group arrival.  It
+        completes after every earlier operation of its unit.
+      * "tma": a copy, which may complete at any time.
+      * any other tag names the accumulator of a group of MMAs.  tcgen05.mma
+        instructions of one thread are pipelined (kept in order) only when they
+        share the accumulator and shape, so the group completes after the
+        earlier groups of its unit on the same accumulator, in any order
+        relative to the rest.
+    With in_order=True every unit completes in issue order instead."""
+
+    def __init__(self, in_order=False):
+        self.units = {}
+        self.in_order = in_order
+
+    def push(self, unit, fn, tag="commit"):
+        self.units.setdefault(unit, []).append((fn, tag))
+
+    def pending(self):
+        return any(self.units.values())
+
+    def _eligible(self, ops, i):
+        tag = ops[i][1]
+        if self.in_order or tag == "commit":
+            return i == 0
+        if tag == "tma":
+            return True
+        return all(t != tag for _, t in ops[:i])
+
+    def ready(self):
+        return [(u, i) for u, ops in self.units.items() for i in range(len(ops))
+                if self._eligible(ops, i)]
+
+    def complete(self, unit, i):
+        fn, _ = self.units[unit].pop(i)
+        fn()
+
+
+def push_op(work, op):
+    """An ("async", unit, fn[, tag]) operation of a role."""
+    work.push(op[1], op[2], op[3] if len(op) > 3 else "commit")
+
+
+def group_ready(op):
+    """A role's grouped wait: every barrier is tested (the kernel issues all
+    the tests before it looks at any result), and it passes when all pass."""
+    results = [W.bar(b).test(k) for b, k in op[1]]
+    return all(results)
+
+
 ST = 3          # Q / dO / statistics stages
 NCOMP = 4       # compute agents: (half, quarter) for half in 0,1 and quarter in 0,1
 NDQ = 2         # dQ agents; agent 0 holds the reduction issuer
@@ -98,7 +153,8 @@ NDQ = 2         # dQ agents; agent 0 holds the reduction issuer
 # Roles.  Operations yielded:
 #   ("wait", [(bar, k), ...])          all tests must pass (tested together)
 #   ("arrive", bar, use)
-#   ("async", queue, fn)               fn() runs when the queue delivers it
+#   ("async", unit, fn[, tag])         fn() runs when the unit completes it
+#                                      (completion order: AsyncWork)
 #   ("read", key, version) / ("write", key, version)   a role's own access
 # Every operation of a role is a step of its own, so any other step can fall
 # between two of them; the effects of an MMA or a copy happen at once when it
@@ -118,7 +174,7 @@ def producer(plan, v):
                 W.write(("DO", s), g)
                 W.write(("LD", s), g)
                 W.bar(f"QF{s}").arrive(n)
-            yield ("async", "tma", land)
+            yield ("async", "tma", land, "tma")
         pre = min(ST, n_it)
         for _ in range(pre):
             yield from load_tile(g)
@@ -130,7 +186,7 @@ def producer(plan, v):
             W.write("K", item)
             W.write("V", item)
             W.bar("KV").arrive(item)
-        yield ("async", "tma", land_kv)
+        yield ("async", "tma", land_kv, "tma")
         for _ in range(pre, n_it):
             yield from load_tile(g)
             g += 1
@@ -161,7 +217,7 @@ def issuer_a(plan, v):
                 W.read("V", item)
                 W.read(("DO", s), g)
                 W.write("DP", g)
-            yield ("async", "A", dp)
+            yield ("async", "A", dp, "DP")
             yield ("async", "A", lambda g=g: W.bar("DPF").arrive(g))
             yield ("async", "A", lambda s=s, g=g: W.bar(f"QE{s}", 2).arrive(g // ST))
             if more:
@@ -179,7 +235,7 @@ def mma_s(g, item):
         for q in range(2):
             for r in ("R0", "R1", "R2", "R3"):   # S^T columns 0-15, 16-31, 32-47, 48-63
                 W.write(("S", g & 1, q, r), ("S", g))
-    yield ("async", "A", run)
+    yield ("async", "A", run, f"S{g & 1}")
     yield ("async", "A", lambda g=g: W.bar(f"SF{g & 1}").arrive(g >> 1))
 
 
@@ -199,7 +255,7 @@ def issuer_b(plan, v):
                     W.read(("S", g & 1, q, "R2" if v.own_region_p else "R1"), ("P", g))
                 W.read(("DO", s), g)
                 W.write("DVACC", (item, it + 1))
-            yield ("async", "B", dv)
+            yield ("async", "B", dv, "DV")
             yield ("async", "B", lambda g=g: W.bar(f"DVD{g & 1}").arrive(g >> 1))
             dsf = ("DSF0", g) if v.single_dsf else (f"DSF{g & 1}", g >> 1)
             waits = [dsf]
@@ -209,15 +265,19 @@ def issuer_b(plan, v):
                 waits.append(("KV", item))
             yield ("wait", waits)
 
-            def dkdq(g=g, s=s, item=item, it=it):
-                b = g & 1
+            def dk(g=g, s=s, it=it, item=item):
                 for h in range(2):
-                    W.read(("DS", b, h), g)
+                    W.read(("DS", g & 1, h), g)
                 W.read(("Q", s), g)
-                W.read("K", item)
                 W.write("DKACC", (item, it + 1))
+
+            def dq(g=g, item=item):
+                for h in range(2):
+                    W.read(("DS", g & 1, h), g)
+                W.read("K", item)
                 W.write("DQ", g)
-            yield ("async", "B", dkdq)
+            yield ("async", "B", dk, "DK")
+            yield ("async", "B", dq, "DQ")
             yield ("async", "B", lambda s=s, g=g: W.bar(f"QE{s}", 2).arrive(g // ST))
             yield ("async", "B", lambda g=g: W.bar("DQF").arrive(g))
             yield ("async", "B", lambda g=g: W.bar(f"DSTE{g & 1}").arrive(g >> 1))
@@ -387,9 +447,10 @@ def dq_role(agent, plan, v):
 W = None  # the world of the schedule being run (the roles read it as a global)
 
 
-def run_schedule(plan, seed, variant=None, max_steps=200000):
+def run_schedule(plan, seed, variant=None, max_steps=200000, in_order=False):
     """Runs one random schedule of one CTA working through `plan`; raises
-    ProtocolError on a violation or a deadlock."""
+    ProtocolError on a violation or a deadlock.  in_order: complete each
+    unit's asynchronous work in issue order (a narrower set of schedules)."""
     global W
     v = variant or Variant()
     W = World()
@@ -418,7 +479,7 @@ def run_schedule(plan, seed, variant=None, max_steps=200000):
     for a in range(NDQ):
         roles[f"dq{a}"] = dq_role(a, plan, v)
     nxt = {name: None for name in roles}       # pending operation of each role
-    queues = {"tma": [], "A": [], "B": [], "store": []}
+    work = AsyncWork(in_order)
     done = set()
 
     def advance(name):
@@ -431,32 +492,26 @@ def run_schedule(plan, seed, variant=None, max_steps=200000):
     for name in roles:
         advance(name)
     for _ in range(max_steps):
-        if len(done) == len(roles) and not any(queues.values()):
+        if len(done) == len(roles) and not work.pending():
             return
         choices = []
         for name, op in nxt.items():
             if op is None:
                 continue
-            if op[0] == "wait":
-                # the kernel tests all barriers of a group; each test is checked
-                if all(W.bar(b).test(k) for b, k in op[1]):
-                    choices.append(("role", name))
-            else:
+            if op[0] != "wait" or group_ready(op):
                 choices.append(("role", name))
-        for qn, q in queues.items():
-            if q:
-                choices.append(("queue", qn))
+        choices += [("work", r) for r in work.ready()]
         if not choices:
             raise ProtocolError(f"deadlock: pending {[(n, o[0], o[1] if o[0] == 'wait' else '') for n, o in nxt.items() if o]}")
         kind, name = rng.choice(choices)
-        if kind == "queue":
-            queues[name].pop(0)()
+        if kind == "work":
+            work.complete(*name)
             continue
         op = nxt[name]
         if op[0] == "arrive":
             W.bar(op[1]).arrive(op[2])
         elif op[0] == "async":
-            queues[op[1]].append(op[2])
+            push_op(work, op)
         elif op[0] == "read":
             W.read(op[1], op[2])
         elif op[0] == "write":

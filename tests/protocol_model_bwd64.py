@@ -14,21 +14,25 @@ each group after its barriers); the compute warps (two column halves x row
 quarters, modelled as four agents) write P^T over S^T (half 1 over columns half
 0 reads, after the shared-read barrier), dS^T into shared memory, and drain dQ
 into the accumulator.  The per-head completion counters after the epilogue
-are outside the model.
+are outside the model.  Asynchronous work completes in any order the hardware
+allows (protocol_model.AsyncWork).
 """
 
 import random
 
-from protocol_model import ProtocolError, World
+from protocol_model import AsyncWork, ProtocolError, World
 
 QST = DOST = 2
 NCOMP = 4    # (half, quarter) agents
 
 
 class Variant:
-    def __init__(self, no_srd=False, no_dsf_wait=False, no_acce=False):
+    def __init__(self, no_srd=False, no_dsf_wait=False, no_acce=False, s_without_dvd_wait=False):
         self.no_srd = no_srd              # mistake: half 1 writes P^T without the SRD wait
         self.no_dsf_wait = no_dsf_wait    # mistake: dK / dQ issued without waiting for dS^T
+        # mistake: S^T(g+1) issued without waiting for dV(g), which reads P^T
+        # from the same columns, trusting the issue order of one thread's MMAs
+        self.s_without_dvd_wait = s_without_dvd_wait
         # persistent: the next item's first dV without the accumulator-release
         # wait.  Not a mistake: the compute warps read dV/dK in the epilogue
         # before they write the next item's P^T, which that dV waits for, so
@@ -49,7 +53,7 @@ def producer(plan, v):
             W.write("K", item)
             W.write("V", item)
             W.bar("KV").arrive(item)
-        yield ("async", "tma", land_kv)
+        yield ("async", "tma", land_kv, "tma")
         for _ in range(n_it):
             qs, qn, ds, dn = g % QST, g // QST, g % DOST, g // DOST
             yield ("wait", [(f"QE{qs}", qn - 1)])
@@ -58,13 +62,13 @@ def producer(plan, v):
                 W.write(("Q", qs), g)
                 W.write(("LD", qs), g)
                 W.bar(f"QF{qs}").arrive(qn)
-            yield ("async", "tma", land_q)
+            yield ("async", "tma", land_q, "tma")
             yield ("wait", [(f"DOE{ds}", dn - 1)])
 
             def land_do(g=g, ds=ds, dn=dn):
                 W.write(("DO", ds), g)
                 W.bar(f"DOF{ds}").arrive(dn)
-            yield ("async", "tma", land_do)
+            yield ("async", "tma", land_do, "tma")
             g += 1
 
 
@@ -75,7 +79,7 @@ def issuer(plan, v):
         for it in range(n_it):
             qs, qn, ds, dn = g % QST, g // QST, g % DOST, g // DOST
             waits = [(f"QF{qs}", qn)]
-            if g > 0:
+            if g > 0 and not v.s_without_dvd_wait:
                 waits.append(("DVD", g - 1))
             yield ("wait", waits)
 
@@ -85,7 +89,7 @@ def issuer(plan, v):
                 for q in range(2):
                     for r in ("R0", "R1", "R2", "R3"):
                         W.write(("S", q, r), ("S", g))
-            yield ("async", "mma", s_mma)
+            yield ("async", "mma", s_mma, "S")
             yield ("async", "mma", lambda g=g: W.bar("SF").arrive(g))
             yield ("wait", [(f"DOF{ds}", dn)])
 
@@ -93,7 +97,7 @@ def issuer(plan, v):
                 W.read("V", item)
                 W.read(("DO", ds), g)
                 W.write("DP", g)
-            yield ("async", "mma", dp_mma)
+            yield ("async", "mma", dp_mma, "DP")
             yield ("async", "mma", lambda g=g: W.bar("DPF").arrive(g))
             waits = [("PTF", g)]
             if it == 0 and item > 0 and not v.no_acce:
@@ -106,7 +110,7 @@ def issuer(plan, v):
                     W.read(("S", q, "R1"), ("P", g))
                 W.read(("DO", ds), g)
                 W.write("DVACC", (item, it + 1))
-            yield ("async", "mma", dv_mma)
+            yield ("async", "mma", dv_mma, "DV")
             yield ("async", "mma", lambda g=g: W.bar("DVD").arrive(g))
             yield ("async", "mma", lambda ds=ds, dn=dn: W.bar(f"DOE{ds}").arrive(dn))
             waits = [] if v.no_dsf_wait else [("DSF", g)]
@@ -115,14 +119,19 @@ def issuer(plan, v):
             if waits:
                 yield ("wait", waits)
 
-            def dkdq_mma(g=g, qs=qs, item=item, it=it):
+            def dk_mma(g=g, qs=qs, item=item, it=it):
                 for h in range(2):
                     W.read(("DS", h), g)
                 W.read(("Q", qs), g)
-                W.read("K", item)
                 W.write("DKACC", (item, it + 1))
+
+            def dq_mma(g=g, item=item):
+                for h in range(2):
+                    W.read(("DS", h), g)
+                W.read("K", item)
                 W.write("DQ", g)
-            yield ("async", "mma", dkdq_mma)
+            yield ("async", "mma", dk_mma, "DK")
+            yield ("async", "mma", dq_mma, "DQ")
             yield ("async", "mma", lambda qs=qs, qn=qn: W.bar(f"QE{qs}").arrive(qn))
             yield ("async", "mma", lambda g=g: W.bar("DQF").arrive(g))
             g += 1
@@ -165,9 +174,10 @@ def compute(agent, plan, v):
         yield ("arrive", "ACCE", item)
 
 
-def run_schedule(plan, seed, variant=None, max_steps=200000):
+def run_schedule(plan, seed, variant=None, max_steps=200000, in_order=False):
     """plan: the number of 128-query tiles of one work item (an int: the kernel
-    as it is, one item per CTA), or of each item a persistent CTA takes."""
+    as it is, one item per CTA), or of each item a persistent CTA takes.
+    in_order: complete each unit's asynchronous work in issue order."""
     global W
     v = variant or Variant()
     plan = [plan] if isinstance(plan, int) else list(plan)
@@ -180,7 +190,7 @@ def run_schedule(plan, seed, variant=None, max_steps=200000):
     for a in range(NCOMP):
         roles[f"comp{a}"] = compute(a, plan, v)
     nxt = {n: None for n in roles}
-    queues = {"tma": [], "mma": []}
+    work = AsyncWork(in_order)
     done = set()
 
     def advance(name):
@@ -193,26 +203,26 @@ def run_schedule(plan, seed, variant=None, max_steps=200000):
     for name in roles:
         advance(name)
     for _ in range(max_steps):
-        if len(done) == len(roles) and not any(queues.values()):
+        if len(done) == len(roles) and not work.pending():
             return
         choices = []
         for name, op in nxt.items():
             if op is None:
                 continue
-            if op[0] != "wait" or all(W.bar(b).test(k) for b, k in op[1]):
+            if op[0] != "wait" or all([W.bar(b).test(k) for b, k in op[1]]):
                 choices.append(("role", name))
-        choices += [("queue", qn) for qn, qu in queues.items() if qu]
+        choices += [("work", r) for r in work.ready()]
         if not choices:
             raise ProtocolError("deadlock: " + str([(n, o) for n, o in nxt.items() if o]))
         kind, name = rng.choice(choices)
-        if kind == "queue":
-            queues[name].pop(0)()
+        if kind == "work":
+            work.complete(*name)
             continue
         op = nxt[name]
         if op[0] == "arrive":
             W.bar(op[1]).arrive(op[2])
         elif op[0] == "async":
-            queues[op[1]].append(op[2])
+            work.push(op[1], op[2], op[3] if len(op) > 3 else "commit")
         elif op[0] == "read":
             W.read(op[1], op[2])
         elif op[0] == "write":

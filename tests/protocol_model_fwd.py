@@ -11,7 +11,9 @@ the data in the kernel; the model decides it at random.
 
 Every operation of a role (barrier tests and arrivals, its own reads and
 writes) is a step of its own; the effects of an MMA or a copy happen at once
-when it completes.
+when it completes, in any order the hardware allows (protocol_model.AsyncWork:
+MMA groups in issue order only per accumulator, a commit after all earlier
+work of its thread, copies in any order).
 
 A work item is given by (nkv_0, nkv_1), the key-tile steps of its two query
 tiles: equal without the mask; under the causal mask tile 1 has one more, and
@@ -20,7 +22,7 @@ the last pair of an odd tile count has nkv_1 = 0.
 
 import random
 
-from protocol_model import Barrier, ProtocolError, World
+from protocol_model import AsyncWork, ProtocolError, World
 
 ST = 2      # K/V stages (d = 128)
 NSM = 2     # softmax agents per query tile
@@ -28,7 +30,7 @@ NSM = 2     # softmax agents per query tile
 
 class Variant:
     def __init__(self, ke_before_pv=False, epilogue_no_od_wait=False, split=False,
-                 split_no_exchange_wait=False):
+                 split_no_exchange_wait=False, order_c=False, s_without_od_wait=False):
         # release the K/V stage before the tile-1 P V of the step is issued
         self.ke_before_pv = ke_before_pv
         # the epilogue reads O without waiting for the last P V
@@ -41,6 +43,14 @@ class Variant:
         # mistake for the split design: read the other half's max without
         # waiting for the exchange barrier
         self.split_no_exchange_wait = split_no_exchange_wait
+        # design variant: per key tile both tiles' P V first, then both next S
+        # (each after its own P V has completed), so that each wait for a P V
+        # is covered by MMAs already in the tensor pipe
+        self.order_c = order_c
+        # mistake: the next S issued without waiting for the P V that reads
+        # its columns, trusting the issue order (which the hardware keeps only
+        # between MMAs on the same accumulator)
+        self.s_without_od_wait = s_without_od_wait
 
 
 W = None
@@ -56,7 +66,7 @@ def producer(plan, v):
         def land_q(item=item):
             W.write("Q", item)
             W.bar("Q").arrive(item)
-        yield ("async", "tma", land_q)
+        yield ("async", "tma", land_q, "tma")
         for j in range(nkv):
             kvj = kv + j
             s, n = kvj % ST, kvj // ST
@@ -69,8 +79,8 @@ def producer(plan, v):
             def land_v(kvj=kvj, s=s, n=n):
                 W.write(("V", s), kvj)
                 W.bar(f"VF{s}").arrive(n)
-            yield ("async", "tma", land_k)
-            yield ("async", "tma", land_v)
+            yield ("async", "tma", land_k, "tma")
+            yield ("async", "tma", land_v, "tma")
         kv += nkv
 
 
@@ -86,7 +96,7 @@ def issuer(plan, v):
             W.read(("K", s), kvi)
             for a in range(nagents(v)):
                 W.write(("S", t, a), ("S", kvi))
-        yield ("async", "mma", run)
+        yield ("async", "mma", run, f"S{t}")
         k = n_s[t]
         n_s[t] += 1
         yield ("async", "mma", lambda t=t, k=k: W.bar(f"SF{t}").arrive(k))
@@ -107,7 +117,18 @@ def issuer(plan, v):
             kvj = kv + j
             s, n = kvj % ST, kvj // ST
             k1 = kvj + 1
-            k_next = False
+            k_next = [False]  # K_{j+1} has been waited for
+
+            def next_s(t, k1=k1, k_next=k_next, item=item):
+                # S_t(j+1) takes the columns P_t(j) V read: wait for that P V
+                waits = [] if v.s_without_od_wait else [(f"OD{t}", n_pv[t] - 1)]
+                if not k_next[0]:
+                    waits.append((f"KF{k1 % ST}", k1 // ST))
+                if waits:
+                    yield ("wait", waits)
+                k_next[0] = True
+                yield from issue_s(t, k1, item)
+
             for t in range(2):
                 act = j < nkv_t[t]
                 waits = []
@@ -130,18 +151,19 @@ def issuer(plan, v):
                     W.read(("V", s), kvj)
                     for hh in range(2 if v.split else 1):
                         W.write(("O", t, hh), (item, j + 1))
-                yield ("async", "mma", pv)
+                yield ("async", "mma", pv, f"O{t}")
                 k = n_pv[t]
                 n_pv[t] += 1
                 yield ("async", "mma", lambda t=t, k=k: W.bar(f"OD{t}").arrive(k))
-                if j + 1 < nkv_t[t]:
-                    waits = [(f"OD{t}", n_pv[t] - 1)]
-                    if not k_next:
-                        waits.append((f"KF{k1 % ST}", k1 // ST))
-                    yield ("wait", waits)
-                    k_next = True
-                    yield from issue_s(t, k1, item)
-            if not v.ke_before_pv:
+                if j + 1 < nkv_t[t] and not v.order_c:
+                    yield from next_s(t)
+            if v.order_c:
+                if not v.ke_before_pv:
+                    yield ("async", "mma", lambda s=s, n=n: W.bar(f"KE{s}").arrive(n))
+                for t in range(2):
+                    if j + 1 < nkv_t[t]:
+                        yield from next_s(t)
+            elif not v.ke_before_pv:
                 yield ("async", "mma", lambda s=s, n=n: W.bar(f"KE{s}").arrive(n))
         yield ("async", "mma", lambda item=item: W.bar("QE").arrive(item))
         kv += nkv
@@ -219,7 +241,10 @@ def softmax_split(t, h, qq, plan, v, seed):
         kv += nkv
 
 
-def run_schedule(plan, seed, variant=None, max_steps=200000):
+def run_schedule(plan, seed, variant=None, max_steps=200000, in_order=False):
+    """One random schedule of one CTA working through `plan`; raises
+    ProtocolError on a violation or a deadlock.  in_order: complete each
+    unit's asynchronous work in issue order."""
     global W
     v = variant or Variant()
     W = World()
@@ -241,7 +266,7 @@ def run_schedule(plan, seed, variant=None, max_steps=200000):
             for a in range(NSM):
                 roles[f"sm{t}{a}"] = softmax(t, a, plan, v, random.Random(seed * 7 + 2 * t + a))
     nxt = {n: None for n in roles}
-    queues = {"tma": [], "mma": []}
+    work = AsyncWork(in_order)
     done = set()
 
     def advance(name):
@@ -254,31 +279,26 @@ def run_schedule(plan, seed, variant=None, max_steps=200000):
     for name in roles:
         advance(name)
     for _ in range(max_steps):
-        if len(done) == len(roles) and not any(queues.values()):
+        if len(done) == len(roles) and not work.pending():
             return
         choices = []
         for name, op in nxt.items():
             if op is None:
                 continue
-            if op[0] == "wait":
-                if all(W.bar(b).test(k) for b, k in op[1]):
-                    choices.append(("role", name))
-            else:
+            if op[0] != "wait" or all([W.bar(b).test(k) for b, k in op[1]]):
                 choices.append(("role", name))
-        for qn, q in queues.items():
-            if q:
-                choices.append(("queue", qn))
+        choices += [("work", r) for r in work.ready()]
         if not choices:
             raise ProtocolError("deadlock: " + str([(n, o) for n, o in nxt.items() if o]))
         kind, name = rng.choice(choices)
-        if kind == "queue":
-            queues[name].pop(0)()
+        if kind == "work":
+            work.complete(*name)
             continue
         op = nxt[name]
         if op[0] == "arrive":
             W.bar(op[1]).arrive(op[2])
         elif op[0] == "async":
-            queues[op[1]].append(op[2])
+            work.push(op[1], op[2], op[3] if len(op) > 3 else "commit")
         elif op[0] == "read":
             W.read(op[1], op[2])
         elif op[0] == "write":

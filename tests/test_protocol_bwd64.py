@@ -1,7 +1,7 @@
 """The d = 64 backward kernel's mbarrier protocol on the CPU under random
 schedules (tests/protocol_model_bwd64.py mirrors the kernel's roles): the
 kernel as it is (one work item per CTA), the persistent design for it, and the
-checker rejecting two mistakes."""
+checker rejecting mistakes."""
 
 import pytest
 
@@ -33,6 +33,22 @@ def test_checker_rejects_d64_mistakes(mistake, plan):
     for seed in range(300):
         try:
             pm.run_schedule(plan, seed, pm.Variant(**{mistake: True}))
+        except pm.ProtocolError:
+            caught += 1
+    assert caught > 0
+
+
+def test_next_s_needs_the_dv_wait_although_issued_later():
+    """S^T(g+1) overwrites the columns dV(g) reads P^T from, on another
+    accumulator: completed in issue order the missing wait goes unseen; with
+    the completion order the hardware allows, it is caught."""
+    v = pm.Variant(s_without_dvd_wait=True)
+    for seed in range(100):
+        pm.run_schedule(4, seed, v, in_order=True)
+    caught = 0
+    for seed in range(300):
+        try:
+            pm.run_schedule(4, seed, v)
         except pm.ProtocolError:
             caught += 1
     assert caught > 0

@@ -29,6 +29,32 @@ def test_split_softmax_design_holds(name):
         pf.run_schedule(PLANS[name], seed, pf.Variant(split=True))
 
 
+@pytest.mark.parametrize("name", sorted(PLANS))
+@pytest.mark.parametrize("split", [False, True], ids=["one-group", "split"])
+def test_order_c_design_holds(name, split):
+    # next-step design: per key tile both P V first, then both next S
+    for seed in range(100):
+        pf.run_schedule(PLANS[name], seed, pf.Variant(order_c=True, split=split))
+
+
+@pytest.mark.parametrize("order_c", [False, True], ids=["order-a", "order-c"])
+def test_next_s_needs_the_pv_wait_although_issued_later(order_c):
+    """S_t(j+1) overwrites the columns P_t(j) V reads.  Completed in issue
+    order the mistake would go unseen; with MMAs on different accumulators
+    free to complete out of order, as the hardware allows, it is caught."""
+    plan = [(3, 4), (2, 2)]
+    v = pf.Variant(order_c=order_c, s_without_od_wait=True)
+    for seed in range(100):
+        pf.run_schedule(plan, seed, v, in_order=True)
+    caught = 0
+    for seed in range(300):
+        try:
+            pf.run_schedule(plan, seed, v)
+        except pf.ProtocolError:
+            caught += 1
+    assert caught > 0
+
+
 @pytest.mark.parametrize("mistake", ["ke_before_pv", "epilogue_no_od_wait",
                                      "split_no_exchange_wait"])
 def test_checker_rejects_forward_mistakes(mistake):
