@@ -9,7 +9,10 @@ the bulk stores) is queued and completed at random later points, in any order
 the hardware allows (`AsyncWork`): a commit after everything its thread issued
 before it, an MMA after the earlier MMAs of its thread on the same
 accumulator, a copy at any time.  Buffers carry a version tag: every read
-states the version it must see, every write sets one.
+states the version it must see, every write sets one.  The work-item stream
+(cluster launch control responses in two slots, a full and an empty barrier
+each) is modelled for every role.  Each schedule gives every role a random
+speed, so that some fall far behind the others.
 
 Groups of threads that run the same code are modelled by a few agents each
 (two per column half of the compute warps, two dQ warps), so the barriers'
@@ -49,6 +52,10 @@ class Variant:
     # after issuer A's wait for DPE(g).
     pd_split: bool = False
     pd_split_early_dpe: bool = False  # mistake: DPE before the dS group reads P^T
+    # work items dealt in a fixed order (no mask) instead of taken through
+    # cluster launch control responses (causal)
+    static_items: bool = False
+    clc_no_empty_wait: bool = False   # request into a slot without its consumers' release
 
 
 class Barrier:
@@ -132,16 +139,87 @@ class AsyncWork:
         fn()
 
 
-def push_op(work, op):
-    """An ("async", unit, fn[, tag]) operation of a role."""
-    work.push(op[1], op[2], op[3] if len(op) > 3 else "commit")
+def item_request(world, t, dynamic, wait_empty=True):
+    """The producer, once work item t's loads are issued, asks for the item
+    after it (ItemStream::request): response k = t + 1 goes to slot k & 1,
+    whose previous response every consumer must have read first."""
+    if not dynamic:
+        return
+    k, slot, u = t + 1, (t + 1) & 1, t >> 1
+
+    if u >= 1 and wait_empty:
+        yield ("wait", [(f"CLCE{slot}", u - 1)])
+
+    def land(k=k, slot=slot, u=u):
+        world.write(("CLC", slot), k)
+        world.bar(f"CLCF{slot}").arrive(u)
+    yield ("async", "clc", land, "tma")
 
 
-def group_ready(op):
-    """A role's grouped wait: every barrier is tested (the kernel issues all
-    the tests before it looks at any result), and it passes when all pass."""
-    results = [W.bar(b).test(k) for b, k in op[1]]
-    return all(results)
+def item_advance(world, t, dynamic):
+    """Every role (one agent of it) after work item t: waits for response
+    t + 1, reads it and frees its slot (ItemStream::advance)."""
+    if not dynamic:
+        return
+    k, slot, u = t + 1, (t + 1) & 1, t >> 1
+    yield ("wait", [(f"CLCF{slot}", u)])
+    yield ("read", ("CLC", slot), k)
+    yield ("arrive", f"CLCE{slot}", u)
+
+
+def run_roles(world, roles, seed, in_order=False, max_steps=200000):
+    """Runs the roles (generators of operations) and their asynchronous work
+    under one random schedule; raises ProtocolError on a violation or a
+    deadlock.  Each schedule draws a speed for every role and for the
+    asynchronous units, so that some roles lag far behind the others (a
+    uniform choice at every step rarely lets one fall more than a few steps
+    behind)."""
+    rng = random.Random(seed)
+    speed = {name: rng.choice((0.02, 0.2, 1.0, 1.0, 1.0, 4.0)) for name in roles}
+    work_speed = rng.choice((0.1, 1.0, 1.0, 4.0))
+    nxt = {name: None for name in roles}       # pending operation of each role
+    work = AsyncWork(in_order)
+    done = set()
+
+    def advance(name):
+        try:
+            nxt[name] = next(roles[name])
+        except StopIteration:
+            nxt[name] = None
+            done.add(name)
+
+    def ready(op):
+        # the kernel issues every test of a grouped wait before it looks at
+        # any result, so every test is checked
+        return all([world.bar(b).test(k) for b, k in op[1]])
+
+    for name in roles:
+        advance(name)
+    for _ in range(max_steps):
+        if len(done) == len(roles) and not work.pending():
+            return
+        choices = [("role", n) for n, op in nxt.items()
+                   if op is not None and (op[0] != "wait" or ready(op))]
+        choices += [("work", r) for r in work.ready()]
+        if not choices:
+            raise ProtocolError("deadlock: pending " + str(
+                [(n, o[0], o[1] if o[0] == "wait" else "") for n, o in nxt.items() if o]))
+        weights = [speed[c[1]] if c[0] == "role" else work_speed for c in choices]
+        kind, name = rng.choices(choices, weights)[0]
+        if kind == "work":
+            work.complete(*name)
+            continue
+        op = nxt[name]
+        if op[0] == "arrive":
+            world.bar(op[1]).arrive(op[2])
+        elif op[0] == "async":
+            work.push(op[1], op[2], op[3] if len(op) > 3 else "commit")
+        elif op[0] == "read":
+            world.read(op[1], op[2])
+        elif op[0] == "write":
+            world.write(op[1], op[2])
+        advance(name)
+    raise ProtocolError("schedule did not finish")
 
 
 ST = 3          # Q / dO / statistics stages
@@ -190,6 +268,8 @@ def producer(plan, v):
         for _ in range(pre, n_it):
             yield from load_tile(g)
             g += 1
+        yield from item_request(W, item, not v.static_items, not v.clc_no_empty_wait)
+        yield from item_advance(W, item, not v.static_items)
 
 
 def issuer_a(plan, v):
@@ -224,6 +304,7 @@ def issuer_a(plan, v):
                 yield from mma_s(g1, item)
             g += 1
         yield ("async", "A", lambda item=item: W.bar("KVE", 2).arrive(item))
+        yield from item_advance(W, item, not v.static_items)
 
 
 def mma_s(g, item):
@@ -284,6 +365,7 @@ def issuer_b(plan, v):
             g += 1
         yield ("async", "B", lambda item=item: W.bar("FIN").arrive(item))
         yield ("async", "B", lambda item=item: W.bar("KVE", 2).arrive(item))
+        yield from item_advance(W, item, not v.static_items)
 
 
 def compute(agent, plan, v):
@@ -349,6 +431,7 @@ def compute(agent, plan, v):
                 W.bar("EPF").arrive(item)
             yield ("async", "store", store)
         yield ("wait", [("EPF", item)])
+        yield from item_advance(W, item, not v.static_items)
 
 
 def compute_p(q, plan, v):
@@ -385,6 +468,7 @@ def compute_p(q, plan, v):
                 W.bar("EPF").arrive(item)
             yield ("async", "store", store)
         yield ("wait", [("EPF", item)])
+        yield from item_advance(W, item, not v.static_items)
 
 
 def compute_ds(q, plan, v):
@@ -419,6 +503,7 @@ def compute_ds(q, plan, v):
         yield ("write", ("DS", 1, 1), ("dK", item))
         yield ("arrive", "EPS", item)
         yield ("wait", [("EPF", item)])
+        yield from item_advance(W, item, not v.static_items)
 
 
 def dq_role(agent, plan, v):
@@ -442,6 +527,7 @@ def dq_role(agent, plan, v):
                 if it + 1 == n_it:
                     yield ("arrive", "DQD", item)
             g += 1
+        yield from item_advance(W, item, not v.static_items)
 
 
 W = None  # the world of the schedule being run (the roles read it as a global)
@@ -465,9 +551,10 @@ def run_schedule(plan, seed, variant=None, max_steps=200000, in_order=False):
         half = NCOMP // 2      # 2 P agents, 2 dS agents
         counts.update({"PTF0": half, "PTF1": half, "DPE": half,
                        "DSF0": half, "DSF1": half, "ACCE": NCOMP, "EPS": NCOMP})
+    # one arrival per modelled agent frees a response slot
+    counts["CLCE0"] = counts["CLCE1"] = 3 + NCOMP + NDQ
     for name, c in counts.items():
         W.bar(name, c)
-    rng = random.Random(seed)
     roles = {"prod": producer(plan, v), "A": issuer_a(plan, v), "B": issuer_b(plan, v)}
     if v.pd_split:
         for q in range(NCOMP // 2):
@@ -478,43 +565,4 @@ def run_schedule(plan, seed, variant=None, max_steps=200000, in_order=False):
             roles[f"comp{a}"] = compute(a, plan, v)
     for a in range(NDQ):
         roles[f"dq{a}"] = dq_role(a, plan, v)
-    nxt = {name: None for name in roles}       # pending operation of each role
-    work = AsyncWork(in_order)
-    done = set()
-
-    def advance(name):
-        try:
-            nxt[name] = next(roles[name])
-        except StopIteration:
-            nxt[name] = None
-            done.add(name)
-
-    for name in roles:
-        advance(name)
-    for _ in range(max_steps):
-        if len(done) == len(roles) and not work.pending():
-            return
-        choices = []
-        for name, op in nxt.items():
-            if op is None:
-                continue
-            if op[0] != "wait" or group_ready(op):
-                choices.append(("role", name))
-        choices += [("work", r) for r in work.ready()]
-        if not choices:
-            raise ProtocolError(f"deadlock: pending {[(n, o[0], o[1] if o[0] == 'wait' else '') for n, o in nxt.items() if o]}")
-        kind, name = rng.choice(choices)
-        if kind == "work":
-            work.complete(*name)
-            continue
-        op = nxt[name]
-        if op[0] == "arrive":
-            W.bar(op[1]).arrive(op[2])
-        elif op[0] == "async":
-            push_op(work, op)
-        elif op[0] == "read":
-            W.read(op[1], op[2])
-        elif op[0] == "write":
-            W.write(op[1], op[2])
-        advance(name)
-    raise ProtocolError("schedule did not finish")
+    run_roles(W, roles, seed, in_order, max_steps)

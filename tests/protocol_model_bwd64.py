@@ -18,21 +18,24 @@ are outside the model.  Asynchronous work completes in any order the hardware
 allows (protocol_model.AsyncWork).
 """
 
-import random
 
-from protocol_model import AsyncWork, ProtocolError, World
+from protocol_model import ProtocolError, World, item_advance, item_request, run_roles
 
 QST = DOST = 2
 NCOMP = 4    # (half, quarter) agents
 
 
 class Variant:
-    def __init__(self, no_srd=False, no_dsf_wait=False, no_acce=False, s_without_dvd_wait=False):
+    def __init__(self, no_srd=False, no_dsf_wait=False, no_acce=False, s_without_dvd_wait=False,
+                 static_items=False):
         self.no_srd = no_srd              # mistake: half 1 writes P^T without the SRD wait
         self.no_dsf_wait = no_dsf_wait    # mistake: dK / dQ issued without waiting for dS^T
         # mistake: S^T(g+1) issued without waiting for dV(g), which reads P^T
         # from the same columns, trusting the issue order of one thread's MMAs
         self.s_without_dvd_wait = s_without_dvd_wait
+        # persistent design: items dealt in a fixed order (no mask) instead of
+        # taken through cluster launch control responses
+        self.static_items = static_items
         # persistent: the next item's first dV without the accumulator-release
         # wait.  Not a mistake: the compute warps read dV/dK in the epilogue
         # before they write the next item's P^T, which that dV waits for, so
@@ -41,6 +44,7 @@ class Variant:
 
 
 W = None
+persistent = False  # the schedule runs a list of items (the persistent design)
 
 
 def producer(plan, v):
@@ -70,6 +74,9 @@ def producer(plan, v):
                 W.bar(f"DOF{ds}").arrive(dn)
             yield ("async", "tma", land_do, "tma")
             g += 1
+        if persistent:
+            yield from item_request(W, item, not v.static_items)
+            yield from item_advance(W, item, not v.static_items)
 
 
 def issuer(plan, v):
@@ -137,6 +144,8 @@ def issuer(plan, v):
             g += 1
         yield ("async", "mma", lambda item=item: W.bar("FIN").arrive(item))
         yield ("async", "mma", lambda item=item: W.bar("KVE").arrive(item))
+        if persistent:
+            yield from item_advance(W, item, not v.static_items)
 
 
 def compute(agent, plan, v):
@@ -172,60 +181,25 @@ def compute(agent, plan, v):
         yield ("read", "DVACC", (item, n_it))
         yield ("read", "DKACC", (item, n_it))
         yield ("arrive", "ACCE", item)
+        if persistent:
+            yield from item_advance(W, item, not v.static_items)
 
 
 def run_schedule(plan, seed, variant=None, max_steps=200000, in_order=False):
     """plan: the number of 128-query tiles of one work item (an int: the kernel
     as it is, one item per CTA), or of each item a persistent CTA takes.
     in_order: complete each unit's asynchronous work in issue order."""
-    global W
+    global W, persistent
     v = variant or Variant()
+    persistent = not isinstance(plan, int)
     plan = [plan] if isinstance(plan, int) else list(plan)
     W = World()
     for name, c in {"PTF": NCOMP, "DSF": NCOMP, "DQE": NCOMP, "SRD": NCOMP // 2,
                     "ACCE": NCOMP}.items():
         W.bar(name, c)
-    rng = random.Random(seed)
+    W.bar("CLCE0", 2 + NCOMP)
+    W.bar("CLCE1", 2 + NCOMP)
     roles = {"prod": producer(plan, v), "mma": issuer(plan, v)}
     for a in range(NCOMP):
         roles[f"comp{a}"] = compute(a, plan, v)
-    nxt = {n: None for n in roles}
-    work = AsyncWork(in_order)
-    done = set()
-
-    def advance(name):
-        try:
-            nxt[name] = next(roles[name])
-        except StopIteration:
-            nxt[name] = None
-            done.add(name)
-
-    for name in roles:
-        advance(name)
-    for _ in range(max_steps):
-        if len(done) == len(roles) and not work.pending():
-            return
-        choices = []
-        for name, op in nxt.items():
-            if op is None:
-                continue
-            if op[0] != "wait" or all([W.bar(b).test(k) for b, k in op[1]]):
-                choices.append(("role", name))
-        choices += [("work", r) for r in work.ready()]
-        if not choices:
-            raise ProtocolError("deadlock: " + str([(n, o) for n, o in nxt.items() if o]))
-        kind, name = rng.choice(choices)
-        if kind == "work":
-            work.complete(*name)
-            continue
-        op = nxt[name]
-        if op[0] == "arrive":
-            W.bar(op[1]).arrive(op[2])
-        elif op[0] == "async":
-            work.push(op[1], op[2], op[3] if len(op) > 3 else "commit")
-        elif op[0] == "read":
-            W.read(op[1], op[2])
-        elif op[0] == "write":
-            W.write(op[1], op[2])
-        advance(name)
-    raise ProtocolError("schedule did not finish")
+    run_roles(W, roles, seed, in_order, max_steps)

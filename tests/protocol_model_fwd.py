@@ -22,7 +22,7 @@ the last pair of an odd tile count has nkv_1 = 0.
 
 import random
 
-from protocol_model import AsyncWork, ProtocolError, World
+from protocol_model import ProtocolError, World, item_advance, item_request, run_roles
 
 ST = 2      # K/V stages (d = 128)
 NSM = 2     # softmax agents per query tile
@@ -30,7 +30,8 @@ NSM = 2     # softmax agents per query tile
 
 class Variant:
     def __init__(self, ke_before_pv=False, epilogue_no_od_wait=False, split=False,
-                 split_no_exchange_wait=False, order_c=False, s_without_od_wait=False):
+                 split_no_exchange_wait=False, order_c=False, s_without_od_wait=False,
+                 static_items=False, clc_no_empty_wait=False):
         # release the K/V stage before the tile-1 P V of the step is issued
         self.ke_before_pv = ke_before_pv
         # the epilogue reads O without waiting for the last P V
@@ -51,6 +52,12 @@ class Variant:
         # its columns, trusting the issue order (which the hardware keeps only
         # between MMAs on the same accumulator)
         self.s_without_od_wait = s_without_od_wait
+        # work items dealt in a fixed order (no mask) instead of taken through
+        # cluster launch control responses
+        self.static_items = static_items
+        # mistake: ask for the next item into a response slot before every
+        # consumer has read the slot's previous response
+        self.clc_no_empty_wait = clc_no_empty_wait
 
 
 W = None
@@ -82,6 +89,8 @@ def producer(plan, v):
             yield ("async", "tma", land_k, "tma")
             yield ("async", "tma", land_v, "tma")
         kv += nkv
+        yield from item_request(W, item, not v.static_items, not v.clc_no_empty_wait)
+        yield from item_advance(W, item, not v.static_items)
 
 
 def issuer(plan, v):
@@ -170,6 +179,7 @@ def issuer(plan, v):
         for t in range(2):
             if nkv_t[t] > 0:
                 n_done[t] += 1
+        yield from item_advance(W, item, not v.static_items)
 
 
 def softmax(t, agent, plan, v, rng):
@@ -181,6 +191,7 @@ def softmax(t, agent, plan, v, rng):
         nkv = max(nk)
         if my == 0:
             kv += nkv
+            yield from item_advance(W, item, not v.static_items)
             continue
         for j in range(my):
             yield ("wait", [(f"SF{t}", n_s)])
@@ -198,6 +209,7 @@ def softmax(t, agent, plan, v, rng):
         yield ("arrive", f"OE{t}", done)
         done += 1
         kv += nkv
+        yield from item_advance(W, item, not v.static_items)
 
 
 def nagents(v):
@@ -212,6 +224,7 @@ def softmax_split(t, h, qq, plan, v, seed):
         my, nkv = nk[t], max(nk)
         if my == 0:
             kv += nkv
+            yield from item_advance(W, item, not v.static_items)
             continue
         for j in range(my):
             yield ("wait", [(f"SF{t}", n_s)])
@@ -239,6 +252,7 @@ def softmax_split(t, h, qq, plan, v, seed):
         yield ("arrive", f"OE{t}", done)
         done += 1
         kv += nkv
+        yield from item_advance(W, item, not v.static_items)
 
 
 def run_schedule(plan, seed, variant=None, max_steps=200000, in_order=False):
@@ -255,7 +269,10 @@ def run_schedule(plan, seed, variant=None, max_steps=200000, in_order=False):
             W.bar(f"LX{t}{qq}", 2)
             for sl in range(2):
                 W.bar(f"MX{t}{qq}{sl}", 2)
-    rng = random.Random(seed)
+    # one arrival per modelled agent frees a response slot
+    n_consumers = 2 + 2 * nagents(v)
+    W.bar("CLCE0", n_consumers)
+    W.bar("CLCE1", n_consumers)
     roles = {"prod": producer(plan, v), "mma": issuer(plan, v)}
     for t in range(2):
         if v.split:
@@ -265,43 +282,4 @@ def run_schedule(plan, seed, variant=None, max_steps=200000, in_order=False):
         else:
             for a in range(NSM):
                 roles[f"sm{t}{a}"] = softmax(t, a, plan, v, random.Random(seed * 7 + 2 * t + a))
-    nxt = {n: None for n in roles}
-    work = AsyncWork(in_order)
-    done = set()
-
-    def advance(name):
-        try:
-            nxt[name] = next(roles[name])
-        except StopIteration:
-            nxt[name] = None
-            done.add(name)
-
-    for name in roles:
-        advance(name)
-    for _ in range(max_steps):
-        if len(done) == len(roles) and not work.pending():
-            return
-        choices = []
-        for name, op in nxt.items():
-            if op is None:
-                continue
-            if op[0] != "wait" or all([W.bar(b).test(k) for b, k in op[1]]):
-                choices.append(("role", name))
-        choices += [("work", r) for r in work.ready()]
-        if not choices:
-            raise ProtocolError("deadlock: " + str([(n, o) for n, o in nxt.items() if o]))
-        kind, name = rng.choice(choices)
-        if kind == "work":
-            work.complete(*name)
-            continue
-        op = nxt[name]
-        if op[0] == "arrive":
-            W.bar(op[1]).arrive(op[2])
-        elif op[0] == "async":
-            work.push(op[1], op[2], op[3] if len(op) > 3 else "commit")
-        elif op[0] == "read":
-            W.read(op[1], op[2])
-        elif op[0] == "write":
-            W.write(op[1], op[2])
-        advance(name)
-    raise ProtocolError("schedule did not finish")
+    run_roles(W, roles, seed, in_order, max_steps)

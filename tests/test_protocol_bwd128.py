@@ -39,14 +39,21 @@ def test_pipelined_p_ds_groups_design_holds(plan):
         pm.run_schedule(plan, seed, pm.Variant(pd_split=True))
 
 
+def test_static_item_order_holds():
+    # without the mask the items are dealt in a fixed order: no response slots
+    for seed in range(100):
+        pm.run_schedule([3, 2, 4, 1], seed, pm.Variant(static_items=True))
+
+
 @pytest.mark.parametrize("mistake", ["single_srd", "single_dsf", "epilogue_tile_wait",
-                                     "pd_split_early_dpe"])
+                                     "pd_split_early_dpe", "clc_no_empty_wait"])
 def test_checker_rejects_known_mistakes(mistake):
     caught = 0
+    plan = [2, 1, 1, 3] if mistake.startswith("clc") else [3, 2, 4, 1]
     for seed in range(400):
         try:
             kw = {mistake: True, "pd_split": mistake.startswith("pd_split")}
-            pm.run_schedule([3, 2, 4, 1], seed, pm.Variant(**kw))
+            pm.run_schedule(plan, seed, pm.Variant(**kw))
         except pm.ProtocolError:
             caught += 1
     assert caught > 0, f"{mistake} was never caught"

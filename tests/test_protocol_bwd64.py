@@ -21,6 +21,12 @@ def test_persistent_d64_design_holds(plan):
         pm.run_schedule(plan, seed)
 
 
+def test_persistent_d64_static_item_order_holds():
+    # without the mask the items are dealt in a fixed order: no response slots
+    for seed in range(100):
+        pm.run_schedule([3, 1, 4, 2], seed, pm.Variant(static_items=True))
+
+
 def test_accumulator_release_is_implied_by_the_role_order():
     for seed in range(150):
         pm.run_schedule([3, 2, 4, 1], seed, pm.Variant(no_acce=True))

@@ -55,8 +55,14 @@ def test_next_s_needs_the_pv_wait_although_issued_later(order_c):
     assert caught > 0
 
 
+def test_static_item_order_holds():
+    # without the mask the items are dealt in a fixed order: no response slots
+    for seed in range(100):
+        pf.run_schedule(PLANS["noncausal"], seed, pf.Variant(static_items=True))
+
+
 @pytest.mark.parametrize("mistake", ["ke_before_pv", "epilogue_no_od_wait",
-                                     "split_no_exchange_wait"])
+                                     "split_no_exchange_wait", "clc_no_empty_wait"])
 def test_checker_rejects_forward_mistakes(mistake):
     caught = 0
     for seed in range(300):
