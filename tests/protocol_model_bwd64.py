@@ -13,8 +13,10 @@ one thread issues, per tile, S^T, dP^T, dV, then dK and dQ (in that order,
 each group after its barriers); the compute warps (two column halves x row
 quarters, modelled as four agents) write P^T over S^T (half 1 over columns half
 0 reads, after the shared-read barrier), dS^T into shared memory, and drain dQ
-into the accumulator.  The per-head completion counters after the epilogue
-are outside the model.  Asynchronous work completes in any order the hardware
+into the accumulator.  After the epilogue, every agent arrives at ENDA; agent
+0 counts the item on its head and publishes whether this CTA completed the
+head, and all read that flag after ENDB (the counter itself and the dQ
+conversion it gates are outside the model).  Asynchronous work completes in any order the hardware
 allows (protocol_model.AsyncWork).
 """
 
@@ -27,7 +29,7 @@ NCOMP = 4    # (half, quarter) agents
 
 class Variant:
     def __init__(self, no_srd=False, no_dsf_wait=False, no_acce=False, s_without_dvd_wait=False,
-                 static_items=False):
+                 static_items=False, flag_without_endb=False):
         self.no_srd = no_srd              # mistake: half 1 writes P^T without the SRD wait
         self.no_dsf_wait = no_dsf_wait    # mistake: dK / dQ issued without waiting for dS^T
         # mistake: S^T(g+1) issued without waiting for dV(g), which reads P^T
@@ -36,6 +38,8 @@ class Variant:
         # persistent design: items dealt in a fixed order (no mask) instead of
         # taken through cluster launch control responses
         self.static_items = static_items
+        # mistake: read the head-completion flag without waiting for ENDB
+        self.flag_without_endb = flag_without_endb
         # persistent: the next item's first dV without the accumulator-release
         # wait.  Not a mistake: the compute warps read dV/dK in the epilogue
         # before they write the next item's P^T, which that dV waits for, so
@@ -181,6 +185,17 @@ def compute(agent, plan, v):
         yield ("read", "DVACC", (item, n_it))
         yield ("read", "DKACC", (item, n_it))
         yield ("arrive", "ACCE", item)
+        # the end-of-item handshake: every agent has written its dK/dV rows
+        # (ENDA); agent 0 counts the item on its head and publishes whether the
+        # CTA finished the head (the flag); all read the flag after ENDB
+        yield ("arrive", "ENDA", item)
+        if agent == 0:
+            yield ("wait", [("ENDA", item)])
+            yield ("write", "LASTFLAG", item)
+            yield ("arrive", "ENDB", item)
+        if not v.flag_without_endb:
+            yield ("wait", [("ENDB", item)])
+        yield ("read", "LASTFLAG", item)
         if persistent:
             yield from item_advance(W, item, not v.static_items)
 
@@ -195,7 +210,7 @@ def run_schedule(plan, seed, variant=None, max_steps=200000, in_order=False):
     plan = [plan] if isinstance(plan, int) else list(plan)
     W = World()
     for name, c in {"PTF": NCOMP, "DSF": NCOMP, "DQE": NCOMP, "SRD": NCOMP // 2,
-                    "ACCE": NCOMP}.items():
+                    "ACCE": NCOMP, "ENDA": NCOMP}.items():
         W.bar(name, c)
     W.bar("CLCE0", 2 + NCOMP)
     W.bar("CLCE1", 2 + NCOMP)

@@ -32,7 +32,7 @@ def test_accumulator_release_is_implied_by_the_role_order():
         pm.run_schedule([3, 2, 4, 1], seed, pm.Variant(no_acce=True))
 
 
-@pytest.mark.parametrize("mistake", ["no_srd", "no_dsf_wait"])
+@pytest.mark.parametrize("mistake", ["no_srd", "no_dsf_wait", "flag_without_endb"])
 @pytest.mark.parametrize("plan", [5, [3, 2, 4, 1]], ids=["one-item", "persistent"])
 def test_checker_rejects_d64_mistakes(mistake, plan):
     caught = 0
