@@ -8,6 +8,7 @@ dQ, dK, dV relative L2 <= 1e-2.
 from __future__ import annotations
 
 import math
+import os
 
 import numpy as np
 
@@ -97,3 +98,43 @@ def sample_rows(BH, N, per_head=24, seed=1):
 
 def default_scale(d):
     return 1.0 / math.sqrt(d)
+
+
+def _exact(expr):
+    """Value of a fixture expression: numbers, + - * /, parentheses, log()."""
+    import ast
+
+    def ev(n):
+        if isinstance(n, ast.Expression):
+            return ev(n.body)
+        if isinstance(n, ast.Constant) and isinstance(n.value, (int, float)):
+            return float(n.value)
+        if isinstance(n, ast.UnaryOp) and isinstance(n.op, (ast.USub, ast.UAdd)):
+            return -ev(n.operand) if isinstance(n.op, ast.USub) else ev(n.operand)
+        if isinstance(n, ast.BinOp) and isinstance(n.op, (ast.Add, ast.Sub, ast.Mult, ast.Div)):
+            a, b = ev(n.left), ev(n.right)
+            return {ast.Add: a + b, ast.Sub: a - b, ast.Mult: a * b,
+                    ast.Div: a / b if b else math.nan}[type(n.op)]
+        if (isinstance(n, ast.Call) and isinstance(n.func, ast.Name) and n.func.id == "log"
+                and len(n.args) == 1):
+            return math.log(ev(n.args[0]))
+        raise ValueError(f"unsupported expression {expr!r}")
+    return ev(ast.parse(expr, mode="eval"))
+
+
+def load_worked_examples():
+    """The hand-worked examples of tests/golden/worked_examples.txt."""
+    path = os.path.join(os.path.dirname(__file__), "golden", "worked_examples.txt")
+    examples, cur = [], {}
+    for line in open(path, encoding="utf-8").read().splitlines() + [""]:
+        line = line.strip()
+        if line.startswith("#"):
+            continue
+        if not line:
+            if cur:
+                examples.append(cur)
+            cur = {}
+            continue
+        key, _, val = (x.strip() for x in line.partition("="))
+        cur[key] = val if key == "name" else np.array([_exact(t) for t in val.split()])
+    return examples

@@ -3,7 +3,9 @@
 Each mutant is a plausible slip (a dropped term, a wrong sign or index, a
 transposed operand); the copy is compiled to a temporary library on the
 CPU and checked with the same independent references the pins use
-(brute-force softmax and fp64 autograd).  The committed oracle is untouched.
+(brute-force softmax and fp64 autograd), and separately with the hand-worked
+exact examples of tests/golden/worked_examples.txt alone.  The committed
+oracle is untouched.
 """
 
 import ctypes
@@ -16,6 +18,8 @@ import numpy as np
 import pytest
 import scipy.special as sps
 import torch
+
+from helpers import load_worked_examples
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle", "attn_oracle.c")
 
@@ -87,3 +91,41 @@ def test_mutant_is_caught(name):
         text = f.read()
     assert text.count(old) >= 1, f"mutation site missing: {old}"
     assert not _pins_pass(_build(text.replace(old, new, 1)))
+
+
+def _worked_pass(L):
+    """The hand-worked examples, through the library's own entry points."""
+    P = lambda a: a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+    for ex in load_worked_examples():
+        N = ex["q"].size
+        q, k, v = (np.ascontiguousarray(ex[n], dtype=np.float64) for n in ("q", "k", "v"))
+        causal, scale = int(ex["causal"][0]), float(ex["scale"][0])
+        o, lse = np.empty(N), np.empty(N)
+        L.oracle_fwd(P(q), P(k), P(v), P(o), P(lse), 1, N, 1, causal, scale)
+        if not (np.allclose(o, ex["o"], rtol=0, atol=1e-13) and
+                np.allclose(lse, ex["lse"], rtol=0, atol=1e-13)):
+            return False
+        if "dout" in ex:
+            do = np.ascontiguousarray(ex["dout"], dtype=np.float64)
+            dq, dk, dv = np.empty(N), np.empty(N), np.empty(N)
+            heads = np.zeros(1, dtype=np.int64)
+            L.oracle_bwd_heads(P(q), P(k), P(v), P(do), 1, N, 1, causal, scale,
+                               heads.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), 1, P(dq),
+                               P(dk), P(dv))
+            for mine, want in ((dq, ex["dq"]), (dk, ex["dk"]), (dv, ex["dv"])):
+                if not np.allclose(mine, want, rtol=0, atol=1e-13):
+                    return False
+    return True
+
+
+def test_unmutated_copy_passes_worked_examples():
+    with open(SRC) as f:
+        assert _worked_pass(_build(f.read()))
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught_by_worked_examples(name):
+    old, new = MUTANTS[name]
+    with open(SRC) as f:
+        text = f.read()
+    assert not _worked_pass(_build(text.replace(old, new, 1)))

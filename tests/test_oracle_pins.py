@@ -3,9 +3,10 @@
 Each test ties the oracle to something the pages or mathematics fix:
 brute force on the full N x N matrix with library softmax/logsumexp,
 rows of P summing to one, the online recurrence equalling two passes,
-key permutation invariance, constant V, closed forms, a hand-worked
-two-key example, central finite differences and fp64 autograd of the
-brute-force definition for the gradients.
+key permutation invariance, constant V, closed forms, hand-worked
+examples with exact values (tests/golden/worked_examples.txt), central
+finite differences and fp64 autograd of the brute-force definition for the
+gradients.
 """
 
 import math
@@ -16,6 +17,7 @@ import scipy.special as sps
 import torch
 
 import oracle
+from helpers import load_worked_examples
 
 RNG = np.random.default_rng(12345)
 
@@ -124,25 +126,33 @@ def test_zero_query_gives_mean_of_visible_values(causal):
     np.testing.assert_allclose(lse[0, 0], np.log(cnt), rtol=0, atol=1e-14)
 
 
-def test_two_key_worked_example():
-    # q = 1 for both rows, keys 0 and ln 3, values 4 and 8, scale 1:
-    # weights 1/4, 3/4 -> O = 7, LSE = ln 4.  Causal row 0 sees key 0 only.
-    q = np.array([1.0, 1.0]).reshape(1, 1, 2, 1)
-    k = np.array([0.0, math.log(3.0)]).reshape(1, 1, 2, 1)
-    v = np.array([4.0, 8.0]).reshape(1, 1, 2, 1)
-    o, lse = oracle.fwd(q, k, v, False, 1.0)
-    np.testing.assert_allclose(o.ravel(), [7.0, 7.0], rtol=0, atol=1e-14)
-    np.testing.assert_allclose(lse.ravel(), [math.log(4.0)] * 2, rtol=0, atol=1e-15)
-    o, lse = oracle.fwd(q, k, v, True, 1.0)
-    np.testing.assert_allclose(o.ravel(), [4.0, 7.0], rtol=0, atol=1e-14)
-    np.testing.assert_allclose(lse.ravel(), [0.0, math.log(4.0)], rtol=0, atol=1e-15)
-    # Gradients of sum(O * dO) with dO = (1, 0): D_0 = 7, dP_0j = v_j,
-    # dS_00 = (1/4)(4 - 7) = -3/4, dS_01 = (3/4)(8 - 7) = 3/4.
-    dout = np.array([1.0, 0.0]).reshape(1, 1, 2, 1)
-    dq, dk, dv = oracle.bwd(q, k, v, dout, False, 1.0)
-    np.testing.assert_allclose(dq.ravel(), [0.75 * math.log(3.0), 0.0], rtol=0, atol=1e-14)
-    np.testing.assert_allclose(dk.ravel(), [-0.75, 0.75], rtol=0, atol=1e-14)
-    np.testing.assert_allclose(dv.ravel(), [0.25, 0.75], rtol=0, atol=1e-14)
+WORKED = load_worked_examples()
+
+
+def test_worked_examples_fixture_is_complete():
+    names = [e["name"] for e in WORKED]
+    assert names == ["two keys, non-causal", "two keys, causal", "two keys, scale 1/2",
+                     "three keys, non-causal", "three keys, causal"]
+    for e in WORKED:
+        assert {"causal", "scale", "q", "k", "v", "o", "lse"} <= set(e)
+
+
+@pytest.mark.parametrize("ex", WORKED, ids=lambda e: e["name"])
+def test_worked_example(ex):
+    """Exact values worked by hand from the definition (no numeric example is
+    printed on the pages); the derivations are in the fixture's header."""
+    N = ex["q"].size
+    t = {k: ex[k].reshape(1, 1, N, 1) for k in ("q", "k", "v")}
+    causal, scale = bool(ex["causal"][0]), float(ex["scale"][0])
+    o, lse = oracle.fwd(t["q"], t["k"], t["v"], causal, scale)
+    np.testing.assert_allclose(o.ravel(), ex["o"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(lse.ravel(), ex["lse"], rtol=0, atol=1e-14)
+    if "dout" in ex:
+        dq, dk, dv = oracle.bwd(t["q"], t["k"], t["v"], ex["dout"].reshape(1, 1, N, 1), causal,
+                                scale)
+        np.testing.assert_allclose(dq.ravel(), ex["dq"], rtol=0, atol=1e-14)
+        np.testing.assert_allclose(dk.ravel(), ex["dk"], rtol=0, atol=1e-14)
+        np.testing.assert_allclose(dv.ravel(), ex["dv"], rtol=0, atol=1e-14)
 
 
 def test_rows_subset_matches_full():
