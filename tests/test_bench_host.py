@@ -1,6 +1,7 @@
-"""Host-side logic of bench.py, on the CPU: the FLOP convention against the
-survey's per-config table, the traffic lookup and its invalidation when a
-kernel source changes, clock-sample parsing, and the weak-scaling helpers."""
+"""Host-side logic of bench.py, on the CPU: the FLOP convention against FLOP
+counts worked out by hand for the five workloads, the traffic lookup and its
+invalidation when a kernel source changes, clock-sample parsing, and the
+weak-scaling helpers."""
 
 import json
 import os
@@ -14,8 +15,9 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 import bench  # noqa: E402
 
-# (B, H, N, d, causal, forward GFLOP, fwd+bwd GFLOP or None), from the measurement
-# table of the survey (4 B H N^2 d forward, x 3.5 with the backward, halved causal)
+# (B, H, N, d, causal, forward GFLOP, fwd+bwd GFLOP or None), worked out by hand
+# to three significant digits (4 B H N^2 d forward, x 3.5 with the backward,
+# halved when causal)
 TABLE = [
     (1, 2, 256, 64, False, 0.0336, None),
     (8, 16, 512, 64, False, 8.59, None),
