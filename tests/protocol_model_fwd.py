@@ -25,13 +25,15 @@ import random
 from protocol_model import ProtocolError, World, item_advance, item_request, run_roles
 
 ST = 2      # K/V stages (d = 128)
+ST_DOUBLE = 4  # K/V stages of 64-key tiles (the s_double design)
 NSM = 2     # softmax agents per query tile
 
 
 class Variant:
     def __init__(self, ke_before_pv=False, epilogue_no_od_wait=False, split=False,
                  split_no_exchange_wait=False, order_c=False, s_without_od_wait=False,
-                 static_items=False, clc_no_empty_wait=False):
+                 static_items=False, clc_no_empty_wait=False, s_double=False,
+                 s_double_no_od_wait=False):
         # release the K/V stage before the tile-1 P V of the step is issued
         self.ke_before_pv = ke_before_pv
         # the epilogue reads O without waiting for the last P V
@@ -58,12 +60,25 @@ class Variant:
         # mistake: ask for the next item into a response slot before every
         # consumer has read the slot's previous response
         self.clc_no_empty_wait = clc_no_empty_wait
+        # design variant: 64-key K/V tiles (4 stages) and two S buffers per
+        # query tile, so S_t(j + 1) is computed while the softmax works on
+        # S_t(j); per key tile both P V, then both S_t(j + 2) (each after the
+        # P V that read its buffer)
+        self.s_double = s_double
+        # mistake for that design: S_t(j + 2) issued without waiting for
+        # P_t(j) V, which reads the same buffer
+        self.s_double_no_od_wait = s_double_no_od_wait
 
 
 W = None
 
 
+def stages(v):
+    return ST_DOUBLE if v.s_double else ST
+
+
 def producer(plan, v):
+    ST = stages(v)
     kv = 0
     for item, (n0, n1) in enumerate(plan):
         nkv = max(n0, n1)
@@ -182,6 +197,124 @@ def issuer(plan, v):
         yield from item_advance(W, item, not v.static_items)
 
 
+def issuer_sdouble(plan, v):
+    """The s_double design: S in two buffers per query tile."""
+    stg = stages(v)
+    kv = 0
+    n_pv, n_s, n_done = [0, 0], [0, 0], [0, 0]
+
+    def issue_s(t, kvi, item):
+        s, b, use = kvi % stg, n_s[t] & 1, n_s[t] >> 1
+
+        def run(t=t, kvi=kvi, s=s, b=b, item=item):
+            W.read("Q", item)
+            W.read(("K", s), kvi)
+            for a in range(nagents(v)):
+                W.write(("S", t, b, a), ("S", kvi))
+        yield ("async", "mma", run, f"S{t}{b}")
+        n_s[t] += 1
+        yield ("async", "mma", lambda t=t, b=b, use=use: W.bar(f"SF{t}{b}").arrive(use))
+
+    for item, (n0, n1) in enumerate(plan):
+        nkv_t = (n0, n1)
+        nkv = max(n0, n1)
+        base = list(n_s)  # S count of each tile at the item's start
+        # the previous item's last P V (committed after every earlier one)
+        # read the buffers the first S take
+        waits = [("Q", item), (f"KF{kv % stg}", kv // stg)]
+        for t in range(2):
+            if nkv_t[t] > 0 and n_pv[t] > 0:
+                last = n_pv[t] - 1
+                waits.append((f"OD{t}{last & 1}", last >> 1))
+        yield ("wait", waits)
+        for t in range(2):
+            if nkv_t[t] > 0:
+                yield from issue_s(t, kv, item)
+        if nkv > 1:
+            yield ("wait", [(f"KF{(kv + 1) % stg}", (kv + 1) // stg)])
+            for t in range(2):
+                if nkv_t[t] > 1:
+                    yield from issue_s(t, kv + 1, item)
+        for j in range(nkv):
+            kvj = kv + j
+            s, n = kvj % stg, kvj // stg
+            for t in range(2):
+                act = j < nkv_t[t]
+                waits = []
+                if t == 0:
+                    waits.append((f"VF{s}", n))
+                b = (base[t] + j) & 1
+                if act:
+                    # P ready, one barrier per S buffer: with S(j + 1) computed
+                    # early, one agent can run a step ahead of another
+                    waits.append((f"PF{t}{b}", n_pv[t] >> 1))
+                    if j == 0 and n_done[t] > 0:
+                        waits.append((f"OE{t}", n_done[t] - 1))
+                if waits:
+                    yield ("wait", waits)
+                if not act:
+                    continue
+
+                def pv(t=t, kvj=kvj, s=s, b=b, item=item, j=j):
+                    for a in range(nagents(v)):
+                        W.read(("S", t, b, a), ("P", kvj))
+                    W.read(("V", s), kvj)
+                    W.write(("O", t, 0), (item, j + 1))
+                yield ("async", "mma", pv, f"O{t}")
+                k = n_pv[t]
+                n_pv[t] += 1
+                # P V done, one barrier per S buffer: two P V of a tile can be
+                # in flight, and a parity test is only valid for the newest
+                # phase or the one before
+                yield ("async", "mma", lambda t=t, k=k: W.bar(f"OD{t}{k & 1}").arrive(k >> 1))
+            yield ("async", "mma", lambda s=s, n=n: W.bar(f"KE{s}").arrive(n))
+            k2, k_waited = kvj + 2, False
+            for t in range(2):
+                if j + 2 < nkv_t[t]:
+                    k = n_pv[t] - 1
+                    waits = [] if v.s_double_no_od_wait else [(f"OD{t}{k & 1}", k >> 1)]
+                    if not k_waited:
+                        waits.append((f"KF{k2 % stg}", k2 // stg))
+                    k_waited = True
+                    yield ("wait", waits)
+                    yield from issue_s(t, k2, item)
+        yield ("async", "mma", lambda item=item: W.bar("QE").arrive(item))
+        kv += nkv
+        for t in range(2):
+            if nkv_t[t] > 0:
+                n_done[t] += 1
+        yield from item_advance(W, item, not v.static_items)
+
+
+def softmax_sdouble(t, agent, plan, v, rng):
+    kv = n_s = done = 0
+    for item, nk in enumerate(plan):
+        my, nkv = nk[t], max(nk)
+        if my == 0:
+            kv += nkv
+            yield from item_advance(W, item, not v.static_items)
+            continue
+        for j in range(my):
+            b, use = n_s & 1, n_s >> 1
+            yield ("wait", [(f"SF{t}{b}", use)])
+            n_s += 1
+            yield ("read", ("S", t, b, agent), ("S", kv + j))
+            if j > 0 and rng.random() < 0.3:
+                # the kept max moves: O is rescaled, which needs P V(j-1)
+                k = n_s - 2
+                yield ("wait", [(f"OD{t}{k & 1}", k >> 1)])
+                yield ("read", ("O", t, 0), (item, j))
+            yield ("write", ("S", t, b, agent), ("P", kv + j))
+            yield ("arrive", f"PF{t}{b}", use)
+        k = n_s - 1
+        yield ("wait", [(f"OD{t}{k & 1}", k >> 1)])
+        yield ("read", ("O", t, 0), (item, my))
+        yield ("arrive", f"OE{t}", done)
+        done += 1
+        kv += nkv
+        yield from item_advance(W, item, not v.static_items)
+
+
 def softmax(t, agent, plan, v, rng):
     kv = 0
     n_s = 0
@@ -264,6 +397,8 @@ def run_schedule(plan, seed, variant=None, max_steps=200000, in_order=False):
     W = World()
     for t in range(2):
         W.bar(f"PF{t}", nagents(v))
+        for b in range(2):
+            W.bar(f"PF{t}{b}", nagents(v))
         W.bar(f"OE{t}", nagents(v))
         for qq in range(NSM):
             W.bar(f"LX{t}{qq}", 2)
@@ -273,9 +408,14 @@ def run_schedule(plan, seed, variant=None, max_steps=200000, in_order=False):
     n_consumers = 2 + 2 * nagents(v)
     W.bar("CLCE0", n_consumers)
     W.bar("CLCE1", n_consumers)
-    roles = {"prod": producer(plan, v), "mma": issuer(plan, v)}
+    roles = {"prod": producer(plan, v),
+             "mma": issuer_sdouble(plan, v) if v.s_double else issuer(plan, v)}
     for t in range(2):
-        if v.split:
+        if v.s_double:
+            for a in range(NSM):
+                roles[f"sm{t}{a}"] = softmax_sdouble(t, a, plan, v,
+                                                     random.Random(seed * 7 + 2 * t + a))
+        elif v.split:
             for h in range(2):
                 for qq in range(NSM):
                     roles[f"sm{t}{h}{qq}"] = softmax_split(t, h, qq, plan, v, seed)

@@ -55,6 +55,32 @@ def test_next_s_needs_the_pv_wait_although_issued_later(order_c):
     assert caught > 0
 
 
+SD_PLANS = {
+    "noncausal": [(6, 6), (6, 6), (2, 2)],
+    "causal": [(2, 4), (6, 8), (10, 0)],
+    "causal-repeat": [(3, 5), (3, 5), (1, 1), (8, 10)],
+}
+
+
+@pytest.mark.parametrize("name", sorted(SD_PLANS))
+def test_double_buffered_s_design_holds(name):
+    # next-step design: 64-key tiles, two S buffers per query tile; P ready and
+    # P V done are one barrier per S buffer
+    for seed in range(120):
+        pf.run_schedule(SD_PLANS[name], seed, pf.Variant(s_double=True))
+
+
+def test_double_buffered_s_needs_the_pv_wait():
+    caught = 0
+    for seed in range(300):
+        try:
+            pf.run_schedule(SD_PLANS["causal"], seed,
+                            pf.Variant(s_double=True, s_double_no_od_wait=True))
+        except pf.ProtocolError:
+            caught += 1
+    assert caught > 0
+
+
 def test_static_item_order_holds():
     # without the mask the items are dealt in a fixed order: no response slots
     for seed in range(100):
