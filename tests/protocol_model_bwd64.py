@@ -53,7 +53,30 @@ persistent = False  # the schedule runs a list of items (the persistent design)
 
 def producer(plan, v):
     g = 0
+
+    def load_tile(g):
+        qs, qn, ds, dn = g % QST, g // QST, g % DOST, g // DOST
+        yield ("wait", [(f"QE{qs}", qn - 1)])
+
+        def land_q(g=g, qs=qs, qn=qn):
+            W.write(("Q", qs), g)
+            W.write(("LD", qs), g)
+            W.bar(f"QF{qs}").arrive(qn)
+        yield ("async", "tma", land_q, "tma")
+        yield ("wait", [(f"DOE{ds}", dn - 1)])
+
+        def land_do(g=g, ds=ds, dn=dn):
+            W.write(("DO", ds), g)
+            W.bar(f"DOF{ds}").arrive(dn)
+        yield ("async", "tma", land_do, "tma")
+
     for item, n_it in enumerate(plan):
+        # the persistent design loads an item's first query tiles ahead of its
+        # K/V, which wait until the previous item's MMAs are done with K and V
+        pre = min(QST, n_it) if persistent else 0
+        for _ in range(pre):
+            yield from load_tile(g)
+            g += 1
         if item > 0:
             yield ("wait", [("KVE", item - 1)])
 
@@ -62,21 +85,8 @@ def producer(plan, v):
             W.write("V", item)
             W.bar("KV").arrive(item)
         yield ("async", "tma", land_kv, "tma")
-        for _ in range(n_it):
-            qs, qn, ds, dn = g % QST, g // QST, g % DOST, g // DOST
-            yield ("wait", [(f"QE{qs}", qn - 1)])
-
-            def land_q(g=g, qs=qs, qn=qn):
-                W.write(("Q", qs), g)
-                W.write(("LD", qs), g)
-                W.bar(f"QF{qs}").arrive(qn)
-            yield ("async", "tma", land_q, "tma")
-            yield ("wait", [(f"DOE{ds}", dn - 1)])
-
-            def land_do(g=g, ds=ds, dn=dn):
-                W.write(("DO", ds), g)
-                W.bar(f"DOF{ds}").arrive(dn)
-            yield ("async", "tma", land_do, "tma")
+        for _ in range(pre, n_it):
+            yield from load_tile(g)
             g += 1
         if persistent:
             yield from item_request(W, item, not v.static_items)
