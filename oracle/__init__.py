@@ -37,6 +37,12 @@ def lib():
         L.oracle_fwd_online.restype = None
         L.oracle_bwd_heads.argtypes = [dp, dp, dp, dp, i64, i64, i64, ci, cd, lp, i64, dp, dp, dp]
         L.oracle_bwd_heads.restype = None
+        u8 = ctypes.POINTER(ctypes.c_uint8)
+        L.oracle_fwd_blocksparse.argtypes = [dp, dp, dp, dp, dp, i64, i64, i64, ci, cd, u8, i64]
+        L.oracle_fwd_blocksparse.restype = None
+        L.oracle_bwd_blocksparse_heads.argtypes = [dp, dp, dp, dp, i64, i64, i64, ci, cd, u8, i64,
+                                                   lp, i64, dp, dp, dp]
+        L.oracle_bwd_blocksparse_heads.restype = None
         L.oracle_num_threads.argtypes = []
         L.oracle_num_threads.restype = ci
         L.oracle_set_num_threads.argtypes = [ci]
@@ -130,4 +136,54 @@ def bwd(q, k, v, dout, causal: bool, scale: float):
     """Exact gradients for every head, shaped like q."""
     shape = np.shape(q)
     dq, dk, dv = bwd_heads(q, k, v, dout, causal, scale)
+    return dq.reshape(shape), dk.reshape(shape), dv.reshape(shape)
+
+
+def _block_mask(mask, N, blk):
+    mask = np.ascontiguousarray(mask, dtype=np.uint8)
+    nb = (N + blk - 1) // blk
+    if mask.shape != (nb, nb):
+        raise ValueError(f"block mask must be ({nb}, {nb}) for N={N}, block {blk}")
+    return mask
+
+
+def fwd_blocksparse(q, k, v, mask, causal: bool, scale: float, block: int = 128):
+    """Block-sparse forward: key j is visible to query i iff
+    mask[i // block, j // block] != 0 (and j <= i when causal).  Rows with no
+    visible key get O = 0 and LSE = -inf.  Returns (O, LSE)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    BH, N, d = _dims(q)
+    mask = _block_mask(mask, N, block)
+    o = np.empty_like(q)
+    lse = np.empty(q.shape[:-1], dtype=np.float64)
+    lib().oracle_fwd_blocksparse(_p(q), _p(k), _p(v), _p(o), _p(lse), BH, N, d,
+                                 int(bool(causal)), float(scale), _p(mask, ctypes.c_uint8),
+                                 int(block))
+    return o, lse
+
+
+def bwd_blocksparse_heads(q, k, v, dout, mask, causal: bool, scale: float, heads=None,
+                          block: int = 128):
+    """Exact gradients of sum(O * dO) under the block mask, for the listed heads."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    BH, N, d = _dims(q)
+    mask = _block_mask(mask, N, block)
+    if heads is None:
+        heads = np.arange(BH)
+    heads = np.ascontiguousarray(heads, dtype=np.int64)
+    if heads.size and (heads.min() < 0 or heads.max() >= BH):
+        raise IndexError("head index out of range")
+    shp = (heads.size, N, d)
+    dq, dk, dv = np.empty(shp), np.empty(shp), np.empty(shp)
+    lib().oracle_bwd_blocksparse_heads(_p(q), _p(k), _p(v), _p(dout), BH, N, d,
+                                       int(bool(causal)), float(scale), _p(mask, ctypes.c_uint8),
+                                       int(block), _p(heads, ctypes.c_int64), heads.size,
+                                       _p(dq), _p(dk), _p(dv))
+    return dq, dk, dv
+
+
+def bwd_blocksparse(q, k, v, dout, mask, causal: bool, scale: float, block: int = 128):
+    """Block-sparse gradients for every head, shaped like q."""
+    shape = np.shape(q)
+    dq, dk, dv = bwd_blocksparse_heads(q, k, v, dout, mask, causal, scale, block=block)
     return dq.reshape(shape), dk.reshape(shape), dv.reshape(shape)

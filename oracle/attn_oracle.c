@@ -236,6 +236,151 @@ void oracle_bwd_heads(const double* q, const double* k, const double* v, const d
     free(part);
 }
 
+/*
+ * Block-sparse attention: "FlashAttention の概要" (zenn.dev), the paragraph on
+ * Block-Sparse FlashAttention, which approximates attention by computing only
+ * the (query block, key block) pairs a block mask marks and is otherwise the
+ * same algorithm.  The page describes no more; the readings taken here:
+ *  - one mask for every (batch, head): mask[(i / blk) * nb + (j / blk)] != 0
+ *    marks the pair of query block i / blk and key block j / blk, with
+ *    nb = ceil(N / blk) blocks per side;
+ *  - key j is visible to query i iff its block pair is marked and, with the
+ *    causal flag, j <= i (the causal rule of "causal masking" on the
+ *    marketmaker.cc page still applies inside marked blocks);
+ *  - over the visible keys the result is exact softmax attention; a row with
+ *    no visible key has O = 0 and LSE = -inf (the empty sum).
+ * The forward and backward below are the definitions above written out on an
+ * explicit list of each row's visible keys.
+ */
+static int64_t visible_list(int64_t i, int64_t N, int causal, const uint8_t* mask, int64_t blk,
+                            int64_t* idx) {
+    int64_t nb = (N + blk - 1) / blk, n = 0;
+    for (int64_t j = 0; j < N; ++j)
+        if (mask[(i / blk) * nb + j / blk] && (!causal || j <= i)) idx[n++] = j;
+    return n;
+}
+
+/* One query row over the keys idx[0..nvis): s[0..nvis) gets P, returns LSE. */
+static double row_forward_list(const double* qi, const double* K, const double* V,
+                               const int64_t* idx, int64_t nvis, int64_t d, double scale,
+                               double* s, double* oi) {
+    for (int64_t t = 0; t < d; ++t) oi[t] = 0.0;
+    if (nvis == 0) return -INFINITY;
+    double M = -INFINITY;
+    for (int64_t r = 0; r < nvis; ++r) {          /* scores and pass 1: max */
+        s[r] = scale * dot(qi, K + idx[r] * d, d);
+        if (s[r] > M) M = s[r];
+    }
+    double Z = 0.0;
+    for (int64_t r = 0; r < nvis; ++r) {          /* pass 2: exponentiate, sum */
+        s[r] = exp(s[r] - M);
+        Z += s[r];
+    }
+    for (int64_t r = 0; r < nvis; ++r) {          /* normalise, weight V */
+        s[r] /= Z;
+        const double* vj = V + idx[r] * d;
+        for (int64_t t = 0; t < d; ++t) oi[t] += s[r] * vj[t];
+    }
+    return M + log(Z);
+}
+
+/* Block-sparse forward: O (BH, N, d), LSE (BH, N). */
+void oracle_fwd_blocksparse(const double* q, const double* k, const double* v, double* o,
+                            double* lse, int64_t BH, int64_t N, int64_t d, int causal,
+                            double scale, const uint8_t* mask, int64_t blk) {
+#pragma omp parallel
+    {
+        double* s = (double*)malloc((size_t)N * sizeof(double));
+        int64_t* idx = (int64_t*)malloc((size_t)N * sizeof(int64_t));
+#pragma omp for collapse(2) schedule(dynamic, 16)
+        for (int64_t bh = 0; bh < BH; ++bh)
+            for (int64_t i = 0; i < N; ++i) {
+                int64_t row = bh * N + i;
+                int64_t nv = visible_list(i, N, causal, mask, blk, idx);
+                lse[row] = row_forward_list(q + row * d, k + bh * N * d, v + bh * N * d, idx, nv,
+                                            d, scale, s, o + row * d);
+            }
+        free(idx);
+        free(s);
+    }
+}
+
+/* Block-sparse backward of L = sum(O * dO) for the listed heads; same chain
+ * rule as oracle_bwd_heads, over each row's visible keys only. */
+void oracle_bwd_blocksparse_heads(const double* q, const double* k, const double* v,
+                                  const double* dout, int64_t BH, int64_t N, int64_t d,
+                                  int causal, double scale, const uint8_t* mask, int64_t blk,
+                                  const int64_t* heads, int64_t nheads, double* dq, double* dk,
+                                  double* dv) {
+    (void)BH;
+    int nthr = 1;
+#ifdef _OPENMP
+    nthr = omp_get_max_threads();
+#endif
+    size_t nd = (size_t)N * (size_t)d;
+    double* part = (double*)calloc((size_t)nthr * 2 * nd, sizeof(double));
+    for (int64_t hh = 0; hh < nheads; ++hh) {
+        int64_t bh = heads[hh];
+        const double* Q = q + bh * N * d;
+        const double* K = k + bh * N * d;
+        const double* V = v + bh * N * d;
+        const double* dO = dout + bh * N * d;
+        double* dQ = dq + hh * N * d;
+        memset(part, 0, (size_t)nthr * 2 * nd * sizeof(double));
+#pragma omp parallel
+        {
+            int tid = 0;
+#ifdef _OPENMP
+            tid = omp_get_thread_num();
+#endif
+            double* dKp = part + (size_t)tid * 2 * nd;
+            double* dVp = dKp + nd;
+            double* p = (double*)malloc((size_t)N * sizeof(double));
+            int64_t* idx = (int64_t*)malloc((size_t)N * sizeof(int64_t));
+            double* oi = (double*)malloc((size_t)d * sizeof(double));
+#pragma omp for schedule(dynamic, 8)
+            for (int64_t i = 0; i < N; ++i) {
+                int64_t nv = visible_list(i, N, causal, mask, blk, idx);
+                const double* qi = Q + i * d;
+                const double* doi = dO + i * d;
+                row_forward_list(qi, K, V, idx, nv, d, scale, p, oi);
+                double Di = dot(doi, oi, d);
+                double* dqi = dQ + i * d;
+                for (int64_t t = 0; t < d; ++t) dqi[t] = 0.0;
+                for (int64_t r = 0; r < nv; ++r) {
+                    int64_t j = idx[r];
+                    const double* vj = V + j * d;
+                    const double* kj = K + j * d;
+                    double dpij = dot(doi, vj, d);
+                    double dsij = p[r] * (dpij - Di);
+                    double* dkj = dKp + j * d;
+                    double* dvj = dVp + j * d;
+                    for (int64_t t = 0; t < d; ++t) {
+                        dqi[t] += scale * dsij * kj[t];
+                        dkj[t] += scale * dsij * qi[t];
+                        dvj[t] += p[r] * doi[t];
+                    }
+                }
+            }
+            free(oi);
+            free(idx);
+            free(p);
+        }
+        double* dK = dk + hh * N * d;
+        double* dV = dv + hh * N * d;
+        for (size_t e = 0; e < nd; ++e) {
+            double sk = 0.0, sv = 0.0;
+            for (int t = 0; t < nthr; ++t) {
+                sk += part[(size_t)t * 2 * nd + e];
+                sv += part[(size_t)t * 2 * nd + nd + e];
+            }
+            dK[e] = sk;
+            dV[e] = sv;
+        }
+    }
+    free(part);
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

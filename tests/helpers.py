@@ -138,3 +138,75 @@ def load_worked_examples():
         key, _, val = (x.strip() for x in line.partition("="))
         cur[key] = val if key == "name" else np.array([_exact(t) for t in val.split()])
     return examples
+
+
+# ---- inputs that make the forward move its running max (and rescale O) ------
+# The forward keeps a stale running max until a key tile's row max exceeds it
+# by more than 2^8 (8 in log2 units), then moves it and rescales the output
+# accumulator.  Gaussian inputs at the workloads' sigma never get there; these
+# patterns do, in many rows and several times per row.
+RESCALE_LOG2_THRESHOLD = 8.0
+
+
+def rescale_inputs(pattern, B, H, N, d, dtype="bf16", seed=0):
+    """Seeded Q, K, V, dO (storage arrays and exact f64 values) shaped so that
+    row maxima keep growing along the keys.
+
+    ``ramp``: key row j is scaled by 1 + 3 j / 64, so each later key tile
+    holds larger scores; odd query rows are scaled by 0.2, so within a warp
+    some rows move their max at a tile and others do not.
+    ``shared``: K = Q (sigma 1.2), so under the causal mask a row's own
+    diagonal score (about sqrt(d) sigma^2) dwarfs those of the first key tile.
+    """
+    arrs = synth.attention_inputs(B, H, N, d, seed=seed, sigma=1.0, dtype=dtype, with_dout=True)
+    z = [synth.to_f64(a, dtype) for a in arrs]
+    if pattern == "ramp":
+        rq = np.where(np.arange(N) % 2 == 0, 1.0, 0.2)[:, None]
+        rk = (1.0 + 3.0 * np.arange(N) / 64.0)[:, None]
+        q, k = z[0] * rq, z[1] * rk
+    elif pattern == "shared":
+        q = z[0] * 1.2
+        k = q
+    else:
+        raise ValueError(pattern)
+
+    def store(x):
+        return synth.round_bf16_bits(x) if dtype == "bf16" else x.astype(np.float16)
+
+    stored = [store(q), store(k), arrs[2], arrs[3]]
+    return stored, [synth.to_f64(a, dtype) for a in stored]
+
+
+def rescale_moves(q, k, causal, scale, key_tile, margin=0.05):
+    """For one head (q, k: (N, d) f64), replay the forward's max-keeping rule
+    over key tiles of ``key_tile`` columns in fp64.  Returns boolean arrays
+    (N, tiles): ``moved[i, j]`` where row i's max surely moves at tile j > 0
+    (growth above the threshold by ``margin``) and ``kept[i, j]`` where it
+    surely stays (growth below it by ``margin``)."""
+    N = q.shape[0]
+    s = (q @ k.T) * scale / math.log(2.0)
+    if causal:
+        s = np.where(np.arange(N)[None, :] <= np.arange(N)[:, None], s, -np.inf)
+    nt = (N + key_tile - 1) // key_tile
+    tmax = np.stack([s[:, j * key_tile:(j + 1) * key_tile].max(1) for j in range(nt)], 1)
+    moved = np.zeros((N, nt), bool)
+    kept = np.zeros((N, nt), bool)
+    m = tmax[:, 0].copy()
+    for j in range(1, nt):
+        vis = np.isfinite(tmax[:, j])
+        grow = tmax[:, j] - m
+        moved[:, j] = vis & (grow > RESCALE_LOG2_THRESHOLD + margin)
+        kept[:, j] = vis & (grow < RESCALE_LOG2_THRESHOLD - margin)
+        m = np.where(vis & (grow > RESCALE_LOG2_THRESHOLD), tmax[:, j], m)
+    return moved, kept
+
+
+def mixed_warps(moved, kept):
+    """Count (32-row warp, key tile) pairs where some rows surely move their
+    max and others surely keep it."""
+    N, nt = moved.shape
+    n = 0
+    for r0 in range(0, N - 31, 32):
+        for j in range(1, nt):
+            n += bool(moved[r0:r0 + 32, j].any() and kept[r0:r0 + 32, j].any())
+    return n

@@ -10,7 +10,7 @@ import numpy as np
 import pytest
 
 import oracle
-from helpers import CONFIGS, check_grads, default_scale, inputs, to_device
+from helpers import CONFIGS, check_fwd, check_grads, default_scale, inputs, to_device
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -57,7 +57,7 @@ def test_bwd_small_full_compare(B, H, N, d, causal, dtype):
     check_grads(g, ref, f"{(B, H, N, d, causal, dtype)}")
 
 
-@pytest.mark.parametrize("name,heads", [("gpt2_causal", [0, 50, 95]), ("large_head", [0, 63])])
+@pytest.mark.parametrize("name,heads", [("gpt2_causal", [0, 47, 50, 95]), ("large_head", [0, 31, 63])])
 def test_bwd_full_size_selected_heads(name, heads):
     B, H, N, d, causal, dtype, sigma, with_bwd = CONFIGS[name]
     assert with_bwd
@@ -116,8 +116,7 @@ def test_fwd_bwd_many_items_per_cta(B, H, N, d, causal):
         b, h = divmod(bh, H)
         sel = [x[b:b + 1, h:h + 1] for x in f64]
         o_ref, lse_ref = oracle.fwd(*sel[:3], causal, scale)
-        o_err = float(np.abs(got[0][b:b + 1, h:h + 1] - o_ref).max())
-        l_err = float(np.abs(got[1][b:b + 1, h:h + 1] - lse_ref).max())
-        assert o_err <= 1e-2 and l_err <= 1e-3, (bh, o_err, l_err)
+        check_fwd(got[0][b:b + 1, h:h + 1], got[1][b:b + 1, h:h + 1], o_ref, lse_ref,
+                  f"{(B, H, N, d, causal)} head {bh}")
         ref = oracle.bwd(*sel, causal, scale)
         check_grads([x[b:b + 1, h:h + 1] for x in got[2:]], ref, f"{(B, H, N, d, causal)} head {bh}")

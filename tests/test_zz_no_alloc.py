@@ -7,7 +7,8 @@ runs.  For them the library keeps a fixed scratch array of its own on each
 device.  These tests call that entry point through the C ABI and check that
 it gives the same gradients as attn_bwd with a caller-supplied workspace,
 twice in a row (the second call starts from whatever the first left in the
-shared array), and that a problem too big for the array is refused.
+shared array), that those gradients also match the fp64 oracle, and that a
+problem too big for the array is refused.
 
 This file is collected last on purpose, and passes alone or after the rest.
 """
@@ -17,7 +18,8 @@ import ctypes
 import numpy as np
 import pytest
 
-from helpers import GRAD_REL_L2, inputs, rel_l2, to_device
+import oracle
+from helpers import GRAD_REL_L2, check_grads, default_scale, inputs, rel_l2, to_device
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -29,7 +31,7 @@ from io_aware_exact_30_b200 import attn  # noqa: E402
                                                   (1, 4, 1029, 64, True, "fp16")])
 def test_noalloc_matches_workspace_backward_twice(B, H, N, d, causal, dtype):
     assert attn.attn_bwd_workspace_bytes(B, H, N, d) <= attn.NOALLOC_SCRATCH_BYTES
-    arrs, _ = inputs(B, H, N, d, dtype=dtype, seed=N, with_dout=True)
+    arrs, f64 = inputs(B, H, N, d, dtype=dtype, seed=N, with_dout=True)
     q, k, v, do = (to_device(a, dtype) for a in arrs)
     o, lse = attn.forward(q, k, v, causal)
     ref = attn.backward(q, k, v, o, lse, do, causal)  # existing entry point, own workspace
@@ -45,6 +47,10 @@ def test_noalloc_matches_workspace_backward_twice(B, H, N, d, causal, dtype):
             assert np.all(np.isfinite(got)), (call, name)
             err = rel_l2(got, want)
             assert err <= GRAD_REL_L2, f"call {call} {name} rel-L2 {err}"
+        if call == 1:  # and against the oracle, on the last head
+            exact = oracle.bwd_heads(*f64, causal, default_scale(d), heads=[B * H - 1])
+            got = [t.double().cpu().numpy().reshape(B * H, N, d)[-1:] for t in (dq, dk, dv)]
+            check_grads(got, exact, f"noalloc {(B, H, N, d, causal, dtype)}")
 
 
 def test_noalloc_refuses_problems_larger_than_its_scratch():
