@@ -43,6 +43,14 @@ def lib():
         L.oracle_bwd_blocksparse_heads.argtypes = [dp, dp, dp, dp, i64, i64, i64, ci, cd, u8, i64,
                                                    lp, i64, dp, dp, dp]
         L.oracle_bwd_blocksparse_heads.restype = None
+        fp = ctypes.POINTER(ctypes.c_float)
+        L.oracle_e4m3_round.argtypes = [ctypes.c_float]
+        L.oracle_e4m3_round.restype = ctypes.c_float
+        L.oracle_fwht32.argtypes = [fp, i64, i64]
+        L.oracle_fwht32.restype = None
+        L.oracle_fp8_quantize.argtypes = [dp, i64, i64, i64, ctypes.POINTER(ctypes.c_int8), ci,
+                                          fp, fp]
+        L.oracle_fp8_quantize.restype = None
         L.oracle_num_threads.argtypes = []
         L.oracle_num_threads.restype = ci
         L.oracle_set_num_threads.argtypes = [ci]
@@ -187,3 +195,56 @@ def bwd_blocksparse(q, k, v, dout, mask, causal: bool, scale: float, block: int 
     shape = np.shape(q)
     dq, dk, dv = bwd_blocksparse_heads(q, k, v, dout, mask, causal, scale, block=block)
     return dq.reshape(shape), dk.reshape(shape), dv.reshape(shape)
+
+
+def e4m3_round(x: float) -> float:
+    """Nearest e4m3 value of an fp32 number (ties to even, saturating at 448)."""
+    return float(lib().oracle_e4m3_round(float(x)))
+
+
+def fwht32(x):
+    """Unnormalised Walsh-Hadamard transform of each row of x in fp32 butterflies."""
+    y = np.ascontiguousarray(x, dtype=np.float32).copy()
+    d = y.shape[-1]
+    lib().oracle_fwht32(_p(y, ctypes.c_float), y.size // d, d)
+    return y
+
+
+def fp8_quantize(x, signs=None, rotate: bool = True):
+    """Block-wise e4m3 quantisation of x (B, H, N, d) or (BH, N, d), after the
+    randomised Hadamard rotation when `rotate`.  Returns (codes, scales): codes
+    shaped like x (the e4m3 values, as float32), scales (..., ceil(N / 128))."""
+    x = _f64(x)
+    BH, N, d = _dims(x)
+    nb = (N + 127) // 128
+    codes = np.empty(x.shape, dtype=np.float32)
+    scales = np.empty(x.shape[:-2] + (nb,), dtype=np.float32)
+    sg = None
+    if signs is not None:
+        sg = np.ascontiguousarray(signs, dtype=np.int8)
+        if sg.shape != (d,):
+            raise ValueError("signs must have d entries")
+    lib().oracle_fp8_quantize(_p(x), BH, N, d,
+                              None if sg is None else _p(sg, ctypes.c_int8), int(bool(rotate)),
+                              _p(codes, ctypes.c_float), _p(scales, ctypes.c_float))
+    return codes, scales
+
+
+def fp8_dequantize(codes, scales):
+    """codes * their block's scale, in fp64 (exact)."""
+    codes = np.asarray(codes, dtype=np.float64)
+    N = codes.shape[-2]
+    per_row = np.repeat(np.asarray(scales, dtype=np.float64), 128, axis=-1)[..., :N]
+    return codes * per_row[..., None]
+
+
+def fwd_fp8(q, k, v, causal: bool, scale: float, signs=None, rotate: bool = True):
+    """The FP8 forward as the method computes it: Q and K rotated and quantised
+    block-wise to e4m3 (fp8_quantize), the scores scale (q~ . k~) / d (the
+    rotation multiplies dot products by d; 1 without it), then the exact
+    two-pass attention in fp64 with the 16-bit V.  Returns (O, LSE)."""
+    d = np.shape(q)[-1]
+    qc, qs = fp8_quantize(q, signs, rotate)
+    kc, ks = fp8_quantize(k, signs, rotate)
+    return fwd(fp8_dequantize(qc, qs), fp8_dequantize(kc, ks), v, causal,
+               scale / (d if rotate else 1.0))

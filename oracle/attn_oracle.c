@@ -381,6 +381,101 @@ void oracle_bwd_blocksparse_heads(const double* q, const double* k, const double
     free(part);
 }
 
+/*
+ * FP8 with incoherent processing: "Is a full day of context better than ten
+ * minutes?" (marketmaker.cc), section "FA3: Hopper", third item: naive FP8
+ * attention is hurt by outliers, so the vectors are randomly rotated before
+ * block-wise quantisation, which spreads an outlier's magnitude over all
+ * coordinates (reported 2.6x lower error than naive FP8).  The page gives no
+ * formulas; the readings taken:
+ *  - the rotation is a randomised Hadamard transform of each row of Q and K
+ *    along the head dimension: y = H (s o x), with s a random +-1 vector (an
+ *    input) and H the d x d Sylvester-Hadamard matrix, unnormalised (entries
+ *    +-1).  H^T H = d I, so (H s o q) . (H s o k) = d (q . k): the scores are
+ *    recovered exactly by dividing by d, and no rounding is added by a
+ *    1/sqrt(d) factor.  Without rotation (naive FP8) y = x.
+ *  - quantisation is per block of 128 rows of one (batch, head): amax = max
+ *    |y| over the block, codes e4m3(y * (448 / amax)) rounded to nearest even
+ *    with saturation, dequantisation scale amax / 448 (a block of zeros gets
+ *    scale 0 and codes 0);
+ *  - only the S = Q K^T product runs in FP8; P V keeps the 16-bit V.
+ * The rotation and quantisation decide integer codes, so they are taken in
+ * fp32 exactly as stated (the butterflies below in this order, IEEE single
+ * operations), the precision the kernel uses; the attention on the
+ * dequantised values is then the exact two-pass definition in fp64.
+ */
+
+/* fp32 -> nearest e4m3 value (1 sign, 4 exponent bits with bias 7, 3 mantissa
+ * bits; normals 2^-6 .. 448, subnormals multiples of 2^-9), ties to even,
+ * magnitudes beyond 448 saturate to 448.  Returned as a float (exact). */
+float oracle_e4m3_round(float x) {
+    if (x != x) return x;
+    double a = fabs((double)x), r;
+    if (a >= 448.0) {
+        r = 448.0;
+    } else if (a < 0.015625) {                  /* below 2^-6: subnormal grid 2^-9 */
+        r = nearbyint(a * 512.0) / 512.0;
+    } else {
+        int e;
+        frexp(a, &e);                           /* a = f 2^e, f in [0.5, 1) */
+        double quantum = ldexp(1.0, e - 4);     /* 3 mantissa bits below 2^(e-1) */
+        r = nearbyint(a / quantum) * quantum;
+        if (r > 448.0) r = 448.0;
+    }
+    return (float)(x < 0 ? -r : r);
+}
+
+/* In-place Walsh-Hadamard butterflies on d floats (d a power of two), in fp32:
+ * for h = 1, 2, 4, ..: (x[j], x[j + h]) <- (x[j] + x[j + h], x[j] - x[j + h]). */
+static void fwht32(float* x, int64_t d) {
+    for (int64_t h = 1; h < d; h *= 2)
+        for (int64_t i = 0; i < d; i += 2 * h)
+            for (int64_t j = i; j < i + h; ++j) {
+                float a = x[j], b = x[j + h];
+                x[j] = a + b;
+                x[j + h] = a - b;
+            }
+}
+
+void oracle_fwht32(float* x, int64_t rows, int64_t d) {
+    for (int64_t r = 0; r < rows; ++r) fwht32(x + r * d, d);
+}
+
+/*
+ * Quantise x (BH, N, d; values exactly representable in fp32) as described
+ * above: codes (BH, N, d) as e4m3 values, scales (BH, ceil(N / 128)).
+ * signs: d entries +-1 (NULL: no sign flip); rotate: apply H.
+ */
+void oracle_fp8_quantize(const double* x, int64_t BH, int64_t N, int64_t d,
+                         const int8_t* signs, int rotate, float* codes, float* scales) {
+    int64_t nb = (N + 127) / 128;
+#pragma omp parallel for collapse(2) schedule(dynamic, 4)
+    for (int64_t bh = 0; bh < BH; ++bh)
+        for (int64_t b = 0; b < nb; ++b) {
+            int64_t r0 = b * 128, r1 = r0 + 128 < N ? r0 + 128 : N;
+            float* y = codes + (bh * N + r0) * d;
+            float amax = 0.0f;
+            for (int64_t r = r0; r < r1; ++r) {
+                float* yr = y + (r - r0) * d;
+                for (int64_t t = 0; t < d; ++t) {
+                    float v = (float)x[(bh * N + r) * d + t];
+                    yr[t] = signs ? (signs[t] < 0 ? -v : v) : v;
+                }
+                if (rotate) fwht32(yr, d);
+                for (int64_t t = 0; t < d; ++t) {
+                    float m = fabsf(yr[t]);
+                    if (m > amax) amax = m;
+                }
+            }
+            float inv = amax > 0.0f ? 448.0f / amax : 0.0f;
+            for (int64_t e = 0; e < (r1 - r0) * d; ++e) {
+                float t = y[e] * inv;
+                y[e] = oracle_e4m3_round(t);
+            }
+            scales[bh * nb + b] = amax / 448.0f;
+        }
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

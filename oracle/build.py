@@ -1,7 +1,8 @@
 """Compile the fp64 oracle (plain C + OpenMP) into oracle/_build/liboracle.so.
 
 Test infrastructure: the product library never links or loads this.
-Plain -O2 without fast-math, so IEEE double semantics are kept.
+Plain -O2 without fast-math or contraction, so IEEE single and double
+semantics are kept.
 """
 
 from __future__ import annotations
@@ -21,7 +22,7 @@ def build(force: bool = False) -> str:
         return LIB
     os.makedirs(OUT_DIR, exist_ok=True)
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = ["gcc", "-O2", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+    cmd = ["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp", "-fPIC", "-shared", "-std=c11",
            "-o", tmp, SRC, "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
