@@ -45,13 +45,19 @@ WORKLOADS = {
     "gpt2_causal": (8, 12, 1024, 64, True, "bf16", 1.0, "fwdbwd"),
     "long_day": (1, 12, 23400, 64, True, "fp16", 0.5, "fwd"),
     "large_head": (4, 16, 4096, 128, True, "bf16", 1.0, "fwdbwd"),
+    "large_head_blocksparse": (4, 16, 4096, 128, False, "bf16", 1.0, "fwdbwd"),
 }
+# Block-sparse workloads: density of the seeded 128 x 128 block mask (the
+# diagonal is always marked, so no row is empty).
+BLOCK_MASKS = {"large_head_blocksparse": 0.5}
 DESCRIPTION = {
     "tiny": "tiny exact attention fwd B=1 H=2 N=256 d=64 non-causal bf16",
     "bert_large": "BERT-large-shaped fwd B=8 H=16 N=512 d=64 non-causal bf16",
     "gpt2_causal": "GPT-2-shaped causal fwd+bwd B=8 H=12 N=1024 d=64 bf16",
     "long_day": "long single-sequence causal fwd B=1 H=12 N=23400 d=64 fp16 sigma=0.5",
     "large_head": "large-head causal fwd+bwd B=4 H=16 N=4096 d=128 bf16",
+    "large_head_blocksparse": "block-sparse fwd+bwd B=4 H=16 N=4096 d=128 bf16, "
+                              "half of the 128x128 blocks marked (seeded, diagonal kept)",
 }
 METRIC = "attention fwd and fwd+bwd TFLOP/s on 1 B200; % of dense BF16 tensor peak"
 L2_BYTES = 126 * 1024 * 1024
@@ -62,6 +68,30 @@ def flops(B, H, N, d, causal):
     if causal:
         f /= 2
     return f, 2.5 * f  # forward, backward
+
+
+def block_mask(N, density, seed=1):
+    """Seeded (nb, nb) uint8 block mask with the diagonal marked."""
+    nb = (N + 127) // 128
+    m = (np.random.default_rng(seed).random((nb, nb)) < density).astype(np.uint8)
+    np.fill_diagonal(m, 1)
+    return m
+
+
+def blocksparse_flops(B, H, N, d, mask):
+    """Forward and backward FLOPs of the marked blocks (the same convention as
+    flops(): 4 d per visible query-key pair forward, 10 d backward)."""
+    sizes = np.minimum(128, N - 128 * np.arange(mask.shape[0]))
+    pairs = float(sizes @ mask.astype(np.float64) @ sizes)
+    f = 4.0 * B * H * d * pairs
+    return f, 2.5 * f
+
+
+def workload_flops(wl):
+    B, H, N, d, causal, _, _, _ = WORKLOADS[wl]
+    if wl in BLOCK_MASKS:
+        return blocksparse_flops(B, H, N, d, block_mask(N, BLOCK_MASKS[wl]))
+    return flops(B, H, N, d, causal)
 
 
 def kernel_traffic(kernels):
@@ -128,7 +158,10 @@ class ClockSampler:
             self.t1 = time.time()
 
     def stop(self):
+        """Ends sampling; returns the csv text (None if nvidia-smi never ran)."""
         if self.proc is None:
+            self.file.close()
+            os.unlink(self.file.name)
             return None
         time.sleep(0.2)
         self.proc.terminate()
@@ -140,7 +173,7 @@ class ClockSampler:
         self.file.seek(0)
         text = self.file.read()
         os.unlink(self.file.name)
-        return parse_clock_samples(text, self.t0, self.t1)
+        return text
 
 
 def parse_clock_samples(text, t0, t1):
@@ -192,65 +225,193 @@ def job_tflops(flop_per_rank_step: float, world: int, max_ms_per_step: float) ->
     return world * flop_per_rank_step / (max_ms_per_step * 1e-3) / 1e12
 
 
-def host_inputs(wl, seed):
-    B, H, N, d, causal, dtype, sigma, passes = WORKLOADS[wl]
+def _device_tensors(wl, seed, dev, passes):
+    """Seeded host inputs (pinned) and their device copies for workload `wl`."""
+    import torch
+    B, H, N, d, causal, dtype, sigma, _ = WORKLOADS[wl]
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float16
     arrs = synth.attention_inputs(B, H, N, d, seed=seed, sigma=sigma, dtype=dtype,
                                   with_dout=(passes == "fwdbwd"))
-    return arrs
+    pinned = []
+    for a in arrs:
+        t = torch.from_numpy(a.view(np.int16)).view(tdt) if dtype == "bf16" else torch.from_numpy(a)
+        pinned.append(t.pin_memory())
+    return pinned, [t.to(dev) for t in pinned]
+
+
+class DeviceRun:
+    """Buffers and one step (forward, then the backward's two phases) of a
+    workload on one device, with CUDA events on the launching stream."""
+
+    def __init__(self, wl, passes, seed, dev):
+        import torch
+        from io_aware_exact_30_b200 import attn
+        self.attn = attn
+        B, H, N, d, causal, dtype, sigma, _ = WORKLOADS[wl]
+        self.wl, self.passes, self.causal, self.scale = wl, passes, causal, 1.0 / math.sqrt(d)
+        self.shape = (B, H, N, d)
+        self.pinned, self.dev_in = _device_tensors(wl, seed, dev, passes)
+        self.q, self.k, self.v = self.dev_in[:3]
+        self.do = self.dev_in[3] if passes == "fwdbwd" else None
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        if passes == "fwdbwd":
+            self.dq, self.dk, self.dv = (torch.empty_like(self.q) for _ in range(3))
+            self.ws = torch.empty(attn.attn_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8,
+                                  device=dev)
+        self.working_set = sum(t.numel() * t.element_size() for t in self.dev_in) + \
+            self.o.numel() * self.o.element_size()
+        self.flush = None
+        if self.working_set < 2 * L2_BYTES:
+            self.flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+        self.mask = None
+        if wl in BLOCK_MASKS:
+            self.mask = torch.from_numpy(block_mask(N, BLOCK_MASKS[wl])).to(dev)
+        self.stream = torch.cuda.current_stream(dev)
+        self.n_launch = 1 + (attn.bwd_launches(d) if passes == "fwdbwd" else 0)
+        self.n_events = 4 if passes == "fwdbwd" else 2
+
+    def l2_note(self):
+        if self.flush is None:
+            return "inputs larger than L2 (working set %.0f MB)" % (self.working_set / 1e6)
+        return "L2 flushed between steps (256 MB write, outside the per-step events)"
+
+    def step(self, evs=None):
+        a, st = self.attn, self.stream
+        if self.flush is not None:
+            self.flush.zero_()
+        if evs:
+            evs[0].record(st)
+        if self.mask is None:
+            a.attn_fwd(self.q, self.k, self.v, self.o, self.lse, self.causal, self.scale)
+        else:
+            a.attn_fwd_blocksparse(self.q, self.k, self.v, self.o, self.lse, self.mask,
+                                   self.causal, self.scale)
+        if evs:
+            evs[1].record(st)
+        if self.passes == "fwdbwd":
+            if self.mask is None:
+                a.attn_bwd_prep(self.o, self.do, self.lse, self.ws)
+                if evs:
+                    evs[2].record(st)
+                a.attn_bwd_main(self.q, self.k, self.v, self.do, self.dq, self.dk, self.dv,
+                                self.ws, self.causal, self.scale)
+            else:  # one call (prep + main): the prep share is timed with the main phase
+                if evs:
+                    evs[2].record(st)
+                a.attn_bwd_blocksparse(self.q, self.k, self.v, self.o, self.lse, self.do, self.dq,
+                                       self.dk, self.dv, self.ws, self.mask, self.causal,
+                                       self.scale)
+            if evs:
+                evs[3].record(st)
+
+    def events(self, steps):
+        import torch
+        return [[torch.cuda.Event(enable_timing=True) for _ in range(self.n_events)]
+                for _ in range(steps)]
+
+    @staticmethod
+    def medians(per_step):
+        """Median per-step times (ms): whole step, forward, backward prep, backward main."""
+        med = lambda xs: statistics.median(xs) if xs else 0.0
+        step = med([e[0].elapsed_time(e[-1]) for e in per_step])
+        fwd = med([e[0].elapsed_time(e[1]) for e in per_step])
+        prep = med([e[1].elapsed_time(e[2]) for e in per_step]) if len(per_step[0]) > 2 else 0.0
+        main = med([e[2].elapsed_time(e[3]) for e in per_step]) if len(per_step[0]) > 2 else 0.0
+        return step, fwd, prep, main
+
+
+def roofline_entry(d, passes, f_fwd, f_bwd, fwd_ms, main_ms, traffic):
+    """Roofline of the dominant kernel call: the backward main call (main kernel,
+    plus the dQ conversion it launches at d = 128) when the backward runs, else
+    the forward.  The peak is the measured burst bf16 rate: the kernels are timed
+    over a timed region of milliseconds at full clock, not a seconds-long loop
+    under the power cap (fp16 contractions run at the same tensor rate)."""
+    burst, _, _, src = peaks()
+    if passes == "fwdbwd":
+        kern = (["attn_bwd_main128_kernel", "attn_bwd_dq_convert_kernel"] if d == 128
+                else ["attn_bwd_main_kernel"])
+        flop, ms = f_bwd, main_ms
+    else:
+        kern, flop, ms = ["attn_fwd_kernel"], f_fwd, fwd_ms
+    achieved = flop / (ms * 1e-3) / 1e12
+    return {
+        "kernel": " + ".join(kern),
+        "bound": "tensor",
+        "achieved": round(achieved, 2),
+        "peak": burst,
+        "peak_kind": f"bf16_tflops burst ({src}); fp16 runs at the same tensor rate",
+        "unit": "TFLOP/s",
+        "frac": round(achieved / burst, 4),
+        "traffic": traffic,
+        "traffic_unit": "bytes per launch (ncu dram read+write; profiles/traffic.json)",
+    }, kern
+
+
+def side_workloads(args, dev, clocks):
+    """Every other configuration, timed the same way (median of per-step CUDA
+    events after warm-up, L2 flushed between steps when the inputs fit in L2);
+    parity cases for the tests, reported here so each has a measured number."""
+    import torch
+    out = {}
+    burst, _, _, _ = peaks()
+    for wl in WORKLOADS:
+        if wl == args.workload:
+            continue
+        B, H, N, d, causal, dtype, sigma, passes = WORKLOADS[wl]
+        run = DeviceRun(wl, passes, args.seed, dev)
+        for _ in range(max(3, args.warmup)):
+            run.step()
+        torch.cuda.synchronize()
+        steps = max(20, min(args.steps, 50))
+        per = run.events(steps)
+        t0 = time.time()
+        for i in range(steps):
+            run.step(per[i])
+        torch.cuda.synchronize()
+        t1 = time.time()
+        if run.attn.attn_last_device_status() != 0:
+            raise RuntimeError(f"device status not OK after {wl}")
+        step_ms, fwd_ms, prep_ms, main_ms = DeviceRun.medians(per)
+        f_fwd, f_bwd = workload_flops(wl)
+        f_step = f_fwd + (f_bwd if passes == "fwdbwd" else 0.0)
+        roof, _ = roofline_entry(d, passes, f_fwd, f_bwd, fwd_ms, main_ms, None)
+        roof.pop("traffic")
+        roof.pop("traffic_unit")
+        e = {
+            "workload": DESCRIPTION[wl], "passes": passes, "steps": steps,
+            "ms_per_step": round(step_ms, 4),
+            "tflops": round(f_step / (step_ms * 1e-3) / 1e12, 2),
+            "fwd_ms": round(fwd_ms, 4), "fwd_tflops": round(f_fwd / (fwd_ms * 1e-3) / 1e12, 2),
+            "pct_of_2250_spec": round(100 * f_step / (step_ms * 1e-3) / 1e12 / 2250.0, 2),
+            "frac_of_measured_burst": round(f_step / (step_ms * 1e-3) / 1e12 / burst, 4),
+            "roofline": roof, "l2": run.l2_note(),
+        }
+        if passes == "fwdbwd":
+            e["bwd_prep_ms"] = round(prep_ms, 4)
+            e["bwd_main_ms"] = round(main_ms, 4)
+            e["bwd_tflops"] = round(f_bwd / ((prep_ms + main_ms) * 1e-3) / 1e12, 2)
+        e["clocks_window"] = [t0, t1]
+        out[wl] = e
+        del run
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
-    from io_aware_exact_30_b200 import attn
 
     B, H, N, d, causal, dtype, sigma, passes = WORKLOADS[args.workload]
     if args.passes:
         passes = args.passes
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    tdt = torch.bfloat16 if dtype == "bf16" else torch.float16
-    scale = 1.0 / math.sqrt(d)
-
-    arrs = host_inputs(args.workload, seed=rank_seed(args.seed, rank))
-    pinned = []
-    for a in arrs:
-        t = torch.from_numpy(a.view(np.int16)).view(tdt) if dtype == "bf16" else torch.from_numpy(a)
-        pinned.append(t.pin_memory())
-    dev_in = [t.to(dev) for t in pinned]
-    q, k, v = dev_in[:3]
-    do = dev_in[3] if passes == "fwdbwd" else None
-    o = torch.empty_like(q)
-    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-    if passes == "fwdbwd":
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
-        ws = torch.empty(attn.attn_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
-    working_set = sum(t.numel() * t.element_size() for t in dev_in) + o.numel() * 2
-    flush = None
-    if working_set < 2 * L2_BYTES:
-        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
-
-    stream = torch.cuda.current_stream(dev)
-    n_launch = {"fwd": 1, "fwdbwd": 1 + attn.bwd_launches(d)}[passes]
-
-    def step(evs=None):
-        if flush is not None:
-            flush.zero_()
-        if evs:
-            evs[0].record(stream)
-        attn.attn_fwd(q, k, v, o, lse, causal, scale)
-        if evs:
-            evs[1].record(stream)
-        if passes == "fwdbwd":
-            attn.attn_bwd_prep(o, do, lse, ws)
-            if evs:
-                evs[2].record(stream)
-            attn.attn_bwd_main(q, k, v, do, dq, dk, dv, ws, causal, scale)
-            if evs:
-                evs[3].record(stream)
+    run = DeviceRun(args.workload, passes, rank_seed(args.seed, rank), dev)
+    attn = run.attn
 
     for _ in range(args.warmup):
-        step()
+        run.step()
     torch.cuda.synchronize()
     if attn.attn_last_device_status() != 0:
         raise RuntimeError("device status not OK after warm-up")
@@ -258,82 +419,87 @@ def run_ours(args, rank, world, local_rank):
     clocks = ClockSampler(local_rank)
     if rank == 0:
         clocks.start()
-    per_step = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    per_step = run.events(args.steps)
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clocks.mark(True)
-    t_start.record(stream)
+    t_start.record(run.stream)
     for i in range(args.steps):
-        step(per_step[i])
-    t_end.record(stream)
+        run.step(per_step[i])
+    t_end.record(run.stream)
     torch.cuda.synchronize()
     clocks.mark(False)
     if world > 1:
         dist.barrier()
     status = attn.attn_last_device_status()
-    total_ms = t_start.elapsed_time(t_end)
-    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in per_step)
-    prep_ms = main_ms = 0.0
-    if passes == "fwdbwd":
-        prep_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in per_step)
-        main_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in per_step)
+    bracket_ms = t_start.elapsed_time(t_end)
+    step_ms, fwd_ms, prep_ms, main_ms = DeviceRun.medians(per_step)
 
-    # whole-job time = slowest rank
-    max_ms = reduce_max(total_ms, world, dev)
-    clk = clocks.stop() if rank == 0 else None
+    # whole-job time per step = slowest rank's median step
+    max_step_ms = reduce_max(step_ms, world, dev)
+    max_bracket_ms = reduce_max(bracket_ms, world, dev)
 
     # ---- end to end through the public API with host buffers -------------
+    # attn_sdpa_host: the inputs come from pinned host memory and the results
+    # go back there inside the call, chunk by chunk over heads with copies in,
+    # kernels and copies out overlapped on the library's internal streams.
     e2e_steps = max(3, min(args.steps, 20))
+    pinned = run.pinned
     host_out = [torch.empty_like(pinned[0]).pin_memory() for _ in range(3 if passes == "fwdbwd" else 1)]
     host_lse = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+    with_bwd = passes == "fwdbwd"
+    scratch = torch.empty(attn.attn_sdpa_host_scratch_bytes(B, H, N, d, with_bwd),
+                          dtype=torch.uint8, device=dev)
 
     def e2e_step():
-        for src, dst in zip(pinned, dev_in):
-            dst.copy_(src, non_blocking=True)
-        attn.attn_fwd(q, k, v, o, lse, causal, scale)
-        if passes == "fwdbwd":
-            attn.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, causal, scale)
-            for src, dst in zip((dq, dk, dv), host_out):
-                dst.copy_(src, non_blocking=True)
+        if with_bwd:
+            attn.attn_sdpa_host(pinned[0], pinned[1], pinned[2], pinned[3], None, None,
+                                host_out[0], host_out[1], host_out[2], scratch, causal, run.scale)
         else:
-            host_out[0].copy_(o, non_blocking=True)
-            host_lse.copy_(lse, non_blocking=True)
+            attn.attn_sdpa_host(pinned[0], pinned[1], pinned[2], None, host_out[0], host_lse,
+                                None, None, None, scratch, causal, run.scale)
 
     e2e_step()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    e0.record(run.stream)
     for _ in range(e2e_steps):
         e2e_step()
-    e1.record(stream)
+    e1.record(run.stream)
     torch.cuda.synchronize()
     e2e_ms = reduce_max(e0.elapsed_time(e1) / e2e_steps, world, dev)
     h2d = sum(t.numel() * t.element_size() for t in pinned)
     d2h = sum(t.numel() * t.element_size() for t in host_out) + (
-        0 if passes == "fwdbwd" else host_lse.numel() * 4)
+        0 if with_bwd else host_lse.numel() * 4)
+    del scratch
     if attn.attn_last_device_status() != 0 or status != 0:
         raise RuntimeError("device status not OK after timing")
+    l2_note = run.l2_note()
+    del run
+    torch.cuda.empty_cache()
 
     if rank != 0:
+        clocks.stop()
         return None
-    f_fwd, f_bwd = flops(B, H, N, d, causal)
+    others = side_workloads(args, dev, clocks) if (world == 1 and not args.headline_only) else None
+    clocks_text = clocks.stop()
+    clk = parse_clock_samples(clocks_text, clocks.t0, clocks.t1) if clocks_text is not None else None
+    if others:
+        for e in others.values():
+            t0, t1 = e.pop("clocks_window")
+            if clocks_text is not None:
+                e["clocks"] = parse_clock_samples(clocks_text, t0, t1)
+
+    f_fwd, f_bwd = workload_flops(args.workload)
     f_step = f_fwd + (f_bwd if passes == "fwdbwd" else 0.0)
-    ms_step = max_ms / args.steps
-    value = job_tflops(f_step, world, ms_step)
+    value = job_tflops(f_step, world, max_step_ms)
     burst, sustained, hbm, src = peaks()
-    # The backward-main call launches, for d = 128, the main kernel and then the dQ
-    # conversion; they are timed together and their traffic is summed.
-    if passes == "fwdbwd":
-        dom = (["attn_bwd_main128_kernel", "attn_bwd_dq_convert_kernel"] if d == 128
-               else ["attn_bwd_main_kernel"], f_bwd, main_ms)
-    else:
-        dom = (["attn_fwd_kernel"], f_fwd, fwd_ms)
-    traffic = kernel_traffic(dom[0]) if args.workload == "large_head" else None
-    achieved = dom[1] / (dom[2] * 1e-3) / 1e12
+    roof, kern = roofline_entry(d, passes, f_fwd, f_bwd, fwd_ms, main_ms, None)
+    roof["traffic"] = kernel_traffic(kern) if args.workload == "large_head" else None
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -341,7 +507,7 @@ def run_ours(args, rank, world, local_rank):
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(ms_step, 4),
+        "ms_per_step": round(max_step_ms, 4),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -352,44 +518,50 @@ def run_ours(args, rank, world, local_rank):
             "B": B, "H": H, "N": N, "d": d, "causal": causal, "passes": passes,
             "flop_per_step": f_step,
             "flop_convention": "fwd 4BHN^2d, bwd 10BHN^2d, halved when causal",
-            "l2": "inputs larger than L2 (working set %.0f MB)" % (working_set / 1e6)
-            if flush is None else "L2 flushed between steps (256 MB write)",
+            "l2": l2_note,
+            "timing": "ms_per_step = median over the timed steps of per-step CUDA events "
+                      "(max over ranks); ms_bracket_mean = barrier-to-barrier events / steps",
             "parallelism": f"dp{world} (independent heads per rank, no collective)",
         },
+        "ms_bracket_mean": round(max_bracket_ms / args.steps, 4),
         "fwd_tflops": round(f_fwd / (fwd_ms * 1e-3) / 1e12, 2),
         "fwd_ms": round(fwd_ms, 4),
         "pct_of_2250_spec": round(100 * value / world / 2250.0, 2),
         "pct_of_measured_burst": round(100 * value / world / burst, 2),
-        "pct_of_measured_sustained": round(100 * value / world / sustained, 2),
-        "roofline": {
-            "kernel": " + ".join(dom[0]),
-            "bound": "tensor",
-            "achieved": round(achieved, 2),
-            "peak": sustained,
-            "peak_kind": f"bf16_tflops_sustained ({src})",
-            "unit": "TFLOP/s",
-            "frac": round(achieved / sustained, 4),
-            "traffic": traffic,
-            "traffic_unit": "bytes per launch (ncu dram read+write; profiles/traffic.json)",
-        },
+        "roofline": roof,
         "e2e": {"value": round(job_tflops(f_step, world, e2e_ms), 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": round(e2e_ms, 4)},
-        "gpu_launches": n_launch * args.steps,
+                "ms_per_step": round(e2e_ms, 4),
+                "api": "attn_sdpa_host (pinned host buffers in and out, copies inside the call)"},
+        "gpu_launches": (1 + (attn.bwd_launches(d) if passes == "fwdbwd" else 0)) * args.steps,
         "clocks": clk,
     }
     if passes == "fwdbwd":
         line["bwd_prep_ms"] = round(prep_ms, 4)
         line["bwd_main_ms"] = round(main_ms, 4)
         line["bwd_tflops"] = round(f_bwd / ((prep_ms + main_ms) * 1e-3) / 1e12, 2)
+    if others is not None:
+        line["workloads"] = others
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.workload, passes, args.cpu_seconds)
+        if others is not None:
+            for wl in ("tiny", "bert_large"):
+                if wl in others:
+                    others[wl]["cpu_baseline_1thread"] = cpu_baseline(wl, "fwd", 3.0, threads=1)
     return line
 
 
-def cpu_baseline(workload, passes, budget_s):
-    """The fp64 oracle as it stands, on the host cores, on a bounded sample."""
+def cpu_baseline(workload, passes, budget_s, threads=None):
+    """The fp64 oracle as it stands, on the host cores (or `threads` of them), on
+    a bounded sample."""
     import oracle
+    if threads is not None:
+        prev = oracle.num_threads()
+        oracle.set_num_threads(threads)
+        try:
+            return cpu_baseline(workload, passes, budget_s)
+        finally:
+            oracle.set_num_threads(prev)
     B, H, N, d, causal, dtype, sigma, _ = WORKLOADS[workload]
     scale = 1.0 / math.sqrt(d)
     arrs = synth.attention_inputs(1, 1, N, d, seed=0, sigma=sigma, dtype=dtype, with_dout=True)
@@ -431,11 +603,16 @@ def cpu_baseline(workload, passes, budget_s):
         per_row = probe / rows.size
         nrows = int(min(rows_all, max(64, budget_s / per_row)))
         rows = np.linspace(0, N - 1, nrows).astype(np.int64)
-        t0 = time.time()
-        oracle.fwd_rows(*f64[:3], causal, scale, rows)
-        dt = time.time() - t0
-        fl = 4.0 * d * float(np.sum(rows + 1 if causal else np.full(rows.size, N)))
-        sample = f"{rows.size} query rows of one head, fp64 two-pass forward"
+        reps, t0 = 0, time.time()
+        while True:  # repeat small samples until at least a second has passed
+            oracle.fwd_rows(*f64[:3], causal, scale, rows)
+            reps += 1
+            dt = time.time() - t0
+            if dt >= min(1.0, budget_s):
+                break
+        fl = reps * 4.0 * d * float(np.sum(rows + 1 if causal else np.full(rows.size, N)))
+        sample = (f"{rows.size} query rows of one head, fp64 two-pass forward"
+                  + (f", repeated {reps} times" if reps > 1 else ""))
     return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": sample, "seconds": round(dt, 2)}
 
@@ -477,12 +654,15 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="large_head", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="large_head",
+                    choices=sorted(w for w in WORKLOADS if w not in BLOCK_MASKS))
     ap.add_argument("--passes", choices=["fwd", "fwdbwd"], default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the other workloads (timed after the headline at N=1)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

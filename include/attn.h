@@ -66,7 +66,8 @@ typedef enum {
     ATTN_ERR_LAUNCH = -7,   /* the CUDA runtime rejected a launch */
     ATTN_ERR_TIMEOUT = -8,  /* a bounded in-kernel wait ran out (device status) */
     ATTN_ERR_ARG = -9,      /* scale not finite and positive, or another bad scalar */
-    ATTN_ERR_SCRATCH = -10  /* attn_bwd_noalloc: problem exceeds the built-in scratch */
+    ATTN_ERR_SCRATCH = -10  /* attn_bwd_noalloc: problem exceeds the built-in scratch;
+                               attn_sdpa_host: scratch_bytes too small */
 } attn_status_t;
 
 /*
@@ -129,6 +130,35 @@ int attn_bwd_main(const void* q, const void* k, const void* v, const void* dout,
                   float scale, attn_dtype_t dtype, void* stream);
 
 /*
+ * Block-sparse attention: the forward and backward above restricted to the
+ * (query tile, key tile) pairs a block mask marks, with tiles of 128 rows and
+ * 128 keys; blocks not marked are skipped entirely (neither loaded nor
+ * computed), as blocks in the future of a query tile are under the causal
+ * mask.  Source: "FlashAttention の概要" (zenn.dev), the paragraph on
+ * Block-Sparse FlashAttention (an approximation of attention that computes
+ * only the blocks of a block mask, otherwise the same algorithm).
+ *
+ * block_mask: device memory, nb x nb bytes with nb = ceil(N / 128), row-major;
+ * block_mask[i * nb + j] != 0 lets the 128 queries of tile i attend to the
+ * 128 keys of tile j.  One mask serves every (batch, head).  With causal != 0
+ * the causal rule applies as well (key j visible to query i iff its block is
+ * marked and j <= i).  Over its visible keys each row is exact softmax
+ * attention; a row with no visible key gets O = 0 and lse = -inf (the empty
+ * sum), and contributes nothing to the gradients (its dq row is 0).
+ * Everything else (layouts, workspace, streams, errors) is as for attn_fwd
+ * and attn_bwd; ATTN_ERR_NULL if block_mask is NULL, ATTN_ERR_DEVICE if it is
+ * not device memory of the current device.
+ */
+int attn_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                         const unsigned char* block_mask, int B, int H, int N, int d,
+                         int causal, float scale, attn_dtype_t dtype, void* stream);
+
+int attn_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                         void* workspace, const unsigned char* block_mask, int B, int H, int N,
+                         int d, int causal, float scale, attn_dtype_t dtype, void* stream);
+
+/*
  * Backward that allocates nothing, for callers that cannot get device memory
  * for a workspace: for example a plugin inside a host framework that owns
  * every device allocation through its own pool and hands the plugin only the
@@ -157,6 +187,42 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                      const float* lse, const void* dout, void* dq, void* dk, void* dv,
                      int B, int H, int N, int d, int causal, float scale,
                      attn_dtype_t dtype, void* stream);
+
+/*
+ * End-to-end attention from host buffers, for callers whose tensors live in
+ * host memory (the pages have no counterpart; it keeps the host link busy in
+ * both directions while the kernels run).  q, k, v (and dout for the
+ * backward) are read from host memory, and the outputs are written back
+ * there: o and lse for the forward alone (dout == NULL; o and lse required);
+ * with the backward dq, dk, dv (required), and o, lse too when not NULL.  All
+ * tensors have the layouts of attn_fwd / attn_bwd.  Host memory should be
+ * page-locked: pageable memory works, but its copies do not overlap.
+ *
+ * The heads are processed in chunks of `heads_per_chunk` heads (<= 0: about
+ * an eighth of B*H, at least 256 query tiles of work per chunk).  The
+ * host-to-device copies of chunk c + 1, the kernels of chunk c and the
+ * device-to-host copies of chunk c - 1 run on three streams the library
+ * creates once per device, in three chunk slots of `scratch`: caller-owned
+ * device memory of at least attn_sdpa_host_scratch_bytes() bytes, 16-byte
+ * aligned.  The call is asynchronous with respect to the host.  Work queued
+ * on `stream` before the call comes first; work queued on `stream` after it
+ * waits for the last copy back, also after an error.  Calls are serialised
+ * by a per-device lock on the host.
+ *
+ * Results equal attn_fwd / attn_bwd on the same inputs: o, lse, dk and dv
+ * bit for bit, dq up to the order of its fp32 additions.
+ * Errors: ATTN_ERR_NULL, _SHAPE, _HEADDIM, _DTYPE and _ARG as attn_fwd;
+ * ATTN_ERR_SCRATCH if scratch_bytes is too small; ATTN_ERR_ALIGN if scratch
+ * is not 16-byte aligned; ATTN_ERR_DEVICE if scratch is not device memory of
+ * the current device; ATTN_ERR_LAUNCH if a copy or launch was refused.
+ */
+size_t attn_sdpa_host_scratch_bytes(int B, int H, int N, int d, int with_backward,
+                                    int heads_per_chunk);
+
+int attn_sdpa_host(const void* q, const void* k, const void* v, const void* dout, void* o,
+                   float* lse, void* dq, void* dk, void* dv, void* scratch,
+                   size_t scratch_bytes, int B, int H, int N, int d, int causal, float scale,
+                   attn_dtype_t dtype, int heads_per_chunk, void* stream);
 
 /*
  * Synchronises `stream`, then returns ATTN_OK, ATTN_ERR_TIMEOUT if a kernel

@@ -33,7 +33,9 @@ def bwd_launches(d: int) -> int:
 
 # Every symbol include/attn.h declares.
 EXPORTS = ("attn_fwd", "attn_bwd", "attn_bwd_prep", "attn_bwd_main", "attn_bwd_workspace_bytes",
-           "attn_bwd_noalloc", "attn_last_device_status", "attn_selftest_wait_timeout",
+           "attn_bwd_noalloc", "attn_sdpa_host", "attn_sdpa_host_scratch_bytes",
+           "attn_fwd_blocksparse", "attn_bwd_blocksparse",
+           "attn_last_device_status", "attn_selftest_wait_timeout",
            "attn_last_cuda_error_string", "attn_strerror", "attn_version")
 
 # Size of the built-in scratch attn_bwd_noalloc uses (bytes, per device).
@@ -70,6 +72,14 @@ def lib() -> ctypes.CDLL:
         L.attn_bwd_main.restype = ci
         L.attn_bwd_noalloc.argtypes = [vp] * 9 + [ci, ci, ci, ci, ci, cf, ci, vp]
         L.attn_bwd_noalloc.restype = ci
+        L.attn_fwd_blocksparse.argtypes = [vp] * 6 + [ci, ci, ci, ci, ci, cf, ci, vp]
+        L.attn_fwd_blocksparse.restype = ci
+        L.attn_bwd_blocksparse.argtypes = [vp] * 11 + [ci, ci, ci, ci, ci, cf, ci, vp]
+        L.attn_bwd_blocksparse.restype = ci
+        L.attn_sdpa_host_scratch_bytes.argtypes = [ci, ci, ci, ci, ci, ci]
+        L.attn_sdpa_host_scratch_bytes.restype = sz
+        L.attn_sdpa_host.argtypes = [vp] * 10 + [sz, ci, ci, ci, ci, ci, cf, ci, ci, vp]
+        L.attn_sdpa_host.restype = ci
         L.attn_bwd_workspace_bytes.argtypes = [ci, ci, ci, ci]
         L.attn_bwd_workspace_bytes.restype = sz
         L.attn_last_device_status.argtypes = [vp]
@@ -206,6 +216,78 @@ def attn_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, causal: bool,
     _check(rc, "attn_bwd_noalloc")
 
 
+# Block size of attn_fwd_blocksparse / attn_bwd_blocksparse masks (rows and keys).
+BLOCK = 128
+
+
+def _check_mask(mask, N, device):
+    nb = (N + BLOCK - 1) // BLOCK
+    if (mask.dtype not in (torch.uint8, torch.bool) or tuple(mask.shape) != (nb, nb)
+            or not mask.is_contiguous() or mask.device != device):
+        raise ValueError(f"block mask must be a contiguous ({nb}, {nb}) uint8/bool tensor on {device}")
+
+
+def attn_fwd_blocksparse(q, k, v, o, lse, block_mask, causal: bool, scale: float | None = None,
+                         stream=None) -> None:
+    """attn_fwd over the 128 x 128 blocks ``block_mask`` marks (one mask for all heads)."""
+    B, H, N, d = _shape(q)
+    _same(q, k, v, o, names=("k", "v", "o"))
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 (B, H, N) tensor")
+    _check_mask(block_mask, N, q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib().attn_fwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(block_mask),
+                                    B, H, N, d, int(bool(causal)), scale, _dtype(q),
+                                    ctypes.c_void_p(_stream(q.device, stream)))
+    _check(rc, "attn_fwd_blocksparse")
+
+
+def attn_bwd_blocksparse(q, k, v, o, lse, dout, dq, dk, dv, workspace, block_mask, causal: bool,
+                         scale: float | None = None, stream=None) -> None:
+    """attn_bwd over the 128 x 128 blocks ``block_mask`` marks."""
+    B, H, N, d = _shape(q)
+    _same(q, k, v, o, dout, dq, dk, dv, names=("k", "v", "o", "dout", "dq", "dk", "dv"))
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 (B, H, N) tensor")
+    _check_mask(block_mask, N, q.device)
+    need = attn_bwd_workspace_bytes(B, H, N, d)
+    if workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace needs {need} bytes")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib().attn_bwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                    _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+                                    _ptr(block_mask), B, H, N, d, int(bool(causal)), scale,
+                                    _dtype(q), ctypes.c_void_p(_stream(q.device, stream)))
+    _check(rc, "attn_bwd_blocksparse")
+
+
+def attn_sdpa_host_scratch_bytes(B: int, H: int, N: int, d: int, with_backward: bool,
+                                 heads_per_chunk: int = 0) -> int:
+    return int(lib().attn_sdpa_host_scratch_bytes(B, H, N, d, int(bool(with_backward)),
+                                                  int(heads_per_chunk)))
+
+
+def attn_sdpa_host(q, k, v, dout, o, lse, dq, dk, dv, scratch, causal: bool,
+                   scale: float | None = None, heads_per_chunk: int = 0, stream=None) -> None:
+    """Attention from host buffers: q, k, v, dout and the outputs are CPU
+    tensors (pinned, for the copies to overlap); ``dout=None`` runs the forward
+    alone (o and lse required).  ``scratch`` is a CUDA uint8 tensor of
+    attn_sdpa_host_scratch_bytes() bytes."""
+    B, H, N, d = _shape(q)
+    host = [t for t in (q, k, v, dout, o, lse, dq, dk, dv) if t is not None]
+    if any(t.device.type != "cpu" or not t.is_contiguous() for t in host):
+        raise ValueError("host tensors must be contiguous CPU tensors")
+    if scratch.device.type != "cuda":
+        raise ValueError("scratch must be device memory")
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib().attn_sdpa_host(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(o), _ptr(lse),
+                              _ptr(dq), _ptr(dk), _ptr(dv), _ptr(scratch),
+                              scratch.numel() * scratch.element_size(), B, H, N, d,
+                              int(bool(causal)), sc, _dtype(q), int(heads_per_chunk),
+                              ctypes.c_void_p(_stream(scratch.device, stream)))
+    _check(rc, "attn_sdpa_host")
+
+
 def attn_last_device_status(stream=None, device=None) -> int:
     st = _stream(device or torch.cuda.current_device(), stream)
     return int(lib().attn_last_device_status(ctypes.c_void_p(st)))
@@ -236,4 +318,23 @@ def backward(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = 
         workspace = torch.empty(attn_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8,
                                 device=q.device)
     attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, causal, scale)
+    return dq, dk, dv
+
+
+def forward_blocksparse(q, k, v, block_mask, causal: bool = False, scale: float | None = None):
+    """Allocates O and LSE and runs attn_fwd_blocksparse; returns (o, lse)."""
+    B, H, N, d = _shape(q)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    attn_fwd_blocksparse(q, k, v, o, lse, block_mask, causal, scale)
+    return o, lse
+
+
+def backward_blocksparse(q, k, v, o, lse, dout, block_mask, causal: bool = False,
+                         scale: float | None = None):
+    """Allocates dQ, dK, dV and the workspace; returns (dq, dk, dv)."""
+    B, H, N, d = _shape(q)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(attn_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=q.device)
+    attn_bwd_blocksparse(q, k, v, o, lse, dout, dq, dk, dv, ws, block_mask, causal, scale)
     return dq, dk, dv

@@ -15,6 +15,7 @@
 #include "fwd_sm100.cuh"
 #include "bwd_sm100.cuh"
 #include "bwd128_sm100.cuh"
+#include "fp8_sm100.cuh"
 
 namespace {
 
@@ -83,6 +84,18 @@ int check_device(int* dev_out) {
     ok &= cudaFuncSetAttribute(attn::attn_fwd_kernel<128, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                FwdCfg<128>::SMEM_BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn::attn_fwd_kernel<64, true, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               FwdCfg<64, true>::SMEM_BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn::attn_fwd_kernel<64, false, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               FwdCfg<64, true>::SMEM_BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn::attn_fwd_kernel<128, true, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               FwdCfg<128, true>::SMEM_BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn::attn_fwd_kernel<128, false, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               FwdCfg<128, true>::SMEM_BYTES) == cudaSuccess;
     ok &= attn::bwd_set_attributes();
     ok &= attn::bwd128_set_attributes();
     if (!ok) {
@@ -136,16 +149,33 @@ bool make_map(CUtensorMap* m, const void* ptr, int dtype, int BH, int N, int d,
     return r == CUDA_SUCCESS;
 }
 
-template <int D, bool BF16>
+// 3-D view (d, N, B*H) of a contiguous (B, H, N, d) e4m3 tensor; box d x 128 x 1
+// (one swizzled box per row: 128-byte swizzle for d = 128, 64-byte for d = 64).
+bool make_map8(CUtensorMap* m, const void* ptr, int BH, int N, int d) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                          static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d),
+                             static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d)};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(d), 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims,
+                             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                             d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int D, bool BF16, bool FP8 = false>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const attn::FwdParams& p, int sm_count, cudaStream_t st) {
     // causal: one CTA per work item, running CTAs take pending CTAs' items;
     // otherwise one CTA per multiprocessor
     const long long items = 1LL * p.n_pairs * p.BH;
     if (items >= (1LL << 31)) return ATTN_ERR_SHAPE;
-    const int nblocks = static_cast<int>(p.causal || items < sm_count ? items : sm_count);
-    attn::attn_fwd_kernel<D, BF16><<<static_cast<unsigned>(nblocks), FwdCfg<D>::NTHREADS,
-                                     FwdCfg<D>::SMEM_BYTES, st>>>(mq, mk, mv, p);
+    const bool dynamic = p.causal || p.bmask != nullptr;
+    const int nblocks = static_cast<int>(dynamic || items < sm_count ? items : sm_count);
+    attn::attn_fwd_kernel<D, BF16, FP8><<<static_cast<unsigned>(nblocks), FwdCfg<D, FP8>::NTHREADS,
+                                          FwdCfg<D, FP8>::SMEM_BYTES, st>>>(mq, mk, mv, p);
     return launch_ok() ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
@@ -190,10 +220,11 @@ int scratch_address(int dev, void** out) {
 
 }  // namespace
 
-extern "C" {
-
-int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
-             int d, int causal, float scale, attn_dtype_t dtype, void* stream) {
+namespace {
+// Forward for attn_fwd (bmask == nullptr) and attn_fwd_blocksparse.
+int fwd_entry(const void* q, const void* k, const void* v, void* o, float* lse,
+              const unsigned char* bmask, int B, int H, int N, int d, int causal, float scale,
+              attn_dtype_t dtype, void* stream) {
     if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
     int rc = check_shape(B, H, N, d, dtype, scale);
     if (rc) return rc;
@@ -202,7 +233,7 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
     int dev;
     if ((rc = check_device(&dev))) return rc;
     if (!on_device(q, dev) || !on_device(k, dev) || !on_device(v, dev) || !on_device(o, dev) ||
-        !on_device(lse, dev))
+        !on_device(lse, dev) || (bmask && !on_device(bmask, dev)))
         return ATTN_ERR_DEVICE;
     const int BH = B * H;
     CUtensorMap mq, mk, mv;
@@ -224,6 +255,9 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
     }
     p.causal = causal ? 1 : 0;
     p.scale_log2 = scale * 1.4426950408889634f;
+    p.bmask = bmask;
+    p.n_ktiles = (N + 127) / 128;
+    p.qscale = p.kscale = nullptr;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool bf = dtype == ATTN_BF16;
     if (d == 64)
@@ -231,6 +265,97 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
                   : launch_fwd<64, false>(mq, mk, mv, p, g_sm_count[dev], st);
     return bf ? launch_fwd<128, true>(mq, mk, mv, p, g_sm_count[dev], st)
               : launch_fwd<128, false>(mq, mk, mv, p, g_sm_count[dev], st);
+}
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+             int d, int causal, float scale, attn_dtype_t dtype, void* stream) {
+    return fwd_entry(q, k, v, o, lse, nullptr, B, H, N, d, causal, scale, dtype, stream);
+}
+
+int attn_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                         const unsigned char* block_mask, int B, int H, int N, int d, int causal,
+                         float scale, attn_dtype_t dtype, void* stream) {
+    if (!block_mask) return ATTN_ERR_NULL;
+    return fwd_entry(q, k, v, o, lse, block_mask, B, H, N, d, causal, scale, dtype, stream);
+}
+
+int attn_fp8_quantize(const void* x, unsigned char* x8, float* scales, const signed char* signs,
+                      int rotate, int B, int H, int N, int d, attn_dtype_t dtype, void* stream) {
+    if (!x || !x8 || !scales) return ATTN_ERR_NULL;
+    int rc = check_shape(B, H, N, d, dtype, 1.f);
+    if (rc) return rc;
+    if (!aligned16(x) || !aligned16(x8) || (reinterpret_cast<uintptr_t>(scales) & 3u))
+        return ATTN_ERR_ALIGN;
+    int dev;
+    if ((rc = check_device(&dev))) return rc;
+    if (!on_device(x, dev) || !on_device(x8, dev) || !on_device(scales, dev) ||
+        (signs && !on_device(signs, dev)))
+        return ATTN_ERR_DEVICE;
+    const long long blocks = 1LL * B * H * ((N + 127) / 128);
+    if (blocks >= (1LL << 31)) return ATTN_ERR_SHAPE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const auto* in = static_cast<const uint8_t*>(x);
+    const auto* sg = reinterpret_cast<const int8_t*>(signs);
+    const bool bf = dtype == ATTN_BF16;
+    const unsigned g = static_cast<unsigned>(blocks);
+    if (d == 64) {
+        if (bf) attn::attn_fp8_quantize_kernel<64, true><<<g, 256, 0, st>>>(in, x8, scales, sg, rotate, N);
+        else attn::attn_fp8_quantize_kernel<64, false><<<g, 256, 0, st>>>(in, x8, scales, sg, rotate, N);
+    } else {
+        if (bf) attn::attn_fp8_quantize_kernel<128, true><<<g, 256, 0, st>>>(in, x8, scales, sg, rotate, N);
+        else attn::attn_fp8_quantize_kernel<128, false><<<g, 256, 0, st>>>(in, x8, scales, sg, rotate, N);
+    }
+    return launch_ok() ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+int attn_fwd_fp8(const unsigned char* q8, const unsigned char* k8, const float* q_scale,
+                 const float* k_scale, const void* v, void* o, float* lse, int B, int H, int N,
+                 int d, int causal, float scale, int rotated, attn_dtype_t dtype, void* stream) {
+    if (!q8 || !k8 || !q_scale || !k_scale || !v || !o || !lse) return ATTN_ERR_NULL;
+    int rc = check_shape(B, H, N, d, dtype, scale);
+    if (rc) return rc;
+    if (!aligned16(q8) || !aligned16(k8) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+        (reinterpret_cast<uintptr_t>(q_scale) & 3u) || (reinterpret_cast<uintptr_t>(k_scale) & 3u))
+        return ATTN_ERR_ALIGN;
+    int dev;
+    if ((rc = check_device(&dev))) return rc;
+    if (!on_device(q8, dev) || !on_device(k8, dev) || !on_device(q_scale, dev) ||
+        !on_device(k_scale, dev) || !on_device(v, dev) || !on_device(o, dev) || !on_device(lse, dev))
+        return ATTN_ERR_DEVICE;
+    const int BH = B * H;
+    CUtensorMap mq, mk, mv;
+    if (!make_map8(&mq, q8, BH, N, d) || !make_map8(&mk, k8, BH, N, d) ||
+        !make_map(&mv, v, dtype, BH, N, d))
+        return ATTN_ERR_LAUNCH;
+    attn::FwdParams p;
+    p.o = o;
+    p.lse = lse;
+    p.BH = BH;
+    p.N = N;
+    p.n_qtiles = (N + 127) / 128;
+    p.n_pairs = (p.n_qtiles + 1) / 2;
+    {
+        const long long kv_head = 1LL * N * d * 3;  // e4m3 K and 16-bit V
+        const long long g = (48LL << 20) / (kv_head > 0 ? kv_head : 1);
+        p.group = static_cast<int>(g < 1 ? 1 : (g > BH ? BH : g));
+    }
+    p.causal = causal ? 1 : 0;
+    // the rotation multiplies every dot product by d
+    p.scale_log2 = scale * 1.4426950408889634f / (rotated ? static_cast<float>(d) : 1.f);
+    p.bmask = nullptr;
+    p.n_ktiles = (N + 127) / 128;
+    p.qscale = q_scale;
+    p.kscale = k_scale;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool bf = dtype == ATTN_BF16;
+    if (d == 64)
+        return bf ? launch_fwd<64, true, true>(mq, mk, mv, p, g_sm_count[dev], st)
+                  : launch_fwd<64, false, true>(mq, mk, mv, p, g_sm_count[dev], st);
+    return bf ? launch_fwd<128, true, true>(mq, mk, mv, p, g_sm_count[dev], st)
+              : launch_fwd<128, false, true>(mq, mk, mv, p, g_sm_count[dev], st);
 }
 
 size_t attn_bwd_workspace_bytes(int B, int H, int N, int d) {
@@ -266,7 +391,8 @@ int bwd_prep_dispatch(const void* o, const void* dout, const float* lse, void* w
 
 int bwd_main_dispatch(const void* q, const void* k, const void* v, const void* dout, void* dq,
                       void* dk, void* dv, void* workspace, int B, int H, int N, int d, int causal,
-                      float scale, attn_dtype_t dtype, cudaStream_t st) {
+                      float scale, attn_dtype_t dtype, cudaStream_t st,
+                      const unsigned char* bmask = nullptr) {
     const int BH = B * H;
     CUtensorMap mq, mk, mv, mdo;
     if (!make_map(&mq, q, dtype, BH, N, d) || !make_map(&mk, k, dtype, BH, N, d) ||
@@ -276,9 +402,9 @@ int bwd_main_dispatch(const void* q, const void* k, const void* v, const void* d
     const int c = causal ? 1 : 0;
     if (d == 64)
         return bf ? attn::bwd_main_launch<64, true>(mq, mk, mv, mdo, dq, dk, dv, workspace, B, H,
-                                                    N, c, scale, st)
+                                                    N, c, scale, st, bmask)
                   : attn::bwd_main_launch<64, false>(mq, mk, mv, mdo, dq, dk, dv, workspace, B, H,
-                                                     N, c, scale, st);
+                                                     N, c, scale, st, bmask);
     // d = 128: 64-query inner tiles
     // (dK and dV leave through TMA stores)
     CUtensorMap mq64, mdo64, mdk, mdv;
@@ -289,9 +415,9 @@ int bwd_main_dispatch(const void* q, const void* k, const void* v, const void* d
     cudaGetDevice(&dev);
     const int sms = g_sm_count[dev];
     return bf ? attn::bwd_main128_launch<true>(mq64, mk, mv, mdo64, mdk, mdv, dq, dk, dv,
-                                               workspace, B, H, N, c, scale, sms, st)
+                                               workspace, B, H, N, c, scale, sms, st, bmask)
               : attn::bwd_main128_launch<false>(mq64, mk, mv, mdo64, mdk, mdv, dq, dk, dv,
-                                                workspace, B, H, N, c, scale, sms, st);
+                                                workspace, B, H, N, c, scale, sms, st, bmask);
 }
 }  // namespace
 
@@ -327,6 +453,22 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
     if ((rc = bwd_prep_dispatch(o, dout, lse, workspace, B, H, N, d, dtype, st))) return rc;
     return bwd_main_dispatch(q, k, v, dout, dq, dk, dv, workspace, B, H, N, d, causal, scale,
                              dtype, st);
+}
+
+int attn_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                         void* workspace, const unsigned char* block_mask, int B, int H, int N,
+                         int d, int causal, float scale, attn_dtype_t dtype, void* stream) {
+    const void* ptrs[11] = {q, k, v, o, lse, dout, dq, dk, dv, workspace, block_mask};
+    int dev;
+    int rc = bwd_common_checks(ptrs, 10, workspace, B, H, N, d, dtype, scale, &dev);
+    if (rc) return rc;
+    if (!block_mask) return ATTN_ERR_NULL;
+    if (!on_device(block_mask, dev)) return ATTN_ERR_DEVICE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((rc = bwd_prep_dispatch(o, dout, lse, workspace, B, H, N, d, dtype, st))) return rc;
+    return bwd_main_dispatch(q, k, v, dout, dq, dk, dv, workspace, B, H, N, d, causal, scale,
+                             dtype, st, block_mask);
 }
 
 int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
@@ -393,7 +535,7 @@ const char* attn_strerror(int status) {
         case ATTN_ERR_LAUNCH: return "the CUDA runtime rejected a launch or reported an error";
         case ATTN_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
         case ATTN_ERR_ARG: return "scale must be finite and > 0 (or a scalar argument is out of range)";
-        case ATTN_ERR_SCRATCH: return "problem needs more backward scratch than the built-in array holds";
+        case ATTN_ERR_SCRATCH: return "not enough scratch: the built-in array (attn_bwd_noalloc) or scratch_bytes (attn_sdpa_host) is too small";
         default: return "unknown status";
     }
 }
@@ -403,3 +545,162 @@ const char* attn_version(void) { return "0.1.0"; }
 const char* attn_last_cuda_error_string(void) { return cudaGetErrorString(g_last_cuda_error); }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Attention from host buffers, chunk by chunk over heads: the host-to-device
+// copies of chunk c + 1, the kernels of chunk c and the device-to-host copies
+// of chunk c - 1 run on three internal streams, so the copies over the host
+// link overlap each other and the kernels.
+namespace {
+
+constexpr int kSlots = 3;  // chunks in flight: loading, computing, draining
+
+struct HostPipe {
+    bool ready = false;
+    cudaStream_t in = nullptr, cmp = nullptr, out = nullptr;
+    cudaEvent_t start = nullptr, done = nullptr;
+    cudaEvent_t loaded[kSlots] = {}, computed[kSlots] = {}, drained[kSlots] = {};
+};
+std::mutex g_pipe_mu;
+HostPipe g_pipe[kMaxDevices];
+
+bool pipe_init(HostPipe& hp) {
+    bool ok = cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.cmp, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.done, cudaEventDisableTiming) == cudaSuccess;
+    for (int s = 0; ok && s < kSlots; ++s)
+        ok = cudaEventCreateWithFlags(&hp.loaded[s], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&hp.computed[s], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&hp.drained[s], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) g_last_cuda_error = cudaGetLastError();
+    hp.ready = ok;
+    return ok;
+}
+
+// Byte offsets of one chunk slot's tensors in the device scratch.
+struct SlotLayout {
+    size_t q, k, v, o, lse, dout, dq, dk, dv, bytes;
+};
+SlotLayout slot_layout(int hc, int N, int d, bool bwd) {
+    const size_t t = attn::align256(static_cast<size_t>(hc) * N * d * 2);
+    const size_t l = attn::align256(static_cast<size_t>(hc) * N * 4);
+    SlotLayout s{};
+    size_t off = 0;
+    s.q = off, off += t;
+    s.k = off, off += t;
+    s.v = off, off += t;
+    s.o = off, off += t;
+    s.lse = off, off += l;
+    if (bwd) {
+        s.dout = off, off += t;
+        s.dq = off, off += t;
+        s.dk = off, off += t;
+        s.dv = off, off += t;
+    }
+    s.bytes = off;
+    return s;
+}
+
+// heads per chunk: the caller's choice, else about an eighth of the heads but
+// at least 256 query tiles' worth of work per chunk
+int chunk_heads(int BH, int N, int want) {
+    if (want > 0) return want < BH ? want : BH;
+    const int n_qtiles = (N + 127) / 128;
+    int hc = (BH + 7) / 8;
+    const int fill = (256 + n_qtiles - 1) / n_qtiles;
+    if (hc < fill) hc = fill;
+    return hc < BH ? hc : BH;
+}
+
+}  // namespace
+
+extern "C" size_t attn_sdpa_host_scratch_bytes(int B, int H, int N, int d, int with_backward,
+                                               int heads_per_chunk) {
+    if (check_shape(B, H, N, d, ATTN_BF16, 1.f) != ATTN_OK) return 0;
+    const int hc = chunk_heads(B * H, N, heads_per_chunk);
+    size_t total = kSlots * slot_layout(hc, N, d, with_backward != 0).bytes;
+    if (with_backward) total += attn::align256(attn_bwd_workspace_bytes(1, hc, N, d));
+    return total;
+}
+
+extern "C" int attn_sdpa_host(const void* q, const void* k, const void* v, const void* dout,
+                              void* o, float* lse, void* dq, void* dk, void* dv, void* scratch,
+                              size_t scratch_bytes, int B, int H, int N, int d, int causal,
+                              float scale, attn_dtype_t dtype, int heads_per_chunk, void* stream) {
+    const bool bwd = dout != nullptr;
+    if (!q || !k || !v || !scratch) return ATTN_ERR_NULL;
+    if (bwd ? (!dq || !dk || !dv) : (!o || !lse)) return ATTN_ERR_NULL;
+    int rc = check_shape(B, H, N, d, dtype, scale);
+    if (rc) return rc;
+    if (scratch_bytes < attn_sdpa_host_scratch_bytes(B, H, N, d, bwd ? 1 : 0, heads_per_chunk))
+        return ATTN_ERR_SCRATCH;
+    if (!aligned16(scratch)) return ATTN_ERR_ALIGN;
+    int dev;
+    if ((rc = check_device(&dev))) return rc;
+    if (!on_device(scratch, dev)) return ATTN_ERR_DEVICE;
+
+    std::lock_guard<std::mutex> lk(g_pipe_mu);
+    HostPipe& hp = g_pipe[dev];
+    if (!hp.ready && !pipe_init(hp)) return ATTN_ERR_DEVICE;
+    cudaStream_t user = static_cast<cudaStream_t>(stream);
+    const int BH = B * H, hc = chunk_heads(BH, N, heads_per_chunk);
+    const SlotLayout L = slot_layout(hc, N, d, bwd);
+    uint8_t* base = static_cast<uint8_t*>(scratch);
+    uint8_t* ws = base + kSlots * L.bytes;
+    const size_t head_t = static_cast<size_t>(N) * d * 2, head_l = static_cast<size_t>(N) * 4;
+
+    // everything the caller queued on its stream before this call comes first
+    bool ok = cudaEventRecord(hp.start, user) == cudaSuccess &&
+              cudaStreamWaitEvent(hp.in, hp.start, 0) == cudaSuccess &&
+              cudaStreamWaitEvent(hp.cmp, hp.start, 0) == cudaSuccess &&
+              cudaStreamWaitEvent(hp.out, hp.start, 0) == cudaSuccess;
+    auto h2d = [&](uint8_t* dst, const void* src, size_t off, size_t n) {
+        ok = ok && cudaMemcpyAsync(dst, static_cast<const uint8_t*>(src) + off, n,
+                                   cudaMemcpyDefault, hp.in) == cudaSuccess;
+    };
+    auto d2h = [&](void* dst, const uint8_t* src, size_t off, size_t n) {
+        ok = ok && cudaMemcpyAsync(static_cast<uint8_t*>(dst) + off, src, n, cudaMemcpyDefault,
+                                   hp.out) == cudaSuccess;
+    };
+    for (int c = 0, h0 = 0; ok && rc == ATTN_OK && h0 < BH; ++c, h0 += hc) {
+        const int n = hc < BH - h0 ? hc : BH - h0, s = c % kSlots;
+        uint8_t* sb = base + s * L.bytes;
+        const size_t tb = n * head_t, lb = n * head_l, ot = h0 * head_t, ol = h0 * head_l;
+        // the slot's previous chunk has left the device (its kernels ran before)
+        ok = cudaStreamWaitEvent(hp.in, hp.drained[s], 0) == cudaSuccess;
+        h2d(sb + L.q, q, ot, tb);
+        h2d(sb + L.k, k, ot, tb);
+        h2d(sb + L.v, v, ot, tb);
+        if (bwd) h2d(sb + L.dout, dout, ot, tb);
+        ok = ok && cudaEventRecord(hp.loaded[s], hp.in) == cudaSuccess &&
+             cudaStreamWaitEvent(hp.cmp, hp.loaded[s], 0) == cudaSuccess;
+        if (!ok) break;
+        float* slse = reinterpret_cast<float*>(sb + L.lse);
+        rc = attn_fwd(sb + L.q, sb + L.k, sb + L.v, sb + L.o, slse, 1, n, N, d, causal, scale,
+                      dtype, hp.cmp);
+        if (rc == ATTN_OK && bwd)
+            rc = attn_bwd(sb + L.q, sb + L.k, sb + L.v, sb + L.o, slse, sb + L.dout, sb + L.dq,
+                          sb + L.dk, sb + L.dv, ws, 1, n, N, d, causal, scale, dtype, hp.cmp);
+        ok = ok && cudaEventRecord(hp.computed[s], hp.cmp) == cudaSuccess &&
+             cudaStreamWaitEvent(hp.out, hp.computed[s], 0) == cudaSuccess;
+        if (o) d2h(o, sb + L.o, ot, tb);
+        if (lse) d2h(lse, sb + L.lse, ol, lb);
+        if (bwd) {
+            d2h(dq, sb + L.dq, ot, tb);
+            d2h(dk, sb + L.dk, ot, tb);
+            d2h(dv, sb + L.dv, ot, tb);
+        }
+        ok = ok && cudaEventRecord(hp.drained[s], hp.out) == cudaSuccess;
+    }
+    // the caller's stream continues after the last copy, also after an error,
+    // so that nothing it frees is still in use
+    const bool fin = cudaEventRecord(hp.done, hp.out) == cudaSuccess &&
+                     cudaStreamWaitEvent(user, hp.done, 0) == cudaSuccess;
+    if (!ok || !fin) {
+        g_last_cuda_error = cudaGetLastError();
+        if (rc == ATTN_OK) rc = ATTN_ERR_LAUNCH;
+    }
+    return rc;
+}

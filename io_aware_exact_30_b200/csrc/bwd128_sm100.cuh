@@ -98,6 +98,32 @@ __device__ __forceinline__ void bwd_item(const BwdParams& p, int k, int& bh, int
     }
 }
 
+// The 64-row query tiles an item (head, key tile j) works through: from the
+// causal start on, and under a block mask only those whose 128-row query tile
+// is marked for key tile j.  Every role walks the same sequence.
+struct Bwd128Tiles {
+    int begin, end;      // candidate 64-row tiles [begin, end)
+    const uint8_t* col;  // mask column of key tile j (stride n_ktiles), nullptr: dense
+    int stride;
+    __device__ Bwd128Tiles(const BwdParams& p, int j, int n_q64)
+        : begin(p.causal ? 2 * j : 0), end(n_q64), col(p.bmask ? p.bmask + j : nullptr),
+          stride(p.n_ktiles) {}
+    __device__ bool act(int i) const { return col == nullptr || col[(i >> 1) * stride] != 0; }
+    __device__ int from(int i) const {
+        if (col == nullptr) return i;
+        while (i < end && !act(i)) ++i;
+        return i;
+    }
+    __device__ int first() const { return from(begin); }
+    __device__ int next(int i) const { return from(i + 1); }
+    __device__ int count() const {
+        if (col == nullptr) return end - begin;
+        int n = 0;
+        for (int i = begin; i < end; ++i) n += act(i);
+        return n;
+    }
+};
+
 template <bool BF16>
 __global__ void __launch_bounds__(480, 1)
     attn_bwd_main128_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -167,8 +193,8 @@ __global__ void __launch_bounds__(480, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    ItemStream cs(p.causal != 0, p.BH * p.n_ktiles, base + C::OFF_CLC, BAR(C::B_CLCF),
-                  BAR(C::B_CLCE));
+    ItemStream cs(p.causal != 0 || p.bmask != nullptr, p.BH * p.n_ktiles, base + C::OFF_CLC,
+                  BAR(C::B_CLCF), BAR(C::B_CLCE));
 
     if (warp == C::WARP_TMA) {
         // ------------------------------------------------------ TMA producer
@@ -202,12 +228,15 @@ __global__ void __launch_bounds__(480, 1)
             };
             while (ok && cs.cur >= 0) {
                 bwd_item(p, cs.cur, bh, j);
-                const int i_begin = p.causal ? 2 * j : 0;
-                const int n_it = n_q64 - i_begin;
+                const Bwd128Tiles tl(p, j, n_q64);
+                const int n_it = tl.count();
                 const int pre = min(C::ST, n_it);
+                int qi = tl.first();
                 // The item's first query tiles go ahead of its K/V, which wait
-                // until the previous item's MMAs are done with K and V.
-                for (int it = 0; ok && it < pre; ++it) ok = load_tile(i_begin + it);
+                // until the previous item's MMAs are done with K and V.  (K and V
+                // are loaded even for an item without query tiles: its dK, dV
+                // are zero, but the per-item handshakes stay in step.)
+                for (int it = 0; ok && it < pre; ++it, qi = tl.next(qi)) ok = load_tile(qi);
                 if (!ok) break;
                 if (items > 0 && !(ok = wait_bounded(BAR(C::B_KVE), (items - 1) & 1, abort_flag)))
                     break;
@@ -220,7 +249,7 @@ __global__ void __launch_bounds__(480, 1)
                                 bh);
                 }
                 ++items;
-                for (int it = pre; ok && it < n_it; ++it) ok = load_tile(i_begin + it);
+                for (int it = pre; ok && it < n_it; ++it, qi = tl.next(qi)) ok = load_tile(qi);
                 // once an item's loads are issued, ask for the next item, and start
                 // its K and V on their way into L2 (they are loaded into shared
                 // memory only when this item's MMAs release K and V)
@@ -273,15 +302,16 @@ __global__ void __launch_bounds__(480, 1)
             };
             while (ok && cs.cur >= 0) {
                 bwd_item(p, cs.cur, bh, j);
-                const int n_it = n_q64 - (p.causal ? 2 * j : 0);
+                const int n_it = Bwd128Tiles(p, j, n_q64).count();
                 if (is_a) {
                     // the item's K, V; Q_g; dV(g-2), the last reader of S buffer g & 1
+                    // (an item without query tiles only waits for its K and V to land)
                     if (!(ok = wait3(BAR(C::B_KV), items & 1, true, BAR(C::B_QF + g % C::ST),
-                                     (g / C::ST) & 1, true, BAR(C::B_DVD + (g & 1)),
-                                     ((g - 2) >> 1) & 1, g >= 2, abort_flag)))
+                                     (g / C::ST) & 1, n_it > 0, BAR(C::B_DVD + (g & 1)),
+                                     ((g - 2) >> 1) & 1, n_it > 0 && g >= 2, abort_flag)))
                         break;
                     tc_fence_after();
-                    issue_s(g);
+                    if (n_it > 0) issue_s(g);
                     for (int it = 0; ok && it < n_it; ++it, ++g) {
                         const int s = g % C::ST, g1 = g + 1;
                         const bool more = it + 1 < n_it;
@@ -380,11 +410,12 @@ __global__ void __launch_bounds__(480, 1)
         bool dq_ok = true;
         while (dq_ok && cs.cur >= 0) {
             bwd_item(p, cs.cur, bh, j);
-            const int i_begin = p.causal ? 2 * j : 0;
-            const int n_it = n_q64 - i_begin;
+            const Bwd128Tiles tl(p, j, n_q64);
+            const int n_it = tl.count();
             float* acc_head = p.dqacc + static_cast<size_t>(bh) * p.N * D;
-            for (int it = 0; it < n_it; ++it, ++g) {
-                const int q0 = (i_begin + it) * 64;
+            int qi = tl.first();
+            for (int it = 0; it < n_it; ++it, ++g, qi = tl.next(qi)) {
+                const int q0 = qi * 64;
                 if (!(dq_ok = __all_sync(0xffffffffu,
                                          wait_bounded(BAR(C::B_DQF), g & 1, abort_flag))))
                     break;
@@ -423,6 +454,8 @@ __global__ void __launch_bounds__(480, 1)
                 dq_ok = __all_sync(0xffffffffu, dq_ok);
                 if (!dq_ok) break;
             }
+            // an item without query tiles leaves the staging tile as it was
+            if (dq_ok && n_it == 0 && issuer) mbar_arrive(BAR(C::B_DQD));
             if (dq_ok) dq_ok = cs.advance(abort_flag, true);
         }
         if (issuer) bulk_wait_all();  // every reduction complete before the CTA exits
@@ -438,12 +471,13 @@ __global__ void __launch_bounds__(480, 1)
         bool ok = true;
         while (ok && cs.cur >= 0) {
             bwd_item(p, cs.cur, bh, j);
-            const int i_begin = p.causal ? 2 * j : 0;
-            const int n_it = n_q64 - i_begin;
+            const Bwd128Tiles tl(p, j, n_q64);
+            const int n_it = tl.count();
             const int key = j * 128 + r;
             const bool key_valid = key < p.N;
-            for (int it = 0; it < n_it; ++it, ++g) {
-                const int q0 = (i_begin + it) * 64;
+            int qi = tl.first();
+            for (int it = 0; it < n_it; ++it, ++g, qi = tl.next(qi)) {
+                const int q0 = qi * 64;
                 const uint32_t ph = g & 1;
                 const int s = g % C::ST;
                 const float4* L4 = reinterpret_cast<const float4*>(sLD + s * 128 + c0);
@@ -558,6 +592,11 @@ __global__ void __launch_bounds__(480, 1)
                 tmem_ld32(lane_addr + C::COL_DK + half * 64u + c * 32u, v);
                 tmem_ld_wait();
                 reg_fence32(v);
+                // no query tile was marked for this key tile: dK = dV = 0 (the
+                // accumulators still hold an earlier item's values)
+                if (n_it == 0)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = 0u;
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
                     hk[16 * c + e] = pack2<BF16>(__uint_as_float(v[2 * e]) * p.scale,
@@ -565,6 +604,9 @@ __global__ void __launch_bounds__(480, 1)
                 tmem_ld32(lane_addr + C::COL_DV + half * 64u + c * 32u, v);
                 tmem_ld_wait();
                 reg_fence32(v);
+                if (n_it == 0)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = 0u;
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
                     hv[16 * c + e] =
@@ -647,8 +689,10 @@ template <bool BF16>
 int bwd_main128_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                        const CUtensorMap& mdo, const CUtensorMap& mdk, const CUtensorMap& mdv,
                        void* dq, void* dk, void* dv, void* ws, int B, int H, int N, int causal,
-                       float scale, int sm_count, cudaStream_t st) {
+                       float scale, int sm_count, cudaStream_t st,
+                       const uint8_t* bmask = nullptr) {
     BwdParams p;
+    p.bmask = bmask;
     uint8_t* w = static_cast<uint8_t*>(ws);
     p.l2pad = reinterpret_cast<const float*>(w);
     p.dpad = reinterpret_cast<const float*>(w + bwd_ws_off_d(B, H, N));
@@ -673,7 +717,8 @@ int bwd_main128_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     }
     const long long items = 1LL * p.n_ktiles * p.BH;
     if (items >= (1LL << 31)) return -2;
-    const int nblocks = static_cast<int>(causal || items < sm_count ? items : sm_count);
+    const bool dynamic = causal || bmask != nullptr;
+    const int nblocks = static_cast<int>(dynamic || items < sm_count ? items : sm_count);
     attn_bwd_main128_kernel<BF16><<<static_cast<unsigned>(nblocks), Bwd128Cfg::NTHREADS,
                                     Bwd128Cfg::SMEM_BYTES, st>>>(mq, mk, mv, mdo, mdk, mdv, p);
     cudaError_t e = cudaGetLastError();

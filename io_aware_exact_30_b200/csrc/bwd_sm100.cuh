@@ -131,6 +131,10 @@ struct BwdParams {
     int causal;
     float scale;
     float scale_log2;
+    // Block-sparse attention: n_qtiles128 x n_ktiles bytes, nonzero where the
+    // 128-row query tile i may attend to key tile j (one mask for every head);
+    // nullptr for dense attention.
+    const uint8_t* bmask = nullptr;
 };
 
 template <int D>
@@ -181,7 +185,19 @@ __global__ void __launch_bounds__(320, 1)
     const int bh = static_cast<int>(blockIdx.x) / p.n_ktiles;
     const int j = static_cast<int>(blockIdx.x) % p.n_ktiles;
     const int i_begin = p.causal ? j : 0;
-    const int n_it = p.n_qtiles - i_begin;
+    // Query tiles i = i_begin .., and under a block mask only those marked for
+    // key tile j; every role walks the same sequence (next_tile).
+    const uint8_t* mcol = p.bmask ? p.bmask + j : nullptr;
+    auto next_tile = [&](int i) {
+        if (mcol != nullptr)
+            while (i < p.n_qtiles && mcol[static_cast<size_t>(i) * p.n_ktiles] == 0) ++i;
+        return i;
+    };
+    int n_it = p.n_qtiles - i_begin;
+    if (mcol != nullptr) {
+        n_it = 0;
+        for (int i = next_tile(i_begin); i < p.n_qtiles; i = next_tile(i + 1)) ++n_it;
+    }
 
     const uint32_t bar0 = base + C::OFF_BAR;
 #define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
@@ -242,8 +258,7 @@ __global__ void __launch_bounds__(320, 1)
             for (int s = 0; s < C::QST; ++s) q_issued[s] = 0;
             for (int s = 0; s < C::DOST; ++s) do_issued[s] = 0;
             const size_t ld_row0 = static_cast<size_t>(bh) * p.Np;
-            for (int it = 0; it < n_it; ++it) {
-                const int i = i_begin + it;
+            for (int it = 0, i = next_tile(i_begin); it < n_it; ++it, i = next_tile(i + 1)) {
                 const int qs = it % C::QST, qn = it / C::QST;
                 const int ds = it % C::DOST, dn = it / C::DOST;
                 if (!wait_bounded(BAR(C::B_QE + qs), (qn & 1) ^ 1, abort_flag)) break;
@@ -357,8 +372,7 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t sDST = base + C::OFF_DST;
         const int c0 = half * 64;  // first query column of this thread's half
         bool ok = true;
-        for (int it = 0; it < n_it; ++it) {
-            const int i = i_begin + it;
+        for (int it = 0, i = next_tile(i_begin); it < n_it; ++it, i = next_tile(i + 1)) {
             const int q0 = i * 128;
             const uint32_t ph = it & 1;
             const float4* L4 = reinterpret_cast<const float4*>(sLD + (it % C::QST) * 256 + c0);
@@ -488,6 +502,9 @@ __global__ void __launch_bounds__(320, 1)
                     tmem_ld32(lane_addr + col + c * 32u, v);
                     tmem_ld_wait();
                     reg_fence32(v);
+                    if (n_it == 0)  // block-sparse: no query tile marked, dK = dV = 0
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) v[e] = 0u;
                     uint32_t h[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
@@ -569,8 +586,10 @@ int bwd_prep_launch(const void* o, const void* dout, const float* lse, void* ws,
 template <int D, bool BF16>
 int bwd_main_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                     const CUtensorMap& mdo, void* dq, void* dk, void* dv, void* ws, int B, int H,
-                    int N, int causal, float scale, cudaStream_t st) {
+                    int N, int causal, float scale, cudaStream_t st,
+                    const uint8_t* bmask = nullptr) {
     BwdParams p;
+    p.bmask = bmask;
     uint8_t* w = static_cast<uint8_t*>(ws);
     p.l2pad = reinterpret_cast<const float*>(w);
     p.dpad = reinterpret_cast<const float*>(w + bwd_ws_off_d(B, H, N));

@@ -54,11 +54,21 @@ struct FwdParams {
     int group;           // heads per scheduling group (their K/V fit in L2)
     int causal;
     float scale_log2;    // scale * log2(e)
+    // Block-sparse attention: n_qtiles x n_ktiles bytes, nonzero where query
+    // tile i may attend to key tile j (128 x 128 blocks, one mask for every
+    // head); nullptr for dense attention.
+    const uint8_t* bmask;
+    int n_ktiles;
+    // FP8 scores (fp8_sm100.cuh): per-(head, 128-row block) dequantisation
+    // scales of the e4m3 Q and K; scale_log2 then also holds the 1/d of the
+    // rotation.  nullptr for 16-bit Q and K.
+    const float* qscale;
+    const float* kscale;
 };
 
 // Persistent schedule.  A work item is (head, pair of query tiles); there are
 // BH * n_pairs of them, taken through an ItemStream: dynamically under the
-// causal mask (unequal costs), in static snake order otherwise.  Heads are taken in groups of
+// causal mask or a block mask (unequal costs), in static snake order otherwise.  Heads are taken in groups of
 // `group` heads whose K/V fit comfortably in L2 together; within a group the
 // items are listed heaviest first — under the causal mask pair p costs 4p + 3
 // key-tile steps, so the group's list runs from the last pair down, heads in
@@ -77,27 +87,56 @@ __device__ __forceinline__ void fwd_item(const FwdParams& p, int k, int& bh, int
     }
 }
 
+// Key tiles of a work item.  Query tile t of the pair attends to key tile j
+// iff act(t, j): j below its causal bound and, under a block mask, marked.
+// K and V are loaded for the union of both tiles' key tiles, walked in order
+// by every role (next() gives the union's next tile); without a mask the
+// union is 0 .. nkv - 1.
 struct FwdItemShape {
     bool has1;
     int nkv_t[2];
     int nkv;
+    const uint8_t* mrow[2];  // mask rows of the two query tiles (nullptr: dense)
     __device__ FwdItemShape(const FwdParams& p, int pair) {
         const int n_kv_all = (p.N + 127) >> 7;
         has1 = 2 * pair + 1 < p.n_qtiles;
         nkv_t[0] = p.causal ? min(n_kv_all, 2 * pair + 1) : n_kv_all;
         nkv_t[1] = has1 ? (p.causal ? min(n_kv_all, 2 * pair + 2) : n_kv_all) : 0;
         nkv = max(nkv_t[0], nkv_t[1]);
+        mrow[0] = p.bmask ? p.bmask + static_cast<size_t>(2 * pair) * p.n_ktiles : nullptr;
+        mrow[1] = p.bmask && has1 ? mrow[0] + p.n_ktiles : nullptr;
+    }
+    __device__ bool act(int t, int j) const {
+        return j < nkv_t[t] && (mrow[t] == nullptr || mrow[t][j] != 0);
+    }
+    __device__ bool any(int j) const { return act(0, j) || act(1, j); }
+    // first union tile at or after j (nkv if none)
+    __device__ int from(int j) const {
+        if (mrow[0] == nullptr) return j;
+        while (j < nkv && !any(j)) ++j;
+        return j;
+    }
+    __device__ int first() const { return from(0); }
+    __device__ int next(int j) const { return from(j + 1); }
+    // number of key tiles query tile t attends to
+    __device__ int count(int t) const {
+        if (mrow[t] == nullptr) return nkv_t[t];
+        int n = 0;
+        for (int j = 0; j < nkv_t[t]; ++j) n += mrow[t][j] != 0;
+        return n;
     }
 };
 
-template <int D>
+template <int D, bool FP8 = false>
 struct FwdCfg {
     static constexpr int KB = D / 64;                 // 64-column swizzle blocks per row
-    static constexpr uint32_t TILE = 128u * D * 2u;   // bytes of a 128 x D half tile
-    static constexpr int STAGES = D == 64 ? 4 : 2;
+    static constexpr uint32_t TILE = 128u * D * 2u;   // bytes of a 128 x D half tile (V)
+    // Q and K tiles: half, or e4m3 (one 128- or 64-byte swizzled box per row)
+    static constexpr uint32_t QKTILE = FP8 ? 128u * D : TILE;
+    static constexpr int STAGES = D == 64 ? 4 : (FP8 ? 3 : 2);
     static constexpr uint32_t OFF_Q = 0;              // two query tiles
-    static constexpr uint32_t OFF_K = OFF_Q + 2 * TILE;
-    static constexpr uint32_t OFF_V = OFF_K + STAGES * TILE;
+    static constexpr uint32_t OFF_K = OFF_Q + 2 * QKTILE;
+    static constexpr uint32_t OFF_V = OFF_K + STAGES * QKTILE;
     static constexpr uint32_t OFF_BAR = OFF_V + STAGES * TILE;
     static constexpr int B_Q = 0, B_KF = 1, B_VF = B_KF + STAGES, B_KE = B_VF + STAGES,
                          B_SF = B_KE + STAGES, B_PF = B_SF + 2, B_OD = B_PF + 2, B_DR = B_OD + 2,
@@ -112,17 +151,18 @@ struct FwdCfg {
     static constexpr uint32_t COL_O = 256;
     static constexpr int NTHREADS = 320;
     static constexpr int WARP_TMA = 8, WARP_MMA = 9;
+    static_assert(SMEM_BYTES <= 232448u, "dynamic shared memory above the sm_100 per-block limit");
 };
 
 // Move the running max (and rescale O) only when the row max grows by more
 // than this many binary orders of magnitude.
 constexpr float kRescaleThreshold = 8.f;
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool FP8 = false>
 __global__ void __launch_bounds__(320, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-    using C = FwdCfg<D>;
+    using C = FwdCfg<D, FP8>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -165,8 +205,8 @@ __global__ void __launch_bounds__(320, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    ItemStream cs(p.causal != 0, p.BH * p.n_pairs, base + C::OFF_CLC, BAR(C::B_CLCF),
-                  BAR(C::B_CLCE));
+    ItemStream cs(p.causal != 0 || p.bmask != nullptr, p.BH * p.n_pairs, base + C::OFF_CLC,
+                  BAR(C::B_CLCF), BAR(C::B_CLCE));
 
     if (warp == C::WARP_TMA) {
         // ------------------------------------------------------ TMA producer
@@ -187,22 +227,33 @@ __global__ void __launch_bounds__(320, 1)
                 // the previous item's S MMAs are done reading the query tiles
                 if (items > 0 && !(ok = wait_bounded(BAR(C::B_QE), (items - 1) & 1, abort_flag)))
                     break;
-                mbar_arrive_expect_tx(BAR(C::B_Q), sh.has1 ? 2 * C::TILE : C::TILE);
-                for (int t = 0; t < (sh.has1 ? 2 : 1); ++t)
+                mbar_arrive_expect_tx(BAR(C::B_Q), sh.has1 ? 2 * C::QKTILE : C::QKTILE);
+                for (int t = 0; t < (sh.has1 ? 2 : 1); ++t) {
+                    if constexpr (FP8) {
+                        tma_load_3d(base + C::OFF_Q + t * C::QKTILE, &tmQ, BAR(C::B_Q), 0,
+                                    (2 * pair + t) * 128, bh);
+                    } else {
 #pragma unroll
-                    for (int kb = 0; kb < C::KB; ++kb)
-                        tma_load_3d(base + C::OFF_Q + t * C::TILE + kb * 16384u, &tmQ, BAR(C::B_Q),
-                                    kb * 64, (2 * pair + t) * 128, bh);
+                        for (int kb = 0; kb < C::KB; ++kb)
+                            tma_load_3d(base + C::OFF_Q + t * C::QKTILE + kb * 16384u, &tmQ,
+                                        BAR(C::B_Q), kb * 64, (2 * pair + t) * 128, bh);
+                    }
+                }
                 ++items;
-                for (int j = 0; j < sh.nkv; ++j, ++kv) {
+                for (int j = sh.first(); j < sh.nkv; j = sh.next(j), ++kv) {
                     const int s = kv % C::STAGES, n = kv / C::STAGES;
                     if (!(ok = wait_bounded(BAR(C::B_KE + s), (n & 1) ^ 1, abort_flag))) break;
-                    const uint32_t sk = base + C::OFF_K + s * C::TILE;
+                    const uint32_t sk = base + C::OFF_K + s * C::QKTILE;
                     const uint32_t sv = base + C::OFF_V + s * C::TILE;
-                    mbar_arrive_expect_tx(BAR(C::B_KF + s), C::TILE);
+                    mbar_arrive_expect_tx(BAR(C::B_KF + s), C::QKTILE);
+                    if constexpr (FP8) {
+                        tma_load_3d(sk, &tmK, BAR(C::B_KF + s), 0, j * 128, bh);
+                    } else {
 #pragma unroll
-                    for (int kb = 0; kb < C::KB; ++kb)
-                        tma_load_3d(sk + kb * 16384u, &tmK, BAR(C::B_KF + s), kb * 64, j * 128, bh);
+                        for (int kb = 0; kb < C::KB; ++kb)
+                            tma_load_3d(sk + kb * 16384u, &tmK, BAR(C::B_KF + s), kb * 64, j * 128,
+                                        bh);
+                    }
                     mbar_arrive_expect_tx(BAR(C::B_VF + s), C::TILE);
 #pragma unroll
                     for (int kb = 0; kb < C::KB; ++kb)
@@ -229,15 +280,30 @@ __global__ void __launch_bounds__(320, 1)
         // running counts across the CTA's work items.
         if (lane == 0) {
             constexpr uint32_t ID_S = idesc_f16(BF16, 128, 128, false, false);
+            constexpr uint32_t ID_S8 = idesc_f16(false, 128, 128, false, false);  // e4m3 x e4m3
             constexpr uint32_t ID_O = idesc_f16(BF16, 128, D, false, true);
             auto issue_s = [&](int t, int kvi) {
-                const uint32_t sq = base + C::OFF_Q + t * C::TILE;
-                const uint32_t sk = base + C::OFF_K + (kvi % C::STAGES) * C::TILE;
+                const uint32_t sq = base + C::OFF_Q + t * C::QKTILE;
+                const uint32_t sk = base + C::OFF_K + (kvi % C::STAGES) * C::QKTILE;
+                if constexpr (FP8) {
+                    // e4m3 rows of D bytes, one swizzled box: K = 32 per step, 32 bytes
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                    mma_ss(tmem + t * 128u, sdesc_sw128(sq + off, 16, 1024),
-                           sdesc_sw128(sk + off, 16, 1024), ID_S, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < D / 32; ++kk) {
+                        const uint32_t off = kk * 32u;
+                        if constexpr (D == 128)
+                            mma_ss_f8(tmem + t * 128u, sdesc_sw128(sq + off, 16, 1024),
+                                      sdesc_sw128(sk + off, 16, 1024), ID_S8, kk > 0 ? 1u : 0u);
+                        else
+                            mma_ss_f8(tmem + t * 128u, sdesc_sw64(sq + off, 16, 512),
+                                      sdesc_sw64(sk + off, 16, 512), ID_S8, kk > 0 ? 1u : 0u);
+                    }
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                        mma_ss(tmem + t * 128u, sdesc_sw128(sq + off, 16, 1024),
+                               sdesc_sw128(sk + off, 16, 1024), ID_S, kk > 0 ? 1u : 0u);
+                    }
                 }
                 mma_commit(BAR(C::B_SF + t));
             };
@@ -246,46 +312,55 @@ __global__ void __launch_bounds__(320, 1)
             for (; ok && cs.cur >= 0; ok = ok && cs.advance(abort_flag, false)) {
                 fwd_item(p, cs.cur, bh, pair);
                 const FwdItemShape sh(p, pair);
-                // Q of this item, K_0, and for each tile t the previous item's
-                // last P_t V, which read the columns S_t is about to take.
-                // Waits test all their barriers at once: a dependent wait stalls
-                // the issue of queued MMAs, so one stall per group.
-                const bool w0 = sh.nkv_t[0] > 0 && n_pv[0] > 0, w1 = sh.nkv_t[1] > 0 && n_pv[1] > 0;
+                const int j0 = sh.first();
+                // Q of this item, K of its first key tile, and for each tile t
+                // that starts there the last P_t V issued (in any earlier item),
+                // which read the columns S_t is about to take.  Waits test all
+                // their barriers at once: a dependent wait stalls the issue of
+                // queued MMAs, so one stall per group.
+                const bool a0 = j0 < sh.nkv && sh.act(0, j0), a1 = j0 < sh.nkv && sh.act(1, j0);
+                const bool w0 = a0 && n_pv[0] > 0, w1 = a1 && n_pv[1] > 0;
                 if (!(ok = wait3(BAR(C::B_Q), items & 1, true, BAR(C::B_KF + kv % C::STAGES),
-                                 (kv / C::STAGES) & 1, true, BAR(C::B_OD), (n_pv[0] - 1) & 1, w0,
-                                 abort_flag)))
+                                 (kv / C::STAGES) & 1, j0 < sh.nkv, BAR(C::B_OD), (n_pv[0] - 1) & 1,
+                                 w0, abort_flag)))
                     break;
                 if (w1 && !(ok = wait_bounded(BAR(C::B_OD + 1), (n_pv[1] - 1) & 1, abort_flag)))
                     break;
                 tc_fence_after();
-                for (int t = 0; t < 2; ++t)
-                    if (sh.nkv_t[t] > 0) issue_s(t, kv);
-                for (int j = 0; ok && j < sh.nkv; ++j) {
-                    const int kvj = kv + j;
+                if (a0) issue_s(0, kv);
+                if (a1) issue_s(1, kv);
+                bool first_pv[2] = {true, true};  // no P_t V of this item issued yet
+                int u = 0;                        // union key tiles of this item so far
+                for (int j = j0, jn; ok && j < sh.nkv; j = jn, ++u) {
+                    jn = sh.next(j);
+                    const int kvj = kv + u;
                     const int s = kvj % C::STAGES, n = kvj / C::STAGES;
                     const uint32_t sv = base + C::OFF_V + s * C::TILE;
                     const int k1 = kvj + 1;
-                    bool k_next = false;  // K_{j+1} has landed
+                    bool k_next = false;  // K of the next union tile has landed
                     for (int t = 0; ok && t < 2; ++t) {
-                        const bool act = j < sh.nkv_t[t];
-                        // V_j (first tile only), P_t, and at an item's first j the
-                        // previous epilogue's read of O_t, which P_t V overwrites
+                        const bool act = sh.act(t, j);
+                        // V_j (first tile only), P_t, and at the item's first P_t V
+                        // the previous epilogue's read of O_t, which P_t V overwrites
                         if (!(ok = wait3(BAR(C::B_VF + s), n & 1, t == 0, BAR(C::B_PF + t),
                                          n_pv[t] & 1, act, BAR(C::B_OE + t), (n_done[t] - 1) & 1,
-                                         act && j == 0 && n_done[t] > 0, abort_flag)))
+                                         act && first_pv[t] && n_done[t] > 0, abort_flag)))
                             break;
-                        if (!act) continue;
-                        tc_fence_after();
+                        if (act) {
+                            tc_fence_after();
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            mma_ts(tmem + C::COL_O + t * D, tmem + t * 128u + kk * 8u,
-                                   sdesc_sw128(sv + kk * 2048u, 16384, 1024), ID_O,
-                                   (j > 0 || kk > 0) ? 1u : 0u);
-                        mma_commit(BAR(C::B_OD + t));
-                        ++n_pv[t];
-                        if (j + 1 < sh.nkv_t[t]) {
-                            // O_t += P_t V_j has read P_t: its columns may take the next S
-                            if (!(ok = wait3(BAR(C::B_OD + t), (n_pv[t] - 1) & 1, true,
+                            for (int kk = 0; kk < 8; ++kk)
+                                mma_ts(tmem + C::COL_O + t * D, tmem + t * 128u + kk * 8u,
+                                       sdesc_sw128(sv + kk * 2048u, 16384, 1024), ID_O,
+                                       (!first_pv[t] || kk > 0) ? 1u : 0u);
+                            mma_commit(BAR(C::B_OD + t));
+                            ++n_pv[t];
+                            first_pv[t] = false;
+                        }
+                        if (jn < sh.nkv && sh.act(t, jn)) {
+                            // S_t of the next union tile, into the columns the last
+                            // P_t V read once it has completed
+                            if (!(ok = wait3(BAR(C::B_OD + t), (n_pv[t] - 1) & 1, n_pv[t] > 0,
                                              BAR(C::B_KF + k1 % C::STAGES), (k1 / C::STAGES) & 1,
                                              !k_next, 0u, 0u, false, abort_flag)))
                                 break;
@@ -299,10 +374,10 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 if (!ok) break;
                 mma_commit(BAR(C::B_QE));  // every S of this item is issued
-                kv += sh.nkv;
+                kv += u;
                 ++items;
                 for (int t = 0; t < 2; ++t)
-                    if (sh.nkv_t[t] > 0) ++n_done[t];
+                    if (!first_pv[t]) ++n_done[t];
             }
             if (*abort_flag) {  // every issued MMA must finish before TMEM is freed
                 mma_commit(BAR(C::B_DR));
@@ -316,17 +391,27 @@ __global__ void __launch_bounds__(320, 1)
         const int r = threadIdx.x & 127;  // row of the tile == TMEM lane
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         const uint32_t colS = t * 128u, colO = C::COL_O + t * D;
-        const float sl = p.scale_log2;
         int n_s = 0, bh, pair;  // S tiles of this query-tile slot seen so far
         bool ok = true;
         for (; ok && cs.cur >= 0; ok = ok && cs.advance(abort_flag, true)) {
             fwd_item(p, cs.cur, bh, pair);
-            const FwdItemShape sh(p, pair);
-            const int my_nkv = sh.nkv_t[t];
-            if (my_nkv == 0) continue;
+            int my_nkv;
+            const uint8_t* my_row;  // this tile's block-mask row (nullptr: dense)
+            {
+                const FwdItemShape sh(p, pair);
+                my_nkv = sh.nkv_t[t];
+                my_row = sh.mrow[t];
+            }
+            if (my_nkv == 0) continue;  // the pair has no second tile
             const int qrow = (2 * pair + t) * 128 + r;
+            float sl_q = p.scale_log2;  // score multiplier (log2 units), times the Q block scale
+            if constexpr (FP8) sl_q *= p.qscale[static_cast<size_t>(bh) * p.n_qtiles + 2 * pair + t];
             float m = -INFINITY, l = 0.f;
+            int seen = 0;  // key tiles of this item this tile has processed
             for (int j = 0; j < my_nkv; ++j) {
+                if (my_row != nullptr && my_row[j] == 0) continue;
+                float sl = sl_q;
+                if constexpr (FP8) sl *= p.kscale[static_cast<size_t>(bh) * p.n_ktiles + j];
                 ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SF + t), n_s & 1, abort_flag));
                 if (!ok) break;
                 ++n_s;
@@ -370,7 +455,7 @@ __global__ void __launch_bounds__(320, 1)
                 if (__any_sync(0xffffffffu, move)) {
                     const float m_new = move ? m_tile : m;
                     const float alpha = ex2(m - m_new);  // 0 on the first tile, 1 if not moved
-                    if (j > 0) {
+                    if (seen > 0) {
                         ok = __all_sync(0xffffffffu,
                                         wait_bounded(BAR(C::B_OD + t), (n_s - 2) & 1, abort_flag));
                         if (!ok) break;
@@ -434,6 +519,20 @@ __global__ void __launch_bounds__(320, 1)
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(BAR(C::B_PF + t));
+                ++seen;
+            }
+            if (ok && seen == 0) {
+                // block-sparse: no key tile is marked for this query tile, so no
+                // row has a visible key; O = 0 and LSE = -inf (the empty sum)
+                if (qrow < p.N) {
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.o) +
+                                                          (static_cast<size_t>(bh) * p.N + qrow) *
+                                                              (D * 2));
+#pragma unroll
+                    for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+                    p.lse[static_cast<size_t>(bh) * p.N + qrow] = -INFINITY;
+                }
+                continue;
             }
             if (ok)
                 ok = __all_sync(0xffffffffu,

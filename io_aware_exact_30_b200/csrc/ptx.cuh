@@ -260,6 +260,17 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// D(tmem) (+)= A(smem desc) * B(smem desc), kind::f8f6f4 (here e4m3 x e4m3 in,
+// fp32 accumulate; K = 32 per instruction).
+__device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 // Arrive once on `bar` when every tcgen05 op issued so far by this thread is done.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile(
@@ -331,7 +342,19 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
            (2ull << 61);
 }
 
-// Instruction descriptor for kind::f16 with fp32 accumulation.
+// The same descriptor for a K-major tile stored with the 64-byte swizzle
+// (8-row, 512-byte atoms; layout code 4); tiles 512-byte aligned.
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr, uint32_t lbo_bytes,
+                                               uint32_t sbo_bytes) {
+    return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) |
+           (static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+           (static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) |
+           (4ull << 61);
+}
+
+// Instruction descriptor for kind::f16 with fp32 accumulation.  (For
+// kind::f8f6f4 the same fields hold e4m3 as format code 0, so
+// idesc_f16(false, ...) also describes an e4m3 x e4m3 -> fp32 product.)
 //   bits 4-5 D format (1 = f32), 7-9 A format, 10-12 B format (0 = f16,
 //   1 = bf16), 15 A major (1 = MN), 16 B major (1 = MN), 17-22 N >> 3,
 //   24-28 M >> 4.

@@ -150,20 +150,31 @@ RESCALE_LOG2_THRESHOLD = 8.0
 
 def rescale_inputs(pattern, B, H, N, d, dtype="bf16", seed=0):
     """Seeded Q, K, V, dO (storage arrays and exact f64 values) shaped so that
-    row maxima keep growing along the keys.
+    row maxima jump along the keys.
 
-    ``ramp``: key row j is scaled by 1 + 3 j / 64, so each later key tile
-    holds larger scores; odd query rows are scaled by 0.2, so within a warp
-    some rows move their max at a tile and others do not.
+    ``steps``: every coordinate of key row j gets the offset 3.5 min(t, 2) /
+    sqrt(d), t = j // 128, and every coordinate of query row i the offset 2
+    (even rows) or 0.6 (odd rows), on top of N(0, 0.5^2) noise.  An even row's
+    scores then step up by about 7 (10 in log2 units) at key tiles 1 and 2 and
+    stay level after, spread within each tile; odd rows step by about 2, so
+    within a warp some rows move their max at a tile and others do not.  (A
+    key offset shared by the keys that carry the weight cancels in
+    dQ = scale dS K and so amplifies the rounding of D = rowsum(dO O), taken
+    from the stored O; the steps therefore stop at tile 2, spreading the
+    weight over several tiles, and the step comes mostly from the query side.)
     ``shared``: K = Q (sigma 1.2), so under the causal mask a row's own
     diagonal score (about sqrt(d) sigma^2) dwarfs those of the first key tile.
+    V is N(0, 0.25^2) in both (a power-of-two scaling of the generator's
+    values, so exact): with only a few keys carrying the weight, O is close to
+    single V rows, and at |O| ~ 4 the output's own bf16 rounding (half an ulp
+    is 2^-6) would exceed the 1e-2 bar.
     """
     arrs = synth.attention_inputs(B, H, N, d, seed=seed, sigma=1.0, dtype=dtype, with_dout=True)
     z = [synth.to_f64(a, dtype) for a in arrs]
-    if pattern == "ramp":
-        rq = np.where(np.arange(N) % 2 == 0, 1.0, 0.2)[:, None]
-        rk = (1.0 + 3.0 * np.arange(N) / 64.0)[:, None]
-        q, k = z[0] * rq, z[1] * rk
+    if pattern == "steps":
+        beta = np.where(np.arange(N) % 2 == 0, 2.0, 0.6)[:, None]
+        offset = (3.5 * np.minimum(np.arange(N) // 128, 2) / math.sqrt(d))[:, None]
+        q, k = 0.5 * z[0] + beta, 0.5 * z[1] + offset
     elif pattern == "shared":
         q = z[0] * 1.2
         k = q
@@ -173,7 +184,7 @@ def rescale_inputs(pattern, B, H, N, d, dtype="bf16", seed=0):
     def store(x):
         return synth.round_bf16_bits(x) if dtype == "bf16" else x.astype(np.float16)
 
-    stored = [store(q), store(k), arrs[2], arrs[3]]
+    stored = [store(q), store(k), store(0.25 * z[2]), arrs[3]]
     return stored, [synth.to_f64(a, dtype) for a in stored]
 
 

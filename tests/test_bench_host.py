@@ -35,6 +35,18 @@ def test_flops_match_the_table(B, H, N, d, causal, gf, gfb):
         assert (f + fb) / 1e9 == pytest.approx(gfb, rel=2e-3)
 
 
+def test_blocksparse_flops():
+    # all blocks marked: the dense non-causal count; a ragged tail counts its
+    # real rows and keys only; one 128 x 60 block by hand
+    import numpy as np
+    f, fb = bench.blocksparse_flops(2, 3, 700, 64, np.ones((6, 6), np.uint8))
+    assert (f, fb) == bench.flops(2, 3, 700, 64, False)
+    m = np.zeros((6, 6), np.uint8)
+    m[1, 5] = 1
+    assert bench.blocksparse_flops(1, 1, 700, 64, m)[0] == 4.0 * 64 * 128 * 60
+    assert bench.block_mask(4096, 0.5).diagonal().all()
+
+
 def test_workloads_cover_the_five_configs():
     shapes = {(w[0], w[1], w[2], w[3], w[4]) for w in bench.WORKLOADS.values()}
     for B, H, N, d, causal, _, _ in TABLE:
@@ -55,7 +67,18 @@ def _copy_tree(dst):
 
 
 def test_traffic_is_summed_and_dropped_when_a_source_changes(tmp_path, monkeypatch):
+    import hashlib
     table = _copy_tree(str(tmp_path))
+    # stamp the copy with the hashes of the copied sources, as a capture does
+    for entry in table.values():
+        if isinstance(entry, dict):
+            m = hashlib.sha1()
+            for src in entry["sources"]:
+                with open(os.path.join(str(tmp_path), src), "rb") as f:
+                    m.update(f.read())
+            entry["source_sha1"] = m.hexdigest()
+    with open(os.path.join(str(tmp_path), "profiles", "traffic.json"), "w") as f:
+        json.dump(table, f)
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     names = [k for k in table if not k.startswith("_")]
     want = sum(table[k]["dram_bytes_read"] + table[k]["dram_bytes_write"] for k in names)

@@ -12,11 +12,11 @@ from helpers import default_scale, mixed_warps, rescale_inputs, rescale_moves
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("key_tile", [64, 128])
 @pytest.mark.parametrize("causal", [True, False])
-def test_ramp_pattern_moves_the_max(d, key_tile, causal):
-    _, f64 = rescale_inputs("ramp", 1, 1, 700, d, seed=3)
+def test_steps_pattern_moves_the_max(d, key_tile, causal):
+    _, f64 = rescale_inputs("steps", 1, 1, 700, d, seed=3)
     moved, kept = rescale_moves(f64[0][0, 0], f64[1][0, 0], causal, default_scale(d), key_tile)
     per_row = moved.sum(1)
-    assert (per_row >= 1).sum() >= 300
+    assert (per_row >= 1).sum() >= 250
     assert (per_row >= 2).sum() >= 150
     assert mixed_warps(moved, kept) >= 20
 
