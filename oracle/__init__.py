@@ -51,6 +51,17 @@ def lib():
         L.oracle_fp8_quantize.argtypes = [dp, i64, i64, i64, ctypes.POINTER(ctypes.c_int8), ci,
                                           fp, fp]
         L.oracle_fp8_quantize.restype = None
+        u32p = ctypes.POINTER(ctypes.c_uint32)
+        L.oracle_philox4x32_10.argtypes = [u32p, u32p, u32p]
+        L.oracle_philox4x32_10.restype = None
+        L.oracle_dropout_mask.argtypes = [i64, i64, ctypes.c_uint64, ci, ctypes.POINTER(ctypes.c_uint8)]
+        L.oracle_dropout_mask.restype = None
+        L.oracle_fwd_dropout.argtypes = [dp, dp, dp, dp, dp, i64, i64, i64, ci, cd,
+                                         ctypes.c_uint64, ci]
+        L.oracle_fwd_dropout.restype = None
+        L.oracle_bwd_dropout_heads.argtypes = [dp, dp, dp, dp, i64, i64, i64, ci, cd,
+                                               ctypes.c_uint64, ci, lp, i64, dp, dp, dp]
+        L.oracle_bwd_dropout_heads.restype = None
         L.oracle_num_threads.argtypes = []
         L.oracle_num_threads.restype = ci
         L.oracle_set_num_threads.argtypes = [ci]
@@ -248,3 +259,57 @@ def fwd_fp8(q, k, v, causal: bool, scale: float, signs=None, rotate: bool = True
     kc, ks = fp8_quantize(k, signs, rotate)
     return fwd(fp8_dequantize(qc, qs), fp8_dequantize(kc, ks), v, causal,
                scale / (d if rotate else 1.0))
+
+
+def dropout_threshold(p: float) -> int:
+    """The 8-bit keep threshold t = round(256 (1 - p)), clamped to 1 .. 256."""
+    return int(min(256, max(1, round(256.0 * (1.0 - float(p))))))
+
+
+def philox4x32_10(ctr, key):
+    """Philox4x32-10 of four 32-bit counter words and two key words."""
+    c = (ctypes.c_uint32 * 4)(*[int(x) & 0xFFFFFFFF for x in ctr])
+    k = (ctypes.c_uint32 * 2)(*[int(x) & 0xFFFFFFFF for x in key])
+    out = (ctypes.c_uint32 * 4)()
+    lib().oracle_philox4x32_10(c, k, out)
+    return [int(x) for x in out]
+
+
+def dropout_mask(BH: int, N: int, seed: int, p: float):
+    """Z (BH, N, N) uint8: 1 where the probability P_ij is kept."""
+    z = np.empty((BH, N, N), dtype=np.uint8)
+    lib().oracle_dropout_mask(BH, N, int(seed), dropout_threshold(p), _p(z, ctypes.c_uint8))
+    return z
+
+
+def fwd_dropout(q, k, v, causal: bool, scale: float, p: float, seed: int):
+    """Forward with dropout on P (kept values scaled by 256 / t): (O, LSE)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    BH, N, d = _dims(q)
+    o = np.empty_like(q)
+    lse = np.empty(q.shape[:-1], dtype=np.float64)
+    lib().oracle_fwd_dropout(_p(q), _p(k), _p(v), _p(o), _p(lse), BH, N, d, int(bool(causal)),
+                             float(scale), int(seed), dropout_threshold(p))
+    return o, lse
+
+
+def bwd_dropout_heads(q, k, v, dout, causal: bool, scale: float, p: float, seed: int,
+                      heads=None):
+    """Exact gradients of sum(O * dO) with the same dropout mask, listed heads."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    BH, N, d = _dims(q)
+    if heads is None:
+        heads = np.arange(BH)
+    heads = np.ascontiguousarray(heads, dtype=np.int64)
+    shp = (heads.size, N, d)
+    dq, dk, dv = np.empty(shp), np.empty(shp), np.empty(shp)
+    lib().oracle_bwd_dropout_heads(_p(q), _p(k), _p(v), _p(dout), BH, N, d, int(bool(causal)),
+                                   float(scale), int(seed), dropout_threshold(p),
+                                   _p(heads, ctypes.c_int64), heads.size, _p(dq), _p(dk), _p(dv))
+    return dq, dk, dv
+
+
+def bwd_dropout(q, k, v, dout, causal: bool, scale: float, p: float, seed: int):
+    shape = np.shape(q)
+    dq, dk, dv = bwd_dropout_heads(q, k, v, dout, causal, scale, p, seed)
+    return dq.reshape(shape), dk.reshape(shape), dv.reshape(shape)

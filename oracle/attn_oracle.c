@@ -476,6 +476,174 @@ void oracle_fp8_quantize(const double* x, int64_t BH, int64_t N, int64_t d,
         }
 }
 
+/*
+ * Dropout on the attention probabilities: the page's integration example
+ * ("Is a full day of context better than ten minutes?" (marketmaker.cc),
+ * section "integration is eight lines") passes dropout_p to the attention
+ * call during training.  The page gives no more; the readings taken:
+ *  - each probability P_ij (after the softmax, whose statistics and LSE are
+ *    unchanged) is kept with probability 1 - p and scaled by 1 / (1 - p), or
+ *    set to 0: O_i = sum_j P_ij Z_ij / (1 - p) V_j, Z_ij in {0, 1};
+ *  - Z comes from a counter-based generator, Philox4x32-10 (Salmon, Moraes,
+ *    Dror and Shaw, "Parallel random numbers: as easy as 1, 2, 3", SC 2011),
+ *    with key (seed low 32 bits, seed high 32 bits) and counter
+ *    (j / 16, i, b H + h, 0): byte j % 16 of its four output words (word
+ *    (j % 16) / 4, little-endian byte j % 4) is the random byte r_ij, and
+ *    Z_ij = [r_ij < t] with the 8-bit threshold t = round(256 (1 - p)) in
+ *    1 .. 256, so the keep probability is t / 256 and kept values are scaled
+ *    by 256 / t (p is taken to the nearest multiple of 1/256);
+ *  - the backward differentiates that: dV_j = sum_i P_ij Z_ij (256/t) dO_i,
+ *    dP_ij = Z_ij (256/t) dO_i . v_j, D_i = dO_i . O_i (still sum_j P_ij
+ *    dP_ij), dS_ij = P_ij (dP_ij - D_i), dQ and dK as without dropout.
+ */
+static uint32_t mulhilo32(uint32_t a, uint32_t b, uint32_t* hi) {
+    uint64_t p = (uint64_t)a * (uint64_t)b;
+    *hi = (uint32_t)(p >> 32);
+    return (uint32_t)p;
+}
+
+/* Philox4x32 with 10 rounds: the round multiplies counter words 0 and 2 by the
+ * paper's constants and mixes the halves with the key; the key is bumped by
+ * the two Weyl constants between rounds. */
+void oracle_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2], uint32_t out[4]) {
+    uint32_t c0 = ctr_in[0], c1 = ctr_in[1], c2 = ctr_in[2], c3 = ctr_in[3];
+    uint32_t k0 = key_in[0], k1 = key_in[1];
+    for (int r = 0; r < 10; ++r) {
+        uint32_t hi0, hi1;
+        uint32_t lo0 = mulhilo32(0xD2511F53u, c0, &hi0);
+        uint32_t lo1 = mulhilo32(0xCD9E8D57u, c2, &hi1);
+        uint32_t n0 = hi1 ^ c1 ^ k0, n1 = lo1, n2 = hi0 ^ c3 ^ k1, n3 = lo0;
+        c0 = n0; c1 = n1; c2 = n2; c3 = n3;
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+static int dropout_keep(uint64_t seed, int64_t bh, int64_t i, int64_t j, int thr) {
+    uint32_t ctr[4] = {(uint32_t)(j >> 4), (uint32_t)i, (uint32_t)bh, 0u};
+    uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    uint32_t w[4];
+    oracle_philox4x32_10(ctr, key, w);
+    uint32_t byte = (w[(j & 15) >> 2] >> (8 * (j & 3))) & 0xFFu;
+    return (int)byte < thr;
+}
+
+/* The dropout mask Z (BH, N, N) as bytes, for tests. */
+void oracle_dropout_mask(int64_t BH, int64_t N, uint64_t seed, int thr, uint8_t* z) {
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t bh = 0; bh < BH; ++bh)
+        for (int64_t i = 0; i < N; ++i)
+            for (int64_t j = 0; j < N; ++j)
+                z[(bh * N + i) * N + j] = (uint8_t)dropout_keep(seed, bh, i, j, thr);
+}
+
+/* Forward with dropout: O (BH, N, d), LSE (BH, N) (LSE of the softmax itself). */
+void oracle_fwd_dropout(const double* q, const double* k, const double* v, double* o,
+                        double* lse, int64_t BH, int64_t N, int64_t d, int causal, double scale,
+                        uint64_t seed, int thr) {
+    double inv_keep = 256.0 / (double)thr;
+#pragma omp parallel
+    {
+        double* s = (double*)malloc((size_t)N * sizeof(double));
+        double* tmp = (double*)malloc((size_t)d * sizeof(double));
+#pragma omp for collapse(2) schedule(dynamic, 16)
+        for (int64_t bh = 0; bh < BH; ++bh)
+            for (int64_t i = 0; i < N; ++i) {
+                int64_t row = bh * N + i, nv = visible(i, N, causal);
+                lse[row] = row_forward(q + row * d, k + bh * N * d, v + bh * N * d, nv, d, scale,
+                                       s, tmp);
+                double* oi = o + row * d;
+                for (int64_t t = 0; t < d; ++t) oi[t] = 0.0;
+                for (int64_t j = 0; j < nv; ++j) {
+                    if (!dropout_keep(seed, bh, i, j, thr)) continue;
+                    const double* vj = v + (bh * N + j) * d;
+                    for (int64_t t = 0; t < d; ++t) oi[t] += s[j] * inv_keep * vj[t];
+                }
+            }
+        free(tmp);
+        free(s);
+    }
+}
+
+/* Backward with dropout for the listed heads (the chain rule above). */
+void oracle_bwd_dropout_heads(const double* q, const double* k, const double* v,
+                              const double* dout, int64_t BH, int64_t N, int64_t d, int causal,
+                              double scale, uint64_t seed, int thr, const int64_t* heads,
+                              int64_t nheads, double* dq, double* dk, double* dv) {
+    (void)BH;
+    double inv_keep = 256.0 / (double)thr;
+    int nthr = 1;
+#ifdef _OPENMP
+    nthr = omp_get_max_threads();
+#endif
+    size_t nd = (size_t)N * (size_t)d;
+    double* part = (double*)calloc((size_t)nthr * 2 * nd, sizeof(double));
+    for (int64_t hh = 0; hh < nheads; ++hh) {
+        int64_t bh = heads[hh];
+        const double* Q = q + bh * N * d;
+        const double* K = k + bh * N * d;
+        const double* V = v + bh * N * d;
+        const double* dO = dout + bh * N * d;
+        double* dQ = dq + hh * N * d;
+        memset(part, 0, (size_t)nthr * 2 * nd * sizeof(double));
+#pragma omp parallel
+        {
+            int tid = 0;
+#ifdef _OPENMP
+            tid = omp_get_thread_num();
+#endif
+            double* dKp = part + (size_t)tid * 2 * nd;
+            double* dVp = dKp + nd;
+            double* p = (double*)malloc((size_t)N * sizeof(double));
+            double* oi = (double*)malloc((size_t)d * sizeof(double));
+#pragma omp for schedule(dynamic, 8)
+            for (int64_t i = 0; i < N; ++i) {
+                int64_t nv = visible(i, N, causal);
+                const double* qi = Q + i * d;
+                const double* doi = dO + i * d;
+                row_forward(qi, K, V, nv, d, scale, p, oi);
+                /* O with dropout, then D = dO . O */
+                for (int64_t t = 0; t < d; ++t) oi[t] = 0.0;
+                for (int64_t j = 0; j < nv; ++j)
+                    if (dropout_keep(seed, bh, i, j, thr))
+                        for (int64_t t = 0; t < d; ++t) oi[t] += p[j] * inv_keep * V[j * d + t];
+                double Di = dot(doi, oi, d);
+                double* dqi = dQ + i * d;
+                for (int64_t t = 0; t < d; ++t) dqi[t] = 0.0;
+                for (int64_t j = 0; j < nv; ++j) {
+                    const double* vj = V + j * d;
+                    const double* kj = K + j * d;
+                    double zj = dropout_keep(seed, bh, i, j, thr) ? inv_keep : 0.0;
+                    double dpij = zj * dot(doi, vj, d);
+                    double dsij = p[j] * (dpij - Di);
+                    double* dkj = dKp + j * d;
+                    double* dvj = dVp + j * d;
+                    for (int64_t t = 0; t < d; ++t) {
+                        dqi[t] += scale * dsij * kj[t];
+                        dkj[t] += scale * dsij * qi[t];
+                        dvj[t] += p[j] * zj * doi[t];
+                    }
+                }
+            }
+            free(oi);
+            free(p);
+        }
+        double* dK = dk + hh * N * d;
+        double* dV = dv + hh * N * d;
+        for (size_t e = 0; e < nd; ++e) {
+            double sk = 0.0, sv = 0.0;
+            for (int t = 0; t < nthr; ++t) {
+                sk += part[(size_t)t * 2 * nd + e];
+                sv += part[(size_t)t * 2 * nd + nd + e];
+            }
+            dK[e] = sk;
+            dV[e] = sv;
+        }
+    }
+    free(part);
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();
