@@ -62,6 +62,10 @@ def lib():
         L.oracle_bwd_dropout_heads.argtypes = [dp, dp, dp, dp, i64, i64, i64, ci, cd,
                                                ctypes.c_uint64, ci, lp, i64, dp, dp, dp]
         L.oracle_bwd_dropout_heads.restype = None
+        L.oracle_linear_attn.argtypes = [dp, dp, dp, dp, i64, i64, i64, cd]
+        L.oracle_linear_attn.restype = None
+        L.oracle_linear_attn_chunked.argtypes = [dp, dp, dp, dp, i64, i64, i64, cd, i64]
+        L.oracle_linear_attn_chunked.restype = None
         L.oracle_num_threads.argtypes = []
         L.oracle_num_threads.restype = ci
         L.oracle_set_num_threads.argtypes = [ci]
@@ -313,3 +317,21 @@ def bwd_dropout(q, k, v, dout, causal: bool, scale: float, p: float, seed: int):
     shape = np.shape(q)
     dq, dk, dv = bwd_dropout_heads(q, k, v, dout, causal, scale, p, seed)
     return dq.reshape(shape), dk.reshape(shape), dv.reshape(shape)
+
+
+def linear_attn(q, k, v, scale: float):
+    """Causal linear attention O_i = scale sum_{j <= i} (q_i . k_j) v_j."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    BH, N, d = _dims(q)
+    o = np.empty_like(q)
+    lib().oracle_linear_attn(_p(q), _p(k), _p(v), _p(o), BH, N, d, float(scale))
+    return o
+
+
+def linear_attn_chunked(q, k, v, scale: float, chunk: int):
+    """The chunked form (in-chunk product + running state), self-check only."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    BH, N, d = _dims(q)
+    o = np.empty_like(q)
+    lib().oracle_linear_attn_chunked(_p(q), _p(k), _p(v), _p(o), BH, N, d, float(scale), int(chunk))
+    return o

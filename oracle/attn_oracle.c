@@ -644,6 +644,72 @@ void oracle_bwd_dropout_heads(const double* q, const double* k, const double* v,
     free(part);
 }
 
+/*
+ * Causal linear attention: "Lightning Attention-2: A Free Lunch for Handling
+ * Unlimited Sequence Lengths in Large Language Models" (chatpaper.ai
+ * summary), abstract: linear attention replaces the softmax so that tokens
+ * cost linear time; the causal form needs a cumulative sum, which
+ * Lightning Attention-2 tiles into intra-block parts (computed like ordinary
+ * attention) and inter-block parts (the linear-attention kernel trick: a
+ * running d x d state).  "[論文レビュー] Gated Linear Attention Transformers
+ * with Hardware-Efficient Training" (nubint.ai), proposed method: chunk-wise
+ * parallel form, recurrence between chunks and parallel computation inside
+ * them.  The pages give no formula; the plainest reading, taken here (no
+ * feature map, no decay, no normalisation):
+ *     O_i = scale * sum_{j <= i} (q_i . k_j) v_j.
+ * oracle_linear_attn is that definition, row by row; oracle_linear_attn_chunked
+ * restates the chunked form (per chunk of C rows: the masked in-chunk product
+ * plus q_i S, S = sum of k_j^T v_j over earlier chunks, updated after the
+ * chunk) as a self-check.
+ */
+void oracle_linear_attn(const double* q, const double* k, const double* v, double* o,
+                        int64_t BH, int64_t N, int64_t d, double scale) {
+#pragma omp parallel for collapse(2) schedule(dynamic, 16)
+    for (int64_t bh = 0; bh < BH; ++bh)
+        for (int64_t i = 0; i < N; ++i) {
+            const double* qi = q + (bh * N + i) * d;
+            double* oi = o + (bh * N + i) * d;
+            for (int64_t t = 0; t < d; ++t) oi[t] = 0.0;
+            for (int64_t j = 0; j <= i; ++j) {
+                double a = scale * dot(qi, k + (bh * N + j) * d, d);
+                const double* vj = v + (bh * N + j) * d;
+                for (int64_t t = 0; t < d; ++t) oi[t] += a * vj[t];
+            }
+        }
+}
+
+void oracle_linear_attn_chunked(const double* q, const double* k, const double* v, double* o,
+                                int64_t BH, int64_t N, int64_t d, double scale, int64_t C) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < BH; ++bh) {
+        double* S = (double*)calloc((size_t)(d * d), sizeof(double));  /* S[a][b] */
+        for (int64_t c0 = 0; c0 < N; c0 += C) {
+            int64_t c1 = c0 + C < N ? c0 + C : N;
+            for (int64_t i = c0; i < c1; ++i) {          /* intra-chunk + inter-chunk */
+                const double* qi = q + (bh * N + i) * d;
+                double* oi = o + (bh * N + i) * d;
+                for (int64_t t = 0; t < d; ++t) {
+                    double acc = 0.0;
+                    for (int64_t a = 0; a < d; ++a) acc += qi[a] * S[a * d + t];
+                    oi[t] = scale * acc;
+                }
+                for (int64_t j = c0; j <= i; ++j) {
+                    double w = scale * dot(qi, k + (bh * N + j) * d, d);
+                    const double* vj = v + (bh * N + j) * d;
+                    for (int64_t t = 0; t < d; ++t) oi[t] += w * vj[t];
+                }
+            }
+            for (int64_t j = c0; j < c1; ++j) {          /* state update after the chunk */
+                const double* kj = k + (bh * N + j) * d;
+                const double* vj = v + (bh * N + j) * d;
+                for (int64_t a = 0; a < d; ++a)
+                    for (int64_t t = 0; t < d; ++t) S[a * d + t] += kj[a] * vj[t];
+            }
+        }
+        free(S);
+    }
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();
