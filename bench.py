@@ -46,10 +46,17 @@ WORKLOADS = {
     "long_day": (1, 12, 23400, 64, True, "fp16", 0.5, "fwd"),
     "large_head": (4, 16, 4096, 128, True, "bf16", 1.0, "fwdbwd"),
     "large_head_blocksparse": (4, 16, 4096, 128, False, "bf16", 1.0, "fwdbwd"),
+    "large_head_fp8_fwd": (4, 16, 4096, 128, True, "bf16", 1.0, "fwd"),
+    "large_head_linear": (4, 16, 4096, 128, True, "bf16", 1.0, "fwd"),
 }
 # Block-sparse workloads: density of the seeded 128 x 128 block mask (the
 # diagonal is always marked, so no row is empty).
 BLOCK_MASKS = {"large_head_blocksparse": 0.5}
+# FP8-score workloads: each step quantises Q and K (rotated) and runs the
+# forward with e4m3 scores.
+FP8_WORKLOADS = {"large_head_fp8_fwd"}
+# Causal linear attention workloads (chunked, three kernels per step).
+LINEAR_WORKLOADS = {"large_head_linear"}
 DESCRIPTION = {
     "tiny": "tiny exact attention fwd B=1 H=2 N=256 d=64 non-causal bf16",
     "bert_large": "BERT-large-shaped fwd B=8 H=16 N=512 d=64 non-causal bf16",
@@ -58,6 +65,10 @@ DESCRIPTION = {
     "large_head": "large-head causal fwd+bwd B=4 H=16 N=4096 d=128 bf16",
     "large_head_blocksparse": "block-sparse fwd+bwd B=4 H=16 N=4096 d=128 bf16, "
                               "half of the 128x128 blocks marked (seeded, diagonal kept)",
+    "large_head_fp8_fwd": "FP8-score causal fwd B=4 H=16 N=4096 d=128 (Q, K rotated and quantised "
+                          "to e4m3 in the step, P V in bf16)",
+    "large_head_linear": "causal linear attention B=4 H=16 N=4096 d=128 bf16, chunks of 128 "
+                         "(K^T V per chunk, prefix of the states, masked in-chunk product + Q S)",
 }
 METRIC = "attention fwd and fwd+bwd TFLOP/s on 1 B200; % of dense BF16 tensor peak"
 L2_BYTES = 126 * 1024 * 1024
@@ -87,8 +98,18 @@ def blocksparse_flops(B, H, N, d, mask):
     return f, 2.5 * f
 
 
+def linear_flops(B, H, N, d, C=128):
+    """Contractions of the chunked linear attention as computed: per chunk of
+    C rows, Q K^T and P V (2 C^2 d each, the masked half included) and Q S and
+    K^T V (2 C d^2 each)."""
+    nc = (N + C - 1) // C
+    return float(B * H * nc) * 4.0 * C * d * (C + d)
+
+
 def workload_flops(wl):
     B, H, N, d, causal, _, _, _ = WORKLOADS[wl]
+    if wl in LINEAR_WORKLOADS:
+        return linear_flops(B, H, N, d), 0.0
     if wl in BLOCK_MASKS:
         return blocksparse_flops(B, H, N, d, block_mask(N, BLOCK_MASKS[wl]))
     return flops(B, H, N, d, causal)
@@ -264,6 +285,19 @@ class DeviceRun:
         self.flush = None
         if self.working_set < 2 * L2_BYTES:
             self.flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+        self.fp8 = None
+        if wl in FP8_WORKLOADS:
+            nb = (N + 127) // 128
+            self.fp8 = dict(
+                q8=torch.empty((B, H, N, d), dtype=torch.uint8, device=dev),
+                k8=torch.empty((B, H, N, d), dtype=torch.uint8, device=dev),
+                qs=torch.empty((B, H, nb), dtype=torch.float32, device=dev),
+                ks=torch.empty((B, H, nb), dtype=torch.float32, device=dev),
+                signs=torch.from_numpy(synth.random_signs(d, seed)).to(dev))
+        self.lin_ws = None
+        if wl in LINEAR_WORKLOADS:
+            self.lin_ws = torch.empty(attn.attn_linear_workspace_bytes(B, H, N, d),
+                                      dtype=torch.uint8, device=dev)
         self.mask = None
         if wl in BLOCK_MASKS:
             self.mask = torch.from_numpy(block_mask(N, BLOCK_MASKS[wl])).to(dev)
@@ -282,7 +316,15 @@ class DeviceRun:
             self.flush.zero_()
         if evs:
             evs[0].record(st)
-        if self.mask is None:
+        if self.lin_ws is not None:
+            a.attn_linear_fwd(self.q, self.k, self.v, self.o, self.lin_ws, self.scale)
+        elif self.fp8 is not None:
+            f = self.fp8
+            a.attn_fp8_quantize(self.q, f["q8"], f["qs"], f["signs"], True)
+            a.attn_fp8_quantize(self.k, f["k8"], f["ks"], f["signs"], True)
+            a.attn_fwd_fp8(f["q8"], f["k8"], f["qs"], f["ks"], self.v, self.o, self.lse,
+                           self.causal, self.scale, True)
+        elif self.mask is None:
             a.attn_fwd(self.q, self.k, self.v, self.o, self.lse, self.causal, self.scale)
         else:
             a.attn_fwd_blocksparse(self.q, self.k, self.v, self.o, self.lse, self.mask,
@@ -378,6 +420,23 @@ def side_workloads(args, dev, clocks):
         roof, _ = roofline_entry(d, passes, f_fwd, f_bwd, fwd_ms, main_ms, None)
         roof.pop("traffic")
         roof.pop("traffic_unit")
+        if wl in LINEAR_WORKLOADS:
+            # memory-bound: Q, K, V read and O written once (algorithmic), against
+            # the measured copy bandwidth; the kernels also move the chunk states
+            _, _, hbm, src = peaks()
+            alg = 4.0 * B * H * N * d * 2
+            roof = {"kernel": "linear_kv_kernel + linear_prefix_kernel + linear_out_kernel",
+                    "bound": "hbm", "achieved": round(alg / (fwd_ms * 1e-3) / 1e9, 1),
+                    "peak": hbm, "peak_kind": f"hbm_gbs ({src})", "unit": "GB/s",
+                    "frac": round(alg / (fwd_ms * 1e-3) / 1e9 / hbm, 4),
+                    "algorithmic_bytes": alg}
+        if wl in FP8_WORKLOADS:
+            # S = Q K^T (half the FLOPs) at the FP8 rate, twice the bf16 rate; P V at
+            # bf16: the attainable peak for the mix is 4/3 of the bf16 peak
+            roof["peak"] = round(burst * 4.0 / 3.0, 1)
+            roof["peak_kind"] = ("bf16_tflops burst (measured) x 4/3: S at the nominal fp8/bf16 "
+                                 "ratio of 2, P V at bf16; step includes the quantisation")
+            roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
         e = {
             "workload": DESCRIPTION[wl], "passes": passes, "steps": steps,
             "ms_per_step": round(step_ms, 4),
@@ -655,7 +714,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="large_head",
-                    choices=sorted(w for w in WORKLOADS if w not in BLOCK_MASKS))
+                    choices=sorted(w for w in WORKLOADS if w not in BLOCK_MASKS
+                                   and w not in FP8_WORKLOADS and w not in LINEAR_WORKLOADS))
     ap.add_argument("--passes", choices=["fwd", "fwdbwd"], default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)

@@ -159,6 +159,84 @@ int attn_bwd_blocksparse(const void* q, const void* k, const void* v, const void
                          int d, int causal, float scale, attn_dtype_t dtype, void* stream);
 
 /*
+ * FP8 scores with incoherent processing: "Is a full day of context better
+ * than ten minutes?" (marketmaker.cc), section "FA3: Hopper", third item
+ * (random rotation of the vectors before block-wise FP8 quantisation spreads
+ * outliers over all coordinates; reported 2.6x lower error than naive FP8).
+ *
+ * attn_fp8_quantize: x is q or k, (B, H, N, d) bf16/fp16.  Each row is
+ * multiplied element-wise by `signs` (d entries of +1/-1, device memory; NULL:
+ * all +1) and, if rotate != 0, transformed by the unnormalised d x d
+ * Sylvester-Hadamard matrix (entries +-1; the butterflies run in fp32 in
+ * ascending stride).  Each block of 128 rows of one (b, h) is quantised with
+ * one scale: x8 = e4m3(y * (448 / amax)) (nearest even, saturating; IEEE fp32
+ * multiply and divide), scales[(b H + h) ceil(N/128) + block] = amax / 448; a
+ * block of zeros gets scale 0.  x8 is (B, H, N, d) bytes (e4m3), scales is
+ * (B, H, ceil(N/128)) fp32; both caller-owned device memory.
+ *
+ * attn_fwd_fp8: the forward of attn_fwd with S = Q K^T computed from the e4m3
+ * q8, k8 on the FP8 tensor cores, each tile's scores multiplied by its two
+ * block scales, and by scale / d when q8 and k8 were rotated (rotated != 0;
+ * the rotation multiplies dot products by d).  P V runs in the dtype of v
+ * (bf16/fp16), o has that dtype, lse is fp32, as for attn_fwd.  q8, k8 and
+ * their scales must come from attn_fp8_quantize with the same signs and
+ * rotate.  Errors as attn_fwd; ATTN_ERR_ALIGN also for scales not 4-byte
+ * aligned.
+ */
+int attn_fp8_quantize(const void* x, unsigned char* x8, float* scales, const signed char* signs,
+                      int rotate, int B, int H, int N, int d, attn_dtype_t dtype, void* stream);
+
+int attn_fwd_fp8(const unsigned char* q8, const unsigned char* k8, const float* q_scale,
+                 const float* k_scale, const void* v, void* o, float* lse, int B, int H, int N,
+                 int d, int causal, float scale, int rotated, attn_dtype_t dtype, void* stream);
+
+/*
+ * Dropout on the attention probabilities, as the dropout_p argument of the
+ * attention call in "Is a full day of context better than ten minutes?"
+ * (marketmaker.cc), section "integration is eight lines".  The forward and
+ * backward of attn_fwd / attn_bwd, with each probability P_ij (after the
+ * softmax; lse is that of P before dropout) kept with probability t / 256 and
+ * then scaled by 256 / t, else set to 0, where t = round(256 (1 - dropout_p))
+ * clamped to 1 .. 256 (dropout_p is taken to the nearest multiple of 1/256;
+ * 0 keeps everything).  The random byte of (b, h, query i, key j) is byte
+ * j % 16 of Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC 2011) with key
+ * (seed & 0xffffffff, seed >> 32) and counter (j / 16, i, b H + h, 0): word
+ * (j % 16) / 4, little-endian byte j % 4; P_ij is kept iff that byte < t.  The
+ * backward regenerates the same mask from the same seed: call attn_bwd_dropout
+ * with the dropout_p and seed given to attn_fwd_dropout.  Errors as attn_fwd /
+ * attn_bwd; ATTN_ERR_ARG unless 0 <= dropout_p < 1.
+ */
+int attn_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int H, int N, int d, int causal, float scale, float dropout_p,
+                     unsigned long long seed, attn_dtype_t dtype, void* stream);
+
+int attn_bwd_dropout(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                     const void* dout, void* dq, void* dk, void* dv, void* workspace, int B,
+                     int H, int N, int d, int causal, float scale, float dropout_p,
+                     unsigned long long seed, attn_dtype_t dtype, void* stream);
+
+/*
+ * Causal linear attention, chunked: O_i = scale * sum_{j <= i} (q_i . k_j) v_j
+ * (no softmax, feature map, decay or normalisation).  Source: "Lightning
+ * Attention-2: A Free Lunch for Handling Unlimited Sequence Lengths in Large
+ * Language Models" (chatpaper.ai summary), abstract (intra-block parts
+ * computed like ordinary attention, inter-block parts by the linear-attention
+ * kernel trick), and "Gated Linear Attention Transformers with
+ * Hardware-Efficient Training" (nubint.ai review), proposed method (the
+ * chunk-wise parallel form).  Chunks of 128 rows: O_c = scale [(Q_c K_c^T) o
+ * causal mask] V_c + Q_c (scale S_c), S_c = sum over earlier chunks of K^T V.
+ * q, k, v, o: (B, H, N, d) bf16/fp16 device memory, d = 128 only (else
+ * ATTN_ERR_HEADDIM).  workspace: caller-owned device memory of
+ * attn_linear_workspace_bytes() bytes, 256-byte aligned: the per-chunk K^T V
+ * in fp32 and the prefix states S_c in the input's type.  The state reaches
+ * the tensor cores rounded to the input's 16-bit type.  Errors as attn_fwd.
+ */
+size_t attn_linear_workspace_bytes(int B, int H, int N, int d);
+
+int attn_linear_fwd(const void* q, const void* k, const void* v, void* o, void* workspace, int B,
+                    int H, int N, int d, float scale, attn_dtype_t dtype, void* stream);
+
+/*
  * Backward that allocates nothing, for callers that cannot get device memory
  * for a workspace: for example a plugin inside a host framework that owns
  * every device allocation through its own pool and hands the plugin only the

@@ -34,7 +34,8 @@ def bwd_launches(d: int) -> int:
 # Every symbol include/attn.h declares.
 EXPORTS = ("attn_fwd", "attn_bwd", "attn_bwd_prep", "attn_bwd_main", "attn_bwd_workspace_bytes",
            "attn_bwd_noalloc", "attn_sdpa_host", "attn_sdpa_host_scratch_bytes",
-           "attn_fwd_blocksparse", "attn_bwd_blocksparse",
+           "attn_fwd_blocksparse", "attn_bwd_blocksparse", "attn_fp8_quantize", "attn_fwd_fp8",
+           "attn_fwd_dropout", "attn_bwd_dropout", "attn_linear_fwd", "attn_linear_workspace_bytes",
            "attn_last_device_status", "attn_selftest_wait_timeout",
            "attn_last_cuda_error_string", "attn_strerror", "attn_version")
 
@@ -76,6 +77,19 @@ def lib() -> ctypes.CDLL:
         L.attn_fwd_blocksparse.restype = ci
         L.attn_bwd_blocksparse.argtypes = [vp] * 11 + [ci, ci, ci, ci, ci, cf, ci, vp]
         L.attn_bwd_blocksparse.restype = ci
+        L.attn_linear_workspace_bytes.argtypes = [ci, ci, ci, ci]
+        L.attn_linear_workspace_bytes.restype = sz
+        L.attn_linear_fwd.argtypes = [vp] * 5 + [ci, ci, ci, ci, cf, ci, vp]
+        L.attn_linear_fwd.restype = ci
+        u64 = ctypes.c_ulonglong
+        L.attn_fwd_dropout.argtypes = [vp] * 5 + [ci, ci, ci, ci, ci, cf, cf, u64, ci, vp]
+        L.attn_fwd_dropout.restype = ci
+        L.attn_bwd_dropout.argtypes = [vp] * 10 + [ci, ci, ci, ci, ci, cf, cf, u64, ci, vp]
+        L.attn_bwd_dropout.restype = ci
+        L.attn_fp8_quantize.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, vp]
+        L.attn_fp8_quantize.restype = ci
+        L.attn_fwd_fp8.argtypes = [vp] * 7 + [ci, ci, ci, ci, ci, cf, ci, ci, vp]
+        L.attn_fwd_fp8.restype = ci
         L.attn_sdpa_host_scratch_bytes.argtypes = [ci, ci, ci, ci, ci, ci]
         L.attn_sdpa_host_scratch_bytes.restype = sz
         L.attn_sdpa_host.argtypes = [vp] * 10 + [sz, ci, ci, ci, ci, ci, cf, ci, ci, vp]
@@ -261,6 +275,90 @@ def attn_bwd_blocksparse(q, k, v, o, lse, dout, dq, dk, dv, workspace, block_mas
     _check(rc, "attn_bwd_blocksparse")
 
 
+def attn_fp8_quantize(x, x8, scales, signs=None, rotate: bool = True, stream=None) -> None:
+    """x8 <- e4m3 codes of x's rows (times ``signs``, Hadamard-rotated when
+    ``rotate``), one scale per 128-row block of each head into ``scales``."""
+    B, H, N, d = _shape(x)
+    nb = (N + 127) // 128
+    if x8.dtype != torch.uint8 or tuple(x8.shape) != (B, H, N, d) or not x8.is_contiguous():
+        raise ValueError("x8 must be a contiguous uint8 (B, H, N, d) tensor")
+    if scales.dtype != torch.float32 or tuple(scales.shape) != (B, H, nb) or not scales.is_contiguous():
+        raise ValueError(f"scales must be a contiguous float32 (B, H, {nb}) tensor")
+    if signs is not None and (signs.dtype != torch.int8 or tuple(signs.shape) != (d,)):
+        raise ValueError("signs must be an int8 tensor of d entries")
+    rc = lib().attn_fp8_quantize(_ptr(x), _ptr(x8), _ptr(scales), _ptr(signs), int(bool(rotate)),
+                                 B, H, N, d, _dtype(x), ctypes.c_void_p(_stream(x.device, stream)))
+    _check(rc, "attn_fp8_quantize")
+
+
+def attn_fwd_fp8(q8, k8, q_scale, k_scale, v, o, lse, causal: bool, scale: float | None = None,
+                 rotated: bool = True, stream=None) -> None:
+    """Forward with e4m3 scores (codes and scales from attn_fp8_quantize)."""
+    B, H, N, d = _shape(v)
+    _same(v, o, names=("o",))
+    for t, n in ((q8, "q8"), (k8, "k8")):
+        if t.dtype != torch.uint8 or tuple(t.shape) != (B, H, N, d) or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous uint8 (B, H, N, d) tensor")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 (B, H, N) tensor")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib().attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(q_scale), _ptr(k_scale), _ptr(v), _ptr(o),
+                            _ptr(lse), B, H, N, d, int(bool(causal)), scale, int(bool(rotated)),
+                            _dtype(v), ctypes.c_void_p(_stream(v.device, stream)))
+    _check(rc, "attn_fwd_fp8")
+
+
+def attn_fwd_dropout(q, k, v, o, lse, causal: bool, dropout_p: float, seed: int,
+                     scale: float | None = None, stream=None) -> None:
+    """attn_fwd with dropout on P (Philox4x32-10 mask from ``seed``)."""
+    B, H, N, d = _shape(q)
+    _same(q, k, v, o, names=("k", "v", "o"))
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 (B, H, N) tensor")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib().attn_fwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                                int(bool(causal)), scale, float(dropout_p),
+                                int(seed) & 0xFFFFFFFFFFFFFFFF, _dtype(q),
+                                ctypes.c_void_p(_stream(q.device, stream)))
+    _check(rc, "attn_fwd_dropout")
+
+
+def attn_bwd_dropout(q, k, v, o, lse, dout, dq, dk, dv, workspace, causal: bool,
+                     dropout_p: float, seed: int, scale: float | None = None, stream=None) -> None:
+    """attn_bwd for attn_fwd_dropout (the same dropout_p and seed)."""
+    B, H, N, d = _shape(q)
+    _same(q, k, v, o, dout, dq, dk, dv, names=("k", "v", "o", "dout", "dq", "dk", "dv"))
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 (B, H, N) tensor")
+    need = attn_bwd_workspace_bytes(B, H, N, d)
+    if workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace needs {need} bytes")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib().attn_bwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), B, H, N, d,
+                                int(bool(causal)), scale, float(dropout_p),
+                                int(seed) & 0xFFFFFFFFFFFFFFFF, _dtype(q),
+                                ctypes.c_void_p(_stream(q.device, stream)))
+    _check(rc, "attn_bwd_dropout")
+
+
+def attn_linear_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(lib().attn_linear_workspace_bytes(B, H, N, d))
+
+
+def attn_linear_fwd(q, k, v, o, workspace, scale: float | None = None, stream=None) -> None:
+    """Causal linear attention O_i = scale sum_{j<=i} (q_i . k_j) v_j (d = 128)."""
+    B, H, N, d = _shape(q)
+    _same(q, k, v, o, names=("k", "v", "o"))
+    need = attn_linear_workspace_bytes(B, H, N, d)
+    if need == 0 or workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace needs {need} bytes (d must be 128)")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib().attn_linear_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(workspace), B, H, N, d,
+                               scale, _dtype(q), ctypes.c_void_p(_stream(q.device, stream)))
+    _check(rc, "attn_linear_fwd")
+
+
 def attn_sdpa_host_scratch_bytes(B: int, H: int, N: int, d: int, with_backward: bool,
                                  heads_per_chunk: int = 0) -> int:
     return int(lib().attn_sdpa_host_scratch_bytes(B, H, N, d, int(bool(with_backward)),
@@ -338,3 +436,51 @@ def backward_blocksparse(q, k, v, o, lse, dout, block_mask, causal: bool = False
     ws = torch.empty(attn_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=q.device)
     attn_bwd_blocksparse(q, k, v, o, lse, dout, dq, dk, dv, ws, block_mask, causal, scale)
     return dq, dk, dv
+
+
+def forward_fp8(q, k, v, causal: bool = False, scale: float | None = None, signs=None,
+                rotate: bool = True):
+    """Quantises q and k (rotated unless ``rotate`` is False) and runs
+    attn_fwd_fp8; returns (o, lse).  ``signs``: int8 (d,) device tensor."""
+    B, H, N, d = _shape(q)
+    nb = (N + 127) // 128
+    q8 = torch.empty((B, H, N, d), dtype=torch.uint8, device=q.device)
+    k8 = torch.empty_like(q8)
+    qs = torch.empty((B, H, nb), dtype=torch.float32, device=q.device)
+    ks = torch.empty_like(qs)
+    attn_fp8_quantize(q, q8, qs, signs, rotate)
+    attn_fp8_quantize(k, k8, ks, signs, rotate)
+    o = torch.empty_like(v)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    attn_fwd_fp8(q8, k8, qs, ks, v, o, lse, causal, scale, rotate)
+    return o, lse
+
+
+def forward_dropout(q, k, v, dropout_p: float, seed: int, causal: bool = False,
+                    scale: float | None = None):
+    """Allocates O and LSE and runs attn_fwd_dropout; returns (o, lse)."""
+    B, H, N, d = _shape(q)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    attn_fwd_dropout(q, k, v, o, lse, causal, dropout_p, seed, scale)
+    return o, lse
+
+
+def backward_dropout(q, k, v, o, lse, dout, dropout_p: float, seed: int, causal: bool = False,
+                     scale: float | None = None):
+    """Allocates dQ, dK, dV and the workspace; runs attn_bwd_dropout."""
+    B, H, N, d = _shape(q)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(attn_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=q.device)
+    attn_bwd_dropout(q, k, v, o, lse, dout, dq, dk, dv, ws, causal, dropout_p, seed, scale)
+    return dq, dk, dv
+
+
+def linear_forward(q, k, v, scale: float | None = None):
+    """Allocates O and the workspace and runs attn_linear_fwd; returns o."""
+    B, H, N, d = _shape(q)
+    o = torch.empty_like(q)
+    ws = torch.empty(max(1, attn_linear_workspace_bytes(B, H, N, d)), dtype=torch.uint8,
+                     device=q.device)
+    attn_linear_fwd(q, k, v, o, ws, scale)
+    return o

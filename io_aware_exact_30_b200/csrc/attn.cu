@@ -16,6 +16,7 @@
 #include "bwd_sm100.cuh"
 #include "bwd128_sm100.cuh"
 #include "fp8_sm100.cuh"
+#include "linear_sm100.cuh"
 
 namespace {
 
@@ -96,6 +97,30 @@ int check_device(int* dev_out) {
     ok &= cudaFuncSetAttribute(attn::attn_fwd_kernel<128, false, true>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                FwdCfg<128, true>::SMEM_BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn::attn_fwd_kernel<64, true, false, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               FwdCfg<64>::SMEM_BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn::attn_fwd_kernel<64, false, false, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               FwdCfg<64>::SMEM_BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn::attn_fwd_kernel<128, true, false, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               FwdCfg<128>::SMEM_BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn::attn_fwd_kernel<128, false, false, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               FwdCfg<128>::SMEM_BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn::linear_kv_kernel<true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               attn::kLinKvSmem) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn::linear_kv_kernel<false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               attn::kLinKvSmem) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn::linear_out_kernel<true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               attn::kLinOutSmem) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn::linear_out_kernel<false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               attn::kLinOutSmem) == cudaSuccess;
     ok &= attn::bwd_set_attributes();
     ok &= attn::bwd128_set_attributes();
     if (!ok) {
@@ -165,7 +190,7 @@ bool make_map8(CUtensorMap* m, const void* ptr, int BH, int N, int d) {
     return r == CUDA_SUCCESS;
 }
 
-template <int D, bool BF16, bool FP8 = false>
+template <int D, bool BF16, bool FP8 = false, bool DROP = false>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const attn::FwdParams& p, int sm_count, cudaStream_t st) {
     // causal: one CTA per work item, running CTAs take pending CTAs' items;
@@ -174,8 +199,9 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
     if (items >= (1LL << 31)) return ATTN_ERR_SHAPE;
     const bool dynamic = p.causal || p.bmask != nullptr;
     const int nblocks = static_cast<int>(dynamic || items < sm_count ? items : sm_count);
-    attn::attn_fwd_kernel<D, BF16, FP8><<<static_cast<unsigned>(nblocks), FwdCfg<D, FP8>::NTHREADS,
-                                          FwdCfg<D, FP8>::SMEM_BYTES, st>>>(mq, mk, mv, p);
+    attn::attn_fwd_kernel<D, BF16, FP8, DROP><<<static_cast<unsigned>(nblocks),
+                                                FwdCfg<D, FP8>::NTHREADS, FwdCfg<D, FP8>::SMEM_BYTES,
+                                                st>>>(mq, mk, mv, p);
     return launch_ok() ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
@@ -222,9 +248,23 @@ int scratch_address(int dev, void** out) {
 
 namespace {
 // Forward for attn_fwd (bmask == nullptr) and attn_fwd_blocksparse.
+// Dropout parameters from (p, seed): keep threshold t = round(256 (1 - p)) in
+// 1 .. 256; ATTN_ERR_ARG unless 0 <= p < 1.
+int dropout_params(float dropout_p, unsigned long long seed, attn::DropoutParams* dp) {
+    if (!(dropout_p >= 0.f && dropout_p < 1.f)) return ATTN_ERR_ARG;
+    long t = std::lround(256.0 * (1.0 - static_cast<double>(dropout_p)));
+    if (t < 1) t = 1;
+    if (t > 256) t = 256;
+    dp->seed_lo = static_cast<uint32_t>(seed);
+    dp->seed_hi = static_cast<uint32_t>(seed >> 32);
+    dp->thr = static_cast<uint32_t>(t);
+    dp->inv_keep = static_cast<float>(256.0 / static_cast<double>(t));
+    return ATTN_OK;
+}
+
 int fwd_entry(const void* q, const void* k, const void* v, void* o, float* lse,
               const unsigned char* bmask, int B, int H, int N, int d, int causal, float scale,
-              attn_dtype_t dtype, void* stream) {
+              attn_dtype_t dtype, void* stream, const attn::DropoutParams* drop = nullptr) {
     if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
     int rc = check_shape(B, H, N, d, dtype, scale);
     if (rc) return rc;
@@ -258,13 +298,22 @@ int fwd_entry(const void* q, const void* k, const void* v, void* o, float* lse,
     p.bmask = bmask;
     p.n_ktiles = (N + 127) / 128;
     p.qscale = p.kscale = nullptr;
+    p.drop = drop ? *drop : attn::DropoutParams{0u, 0u, 256u, 1.f};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool bf = dtype == ATTN_BF16;
+    const int sms = g_sm_count[dev];
+    if (drop) {
+        if (d == 64)
+            return bf ? launch_fwd<64, true, false, true>(mq, mk, mv, p, sms, st)
+                      : launch_fwd<64, false, false, true>(mq, mk, mv, p, sms, st);
+        return bf ? launch_fwd<128, true, false, true>(mq, mk, mv, p, sms, st)
+                  : launch_fwd<128, false, false, true>(mq, mk, mv, p, sms, st);
+    }
     if (d == 64)
-        return bf ? launch_fwd<64, true>(mq, mk, mv, p, g_sm_count[dev], st)
-                  : launch_fwd<64, false>(mq, mk, mv, p, g_sm_count[dev], st);
-    return bf ? launch_fwd<128, true>(mq, mk, mv, p, g_sm_count[dev], st)
-              : launch_fwd<128, false>(mq, mk, mv, p, g_sm_count[dev], st);
+        return bf ? launch_fwd<64, true>(mq, mk, mv, p, sms, st)
+                  : launch_fwd<64, false>(mq, mk, mv, p, sms, st);
+    return bf ? launch_fwd<128, true>(mq, mk, mv, p, sms, st)
+              : launch_fwd<128, false>(mq, mk, mv, p, sms, st);
 }
 }  // namespace
 
@@ -273,6 +322,15 @@ extern "C" {
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
              int d, int causal, float scale, attn_dtype_t dtype, void* stream) {
     return fwd_entry(q, k, v, o, lse, nullptr, B, H, N, d, causal, scale, dtype, stream);
+}
+
+int attn_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int H, int N, int d, int causal, float scale, float dropout_p,
+                     unsigned long long seed, attn_dtype_t dtype, void* stream) {
+    attn::DropoutParams dp;
+    int rc = dropout_params(dropout_p, seed, &dp);
+    if (rc) return rc;
+    return fwd_entry(q, k, v, o, lse, nullptr, B, H, N, d, causal, scale, dtype, stream, &dp);
 }
 
 int attn_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -358,6 +416,58 @@ int attn_fwd_fp8(const unsigned char* q8, const unsigned char* k8, const float* 
               : launch_fwd<128, false, true>(mq, mk, mv, p, g_sm_count[dev], st);
 }
 
+size_t attn_linear_workspace_bytes(int B, int H, int N, int d) {
+    if (check_shape(B, H, N, d, ATTN_BF16, 1.f) || d != 128) return 0;
+    const size_t states = static_cast<size_t>(B) * H * ((N + 127) / 128) * 128 * 128;
+    return attn::align256(states * 4) + attn::align256(states * 2);
+}
+
+int attn_linear_fwd(const void* q, const void* k, const void* v, void* o, void* workspace, int B,
+                    int H, int N, int d, float scale, attn_dtype_t dtype, void* stream) {
+    if (!q || !k || !v || !o || !workspace) return ATTN_ERR_NULL;
+    int rc = check_shape(B, H, N, d, dtype, scale);
+    if (rc) return rc;
+    if (d != 128) return ATTN_ERR_HEADDIM;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return ATTN_ERR_ALIGN;
+    int dev;
+    if ((rc = check_device(&dev))) return rc;
+    if (!on_device(q, dev) || !on_device(k, dev) || !on_device(v, dev) || !on_device(o, dev) ||
+        !on_device(workspace, dev))
+        return ATTN_ERR_DEVICE;
+    const int BH = B * H, nc = (N + 127) / 128;
+    const long long items = 1LL * BH * nc;
+    if (items >= (1LL << 31)) return ATTN_ERR_SHAPE;
+    const size_t states = static_cast<size_t>(items) * 128 * 128;
+    attn::LinearParams p;
+    p.o = o;
+    p.kv = static_cast<float*>(workspace);
+    p.state = static_cast<uint8_t*>(workspace) + attn::align256(states * 4);
+    p.BH = BH;
+    p.N = N;
+    p.n_chunks = nc;
+    p.scale = scale;
+    CUtensorMap mq, mk, mv, ms;
+    if (!make_map(&mq, q, dtype, BH, N, d) || !make_map(&mk, k, dtype, BH, N, d) ||
+        !make_map(&mv, v, dtype, BH, N, d) ||
+        !make_map(&ms, p.state, dtype, static_cast<int>(items), 128, 128))
+        return ATTN_ERR_LAUNCH;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const unsigned g = static_cast<unsigned>(items);
+    const unsigned gp = static_cast<unsigned>((1LL * BH * 4096 + 255) / 256);
+    if (dtype == ATTN_BF16) {
+        attn::linear_kv_kernel<true><<<g, 192, attn::kLinKvSmem, st>>>(mk, mv, p);
+        attn::linear_prefix_kernel<true><<<gp, 256, 0, st>>>(p);
+        attn::linear_out_kernel<true><<<g, 192, attn::kLinOutSmem, st>>>(mq, mk, mv, ms, p);
+    } else {
+        attn::linear_kv_kernel<false><<<g, 192, attn::kLinKvSmem, st>>>(mk, mv, p);
+        attn::linear_prefix_kernel<false><<<gp, 256, 0, st>>>(p);
+        attn::linear_out_kernel<false><<<g, 192, attn::kLinOutSmem, st>>>(mq, mk, mv, ms, p);
+    }
+    return launch_ok() ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
 size_t attn_bwd_workspace_bytes(int B, int H, int N, int d) {
     if (check_shape(B, H, N, d, ATTN_BF16, 1.f)) return 0;
     return attn::bwd_workspace_bytes(B, H, N, d);
@@ -392,7 +502,8 @@ int bwd_prep_dispatch(const void* o, const void* dout, const float* lse, void* w
 int bwd_main_dispatch(const void* q, const void* k, const void* v, const void* dout, void* dq,
                       void* dk, void* dv, void* workspace, int B, int H, int N, int d, int causal,
                       float scale, attn_dtype_t dtype, cudaStream_t st,
-                      const unsigned char* bmask = nullptr) {
+                      const unsigned char* bmask = nullptr,
+                      const attn::DropoutParams* drop = nullptr) {
     const int BH = B * H;
     CUtensorMap mq, mk, mv, mdo;
     if (!make_map(&mq, q, dtype, BH, N, d) || !make_map(&mk, k, dtype, BH, N, d) ||
@@ -402,9 +513,9 @@ int bwd_main_dispatch(const void* q, const void* k, const void* v, const void* d
     const int c = causal ? 1 : 0;
     if (d == 64)
         return bf ? attn::bwd_main_launch<64, true>(mq, mk, mv, mdo, dq, dk, dv, workspace, B, H,
-                                                    N, c, scale, st, bmask)
+                                                    N, c, scale, st, bmask, drop)
                   : attn::bwd_main_launch<64, false>(mq, mk, mv, mdo, dq, dk, dv, workspace, B, H,
-                                                     N, c, scale, st, bmask);
+                                                     N, c, scale, st, bmask, drop);
     // d = 128: 64-query inner tiles
     // (dK and dV leave through TMA stores)
     CUtensorMap mq64, mdo64, mdk, mdv;
@@ -415,9 +526,9 @@ int bwd_main_dispatch(const void* q, const void* k, const void* v, const void* d
     cudaGetDevice(&dev);
     const int sms = g_sm_count[dev];
     return bf ? attn::bwd_main128_launch<true>(mq64, mk, mv, mdo64, mdk, mdv, dq, dk, dv,
-                                               workspace, B, H, N, c, scale, sms, st, bmask)
+                                               workspace, B, H, N, c, scale, sms, st, bmask, drop)
               : attn::bwd_main128_launch<false>(mq64, mk, mv, mdo64, mdk, mdv, dq, dk, dv,
-                                                workspace, B, H, N, c, scale, sms, st, bmask);
+                                                workspace, B, H, N, c, scale, sms, st, bmask, drop);
 }
 }  // namespace
 
@@ -453,6 +564,22 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
     if ((rc = bwd_prep_dispatch(o, dout, lse, workspace, B, H, N, d, dtype, st))) return rc;
     return bwd_main_dispatch(q, k, v, dout, dq, dk, dv, workspace, B, H, N, d, causal, scale,
                              dtype, st);
+}
+
+int attn_bwd_dropout(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                     const void* dout, void* dq, void* dk, void* dv, void* workspace, int B,
+                     int H, int N, int d, int causal, float scale, float dropout_p,
+                     unsigned long long seed, attn_dtype_t dtype, void* stream) {
+    const void* ptrs[10] = {q, k, v, o, lse, dout, dq, dk, dv, workspace};
+    int dev;
+    int rc = bwd_common_checks(ptrs, 10, workspace, B, H, N, d, dtype, scale, &dev);
+    if (rc) return rc;
+    attn::DropoutParams dp;
+    if ((rc = dropout_params(dropout_p, seed, &dp))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((rc = bwd_prep_dispatch(o, dout, lse, workspace, B, H, N, d, dtype, st))) return rc;
+    return bwd_main_dispatch(q, k, v, dout, dq, dk, dv, workspace, B, H, N, d, causal, scale,
+                             dtype, st, nullptr, &dp);
 }
 
 int attn_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o,

@@ -99,32 +99,33 @@ __device__ __forceinline__ void bwd_item(const BwdParams& p, int k, int& bh, int
 }
 
 // The 64-row query tiles an item (head, key tile j) works through: from the
-// causal start on, and under a block mask only those whose 128-row query tile
-// is marked for key tile j.  Every role walks the same sequence.
+// causal start on, and with a block mask (SPARSE) only those whose 128-row
+// query tile is marked for key tile j.  Every role walks the same sequence.
+template <bool SPARSE>
 struct Bwd128Tiles {
     int begin, end;      // candidate 64-row tiles [begin, end)
-    const uint8_t* col;  // mask column of key tile j (stride n_ktiles), nullptr: dense
+    const uint8_t* col;  // mask column of key tile j (stride n_ktiles)
     int stride;
     __device__ Bwd128Tiles(const BwdParams& p, int j, int n_q64)
-        : begin(p.causal ? 2 * j : 0), end(n_q64), col(p.bmask ? p.bmask + j : nullptr),
+        : begin(p.causal ? 2 * j : 0), end(n_q64), col(SPARSE ? p.bmask + j : nullptr),
           stride(p.n_ktiles) {}
-    __device__ bool act(int i) const { return col == nullptr || col[(i >> 1) * stride] != 0; }
+    __device__ bool act(int i) const { return !SPARSE || col[(i >> 1) * stride] != 0; }
     __device__ int from(int i) const {
-        if (col == nullptr) return i;
-        while (i < end && !act(i)) ++i;
+        if constexpr (SPARSE)
+            while (i < end && !act(i)) ++i;
         return i;
     }
     __device__ int first() const { return from(begin); }
     __device__ int next(int i) const { return from(i + 1); }
     __device__ int count() const {
-        if (col == nullptr) return end - begin;
+        if constexpr (!SPARSE) return end - begin;
         int n = 0;
         for (int i = begin; i < end; ++i) n += act(i);
         return n;
     }
 };
 
-template <bool BF16>
+template <bool BF16, bool DROP = false, bool SPARSE = false>
 __global__ void __launch_bounds__(480, 1)
     attn_bwd_main128_kernel(const __grid_constant__ CUtensorMap tmQ,
                             const __grid_constant__ CUtensorMap tmK,
@@ -228,7 +229,7 @@ __global__ void __launch_bounds__(480, 1)
             };
             while (ok && cs.cur >= 0) {
                 bwd_item(p, cs.cur, bh, j);
-                const Bwd128Tiles tl(p, j, n_q64);
+                const Bwd128Tiles<SPARSE> tl(p, j, n_q64);
                 const int n_it = tl.count();
                 const int pre = min(C::ST, n_it);
                 int qi = tl.first();
@@ -302,7 +303,7 @@ __global__ void __launch_bounds__(480, 1)
             };
             while (ok && cs.cur >= 0) {
                 bwd_item(p, cs.cur, bh, j);
-                const int n_it = Bwd128Tiles(p, j, n_q64).count();
+                const int n_it = Bwd128Tiles<SPARSE>(p, j, n_q64).count();
                 if (is_a) {
                     // the item's K, V; Q_g; dV(g-2), the last reader of S buffer g & 1
                     // (an item without query tiles only waits for its K and V to land)
@@ -381,6 +382,16 @@ __global__ void __launch_bounds__(480, 1)
                         mma_commit(BAR(C::B_DSTE + (g & 1)));  // dS^T(g) no longer read
                     }
                     if (!ok) break;
+                    if (n_it == 0) {
+                        // No query tile, no MMA: the commits below would land at once.
+                        // Wait first for the previous item's accumulator release (the
+                        // compute warps are past the previous FIN) and for this item's
+                        // K and V (the producer saw the previous KVE complete), so that
+                        // neither barrier runs two phases ahead of its waiters.
+                        if (!(ok = wait3(BAR(C::B_KV), items & 1, true, BAR(C::B_ACCE),
+                                         (items - 1) & 1, items > 0, 0u, 0u, false, abort_flag)))
+                            break;
+                    }
                     mma_commit(BAR(C::B_FIN));  // dK, dV of this item complete
                     mma_commit(BAR(C::B_KVE));  // B's reads of K
                 }
@@ -406,11 +417,11 @@ __global__ void __launch_bounds__(480, 1)
         const bool issuer = warp == C::WARP_DQ0 && lane == 0;
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
         const uint32_t stg = base + C::OFF_STG + r * 4u;
-        int g = 0, bh = 0, j = 0;
+        int g = 0, items = 0, bh = 0, j = 0;
         bool dq_ok = true;
         while (dq_ok && cs.cur >= 0) {
             bwd_item(p, cs.cur, bh, j);
-            const Bwd128Tiles tl(p, j, n_q64);
+            const Bwd128Tiles<SPARSE> tl(p, j, n_q64);
             const int n_it = tl.count();
             float* acc_head = p.dqacc + static_cast<size_t>(bh) * p.N * D;
             int qi = tl.first();
@@ -454,8 +465,18 @@ __global__ void __launch_bounds__(480, 1)
                 dq_ok = __all_sync(0xffffffffu, dq_ok);
                 if (!dq_ok) break;
             }
-            // an item without query tiles leaves the staging tile as it was
-            if (dq_ok && n_it == 0 && issuer) mbar_arrive(BAR(C::B_DQD));
+            // An item without query tiles leaves the staging tile as it was.  Its
+            // arrival waits for the previous item's epilogue, which follows the
+            // compute warps' wait for the previous one: without it, such items in
+            // a row would run this barrier two phases ahead of that wait.
+            if (dq_ok && n_it == 0 && issuer) {
+                if (items > 0 && !wait_bounded(BAR(C::B_EPF), (items - 1) & 1, abort_flag))
+                    dq_ok = false;
+                else
+                    mbar_arrive(BAR(C::B_DQD));
+            }
+            dq_ok = __all_sync(0xffffffffu, dq_ok);
+            ++items;
             if (dq_ok) dq_ok = cs.advance(abort_flag, true);
         }
         if (issuer) bulk_wait_all();  // every reduction complete before the CTA exits
@@ -471,7 +492,7 @@ __global__ void __launch_bounds__(480, 1)
         bool ok = true;
         while (ok && cs.cur >= 0) {
             bwd_item(p, cs.cur, bh, j);
-            const Bwd128Tiles tl(p, j, n_q64);
+            const Bwd128Tiles<SPARSE> tl(p, j, n_q64);
             const int n_it = tl.count();
             const int key = j * 128 + r;
             const bool key_valid = key < p.N;
@@ -494,6 +515,7 @@ __global__ void __launch_bounds__(480, 1)
                 if (!ok) break;
                 tc_fence_after();
                 float pv[32];
+                uint32_t kw[8];  // dropout keep masks of the 32 query columns (bytes)
                 {
                     uint32_t sv[32];
                     tmem_ld32(lane_addr + colS + c0, sv);
@@ -523,8 +545,25 @@ __global__ void __launch_bounds__(480, 1)
                             if (c < lo) pv[c] = 0.f;
                     }
                     uint32_t pk[16];
+                    if constexpr (DROP) {
+                        // P^T for dV without the dropped values (256 / t is applied to
+                        // dV at the end); dS below uses P and the masked dP
+                        if (p.drop.thr < 256u) {
+                            dropout_keep_keyrows(p.drop, bh, q0 + c0, j * 128 + quarter * 32, kw);
+                        } else {
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) pk[c] = pack2<BF16>(pv[2 * c], pv[2 * c + 1]);
+                            for (int t = 0; t < 8; ++t) kw[t] = 0xFFFFFFFFu;
+                        }
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) {
+                            const uint32_t kb = kw[c >> 1] >> (16 * (c & 1));
+                            pk[c] = pack2<BF16>((kb & 0x1u) ? pv[2 * c] : 0.f,
+                                                (kb & 0x100u) ? pv[2 * c + 1] : 0.f);
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) pk[c] = pack2<BF16>(pv[2 * c], pv[2 * c + 1]);
+                    }
                     if (half == 1) {
                         ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SRD + (g & 1)),
                                                                   (g >> 1) & 1, abort_flag));
@@ -559,9 +598,12 @@ __global__ void __launch_bounds__(480, 1)
                         const float4 d4 = D4[e4];
                         const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            dsv[4 * e4 + e] =
-                                pv[4 * e4 + e] * (__uint_as_float(dpv[4 * e4 + e]) - dd[e]);
+                        for (int e = 0; e < 4; ++e) {
+                            float dpe = __uint_as_float(dpv[4 * e4 + e]);
+                            if constexpr (DROP)
+                                dpe = ((kw[e4] >> (8 * e)) & 1u) ? dpe * p.drop.inv_keep : 0.f;
+                            dsv[4 * e4 + e] = pv[4 * e4 + e] * (dpe - dd[e]);
+                        }
                     }
 #pragma unroll
                     for (int c = 0; c < 4; ++c)  // 16-byte chunks 4 half + c of the 128-byte key row
@@ -607,10 +649,11 @@ __global__ void __launch_bounds__(480, 1)
                 if (n_it == 0)
 #pragma unroll
                     for (int e = 0; e < 32; ++e) v[e] = 0u;
+                const float mv = DROP ? p.drop.inv_keep : 1.f;  // kept P scaled by 256 / t
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
-                    hv[16 * c + e] =
-                        pack2<BF16>(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+                    hv[16 * c + e] = pack2<BF16>(__uint_as_float(v[2 * e]) * mv,
+                                                 __uint_as_float(v[2 * e + 1]) * mv);
             }
             // dK and dV have been read: the next item may overwrite them
             tc_fence_before();
@@ -678,6 +721,18 @@ inline bool bwd128_set_attributes() {
                                 Bwd128Cfg::SMEM_BYTES) == cudaSuccess &&
            cudaFuncSetAttribute(attn_bwd_main128_kernel<false>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Bwd128Cfg::SMEM_BYTES) == cudaSuccess &&
+           cudaFuncSetAttribute(attn_bwd_main128_kernel<true, true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Bwd128Cfg::SMEM_BYTES) == cudaSuccess &&
+           cudaFuncSetAttribute(attn_bwd_main128_kernel<false, true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Bwd128Cfg::SMEM_BYTES) == cudaSuccess &&
+           cudaFuncSetAttribute(attn_bwd_main128_kernel<true, false, true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Bwd128Cfg::SMEM_BYTES) == cudaSuccess &&
+           cudaFuncSetAttribute(attn_bwd_main128_kernel<false, false, true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 Bwd128Cfg::SMEM_BYTES) == cudaSuccess;
 }
 
@@ -690,9 +745,10 @@ int bwd_main128_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
                        const CUtensorMap& mdo, const CUtensorMap& mdk, const CUtensorMap& mdv,
                        void* dq, void* dk, void* dv, void* ws, int B, int H, int N, int causal,
                        float scale, int sm_count, cudaStream_t st,
-                       const uint8_t* bmask = nullptr) {
+                       const uint8_t* bmask = nullptr, const DropoutParams* drop = nullptr) {
     BwdParams p;
     p.bmask = bmask;
+    if (drop) p.drop = *drop;
     uint8_t* w = static_cast<uint8_t*>(ws);
     p.l2pad = reinterpret_cast<const float*>(w);
     p.dpad = reinterpret_cast<const float*>(w + bwd_ws_off_d(B, H, N));
@@ -719,8 +775,17 @@ int bwd_main128_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     if (items >= (1LL << 31)) return -2;
     const bool dynamic = causal || bmask != nullptr;
     const int nblocks = static_cast<int>(dynamic || items < sm_count ? items : sm_count);
-    attn_bwd_main128_kernel<BF16><<<static_cast<unsigned>(nblocks), Bwd128Cfg::NTHREADS,
-                                    Bwd128Cfg::SMEM_BYTES, st>>>(mq, mk, mv, mdo, mdk, mdv, p);
+    if (drop)
+        attn_bwd_main128_kernel<BF16, true><<<static_cast<unsigned>(nblocks), Bwd128Cfg::NTHREADS,
+                                              Bwd128Cfg::SMEM_BYTES, st>>>(mq, mk, mv, mdo, mdk,
+                                                                           mdv, p);
+    else if (bmask)
+        attn_bwd_main128_kernel<BF16, false, true><<<static_cast<unsigned>(nblocks),
+                                                     Bwd128Cfg::NTHREADS, Bwd128Cfg::SMEM_BYTES,
+                                                     st>>>(mq, mk, mv, mdo, mdk, mdv, p);
+    else
+        attn_bwd_main128_kernel<BF16><<<static_cast<unsigned>(nblocks), Bwd128Cfg::NTHREADS,
+                                        Bwd128Cfg::SMEM_BYTES, st>>>(mq, mk, mv, mdo, mdk, mdv, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
         bwd_record_error(e);

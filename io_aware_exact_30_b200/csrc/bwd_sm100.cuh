@@ -46,6 +46,7 @@
 // query row.  For D = 64 it is dQ = dS K (lane = query) in columns 384..447.
 #pragma once
 
+#include "dropout.cuh"
 #include "ptx.cuh"
 
 namespace attn {
@@ -135,6 +136,8 @@ struct BwdParams {
     // 128-row query tile i may attend to key tile j (one mask for every head);
     // nullptr for dense attention.
     const uint8_t* bmask = nullptr;
+    // Dropout on P (kernels instantiated with DROP only).
+    DropoutParams drop{0u, 0u, 256u, 1.f};
 };
 
 template <int D>
@@ -167,7 +170,7 @@ struct BwdCfg {
     static constexpr int WARP_TMA = NCOMPUTE / 32, WARP_MMA = WARP_TMA + 1;
 };
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool DROP = false>
 __global__ void __launch_bounds__(320, 1)
     attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
@@ -386,6 +389,7 @@ __global__ void __launch_bounds__(320, 1)
             if (!ok) break;
             tc_fence_after();
             float pv[64];
+            uint32_t kw[2][8];  // dropout keep masks of the 64 query columns (bytes)
             {
                 uint32_t sv[2][32];
                 tmem_ld32(lane_addr + C::COL_S + c0, sv[0]);
@@ -416,8 +420,26 @@ __global__ void __launch_bounds__(320, 1)
                         if (c < lo) pv[c] = 0.f;
                 }
                 uint32_t pk[32];
+                if constexpr (DROP) {
+                    // P^T for dV without the dropped values (256 / t is applied to dV
+                    // at the end); dS below uses P and the masked dP
+                    if (p.drop.thr < 256u) {
+                        dropout_keep_keyrows(p.drop, bh, q0 + c0, j * 128 + quarter * 32, kw[0]);
+                        dropout_keep_keyrows(p.drop, bh, q0 + c0 + 32, j * 128 + quarter * 32, kw[1]);
+                    } else {
 #pragma unroll
-                for (int c = 0; c < 32; ++c) pk[c] = pack2<BF16>(pv[2 * c], pv[2 * c + 1]);
+                        for (int t = 0; t < 8; ++t) kw[0][t] = kw[1][t] = 0xFFFFFFFFu;
+                    }
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const uint32_t kb = kw[c >> 4][(c >> 1) & 7] >> (16 * (c & 1));
+                        pk[c] = pack2<BF16>((kb & 0x1u) ? pv[2 * c] : 0.f,
+                                            (kb & 0x100u) ? pv[2 * c + 1] : 0.f);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) pk[c] = pack2<BF16>(pv[2 * c], pv[2 * c + 1]);
+                }
                 if (half == 1) {
                     ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SRD), ph, abort_flag));
                     tc_fence_after();
@@ -447,9 +469,12 @@ __global__ void __launch_bounds__(320, 1)
                     const float4 d4 = D4[c4 * 8 + g];
                     const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        dsv[4 * g + e] =
-                            pv[c4 * 32 + 4 * g + e] * (__uint_as_float(dpv[4 * g + e]) - dd[e]);
+                    for (int e = 0; e < 4; ++e) {
+                        float dpe = __uint_as_float(dpv[4 * g + e]);
+                        if constexpr (DROP)
+                            dpe = ((kw[c4][g] >> (8 * e)) & 1u) ? dpe * p.drop.inv_keep : 0.f;
+                        dsv[4 * g + e] = pv[c4 * 32 + 4 * g + e] * (dpe - dd[e]);
+                    }
                 }
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
@@ -495,7 +520,7 @@ __global__ void __launch_bounds__(320, 1)
             for (int which = 0; which < 2; ++which) {
                 uint8_t* out = static_cast<uint8_t*>(which ? p.dv : p.dk) + rowoff;
                 const uint32_t col = (which ? C::COL_DV : C::COL_DK) + half * (D / 2);
-                const float mul = which ? 1.f : p.scale;
+                const float mul = which ? (DROP ? p.drop.inv_keep : 1.f) : p.scale;
 #pragma unroll
                 for (int c = 0; c < D / 64; ++c) {
                     uint32_t v[32];
@@ -561,6 +586,12 @@ inline bool bwd_set_attributes() {
     ok &= cudaFuncSetAttribute(attn_bwd_main_kernel<64, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                BwdCfg<64>::SMEM_BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn_bwd_main_kernel<64, true, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               BwdCfg<64>::SMEM_BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn_bwd_main_kernel<64, false, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               BwdCfg<64>::SMEM_BYTES) == cudaSuccess;
     return ok;
 }
 
@@ -587,9 +618,10 @@ template <int D, bool BF16>
 int bwd_main_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                     const CUtensorMap& mdo, void* dq, void* dk, void* dv, void* ws, int B, int H,
                     int N, int causal, float scale, cudaStream_t st,
-                    const uint8_t* bmask = nullptr) {
+                    const uint8_t* bmask = nullptr, const DropoutParams* drop = nullptr) {
     BwdParams p;
     p.bmask = bmask;
+    if (drop) p.drop = *drop;
     uint8_t* w = static_cast<uint8_t*>(ws);
     p.l2pad = reinterpret_cast<const float*>(w);
     p.dpad = reinterpret_cast<const float*>(w + bwd_ws_off_d(B, H, N));
@@ -608,8 +640,12 @@ int bwd_main_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensor
     p.scale_log2 = scale * 1.4426950408889634f;
     const long long nblocks = 1LL * p.n_ktiles * p.BH;
     if (nblocks >= (1LL << 31)) return -2;
-    attn_bwd_main_kernel<D, BF16><<<static_cast<unsigned>(nblocks), BwdCfg<D>::NTHREADS,
-                                    BwdCfg<D>::SMEM_BYTES, st>>>(mq, mk, mv, mdo, p);
+    if (drop)
+        attn_bwd_main_kernel<D, BF16, true><<<static_cast<unsigned>(nblocks), BwdCfg<D>::NTHREADS,
+                                              BwdCfg<D>::SMEM_BYTES, st>>>(mq, mk, mv, mdo, p);
+    else
+        attn_bwd_main_kernel<D, BF16><<<static_cast<unsigned>(nblocks), BwdCfg<D>::NTHREADS,
+                                        BwdCfg<D>::SMEM_BYTES, st>>>(mq, mk, mv, mdo, p);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) bwd_record_error(e);
     return e == cudaSuccess ? 0 : -7;

@@ -40,6 +40,7 @@
 // Tensor memory: S/P of tile i at column 128 i, O of tile i at 256 + D i.
 #pragma once
 
+#include "dropout.cuh"
 #include "ptx.cuh"
 
 namespace attn {
@@ -64,6 +65,8 @@ struct FwdParams {
     // rotation.  nullptr for 16-bit Q and K.
     const float* qscale;
     const float* kscale;
+    // Dropout on P (kernels instantiated with DROP only).
+    DropoutParams drop;
 };
 
 // Persistent schedule.  A work item is (head, pair of query tiles); there are
@@ -94,37 +97,36 @@ __device__ __forceinline__ void fwd_item(const FwdParams& p, int k, int& bh, int
 // union is 0 .. nkv - 1.
 struct FwdItemShape {
     bool has1;
-    int nkv_t[2];
-    int nkv;
-    const uint8_t* mrow[2];  // mask rows of the two query tiles (nullptr: dense)
+    int nkv0, nkv1;          // key tiles below each query tile's causal bound
+    int nkv;                 // max of the two
+    const uint8_t* mrow0;    // mask rows of the two query tiles (nullptr: dense)
+    const uint8_t* mrow1;
+    // (scalars, not arrays: indexed by a run-time tile they would live in
+    // local memory, on the MMA issuer's critical path)
     __device__ FwdItemShape(const FwdParams& p, int pair) {
         const int n_kv_all = (p.N + 127) >> 7;
         has1 = 2 * pair + 1 < p.n_qtiles;
-        nkv_t[0] = p.causal ? min(n_kv_all, 2 * pair + 1) : n_kv_all;
-        nkv_t[1] = has1 ? (p.causal ? min(n_kv_all, 2 * pair + 2) : n_kv_all) : 0;
-        nkv = max(nkv_t[0], nkv_t[1]);
-        mrow[0] = p.bmask ? p.bmask + static_cast<size_t>(2 * pair) * p.n_ktiles : nullptr;
-        mrow[1] = p.bmask && has1 ? mrow[0] + p.n_ktiles : nullptr;
+        nkv0 = p.causal ? min(n_kv_all, 2 * pair + 1) : n_kv_all;
+        nkv1 = has1 ? (p.causal ? min(n_kv_all, 2 * pair + 2) : n_kv_all) : 0;
+        nkv = max(nkv0, nkv1);
+        mrow0 = p.bmask ? p.bmask + static_cast<size_t>(2 * pair) * p.n_ktiles : nullptr;
+        mrow1 = p.bmask && has1 ? mrow0 + p.n_ktiles : nullptr;
     }
+    __device__ int nk(int t) const { return t ? nkv1 : nkv0; }
+    __device__ const uint8_t* mrow(int t) const { return t ? mrow1 : mrow0; }
     __device__ bool act(int t, int j) const {
-        return j < nkv_t[t] && (mrow[t] == nullptr || mrow[t][j] != 0);
+        const uint8_t* m = mrow(t);
+        return j < nk(t) && (m == nullptr || m[j] != 0);
     }
     __device__ bool any(int j) const { return act(0, j) || act(1, j); }
     // first union tile at or after j (nkv if none)
     __device__ int from(int j) const {
-        if (mrow[0] == nullptr) return j;
+        if (mrow0 == nullptr) return j;
         while (j < nkv && !any(j)) ++j;
         return j;
     }
     __device__ int first() const { return from(0); }
     __device__ int next(int j) const { return from(j + 1); }
-    // number of key tiles query tile t attends to
-    __device__ int count(int t) const {
-        if (mrow[t] == nullptr) return nkv_t[t];
-        int n = 0;
-        for (int j = 0; j < nkv_t[t]; ++j) n += mrow[t][j] != 0;
-        return n;
-    }
 };
 
 template <int D, bool FP8 = false>
@@ -158,7 +160,7 @@ struct FwdCfg {
 // than this many binary orders of magnitude.
 constexpr float kRescaleThreshold = 8.f;
 
-template <int D, bool BF16, bool FP8 = false>
+template <int D, bool BF16, bool FP8 = false, bool DROP = false>
 __global__ void __launch_bounds__(320, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -329,7 +331,7 @@ __global__ void __launch_bounds__(320, 1)
                 tc_fence_after();
                 if (a0) issue_s(0, kv);
                 if (a1) issue_s(1, kv);
-                bool first_pv[2] = {true, true};  // no P_t V of this item issued yet
+                int fresh = 3;  // bit t: no P_t V of this item issued yet
                 int u = 0;                        // union key tiles of this item so far
                 for (int j = j0, jn; ok && j < sh.nkv; j = jn, ++u) {
                     jn = sh.next(j);
@@ -344,7 +346,7 @@ __global__ void __launch_bounds__(320, 1)
                         // the previous epilogue's read of O_t, which P_t V overwrites
                         if (!(ok = wait3(BAR(C::B_VF + s), n & 1, t == 0, BAR(C::B_PF + t),
                                          n_pv[t] & 1, act, BAR(C::B_OE + t), (n_done[t] - 1) & 1,
-                                         act && first_pv[t] && n_done[t] > 0, abort_flag)))
+                                         act && ((fresh >> t) & 1) && n_done[t] > 0, abort_flag)))
                             break;
                         if (act) {
                             tc_fence_after();
@@ -352,10 +354,10 @@ __global__ void __launch_bounds__(320, 1)
                             for (int kk = 0; kk < 8; ++kk)
                                 mma_ts(tmem + C::COL_O + t * D, tmem + t * 128u + kk * 8u,
                                        sdesc_sw128(sv + kk * 2048u, 16384, 1024), ID_O,
-                                       (!first_pv[t] || kk > 0) ? 1u : 0u);
+                                       (!((fresh >> t) & 1) || kk > 0) ? 1u : 0u);
                             mma_commit(BAR(C::B_OD + t));
                             ++n_pv[t];
-                            first_pv[t] = false;
+                            fresh &= ~(1 << t);
                         }
                         if (jn < sh.nkv && sh.act(t, jn)) {
                             // S_t of the next union tile, into the columns the last
@@ -377,7 +379,7 @@ __global__ void __launch_bounds__(320, 1)
                 kv += u;
                 ++items;
                 for (int t = 0; t < 2; ++t)
-                    if (!first_pv[t]) ++n_done[t];
+                    if (!((fresh >> t) & 1)) ++n_done[t];
             }
             if (*abort_flag) {  // every issued MMA must finish before TMEM is freed
                 mma_commit(BAR(C::B_DR));
@@ -399,8 +401,8 @@ __global__ void __launch_bounds__(320, 1)
             const uint8_t* my_row;  // this tile's block-mask row (nullptr: dense)
             {
                 const FwdItemShape sh(p, pair);
-                my_nkv = sh.nkv_t[t];
-                my_row = sh.mrow[t];
+                my_nkv = sh.nk(t);
+                my_row = sh.mrow(t);
             }
             if (my_nkv == 0) continue;  // the pair has no second tile
             const int qrow = (2 * pair + t) * 128 + r;
@@ -489,6 +491,23 @@ __global__ void __launch_bounds__(320, 1)
                     uint32_t nxt[32];
                     if (c < 3) tmem_ld32(lane_addr + colS + (c + 1) * 32u, nxt);
                     uint32_t pk[16];
+                    // dropout: keep masks (0xFF bytes) of this chunk's 32 keys
+                    uint32_t kw[8];
+                    if constexpr (DROP) {
+                        if (p.drop.thr < 256u) {
+                            const uint32_t g = static_cast<uint32_t>(key0 + 32 * c) / 16u;
+                            const uint4 a = dropout_bytes16(p.drop, bh, qrow, g);
+                            const uint4 b = dropout_bytes16(p.drop, bh, qrow, g + 1u);
+                            const uint32_t thr4 = p.drop.thr * 0x01010101u;
+                            kw[0] = keep_bytes(a.x, thr4), kw[1] = keep_bytes(a.y, thr4);
+                            kw[2] = keep_bytes(a.z, thr4), kw[3] = keep_bytes(a.w, thr4);
+                            kw[4] = keep_bytes(b.x, thr4), kw[5] = keep_bytes(b.y, thr4);
+                            kw[6] = keep_bytes(b.z, thr4), kw[7] = keep_bytes(b.w, thr4);
+                        } else {
+#pragma unroll
+                            for (int t = 0; t < 8; ++t) kw[t] = 0xFFFFFFFFu;
+                        }
+                    }
 #pragma unroll
                     for (int q = 0; q < 16; ++q) {
                         uint64_t x = fma2(f2(__uint_as_float(cur[2 * q]), __uint_as_float(cur[2 * q + 1])),
@@ -502,7 +521,12 @@ __global__ void __launch_bounds__(320, 1)
                         const float2 xv = unf2(x);
                         const uint64_t pp = f2(ex2(xv.x), ex2(xv.y));
                         sum2 = add2(sum2, pp);
-                        const float2 pv = unf2(pp);
+                        float2 pv = unf2(pp);
+                        if constexpr (DROP) {  // the row sum keeps the dropped values
+                            const uint32_t kb = kw[q >> 1] >> (16 * (q & 1));
+                            if (!(kb & 0x1u)) pv.x = 0.f;
+                            if (!(kb & 0x100u)) pv.y = 0.f;
+                        }
                         pk[q] = pack2<BF16>(pv.x, pv.y);
                     }
                     tmem_st16(lane_addr + colS + c * 16u, pk);
@@ -539,7 +563,8 @@ __global__ void __launch_bounds__(320, 1)
                                 wait_bounded(BAR(C::B_OD + t), (n_s - 1) & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            const float inv_l = 1.f / l;
+            float inv_l = 1.f / l;
+            if constexpr (DROP) inv_l *= p.drop.inv_keep;  // kept values are scaled by 256 / t
             uint8_t* orow = static_cast<uint8_t*>(p.o) +
                             (static_cast<size_t>(bh) * p.N + qrow) * (D * 2);
 #pragma unroll

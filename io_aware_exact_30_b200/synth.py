@@ -21,7 +21,8 @@ Definition (counter-addressable, so any slice can be regenerated alone):
   fp16 by one round-to-nearest-even step from float64; bf16 by
   round-to-nearest-even to float32 and then round-to-nearest-even to bf16.
 
-Stream ids: Q = 0, K = 1, V = 2, dO = 3.
+Stream ids: Q = 0, K = 1, V = 2, dO = 3; the random signs of the FP8
+rotation use stream 4 (word t >> 63 picks the sign of coordinate t).
 """
 
 from __future__ import annotations
@@ -32,7 +33,7 @@ GAMMA = np.uint64(0x9E3779B97F4A7C15)
 _M1 = np.uint64(0xBF58476D1CE4E5B9)
 _M2 = np.uint64(0x94D049BB133111EB)
 
-STREAM_Q, STREAM_K, STREAM_V, STREAM_DO = 0, 1, 2, 3
+STREAM_Q, STREAM_K, STREAM_V, STREAM_DO, STREAM_SIGNS = 0, 1, 2, 3, 4
 
 _CHUNK = 1 << 22  # elements generated per numpy pass (bounds host memory)
 
@@ -124,3 +125,10 @@ def attention_inputs(B: int, H: int, N: int, d: int, *, seed: int = 0, sigma: fl
     if with_dout:
         out.append(tensor(seed, STREAM_DO, shape, dout_sigma, dtype))
     return out
+
+
+def random_signs(d: int, seed: int = 0) -> np.ndarray:
+    """d random signs (int8, +1 or -1) from stream (seed, 4): the top bit of
+    splitmix64 word t set gives -1."""
+    w = words(seed, STREAM_SIGNS, 0, d)
+    return np.where((w >> np.uint64(63)) == np.uint64(1), -1, 1).astype(np.int8)

@@ -44,18 +44,15 @@ class Variant:
     single_dsf: bool = False      # one barrier (not one per dS^T buffer) for dS^T ready
     epilogue_tile_wait: bool = False  # epilogue waits the per-tile staging barrier, not DQD
     no_dpe: bool = False          # dP^T(g) waits for dS^T(g-1) instead of the dP^T release
-    own_region_p: bool = False    # each half writes P^T over its own S^T columns, no SRD
-    # design variant: P^T and dS^T computed by two warp groups in a pipeline (the
-    # P group writes P^T of tile g+1 while the dS group forms dS^T of tile g,
-    # reading P^T back from tensor memory).  No new barrier: the dS group
-    # releases dP^T (DPE) only after it has read P^T too, and S^T(g+2) is issued
-    # after issuer A's wait for DPE(g).
-    pd_split: bool = False
-    pd_split_early_dpe: bool = False  # mistake: DPE before the dS group reads P^T
     # work items dealt in a fixed order (no mask) instead of taken through
     # cluster launch control responses (causal)
     static_items: bool = False
     clc_no_empty_wait: bool = False   # request into a slot without its consumers' release
+    # an item without query tiles arrives DQD without waiting for the previous
+    # item's epilogue (the mistake the checker found in the block-sparse walk)
+    empty_item_no_epf_wait: bool = False
+    # issuer B commits an empty item's FIN and KVE without waiting (the same)
+    empty_item_no_b_wait: bool = False
 
 
 class Barrier:
@@ -275,11 +272,16 @@ def producer(plan, v):
 def issuer_a(plan, v):
     g = 0
     for item, n_it in enumerate(plan):
-        waits = [("KV", item), (f"QF{g % ST}", g // ST)]
-        if g >= 2:
-            waits.append((f"DVD{g & 1}", (g - 2) >> 1))
+        # an item without query tiles (block-sparse: no query tile marked for
+        # its key tile) only waits for its K and V to land
+        waits = [("KV", item)]
+        if n_it > 0:
+            waits.append((f"QF{g % ST}", g // ST))
+            if g >= 2:
+                waits.append((f"DVD{g & 1}", (g - 2) >> 1))
         yield ("wait", waits)
-        yield from mma_s(g, item)
+        if n_it > 0:
+            yield from mma_s(g, item)
         for it in range(n_it):
             s, g1, more = g % ST, g + 1, it + 1 < n_it
             waits = []
@@ -333,7 +335,7 @@ def issuer_b(plan, v):
             def dv(g=g, s=s, item=item, it=it):
                 for q in range(2):
                     W.read(("S", g & 1, q, "R0"), ("P", g))
-                    W.read(("S", g & 1, q, "R2" if v.own_region_p else "R1"), ("P", g))
+                    W.read(("S", g & 1, q, "R1"), ("P", g))
                 W.read(("DO", s), g)
                 W.write("DVACC", (item, it + 1))
             yield ("async", "B", dv, "DV")
@@ -363,6 +365,16 @@ def issuer_b(plan, v):
             yield ("async", "B", lambda g=g: W.bar("DQF").arrive(g))
             yield ("async", "B", lambda g=g: W.bar(f"DSTE{g & 1}").arrive(g >> 1))
             g += 1
+        if n_it == 0 and not v.empty_item_no_b_wait:
+            # An item without query tiles issues no MMA.  Its FIN and KVE commits
+            # wait for the previous item's accumulator release (the compute
+            # warps have passed the previous FIN) and for this item's K and V
+            # (the producer has seen the previous KVE complete): otherwise
+            # consecutive such items run both barriers two phases ahead.
+            waits = [("KV", item)]
+            if item > 0:
+                waits.append(("ACCE", item - 1))
+            yield ("wait", waits)
         yield ("async", "B", lambda item=item: W.bar("FIN").arrive(item))
         yield ("async", "B", lambda item=item: W.bar("KVE", 2).arrive(item))
         yield from item_advance(W, item, not v.static_items)
@@ -381,17 +393,13 @@ def compute(agent, plan, v):
             if half == 0:
                 yield ("read", ("S", b, q, "R0"), ("S", g))
                 yield ("read", ("S", b, q, "R1"), ("S", g))
-                if not v.own_region_p:
-                    yield ("arrive", srd[0], srd[1])
+                yield ("arrive", srd[0], srd[1])
                 yield ("write", ("S", b, q, "R0"), ("P", g))
             else:
                 yield ("read", ("S", b, q, "R2"), ("S", g))
                 yield ("read", ("S", b, q, "R3"), ("S", g))
-                if v.own_region_p:
-                    yield ("write", ("S", b, q, "R2"), ("P", g))
-                else:
-                    yield ("wait", [srd])
-                    yield ("write", ("S", b, q, "R1"), ("P", g))
+                yield ("wait", [srd])
+                yield ("write", ("S", b, q, "R1"), ("P", g))
             yield ("arrive", f"PTF{b}", g >> 1)
             waits = [("DPF", g)]
             if g >= 2:
@@ -407,8 +415,10 @@ def compute(agent, plan, v):
             g += 1
         # epilogue
         yield ("wait", [("FIN", item)])
-        yield ("read", "DVACC", (item, n_it))
-        yield ("read", "DKACC", (item, n_it))
+        if n_it > 0:
+            yield ("read", "DVACC", (item, n_it))
+            yield ("read", "DKACC", (item, n_it))
+        # (an item without query tiles reads stale accumulators and writes zeros)
         yield ("arrive", "ACCE", item)
         if v.epilogue_tile_wait:
             yield ("wait", [("STGE", g - 1)])
@@ -434,78 +444,6 @@ def compute(agent, plan, v):
         yield from item_advance(W, item, not v.static_items)
 
 
-def compute_p(q, plan, v):
-    """pd_split: P^T of every tile for the key rows of quarter q, and the dV
-    part of the epilogue."""
-    g = 0
-    for item, n_it in enumerate(plan):
-        for it in range(n_it):
-            s, b = g % ST, g & 1
-            yield ("wait", [(f"QF{s}", g // ST)])
-            yield ("wait", [(f"SF{b}", g >> 1)])
-            yield ("read", ("LD", s), g)
-            for r in ("R0", "R1", "R2", "R3"):
-                yield ("read", ("S", b, q, r), ("S", g))
-            yield ("write", ("S", b, q, "R0"), ("P", g))
-            yield ("write", ("S", b, q, "R1"), ("P", g))
-            yield ("arrive", f"PTF{b}", g >> 1)
-            g += 1
-        yield ("wait", [("FIN", item)])
-        yield ("read", "DVACC", (item, n_it))
-        yield ("arrive", "ACCE", item)
-        yield ("wait", [("DQD", item)])
-        yield ("write", ("STG", 0), ("dV", item))
-        yield ("write", ("STG", 1), ("dV", item))
-        yield ("arrive", "EPS", item)
-        if q == 0:
-            yield ("wait", [("EPS", item)])
-
-            def store(item=item):
-                for h in range(2):
-                    W.read(("STG", h), ("dV", item))
-                    W.read(("DS", h, 0), ("dK", item))
-                    W.read(("DS", h, 1), ("dK", item))
-                W.bar("EPF").arrive(item)
-            yield ("async", "store", store)
-        yield ("wait", [("EPF", item)])
-        yield from item_advance(W, item, not v.static_items)
-
-
-def compute_ds(q, plan, v):
-    """pd_split: dS^T of every tile for the key rows of quarter q (P^T read back
-    from tensor memory), and the dK part of the epilogue."""
-    g = 0
-    for item, n_it in enumerate(plan):
-        for it in range(n_it):
-            s, b = g % ST, g & 1
-            waits = [(f"QF{s}", g // ST), (f"PTF{b}", g >> 1), ("DPF", g)]
-            if g >= 2:
-                waits.append((f"DSTE{b}", (g - 2) >> 1))
-            yield ("wait", waits)
-            yield ("read", ("LD", s), g)
-            yield ("read", "DP", g)
-            if v.pd_split_early_dpe:
-                yield ("arrive", "DPE", g)
-            yield ("read", ("S", b, q, "R0"), ("P", g))
-            yield ("read", ("S", b, q, "R1"), ("P", g))
-            if not v.pd_split_early_dpe:
-                yield ("arrive", "DPE", g)
-            yield ("write", ("DS", b, 0), g)
-            yield ("write", ("DS", b, 1), g)
-            yield ("arrive", f"DSF{b}", g >> 1)
-            g += 1
-        yield ("wait", [("FIN", item)])
-        yield ("read", "DKACC", (item, n_it))
-        yield ("arrive", "ACCE", item)
-        yield ("write", ("DS", 0, 0), ("dK", item))
-        yield ("write", ("DS", 0, 1), ("dK", item))
-        yield ("write", ("DS", 1, 0), ("dK", item))
-        yield ("write", ("DS", 1, 1), ("dK", item))
-        yield ("arrive", "EPS", item)
-        yield ("wait", [("EPF", item)])
-        yield from item_advance(W, item, not v.static_items)
-
-
 def dq_role(agent, plan, v):
     g = 0
     for item, n_it in enumerate(plan):
@@ -527,6 +465,14 @@ def dq_role(agent, plan, v):
                 if it + 1 == n_it:
                     yield ("arrive", "DQD", item)
             g += 1
+        if n_it == 0 and agent == 0:
+            # An item without query tiles leaves the staging tile as it was.  Its
+            # DQD arrival waits for the previous item's epilogue (EPF), which
+            # follows the compute warps' wait for the previous DQD: otherwise
+            # consecutive such items run DQD two phases ahead of that wait.
+            if item > 0 and not v.empty_item_no_epf_wait:
+                yield ("wait", [("EPF", item - 1)])
+            yield ("arrive", "DQD", item)
         yield from item_advance(W, item, not v.static_items)
 
 
@@ -547,22 +493,13 @@ def run_schedule(plan, seed, variant=None, max_steps=200000, in_order=False):
         counts[f"QE{s}"] = 2
     if v.single_dsf:
         counts["DSF0"] = NCOMP
-    if v.pd_split:
-        half = NCOMP // 2      # 2 P agents, 2 dS agents
-        counts.update({"PTF0": half, "PTF1": half, "DPE": half,
-                       "DSF0": half, "DSF1": half, "ACCE": NCOMP, "EPS": NCOMP})
     # one arrival per modelled agent frees a response slot
     counts["CLCE0"] = counts["CLCE1"] = 3 + NCOMP + NDQ
     for name, c in counts.items():
         W.bar(name, c)
     roles = {"prod": producer(plan, v), "A": issuer_a(plan, v), "B": issuer_b(plan, v)}
-    if v.pd_split:
-        for q in range(NCOMP // 2):
-            roles[f"p{q}"] = compute_p(q, plan, v)
-            roles[f"d{q}"] = compute_ds(q, plan, v)
-    else:
-        for a in range(NCOMP):
-            roles[f"comp{a}"] = compute(a, plan, v)
+    for a in range(NCOMP):
+        roles[f"comp{a}"] = compute(a, plan, v)
     for a in range(NDQ):
         roles[f"dq{a}"] = dq_role(a, plan, v)
     run_roles(W, roles, seed, in_order, max_steps)

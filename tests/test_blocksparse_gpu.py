@@ -65,6 +65,10 @@ CASES = [
     (1, 2, 513, 128, False, "fp16", 0.3, None, None),
     (2, 40, 1000, 128, True, "bf16", 0.5, 3, 2),  # many items per persistent CTA
     (2, 40, 1000, 64, False, "bf16", 0.5, 3, 2),
+    # mostly empty: runs of key tiles no query tile attends to (items whose
+    # per-item handshakes must still stay in step)
+    (1, 16, 2048, 128, False, "bf16", 0.08, None, None),
+    (1, 16, 2048, 128, True, "bf16", 0.08, None, None),
 ]
 
 

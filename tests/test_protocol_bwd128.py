@@ -5,13 +5,15 @@ Every barrier test must find its barrier in the phase it is for or the next,
 every arrival must land in its phase, every read must see the version it needs,
 and no schedule may deadlock.  The same checker must reject the protocol
 mistakes that were made while building the kernel, which shows it can see
-them."""
+them.  Plans include items without query tiles (block-sparse key tiles no
+query tile attends to), whose handshakes still run once per item."""
 
 import pytest
 
 import protocol_model as pm
 
-PLANS = [[1], [2], [5], [3, 1, 4], [1, 1, 1, 1], [2, 2, 2], [4, 3, 2, 1]]
+PLANS = [[1], [2], [5], [3, 1, 4], [1, 1, 1, 1], [2, 2, 2], [4, 3, 2, 1],
+         [0], [2, 0, 3], [0, 0, 1, 0], [1, 0, 0, 2, 0]]
 
 
 @pytest.mark.parametrize("plan", PLANS, ids=lambda p: "-".join(map(str, p)))
@@ -26,19 +28,6 @@ def test_earlier_correct_design_also_holds():
         pm.run_schedule([3, 2, 4, 1], seed, pm.Variant(no_dpe=True))
 
 
-def test_own_region_p_layout_needs_no_shared_read_barrier():
-    # each half writing P^T over its own S^T columns (dV reading them there)
-    for seed in range(120):
-        pm.run_schedule([3, 2, 4, 1], seed, pm.Variant(own_region_p=True))
-
-
-@pytest.mark.parametrize("plan", PLANS, ids=lambda p: "-".join(map(str, p)))
-def test_pipelined_p_ds_groups_design_holds(plan):
-    # next-step design: P^T and dS^T in two warp groups working on consecutive tiles
-    for seed in range(80):
-        pm.run_schedule(plan, seed, pm.Variant(pd_split=True))
-
-
 def test_static_item_order_holds():
     # without the mask the items are dealt in a fixed order: no response slots
     for seed in range(100):
@@ -46,14 +35,16 @@ def test_static_item_order_holds():
 
 
 @pytest.mark.parametrize("mistake", ["single_srd", "single_dsf", "epilogue_tile_wait",
-                                     "pd_split_early_dpe", "clc_no_empty_wait"])
+                                     "clc_no_empty_wait", "empty_item_no_epf_wait",
+                                     "empty_item_no_b_wait"])
 def test_checker_rejects_known_mistakes(mistake):
     caught = 0
-    plan = [2, 1, 1, 3] if mistake.startswith("clc") else [3, 2, 4, 1]
+    plan = {"clc_no_empty_wait": [2, 1, 1, 3],
+            "empty_item_no_epf_wait": [1, 0, 0, 2, 0],
+            "empty_item_no_b_wait": [2, 0, 3, 0, 0, 1]}.get(mistake, [3, 2, 4, 1])
     for seed in range(400):
         try:
-            kw = {mistake: True, "pd_split": mistake.startswith("pd_split")}
-            pm.run_schedule(plan, seed, pm.Variant(**kw))
+            pm.run_schedule(plan, seed, pm.Variant(**{mistake: True}))
         except pm.ProtocolError:
             caught += 1
     assert caught > 0, f"{mistake} was never caught"

@@ -1,7 +1,10 @@
 """The forward kernel's mbarrier protocol, checked on the CPU under random
 schedules (tests/protocol_model_fwd.py mirrors the kernel's roles): barrier
 tests in the phase they are for or the next, arrivals in their phase, reads of
-the versions they need, no deadlock; and protocol mistakes are rejected."""
+the versions they need, no deadlock; and protocol mistakes are rejected.
+Dense (causal and not) and block-sparse plans, including items where a tile
+starts attending in the middle, tiles with no marked key tile and items with
+none at all."""
 
 import pytest
 
@@ -12,89 +15,64 @@ PLANS = {
     "causal": [(1, 2), (3, 4), (5, 0)],
     "causal-repeat": [(2, 3), (2, 3), (2, 3), (4, 5)],
     "single-step": [(1, 0), (1, 2), (1, 1)],
+    "sparse": [(4, 4, (1, 0, 1, 0), (0, 1, 1, 1)), (3, 3, (0, 0, 1), (1, 0, 0)),
+               (4, 4, (1, 1, 1, 1), (0, 0, 0, 0)), (2, 2, (0, 0), (0, 0)),
+               (3, 3, (0, 1, 0), (0, 1, 1))],
+    "sparse-causal": [(3, 4, (0, 1, 1), (1, 0, 0, 1)), (1, 0, (1,), ()),
+                      (5, 6, (1, 0, 0, 0, 1), (0, 0, 1, 0, 0, 1)), (1, 2, (0,), (0, 1))],
+    "sparse-gaps": [(3, 3, (1, 0, 1), (0, 1, 0))] * 4,
 }
 
 
+@pytest.mark.parametrize("stages", [2, 3, 4])
 @pytest.mark.parametrize("name", sorted(PLANS))
-def test_forward_protocol_holds_under_random_schedules(name):
-    for seed in range(150):
-        pf.run_schedule(PLANS[name], seed)
-
-
-@pytest.mark.parametrize("name", sorted(PLANS))
-def test_split_softmax_design_holds(name):
-    # next-step design: each tile's softmax over two column halves, exchanging
-    # the row max per key tile and the row sum per item
+def test_forward_protocol_holds_under_random_schedules(name, stages):
+    # 2 K/V stages at d = 128, 3 with e4m3 scores at d = 128, 4 at d = 64
     for seed in range(100):
-        pf.run_schedule(PLANS[name], seed, pf.Variant(split=True))
+        pf.run_schedule(PLANS[name], seed, stages=stages)
 
 
-@pytest.mark.parametrize("name", sorted(PLANS))
-@pytest.mark.parametrize("split", [False, True], ids=["one-group", "split"])
-def test_order_c_design_holds(name, split):
-    # next-step design: per key tile both P V first, then both next S
+@pytest.mark.parametrize("plan", ["causal", "sparse"])
+def test_next_s_needs_the_pv_wait_although_issued_later(plan):
+    """S_t of the next key tile overwrites the columns P_t V reads.  Completed
+    in issue order the mistake would go unseen; with MMAs on different
+    accumulators free to complete out of order, as the hardware allows, it is
+    caught."""
+    v = pf.Variant(s_without_od_wait=True)
     for seed in range(100):
-        pf.run_schedule(PLANS[name], seed, pf.Variant(order_c=True, split=split))
-
-
-@pytest.mark.parametrize("order_c", [False, True], ids=["order-a", "order-c"])
-def test_next_s_needs_the_pv_wait_although_issued_later(order_c):
-    """S_t(j+1) overwrites the columns P_t(j) V reads.  Completed in issue
-    order the mistake would go unseen; with MMAs on different accumulators
-    free to complete out of order, as the hardware allows, it is caught."""
-    plan = [(3, 4), (2, 2)]
-    v = pf.Variant(order_c=order_c, s_without_od_wait=True)
-    for seed in range(100):
-        pf.run_schedule(plan, seed, v, in_order=True)
+        pf.run_schedule(PLANS[plan], seed, v, in_order=True)
     caught = 0
     for seed in range(300):
         try:
-            pf.run_schedule(plan, seed, v)
-        except pf.ProtocolError:
-            caught += 1
-    assert caught > 0
-
-
-SD_PLANS = {
-    "noncausal": [(6, 6), (6, 6), (2, 2)],
-    "causal": [(2, 4), (6, 8), (10, 0)],
-    "causal-repeat": [(3, 5), (3, 5), (1, 1), (8, 10)],
-}
-
-
-@pytest.mark.parametrize("name", sorted(SD_PLANS))
-def test_double_buffered_s_design_holds(name):
-    # next-step design: 64-key tiles, two S buffers per query tile; P ready and
-    # P V done are one barrier per S buffer
-    for seed in range(120):
-        pf.run_schedule(SD_PLANS[name], seed, pf.Variant(s_double=True))
-
-
-def test_double_buffered_s_needs_the_pv_wait():
-    caught = 0
-    for seed in range(300):
-        try:
-            pf.run_schedule(SD_PLANS["causal"], seed,
-                            pf.Variant(s_double=True, s_double_no_od_wait=True))
+            pf.run_schedule(PLANS[plan], seed, v)
         except pf.ProtocolError:
             caught += 1
     assert caught > 0
 
 
 def test_static_item_order_holds():
-    # without the mask the items are dealt in a fixed order: no response slots
+    # without a mask of either kind the items are dealt in a fixed order
     for seed in range(100):
         pf.run_schedule(PLANS["noncausal"], seed, pf.Variant(static_items=True))
 
 
-@pytest.mark.parametrize("mistake", ["ke_before_pv", "epilogue_no_od_wait",
-                                     "split_no_exchange_wait", "clc_no_empty_wait"])
-def test_checker_rejects_forward_mistakes(mistake):
+@pytest.mark.parametrize("mistake,plan,stages", [("ke_before_pv", "causal", 2),
+                                                 ("epilogue_no_od_wait", "causal", 2),
+                                                 ("clc_no_empty_wait", "causal", 2),
+                                                 ("s_wait_ignores_fresh_tile", "sparse-gaps", 4)])
+def test_checker_rejects_forward_mistakes(mistake, plan, stages):
     caught = 0
     for seed in range(300):
         try:
-            kw = {mistake: True, "split": mistake.startswith("split")}
-            pf.run_schedule([(1, 2), (3, 4), (5, 0), (2, 2)], seed, pf.Variant(**kw))
+            pf.run_schedule(PLANS[plan] + [(1, 2), (3, 4), (5, 0), (2, 2)], seed,
+                            pf.Variant(**{mistake: True}), stages=stages)
         except pf.ProtocolError:
             caught += 1
     assert caught > 0, f"{mistake} was never caught"
+
+
+def test_skipped_wait_is_implied_with_two_stages():
+    # the same skipped wait is harmless with two K/V stages (see Variant)
+    for seed in range(150):
+        pf.run_schedule(PLANS["sparse-gaps"], seed, pf.Variant(s_wait_ignores_fresh_tile=True),
+                        stages=2)
