@@ -457,6 +457,26 @@ def side_workloads(args, dev, clocks):
     return out
 
 
+def profile_workload(args):
+    """One workload's steps alone, on cuda:0: W warm-up and K timed steps."""
+    import torch
+    wl = args.profile_workload
+    passes = WORKLOADS[wl][7]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    run = DeviceRun(wl, passes, args.seed, dev)
+    for _ in range(args.warmup):
+        run.step()
+    per = run.events(args.steps)
+    for i in range(args.steps):
+        run.step(per[i])
+    torch.cuda.synchronize()
+    if run.attn.attn_last_device_status() != 0:
+        raise RuntimeError("device status not OK")
+    step_ms = DeviceRun.medians(per)[0]
+    return {"workload": DESCRIPTION[wl], "steps": args.steps, "ms_per_step": round(step_ms, 4)}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -723,10 +743,16 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--headline-only", action="store_true",
                     help="skip the other workloads (timed after the headline at N=1)")
+    ap.add_argument("--profile-workload", default=None, choices=sorted(WORKLOADS),
+                    help="run only this workload's steps (for a profiler) and print their "
+                         "median time; no end-to-end leg, no CPU baseline")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
+    if args.profile_workload:
+        print(json.dumps(profile_workload(args)), flush=True)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
