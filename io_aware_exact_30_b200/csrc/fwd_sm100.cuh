@@ -37,7 +37,8 @@
 // Roles (320 threads): warps 0-3 softmax of tile 0, warps 4-7 softmax of tile
 // 1 (thread t of a group owns query row t = TMEM lane t), warp 8 TMA
 // producer, warp 9 TMEM owner and MMA issuer.
-// Tensor memory: S/P of tile i at column 128 i, O of tile i at 256 + D i.
+// Tensor memory: S of tile i at column 128 i, O of tile i at 256 + D i; P of
+// tile i over its S (d = 128) or, at d = 64, in columns 384 + 64 i of its own.
 #pragma once
 
 #include "dropout.cuh"
@@ -151,6 +152,10 @@ struct FwdCfg {
     static constexpr int CLC_CONSUMERS = 10;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_O = 256;
+    // At d = 64, S (256 columns) and O (128) leave 128 columns free: P_t gets
+    // columns of its own there, so the next S_t need not wait for P_t V.
+    static constexpr bool P_OWN = D == 64;
+    static constexpr uint32_t COL_P = 384;
     static constexpr int NTHREADS = 320;
     static constexpr int WARP_TMA = 8, WARP_MMA = 9;
     static_assert(SMEM_BYTES <= 232448u, "dynamic shared memory above the sm_100 per-block limit");
@@ -321,7 +326,8 @@ __global__ void __launch_bounds__(320, 1)
                 // their barriers at once: a dependent wait stalls the issue of
                 // queued MMAs, so one stall per group.
                 const bool a0 = j0 < sh.nkv && sh.act(0, j0), a1 = j0 < sh.nkv && sh.act(1, j0);
-                const bool w0 = a0 && n_pv[0] > 0, w1 = a1 && n_pv[1] > 0;
+                const bool w0 = !C::P_OWN && a0 && n_pv[0] > 0,
+                           w1 = !C::P_OWN && a1 && n_pv[1] > 0;
                 if (!(ok = wait3(BAR(C::B_Q), items & 1, true, BAR(C::B_KF + kv % C::STAGES),
                                  (kv / C::STAGES) & 1, j0 < sh.nkv, BAR(C::B_OD), (n_pv[0] - 1) & 1,
                                  w0, abort_flag)))
@@ -352,7 +358,8 @@ __global__ void __launch_bounds__(320, 1)
                             tc_fence_after();
 #pragma unroll
                             for (int kk = 0; kk < 8; ++kk)
-                                mma_ts(tmem + C::COL_O + t * D, tmem + t * 128u + kk * 8u,
+                                mma_ts(tmem + C::COL_O + t * D,
+                                       tmem + (C::P_OWN ? C::COL_P + t * 64u : t * 128u) + kk * 8u,
                                        sdesc_sw128(sv + kk * 2048u, 16384, 1024), ID_O,
                                        (!((fresh >> t) & 1) || kk > 0) ? 1u : 0u);
                             mma_commit(BAR(C::B_OD + t));
@@ -361,8 +368,11 @@ __global__ void __launch_bounds__(320, 1)
                         }
                         if (jn < sh.nkv && sh.act(t, jn)) {
                             // S_t of the next union tile, into the columns the last
-                            // P_t V read once it has completed
-                            if (!(ok = wait3(BAR(C::B_OD + t), (n_pv[t] - 1) & 1, n_pv[t] > 0,
+                            // P_t V read once it has completed (with P in columns of
+                            // its own, the P-ready wait before that P V suffices: the
+                            // softmax had finished reading S_t)
+                            if (!(ok = wait3(BAR(C::B_OD + t), (n_pv[t] - 1) & 1,
+                                             !C::P_OWN && n_pv[t] > 0,
                                              BAR(C::B_KF + k1 % C::STAGES), (k1 / C::STAGES) & 1,
                                              !k_next, 0u, 0u, false, abort_flag)))
                                 break;
@@ -393,6 +403,10 @@ __global__ void __launch_bounds__(320, 1)
         const int r = threadIdx.x & 127;  // row of the tile == TMEM lane
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         const uint32_t colS = t * 128u, colO = C::COL_O + t * D;
+        // where P_t is written.  At d = 64 its own columns were last read by
+        // the previous P_t V, which the issuer queued before this S_t: the
+        // S-full commit covers every earlier MMA of the issuing thread.
+        const uint32_t colP = C::P_OWN ? C::COL_P + t * 64u : colS;
         int n_s = 0, bh, pair;  // S tiles of this query-tile slot seen so far
         bool ok = true;
         for (; ok && cs.cur >= 0; ok = ok && cs.advance(abort_flag, true)) {
@@ -529,7 +543,7 @@ __global__ void __launch_bounds__(320, 1)
                         }
                         pk[q] = pack2<BF16>(pv.x, pv.y);
                     }
-                    tmem_st16(lane_addr + colS + c * 16u, pk);
+                    tmem_st16(lane_addr + colP + c * 16u, pk);
                     if (c < 3) {
                         tmem_ld_wait();
                         reg_fence32(nxt);

@@ -25,6 +25,13 @@ work of its thread, copies in any order).
 
 Plan items: (n0, n1) for dense tiles (tile t attends to j < n_t), or
 (n0, n1, mask0, mask1) with mask_t a sequence of 0/1 per key tile.
+
+Two tensor-memory layouts: at d = 128 P_t is written over S_t (the next S_t
+waits for the last P_t V); at d = 64 (p_own) P_t has columns of its own, so
+the next S_t waits only for the softmax to have read S_t (the P-ready barrier
+the P V already waited on).  The softmax then writes P_t with no wait of its
+own: the S-full commit it waited on follows the last P_t V in issue order and
+so covers it.
 """
 
 from protocol_model import ProtocolError, World, item_advance, item_request, run_roles  # noqa: F401
@@ -35,7 +42,8 @@ NSM = 2     # softmax agents per query tile
 
 class Variant:
     def __init__(self, ke_before_pv=False, epilogue_no_od_wait=False, s_without_od_wait=False,
-                 static_items=False, clc_no_empty_wait=False, s_wait_ignores_fresh_tile=False):
+                 static_items=False, clc_no_empty_wait=False, s_wait_ignores_fresh_tile=False,
+                 s_before_pv=False):
         # release the K/V stage before the tile-1 P V of the step is issued
         self.ke_before_pv = ke_before_pv
         # the epilogue reads O without waiting for the last P V
@@ -59,9 +67,19 @@ class Variant:
         # an item needs no such wait either: the item's Q load follows the
         # previous item's last commit, which covers every earlier MMA.)
         self.s_wait_ignores_fresh_tile = s_wait_ignores_fresh_tile
+        # mistake (P in columns of its own): the next S_t is issued before this
+        # step's P_t V, so its S-full commit no longer covers that P V and the
+        # softmax may write P_t under it
+        self.s_before_pv = s_before_pv
 
 
 W = None
+P_OWN = False  # d = 64: P_t in tensor-memory columns of its own
+
+
+def p_cols(t, a):
+    """Where agent a of tile t writes P_t (and P_t V reads it)."""
+    return ("P", t, a) if P_OWN else ("S", t, a)
 
 
 class Item:
@@ -132,10 +150,10 @@ def issuer(plan, v):
         waits = [("Q", item)]
         if U:
             waits.append((f"KF{kv % ST}", kv // ST))
-        if a0[0] and n_pv[0] > 0:
+        if a0[0] and n_pv[0] > 0 and not P_OWN:
             waits.append(("OD0", n_pv[0] - 1))
         yield ("wait", waits)
-        if a0[1] and n_pv[1] > 0:
+        if a0[1] and n_pv[1] > 0 and not P_OWN:
             yield ("wait", [("OD1", n_pv[1] - 1)])
         for t in range(2):
             if a0[t]:
@@ -160,30 +178,43 @@ def issuer(plan, v):
                     yield ("wait", waits)
                 if t == 1 and v.ke_before_pv:
                     yield ("async", "mma", lambda s=s, n=n: W.bar(f"KE{s}").arrive(n))
-                if act:
-                    def pv(t=t, kvj=kvj, s=s, item=item, u=u):
-                        for a in range(NSM):
-                            W.read(("S", t, a), ("P", kvj))
-                        W.read(("V", s), kvj)
-                        W.write(("O", t), (item, u))
-                    yield ("async", "mma", pv, f"O{t}")
-                    k = n_pv[t]
-                    n_pv[t] += 1
-                    fresh[t] = False
-                    yield ("async", "mma", lambda t=t, k=k: W.bar(f"OD{t}").arrive(k))
-                if jn is not None and it.act[t][jn]:
-                    # S_t of the next union tile takes the columns the last P_t V
-                    # read: wait for that P V (of this item or an earlier one)
-                    waits = []
-                    skip = v.s_without_od_wait or (v.s_wait_ignores_fresh_tile and not act)
-                    if n_pv[t] > 0 and not skip:
-                        waits.append((f"OD{t}", n_pv[t] - 1))
-                    if not k_next:
-                        waits.append((f"KF{k1 % ST}", k1 // ST))
-                    if waits:
-                        yield ("wait", waits)
-                    k_next = True
-                    yield from issue_s(t, k1, item)
+                def do_pv(t=t, act=act, kvj=kvj, s=s, item=item, u=u):
+                    if act:
+                        def pv(t=t, kvj=kvj, s=s, item=item, u=u):
+                            for a in range(NSM):
+                                W.read(p_cols(t, a), ("P", kvj))
+                            W.read(("V", s), kvj)
+                            W.write(("O", t), (item, u))
+                        yield ("async", "mma", pv, f"O{t}")
+                        k = n_pv[t]
+                        n_pv[t] += 1
+                        fresh[t] = False
+                        yield ("async", "mma", lambda t=t, k=k: W.bar(f"OD{t}").arrive(k))
+
+                def do_next_s(t=t, act=act, k1=k1, item=item):
+                    nonlocal k_next
+                    if jn is not None and it.act[t][jn]:
+                        # S_t of the next union tile takes the columns the last P_t V
+                        # read: wait for that P V (of this item or an earlier one);
+                        # with P in columns of its own, the softmax read S_t before
+                        # the P-ready arrival the last P_t V waited for
+                        waits = []
+                        skip = (P_OWN or v.s_without_od_wait
+                                or (v.s_wait_ignores_fresh_tile and not act))
+                        if n_pv[t] > 0 and not skip:
+                            waits.append((f"OD{t}", n_pv[t] - 1))
+                        if not k_next:
+                            waits.append((f"KF{k1 % ST}", k1 // ST))
+                        if waits:
+                            yield ("wait", waits)
+                        k_next = True
+                        yield from issue_s(t, k1, item)
+                if v.s_before_pv:
+                    yield from do_next_s()
+                    yield from do_pv()
+                else:
+                    yield from do_pv()
+                    yield from do_next_s()
             if not v.ke_before_pv:
                 yield ("async", "mma", lambda s=s, n=n: W.bar(f"KE{s}").arrive(n))
         yield ("async", "mma", lambda item=item: W.bar("QE").arrive(item))
@@ -219,7 +250,7 @@ def softmax(t, agent, plan, v, rng):
                 # the kept max moves: O is rescaled, which needs the last P V
                 yield ("wait", [(f"OD{t}", n_s - 2)])
                 yield ("read", ("O", t), (item, prev_u))
-            yield ("write", ("S", t, agent), ("P", kv + u))
+            yield ("write", p_cols(t, agent), ("P", kv + u))
             yield ("arrive", f"PF{t}", n_s - 1)
             seen += 1
             prev_u = u
@@ -232,13 +263,16 @@ def softmax(t, agent, plan, v, rng):
         yield from item_advance(W, item, not v.static_items)
 
 
-def run_schedule(plan, seed, variant=None, max_steps=200000, in_order=False, stages=2):
+def run_schedule(plan, seed, variant=None, max_steps=200000, in_order=False, stages=2,
+                 p_own=False):
     """One random schedule of one CTA working through `plan`; raises
     ProtocolError on a violation or a deadlock.  in_order: complete each
-    unit's asynchronous work in issue order.  stages: K/V pipeline depth."""
+    unit's asynchronous work in issue order.  stages: K/V pipeline depth.
+    p_own: the d = 64 layout (P_t in columns of its own)."""
     import random
-    global W, ST
+    global W, ST, P_OWN
     ST = stages
+    P_OWN = p_own
     v = variant or Variant()
     W = World()
     for t in range(2):

@@ -50,6 +50,29 @@ def test_next_s_needs_the_pv_wait_although_issued_later(plan):
     assert caught > 0
 
 
+@pytest.mark.parametrize("stages", [2, 4])
+@pytest.mark.parametrize("name", sorted(PLANS))
+def test_forward_protocol_with_p_in_own_columns(name, stages):
+    # the d = 64 layout: P_t in columns of its own, next S_t after P-ready only
+    for seed in range(100):
+        pf.run_schedule(PLANS[name], seed, stages=stages, p_own=True)
+
+
+@pytest.mark.parametrize("plan", ["causal", "sparse"])
+def test_p_write_relies_on_the_issue_order(plan):
+    """With P in columns of its own, nothing waits for P_t V before P_t is
+    written again but the S-full commit queued after it; issuing the next S_t
+    ahead of the P V breaks that, and is caught."""
+    caught = 0
+    for seed in range(300):
+        try:
+            pf.run_schedule(PLANS[plan] + [(3, 3), (2, 4)], seed,
+                            pf.Variant(s_before_pv=True), stages=4, p_own=True)
+        except pf.ProtocolError:
+            caught += 1
+    assert caught > 0
+
+
 def test_static_item_order_holds():
     # without a mask of either kind the items are dealt in a fixed order
     for seed in range(100):
