@@ -229,7 +229,11 @@ int attn_bwd_dropout(const void* q, const void* k, const void* v, const void* o,
  * ATTN_ERR_HEADDIM).  workspace: caller-owned device memory of
  * attn_linear_workspace_bytes() bytes, 256-byte aligned: the per-chunk K^T V
  * in fp32 and the prefix states S_c in the input's type.  The state reaches
- * the tensor cores rounded to the input's 16-bit type.  Errors as attn_fwd.
+ * the tensor cores rounded to the input's 16-bit type.  With B * H >= 32 one
+ * fused kernel runs instead (one CTA per head and half of the value features,
+ * walking the chunks in order with the state kept on chip) and the workspace
+ * is left untouched; it forms the same fp32 sums in the same order.  Errors
+ * as attn_fwd.
  */
 size_t attn_linear_workspace_bytes(int B, int H, int N, int d);
 

@@ -121,6 +121,12 @@ int check_device(int* dev_out) {
     ok &= cudaFuncSetAttribute(attn::linear_out_kernel<false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                attn::kLinOutSmem) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn::linear_fused_kernel<true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               attn::LinFusedCfg::SMEM_BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn::linear_fused_kernel<false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               attn::LinFusedCfg::SMEM_BYTES) == cudaSuccess;
     ok &= attn::bwd_set_attributes();
     ok &= attn::bwd128_set_attributes();
     if (!ok) {
@@ -450,10 +456,21 @@ int attn_linear_fwd(const void* q, const void* k, const void* v, void* o, void* 
     p.scale = scale;
     CUtensorMap mq, mk, mv, ms;
     if (!make_map(&mq, q, dtype, BH, N, d) || !make_map(&mk, k, dtype, BH, N, d) ||
-        !make_map(&mv, v, dtype, BH, N, d) ||
-        !make_map(&ms, p.state, dtype, static_cast<int>(items), 128, 128))
+        !make_map(&mv, v, dtype, BH, N, d))
         return ATTN_ERR_LAUNCH;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (BH >= attn::kLinFusedMinHeads) {
+        // one CTA per (head, half of the value features), the state on chip
+        const unsigned gf = static_cast<unsigned>(2 * BH);
+        if (dtype == ATTN_BF16)
+            attn::linear_fused_kernel<true>
+                <<<gf, 320, attn::LinFusedCfg::SMEM_BYTES, st>>>(mq, mk, mv, p);
+        else
+            attn::linear_fused_kernel<false>
+                <<<gf, 320, attn::LinFusedCfg::SMEM_BYTES, st>>>(mq, mk, mv, p);
+        return launch_ok() ? ATTN_OK : ATTN_ERR_LAUNCH;
+    }
+    if (!make_map(&ms, p.state, dtype, static_cast<int>(items), 128, 128)) return ATTN_ERR_LAUNCH;
     const unsigned g = static_cast<unsigned>(items);
     const unsigned gp = static_cast<unsigned>((1LL * BH * 4096 + 255) / 256);
     if (dtype == ATTN_BF16) {

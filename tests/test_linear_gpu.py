@@ -31,9 +31,14 @@ def check(got, want, label):
     assert ma <= LIN_MAX_REL, f"{label} max-abs / max|O| {ma}"
 
 
+# B H < 32 runs the three chunk-parallel kernels, B H >= 32 the fused one
+# (one CTA per head and half of the value features, walking the chunks)
 @pytest.mark.parametrize("B,H,N,dtype", [(1, 2, 700, "bf16"), (1, 3, 513, "fp16"),
                                          (2, 1, 1, "bf16"), (1, 2, 129, "bf16"),
-                                         (1, 1, 128, "fp16"), (2, 40, 1000, "bf16")])
+                                         (1, 1, 128, "fp16"), (2, 40, 1000, "bf16"),
+                                         (1, 31, 300, "bf16"), (1, 32, 300, "fp16"),
+                                         (4, 8, 1, "bf16"), (8, 4, 129, "fp16"),
+                                         (2, 16, 128, "bf16"), (1, 33, 1535, "bf16")])
 def test_linear_attention_parity(B, H, N, dtype):
     d = 128
     arrs, f64 = inputs(B, H, N, d, dtype=dtype, seed=N)
