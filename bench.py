@@ -68,7 +68,8 @@ DESCRIPTION = {
     "large_head_fp8_fwd": "FP8-score causal fwd B=4 H=16 N=4096 d=128 (Q, K rotated and quantised "
                           "to e4m3 in the step, P V in bf16)",
     "large_head_linear": "causal linear attention B=4 H=16 N=4096 d=128 bf16, chunks of 128 "
-                         "(K^T V per chunk, prefix of the states, masked in-chunk product + Q S)",
+                         "(fused: per head and half of the value features, the chunks in order "
+                         "with the state on chip; masked in-chunk product + Q S)",
 }
 METRIC = "attention fwd and fwd+bwd TFLOP/s on 1 B200; % of dense BF16 tensor peak"
 L2_BYTES = 126 * 1024 * 1024
@@ -422,10 +423,11 @@ def side_workloads(args, dev, clocks):
         roof.pop("traffic_unit")
         if wl in LINEAR_WORKLOADS:
             # memory-bound: Q, K, V read and O written once (algorithmic), against
-            # the measured copy bandwidth; the kernels also move the chunk states
+            # the measured copy bandwidth (64 heads: the fused kernel, whose state
+            # stays on chip)
             _, _, hbm, src = peaks()
             alg = 4.0 * B * H * N * d * 2
-            roof = {"kernel": "linear_kv_kernel + linear_prefix_kernel + linear_out_kernel",
+            roof = {"kernel": "linear_fused_kernel",
                     "bound": "hbm", "achieved": round(alg / (fwd_ms * 1e-3) / 1e9, 1),
                     "peak": hbm, "peak_kind": f"hbm_gbs ({src})", "unit": "GB/s",
                     "frac": round(alg / (fwd_ms * 1e-3) / 1e9 / hbm, 4),

@@ -42,22 +42,34 @@ __global__ void __launch_bounds__(256) attn_fp8_quantize_kernel(
 #pragma unroll
     for (int e = 0; e < E; ++e) sgn[e] = (signs != nullptr && signs[lane * E + e] < 0) ? -1.f : 1.f;
 
-    float y[RPW][E];
-    float amax = 0.f;
+    // every row's load is issued before the first is used, so that a warp has
+    // all 16 in flight (the kernel is bound by HBM latency and bandwidth)
+    uint32_t raw[RPW][E / 2];
 #pragma unroll
     for (int i = 0; i < RPW; ++i) {
         const int r = row0 + warp + 8 * i;
 #pragma unroll
-        for (int e = 0; e < E; ++e) y[i][e] = 0.f;
+        for (int e = 0; e < E / 2; ++e) raw[i][e] = 0u;
         if (r < N) {
             const size_t off = (static_cast<size_t>(bh) * N + r) * D + lane * E;  // elements
-            const uint32_t* src = reinterpret_cast<const uint32_t*>(x + off * 2);
-#pragma unroll
-            for (int e = 0; e < E; e += 2) {
-                const float2 v = unpack2<BF16>(src[e / 2]);
-                y[i][e] = v.x * sgn[e];
-                y[i][e + 1] = v.y * sgn[e + 1];
+            if constexpr (E == 4) {
+                const uint2 w = __ldg(reinterpret_cast<const uint2*>(x + off * 2));
+                raw[i][0] = w.x;
+                raw[i][1] = w.y;
+            } else {
+                raw[i][0] = __ldg(reinterpret_cast<const uint32_t*>(x + off * 2));
             }
+        }
+    }
+    float y[RPW][E];
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < RPW; ++i) {
+#pragma unroll
+        for (int e = 0; e < E; e += 2) {
+            const float2 v = unpack2<BF16>(raw[i][e / 2]);
+            y[i][e] = v.x * sgn[e];
+            y[i][e + 1] = v.y * sgn[e + 1];
         }
         if (rotate) {
             // butterflies of stride h < E inside the thread, then stride E m

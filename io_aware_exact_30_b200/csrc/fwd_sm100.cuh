@@ -436,75 +436,15 @@ __global__ void __launch_bounds__(320, 1)
                 const int key0 = j * 128;
                 int limit = p.N - key0;
                 if (p.causal) limit = min(limit, qrow - key0 + 1);
-                // pass 1: row max over the 128 scores (two chunks of 64 in flight);
                 // tiles without masked columns (all but diagonal and tail tiles)
                 // take the unmasked path
                 const bool full = __all_sync(0xffffffffu, limit >= 128);
-                float mx = -INFINITY;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t a[32], b[32];
-                    tmem_ld32(lane_addr + colS + h * 64u, a);
-                    tmem_ld32(lane_addr + colS + h * 64u + 32u, b);
-                    tmem_ld_wait();
-                    reg_fence32(a);
-                    reg_fence32(b);
-                    if (full) {
-#pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            mx = max3(mx, __uint_as_float(a[e]), __uint_as_float(a[e + 1]));
-                            mx = max3(mx, __uint_as_float(b[e]), __uint_as_float(b[e + 1]));
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const int ca = h * 64 + e, cb = ca + 32;
-                            if (ca < limit) mx = fmaxf(mx, __uint_as_float(a[e]));
-                            if (cb < limit) mx = fmaxf(mx, __uint_as_float(b[e]));
-                        }
-                    }
-                }
-                const float m_tile = mx * sl;
-                // Move the max only when it grows past the threshold (the first
-                // tile always sets it); rescaling O needs O(j-1) complete.
-                const bool move = m_tile > m + kRescaleThreshold;
-                if (__any_sync(0xffffffffu, move)) {
-                    const float m_new = move ? m_tile : m;
-                    const float alpha = ex2(m - m_new);  // 0 on the first tile, 1 if not moved
-                    if (seen > 0) {
-                        ok = __all_sync(0xffffffffu,
-                                        wait_bounded(BAR(C::B_OD + t), (n_s - 2) & 1, abort_flag));
-                        if (!ok) break;
-                        tc_fence_after();
-#pragma unroll
-                        for (int c = 0; c < D / 32; ++c) {
-                            uint32_t o[32];
-                            tmem_ld32(lane_addr + colO + c * 32u, o);
-                            tmem_ld_wait();
-                            reg_fence32(o);
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                            tmem_st32(lane_addr + colO + c * 32u, o);
-                        }
-                        tmem_st_wait();
-                    }
-                    l *= alpha;
-                    m = m_new;
-                }
-                // pass 2: P = 2^(s scale log2e - m) chunk by chunk, written back as
-                // half over columns pass 2 has already read (P chunk c -> 16c..16c+15)
-                uint64_t sum2 = f2(0.f, 0.f);
-                const uint64_t sl2 = f2(sl, sl), negm2 = f2(-m, -m);
-                uint32_t cur[32];
-                tmem_ld32(lane_addr + colS, cur);
-                tmem_ld_wait();
-                reg_fence32(cur);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t nxt[32];
-                    if (c < 3) tmem_ld32(lane_addr + colS + (c + 1) * 32u, nxt);
-                    uint32_t pk[16];
+                const uint64_t sl2 = f2(sl, sl);
+                // P for the 32 keys of chunk c: 2^(s sl - m), masked keys 0, dropped
+                // keys 0 in P but kept in the row sum; xmax gathers the largest
+                // exponent s sl - m of the unmasked keys
+                auto exp_chunk = [&](const uint32_t(&cur)[32], int c, uint64_t negm2,
+                                     uint64_t& sum2, float& xmax, uint32_t(&pk)[16]) {
                     // dropout: keep masks (0xFF bytes) of this chunk's 32 keys
                     uint32_t kw[8];
                     if constexpr (DROP) {
@@ -519,7 +459,7 @@ __global__ void __launch_bounds__(320, 1)
                             kw[6] = keep_bytes(b.z, thr4), kw[7] = keep_bytes(b.w, thr4);
                         } else {
 #pragma unroll
-                            for (int t = 0; t < 8; ++t) kw[t] = 0xFFFFFFFFu;
+                            for (int u = 0; u < 8; ++u) kw[u] = 0xFFFFFFFFu;
                         }
                     }
 #pragma unroll
@@ -533,6 +473,7 @@ __global__ void __launch_bounds__(320, 1)
                             x = f2(xv.x, xv.y);
                         }
                         const float2 xv = unf2(x);
+                        xmax = max3(xmax, xv.x, xv.y);
                         const uint64_t pp = f2(ex2(xv.x), ex2(xv.y));
                         sum2 = add2(sum2, pp);
                         float2 pv = unf2(pp);
@@ -543,12 +484,121 @@ __global__ void __launch_bounds__(320, 1)
                         }
                         pk[q] = pack2<BF16>(pv.x, pv.y);
                     }
-                    tmem_st16(lane_addr + colP + c * 16u, pk);
-                    if (c < 3) {
-                        tmem_ld_wait();
-                        reg_fence32(nxt);
+                };
+                // Past a row's first key tile the kept max usually stands, so the
+                // exponentials are taken against it in a single pass that also
+                // finds the tile's largest exponent.  The pass stands when no row
+                // of the warp exceeds the threshold (exactly when the two-pass
+                // form would keep the max); otherwise the two-pass form below
+                // redoes the tile.  P is written only once the pass stands, so S
+                // is still whole for the redo.
+                // (Not with dropout: its keep masks leave no registers for the
+                // held P.)
+                bool done = false;
+                uint64_t sum2 = f2(0.f, 0.f);
+                if (!DROP && seen > 0) {
+                    const uint64_t negm2 = f2(-m, -m);
+                    float xmax = -INFINITY;
+                    uint32_t pk[4][16];
+                    uint32_t cur[32];
+                    tmem_ld32(lane_addr + colS, cur);
+                    tmem_ld_wait();
+                    reg_fence32(cur);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) cur[e] = nxt[e];
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t nxt[32];
+                        if (c < 3) tmem_ld32(lane_addr + colS + (c + 1) * 32u, nxt);
+                        exp_chunk(cur, c, negm2, sum2, xmax, pk[c]);
+                        if (c < 3) {
+                            tmem_ld_wait();
+                            reg_fence32(nxt);
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) cur[e] = nxt[e];
+                        }
+                    }
+                    if (__all_sync(0xffffffffu, !(xmax > kRescaleThreshold))) {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) tmem_st16(lane_addr + colP + c * 16u, pk[c]);
+                        done = true;
+                    } else {
+                        sum2 = f2(0.f, 0.f);
+                    }
+                }
+                if (!done) {
+                    // pass 1: row max over the 128 scores (two chunks of 64 in flight)
+                    float mx = -INFINITY;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t a[32], b[32];
+                        tmem_ld32(lane_addr + colS + h * 64u, a);
+                        tmem_ld32(lane_addr + colS + h * 64u + 32u, b);
+                        tmem_ld_wait();
+                        reg_fence32(a);
+                        reg_fence32(b);
+                        if (full) {
+#pragma unroll
+                            for (int e = 0; e < 32; e += 2) {
+                                mx = max3(mx, __uint_as_float(a[e]), __uint_as_float(a[e + 1]));
+                                mx = max3(mx, __uint_as_float(b[e]), __uint_as_float(b[e + 1]));
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) {
+                                const int ca = h * 64 + e, cb = ca + 32;
+                                if (ca < limit) mx = fmaxf(mx, __uint_as_float(a[e]));
+                                if (cb < limit) mx = fmaxf(mx, __uint_as_float(b[e]));
+                            }
+                        }
+                    }
+                    const float m_tile = mx * sl;
+                    // Move the max only when it grows past the threshold (the first
+                    // tile always sets it); rescaling O needs O(j-1) complete.
+                    const bool move = m_tile > m + kRescaleThreshold;
+                    if (__any_sync(0xffffffffu, move)) {
+                        const float m_new = move ? m_tile : m;
+                        const float alpha = ex2(m - m_new);  // 0 on the first tile, 1 if not moved
+                        if (seen > 0) {
+                            ok = __all_sync(0xffffffffu,
+                                            wait_bounded(BAR(C::B_OD + t), (n_s - 2) & 1, abort_flag));
+                            if (!ok) break;
+                            tc_fence_after();
+#pragma unroll
+                            for (int c = 0; c < D / 32; ++c) {
+                                uint32_t o[32];
+                                tmem_ld32(lane_addr + colO + c * 32u, o);
+                                tmem_ld_wait();
+                                reg_fence32(o);
+#pragma unroll
+                                for (int i = 0; i < 32; ++i)
+                                    o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                                tmem_st32(lane_addr + colO + c * 32u, o);
+                            }
+                            tmem_st_wait();
+                        }
+                        l *= alpha;
+                        m = m_new;
+                    }
+                    // pass 2: P = 2^(s scale log2e - m) chunk by chunk, written back as
+                    // half over columns pass 2 has already read (P chunk c -> 16c..16c+15)
+                    const uint64_t negm2 = f2(-m, -m);
+                    float xmax = -INFINITY;
+                    uint32_t cur[32];
+                    tmem_ld32(lane_addr + colS, cur);
+                    tmem_ld_wait();
+                    reg_fence32(cur);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t nxt[32];
+                        if (c < 3) tmem_ld32(lane_addr + colS + (c + 1) * 32u, nxt);
+                        uint32_t pk[16];
+                        exp_chunk(cur, c, negm2, sum2, xmax, pk);
+                        tmem_st16(lane_addr + colP + c * 16u, pk);
+                        if (c < 3) {
+                            tmem_ld_wait();
+                            reg_fence32(nxt);
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) cur[e] = nxt[e];
+                        }
                     }
                 }
                 const float2 sv2 = unf2(sum2);
