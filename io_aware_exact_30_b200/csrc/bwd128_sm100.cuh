@@ -60,8 +60,8 @@ struct Bwd128Cfg {
                          B_PTF = B_DPF + 1, B_DVD = B_PTF + 2, B_DSF = B_DVD + 2,
                          B_DSTE = B_DSF + 2, B_DQF = B_DSTE + 2, B_DQE = B_DQF + 1,
                          B_FIN = B_DQE + 1, B_DR = B_FIN + 1, B_KVE = B_DR + 2, B_ACCE = B_KVE + 1,
-                         B_SRD = B_ACCE + 1, B_STGF = B_SRD + 2, B_STGE = B_STGF + 1,
-                         B_CLCF = B_STGE + 1, B_CLCE = B_CLCF + 2, B_DPE = B_CLCE + 2,
+                         B_SRD = B_ACCE + 1, B_STGF = B_SRD + 2, B_STGE = B_STGF + 2,
+                         B_CLCF = B_STGE + 2, B_CLCE = B_CLCF + 2, B_DPE = B_CLCE + 2,
                          B_EPS = B_DPE + 1, B_EPF = B_EPS + 1, B_DQD = B_EPF + 1,
                          NBAR = B_DQD + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
@@ -177,8 +177,10 @@ __global__ void __launch_bounds__(480, 1)
         mbar_init(BAR(C::B_FIN), 1);
         mbar_init(BAR(C::B_SRD), C::NCOMPUTE / 2);
         mbar_init(BAR(C::B_SRD + 1), C::NCOMPUTE / 2);
-        mbar_init(BAR(C::B_STGF), C::NDQ);
-        mbar_init(BAR(C::B_STGE), 1);
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(BAR(C::B_STGF + h), C::NDQ);
+            mbar_init(BAR(C::B_STGE + h), 1);
+        }
         for (int i = 0; i < 2; ++i) {
             mbar_init(BAR(C::B_CLCF + i), 1);
             mbar_init(BAR(C::B_CLCE + i), C::CLC_CONSUMERS);
@@ -439,28 +441,45 @@ __global__ void __launch_bounds__(480, 1)
                 reg_fence32(v[1]);
                 tc_fence_before();
                 mbar_arrive(BAR(C::B_DQE));  // the values are in registers: columns free
-                // the previous tile's bulk reduction has finished reading the staging tile
-                if (g >= 1 && !(dq_ok = __all_sync(0xffffffffu,
-                                                   wait_bounded(BAR(C::B_STGE), (g - 1) & 1,
-                                                                abort_flag))))
-                    break;
+                // The staging tile goes out in two 16 KB halves of 32 queries, each
+                // by its own bulk reduction, so that half 1 is written while half
+                // 0's reduction reads: a half is rewritten once the previous tile's
+                // reduction of it has read it (the issuer waits for all but its
+                // newest bulk group, then releases the half).
 #pragma unroll
-                for (int e = 0; e < 64; ++e)
-                    st_shared_f32(stg + e * 512u, __uint_as_float(v[e >> 5][e & 31]) * p.scale);
-                fence_proxy_async_smem();
-                mbar_arrive(BAR(C::B_STGF));
-                if (issuer) {
-                    if (!wait_bounded(BAR(C::B_STGF), g & 1, abort_flag)) {
-                        dq_ok = false;
-                    } else {
-                        const int nq = min(64, p.N - q0);
-                        bulk_reduce_add_f32(acc_head + static_cast<size_t>(q0) * D,
-                                            base + C::OFF_STG, static_cast<uint32_t>(nq) * 512u);
-                        bulk_commit();
-                        bulk_wait_read_all();
-                        mbar_arrive(BAR(C::B_STGE));
-                        if (it + 1 == n_it) mbar_arrive(BAR(C::B_DQD));  // item's staging done
+                for (int h = 0; h < 2; ++h) {
+                    if (g >= 1) {
+                        if (issuer) {
+                            bulk_wait_read_but1();
+                            mbar_arrive(BAR(C::B_STGE + h));
+                        }
+                        if (!(dq_ok = __all_sync(0xffffffffu,
+                                                 wait_bounded(BAR(C::B_STGE + h), (g - 1) & 1,
+                                                              abort_flag))))
+                            break;
                     }
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        st_shared_f32(stg + (h * 32 + e) * 512u, __uint_as_float(v[h][e]) * p.scale);
+                    fence_proxy_async_smem();
+                    mbar_arrive(BAR(C::B_STGF + h));
+                    if (issuer) {
+                        if (!wait_bounded(BAR(C::B_STGF + h), g & 1, abort_flag)) {
+                            dq_ok = false;
+                        } else {
+                            const int nq = min(32, p.N - q0 - 32 * h);
+                            if (nq > 0)
+                                bulk_reduce_add_f32(acc_head + static_cast<size_t>(q0 + 32 * h) * D,
+                                                    base + C::OFF_STG + h * 16384u,
+                                                    static_cast<uint32_t>(nq) * 512u);
+                            bulk_commit();
+                        }
+                    }
+                    if (!(dq_ok = __all_sync(0xffffffffu, dq_ok))) break;
+                }
+                if (dq_ok && issuer && it + 1 == n_it) {
+                    bulk_wait_read_all();             // the staging tile is free for
+                    mbar_arrive(BAR(C::B_DQD));       // the item's epilogue
                 }
                 dq_ok = __all_sync(0xffffffffu, dq_ok);
                 if (!dq_ok) break;

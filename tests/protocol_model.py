@@ -42,7 +42,7 @@ class ProtocolError(AssertionError):
 class Variant:
     single_srd: bool = False      # one barrier (not one per S buffer) for the shared S^T read
     single_dsf: bool = False      # one barrier (not one per dS^T buffer) for dS^T ready
-    epilogue_tile_wait: bool = False  # epilogue waits the per-tile staging barrier, not DQD
+    epilogue_tile_wait: bool = False  # epilogue waits the last tile's staging-full barrier, not DQD
     no_dpe: bool = False          # dP^T(g) waits for dS^T(g-1) instead of the dP^T release
     # work items dealt in a fixed order (no mask) instead of taken through
     # cluster launch control responses (causal)
@@ -53,6 +53,9 @@ class Variant:
     empty_item_no_epf_wait: bool = False
     # issuer B commits an empty item's FIN and KVE without waiting (the same)
     empty_item_no_b_wait: bool = False
+    # a staging half is released without waiting for the previous tile's
+    # reduction to have read it
+    stg_half_no_read_wait: bool = False
 
 
 class Barrier:
@@ -421,7 +424,7 @@ def compute(agent, plan, v):
         # (an item without query tiles reads stale accumulators and writes zeros)
         yield ("arrive", "ACCE", item)
         if v.epilogue_tile_wait:
-            yield ("wait", [("STGE", g - 1)])
+            yield ("wait", [("STGF1", g - 1)])
         else:
             yield ("wait", [("DQD", item)])
         # half h stages its 64 columns: dV into the staging tile's h-th 16 KB,
@@ -451,19 +454,30 @@ def dq_role(agent, plan, v):
             yield ("wait", [("DQF", g)])
             yield ("read", "DQ", g)
             yield ("arrive", "DQE", g)
-            if g >= 1:
-                yield ("wait", [("STGE", g - 1)])
-            # each dQ warp writes its feature columns in both 16 KB halves
+            # the staging tile in two 16 KB halves (32 queries each), each sent by
+            # its own bulk reduction; agent 0 (the issuing lane) releases a half
+            # once the previous tile's reduction of it has read it
             for h in range(2):
+                if g >= 1:
+                    if agent == 0:
+                        if not v.stg_half_no_read_wait:
+                            yield ("wait", [(f"RD{h}", g - 1)])
+                        yield ("arrive", f"STGE{h}", g - 1)
+                    yield ("wait", [(f"STGE{h}", g - 1)])
+                # each dQ warp writes its feature column of the half
                 yield ("write", ("STG", h), ("dQ", g))
-            yield ("arrive", "STGF", g)
-            if agent == 0:
-                yield ("wait", [("STGF", g)])
-                for h in range(2):
-                    yield ("read", ("STG", h), ("dQ", g))
-                yield ("arrive", "STGE", g)
-                if it + 1 == n_it:
-                    yield ("arrive", "DQD", item)
+                yield ("arrive", f"STGF{h}", g)
+                if agent == 0:
+                    yield ("wait", [(f"STGF{h}", g)])
+
+                    def reduce(h=h, g=g):
+                        W.read(("STG", h), ("dQ", g))
+                        W.bar(f"RD{h}").arrive(g)
+                    yield ("async", "bulk", reduce, "tma")
+            if agent == 0 and it + 1 == n_it:
+                # the epilogue reuses the staging tile once both reductions read it
+                yield ("wait", [("RD0", g), ("RD1", g)])
+                yield ("arrive", "DQD", item)
             g += 1
         if n_it == 0 and agent == 0:
             # An item without query tiles leaves the staging tile as it was.  Its
@@ -488,7 +502,7 @@ def run_schedule(plan, seed, variant=None, max_steps=200000, in_order=False):
     W = World()
     counts = {"KVE": 2, "ACCE": NCOMP, "PTF0": NCOMP, "PTF1": NCOMP, "DSF0": NCOMP,
               "DSF1": NCOMP, "DPE": NCOMP, "SRD0": NCOMP // 2, "SRD1": NCOMP // 2,
-              "EPS": NCOMP, "DQE": NDQ, "STGF": NDQ}
+              "EPS": NCOMP, "DQE": NDQ, "STGF0": NDQ, "STGF1": NDQ}
     for s in range(ST):
         counts[f"QE{s}"] = 2
     if v.single_dsf:

@@ -36,7 +36,7 @@ def test_static_item_order_holds():
 
 @pytest.mark.parametrize("mistake", ["single_srd", "single_dsf", "epilogue_tile_wait",
                                      "clc_no_empty_wait", "empty_item_no_epf_wait",
-                                     "empty_item_no_b_wait"])
+                                     "empty_item_no_b_wait", "stg_half_no_read_wait"])
 def test_checker_rejects_known_mistakes(mistake):
     caught = 0
     plan = {"clc_no_empty_wait": [2, 1, 1, 3],
