@@ -106,19 +106,6 @@ __device__ __forceinline__ bool wait3(uint32_t b0, uint32_t p0, bool e0, uint32_
            (r2 || wait_bounded(b2, p2, abort_flag));
 }
 
-// The same for up to four phases.
-__device__ __forceinline__ bool wait4(uint32_t b0, uint32_t p0, bool e0, uint32_t b1, uint32_t p1,
-                                      bool e1, uint32_t b2, uint32_t p2, bool e2, uint32_t b3,
-                                      uint32_t p3, bool e3, volatile uint32_t* abort_flag) {
-    const bool r0 = !e0 || mbar_test_wait(b0, p0);
-    const bool r1 = !e1 || mbar_test_wait(b1, p1);
-    const bool r2 = !e2 || mbar_test_wait(b2, p2);
-    const bool r3 = !e3 || mbar_test_wait(b3, p3);
-    if (r0 && r1 && r2 && r3) return true;
-    return (r0 || wait_bounded(b0, p0, abort_flag)) && (r1 || wait_bounded(b1, p1, abort_flag)) &&
-           (r2 || wait_bounded(b2, p2, abort_flag)) && (r3 || wait_bounded(b3, p3, abort_flag));
-}
-
 // ---------------------------------------------------- cluster launch control --
 // Asks the scheduler to cancel the launch of a not-yet-running CTA of this
 // grid; a 16-byte response lands at `resp` and completes 16 transaction bytes
