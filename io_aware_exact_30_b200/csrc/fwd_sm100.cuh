@@ -348,12 +348,34 @@ __global__ void __launch_bounds__(320, 1)
                     bool k_next = false;  // K of the next union tile has landed
                     for (int t = 0; ok && t < 2; ++t) {
                         const bool act = sh.act(t, j);
-                        // V_j (first tile only), P_t, and at the item's first P_t V
-                        // the previous epilogue's read of O_t, which P_t V overwrites
-                        if (!(ok = wait3(BAR(C::B_VF + s), n & 1, t == 0, BAR(C::B_PF + t),
-                                         n_pv[t] & 1, act, BAR(C::B_OE + t), (n_done[t] - 1) & 1,
-                                         act && ((fresh >> t) & 1) && n_done[t] > 0, abort_flag)))
-                            break;
+                        const bool nxt = jn < sh.nkv && sh.act(t, jn);  // S_t of the next union tile
+                        if constexpr (C::P_OWN) {
+                            // P in columns of its own: the next S_t goes out first,
+                            // as soon as P-ready shows the softmax is done with S_t
+                            // (and its K has landed), ahead of this P_t V; the
+                            // softmax waits for that P V before it writes P_t again
+                            if (!(ok = wait3(BAR(C::B_VF + s), n & 1, t == 0, BAR(C::B_PF + t),
+                                             n_pv[t] & 1, act, BAR(C::B_KF + k1 % C::STAGES),
+                                             (k1 / C::STAGES) & 1, nxt && !k_next, abort_flag)))
+                                break;
+                            if (nxt) {
+                                k_next = true;
+                                tc_fence_after();
+                                issue_s(t, k1);
+                            }
+                            // the previous epilogue's read of O_t, which the item's
+                            // first P_t V overwrites
+                            if (act && ((fresh >> t) & 1) && n_done[t] > 0 &&
+                                !(ok = wait_bounded(BAR(C::B_OE + t), (n_done[t] - 1) & 1, abort_flag)))
+                                break;
+                        } else {
+                            // V_j (first tile only), P_t, and at the item's first P_t V
+                            // the previous epilogue's read of O_t, which P_t V overwrites
+                            if (!(ok = wait3(BAR(C::B_VF + s), n & 1, t == 0, BAR(C::B_PF + t),
+                                             n_pv[t] & 1, act, BAR(C::B_OE + t), (n_done[t] - 1) & 1,
+                                             act && ((fresh >> t) & 1) && n_done[t] > 0, abort_flag)))
+                                break;
+                        }
                         if (act) {
                             tc_fence_after();
 #pragma unroll
@@ -366,13 +388,10 @@ __global__ void __launch_bounds__(320, 1)
                             ++n_pv[t];
                             fresh &= ~(1 << t);
                         }
-                        if (jn < sh.nkv && sh.act(t, jn)) {
+                        if (!C::P_OWN && nxt) {
                             // S_t of the next union tile, into the columns the last
-                            // P_t V read once it has completed (with P in columns of
-                            // its own, the P-ready wait before that P V suffices: the
-                            // softmax had finished reading S_t)
-                            if (!(ok = wait3(BAR(C::B_OD + t), (n_pv[t] - 1) & 1,
-                                             !C::P_OWN && n_pv[t] > 0,
+                            // P_t V read once it has completed
+                            if (!(ok = wait3(BAR(C::B_OD + t), (n_pv[t] - 1) & 1, n_pv[t] > 0,
                                              BAR(C::B_KF + k1 % C::STAGES), (k1 / C::STAGES) & 1,
                                              !k_next, 0u, 0u, false, abort_flag)))
                                 break;
@@ -403,9 +422,8 @@ __global__ void __launch_bounds__(320, 1)
         const int r = threadIdx.x & 127;  // row of the tile == TMEM lane
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         const uint32_t colS = t * 128u, colO = C::COL_O + t * D;
-        // where P_t is written.  At d = 64 its own columns were last read by
-        // the previous P_t V, which the issuer queued before this S_t: the
-        // S-full commit covers every earlier MMA of the issuing thread.
+        // where P_t is written (at d = 64 its own columns, last read by the
+        // previous P_t V, which the softmax waits for first)
         const uint32_t colP = C::P_OWN ? C::COL_P + t * 64u : colS;
         int n_s = 0, bh, pair;  // S tiles of this query-tile slot seen so far
         bool ok = true;
@@ -431,6 +449,8 @@ __global__ void __launch_bounds__(320, 1)
                 ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SF + t), n_s & 1, abort_flag));
                 if (!ok) break;
                 ++n_s;
+                // (P in columns of its own) the last P_t V has completed
+                bool pv_done = !C::P_OWN || n_s < 2;
                 tc_fence_after();
                 // keys at or past N, and (causal) keys after this query, are masked
                 const int key0 = j * 128;
@@ -517,6 +537,13 @@ __global__ void __launch_bounds__(320, 1)
                         }
                     }
                     if (__all_sync(0xffffffffu, !(xmax > kRescaleThreshold))) {
+                        if (!pv_done) {
+                            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_OD + t),
+                                                                      (n_s - 2) & 1, abort_flag));
+                            if (!ok) break;
+                            pv_done = true;
+                            tc_fence_after();
+                        }
 #pragma unroll
                         for (int c = 0; c < 4; ++c) tmem_st16(lane_addr + colP + c * 16u, pk[c]);
                         done = true;
@@ -561,6 +588,7 @@ __global__ void __launch_bounds__(320, 1)
                             ok = __all_sync(0xffffffffu,
                                             wait_bounded(BAR(C::B_OD + t), (n_s - 2) & 1, abort_flag));
                             if (!ok) break;
+                            pv_done = true;
                             tc_fence_after();
 #pragma unroll
                             for (int c = 0; c < D / 32; ++c) {
@@ -580,6 +608,13 @@ __global__ void __launch_bounds__(320, 1)
                     }
                     // pass 2: P = 2^(s scale log2e - m) chunk by chunk, written back as
                     // half over columns pass 2 has already read (P chunk c -> 16c..16c+15)
+                    if (!pv_done) {
+                        ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_OD + t),
+                                                                  (n_s - 2) & 1, abort_flag));
+                        if (!ok) break;
+                        pv_done = true;
+                        tc_fence_after();
+                    }
                     const uint64_t negm2 = f2(-m, -m);
                     float xmax = -INFINITY;
                     uint32_t cur[32];

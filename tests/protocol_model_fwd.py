@@ -28,10 +28,9 @@ Plan items: (n0, n1) for dense tiles (tile t attends to j < n_t), or
 
 Two tensor-memory layouts: at d = 128 P_t is written over S_t (the next S_t
 waits for the last P_t V); at d = 64 (p_own) P_t has columns of its own, so
-the next S_t waits only for the softmax to have read S_t (the P-ready barrier
-the P V already waited on).  The softmax then writes P_t with no wait of its
-own: the S-full commit it waited on follows the last P_t V in issue order and
-so covers it.
+the next S_t is issued as soon as P-ready shows the softmax is done with S_t,
+ahead of the P_t V, and the softmax waits for that P_t V before it writes
+P_t again.
 """
 
 from protocol_model import ProtocolError, World, item_advance, item_request, run_roles  # noqa: F401
@@ -43,7 +42,7 @@ NSM = 2     # softmax agents per query tile
 class Variant:
     def __init__(self, ke_before_pv=False, epilogue_no_od_wait=False, s_without_od_wait=False,
                  static_items=False, clc_no_empty_wait=False, s_wait_ignores_fresh_tile=False,
-                 s_before_pv=False):
+                 p_write_no_od_wait=False):
         # release the K/V stage before the tile-1 P V of the step is issued
         self.ke_before_pv = ke_before_pv
         # the epilogue reads O without waiting for the last P V
@@ -67,10 +66,10 @@ class Variant:
         # an item needs no such wait either: the item's Q load follows the
         # previous item's last commit, which covers every earlier MMA.)
         self.s_wait_ignores_fresh_tile = s_wait_ignores_fresh_tile
-        # mistake (P in columns of its own): the next S_t is issued before this
-        # step's P_t V, so its S-full commit no longer covers that P V and the
-        # softmax may write P_t under it
-        self.s_before_pv = s_before_pv
+        # mistake (P in columns of its own): the softmax writes P_t without
+        # waiting for the last P_t V, which reads the same columns (the next
+        # S_t goes out ahead of that P V, so S-full does not cover it)
+        self.p_write_no_od_wait = p_write_no_od_wait
 
 
 W = None
@@ -209,7 +208,8 @@ def issuer(plan, v):
                             yield ("wait", waits)
                         k_next = True
                         yield from issue_s(t, k1, item)
-                if v.s_before_pv:
+                if P_OWN:
+                    # the next S_t first: its columns were read before P-ready
                     yield from do_next_s()
                     yield from do_pv()
                 else:
@@ -246,10 +246,15 @@ def softmax(t, agent, plan, v, rng):
             yield ("wait", [(f"SF{t}", n_s)])
             n_s += 1
             yield ("read", ("S", t, agent), ("S", kv + u))
+            od_waited = False  # for the last P_t V
             if seen > 0 and rng.random() < 0.3:
                 # the kept max moves: O is rescaled, which needs the last P V
                 yield ("wait", [(f"OD{t}", n_s - 2)])
+                od_waited = True
                 yield ("read", ("O", t), (item, prev_u))
+            if P_OWN and n_s >= 2 and not od_waited and not v.p_write_no_od_wait:
+                # P_t's columns were last read by the previous P_t V
+                yield ("wait", [(f"OD{t}", n_s - 2)])
             yield ("write", p_cols(t, agent), ("P", kv + u))
             yield ("arrive", f"PF{t}", n_s - 1)
             seen += 1

@@ -59,15 +59,15 @@ def test_forward_protocol_with_p_in_own_columns(name, stages):
 
 
 @pytest.mark.parametrize("plan", ["causal", "sparse"])
-def test_p_write_relies_on_the_issue_order(plan):
-    """With P in columns of its own, nothing waits for P_t V before P_t is
-    written again but the S-full commit queued after it; issuing the next S_t
-    ahead of the P V breaks that, and is caught."""
+def test_p_write_needs_the_pv_wait(plan):
+    """With P in columns of its own the next S_t goes out ahead of P_t V, so
+    nothing but the softmax's own wait keeps its next P_t write off the
+    columns that P V still reads; skipping that wait is caught."""
     caught = 0
     for seed in range(300):
         try:
             pf.run_schedule(PLANS[plan] + [(3, 3), (2, 4)], seed,
-                            pf.Variant(s_before_pv=True), stages=4, p_own=True)
+                            pf.Variant(p_write_no_od_wait=True), stages=4, p_own=True)
         except pf.ProtocolError:
             caught += 1
     assert caught > 0
