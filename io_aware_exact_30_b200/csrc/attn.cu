@@ -366,11 +366,11 @@ int attn_fp8_quantize(const void* x, unsigned char* x8, float* scales, const sig
     const bool bf = dtype == ATTN_BF16;
     const unsigned g = static_cast<unsigned>(blocks);
     if (d == 64) {
-        if (bf) attn::attn_fp8_quantize_kernel<64, true><<<g, 256, 0, st>>>(in, x8, scales, sg, rotate, N);
-        else attn::attn_fp8_quantize_kernel<64, false><<<g, 256, 0, st>>>(in, x8, scales, sg, rotate, N);
+        if (bf) attn::attn_fp8_quantize_kernel<64, true><<<g, 512, 0, st>>>(in, x8, scales, sg, rotate, N);
+        else attn::attn_fp8_quantize_kernel<64, false><<<g, 512, 0, st>>>(in, x8, scales, sg, rotate, N);
     } else {
-        if (bf) attn::attn_fp8_quantize_kernel<128, true><<<g, 256, 0, st>>>(in, x8, scales, sg, rotate, N);
-        else attn::attn_fp8_quantize_kernel<128, false><<<g, 256, 0, st>>>(in, x8, scales, sg, rotate, N);
+        if (bf) attn::attn_fp8_quantize_kernel<128, true><<<g, 512, 0, st>>>(in, x8, scales, sg, rotate, N);
+        else attn::attn_fp8_quantize_kernel<128, false><<<g, 512, 0, st>>>(in, x8, scales, sg, rotate, N);
     }
     return launch_ok() ? ATTN_OK : ATTN_ERR_LAUNCH;
 }

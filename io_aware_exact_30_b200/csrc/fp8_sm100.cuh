@@ -23,107 +23,104 @@
 
 namespace attn {
 
-// One CTA per (head, 128-row block) of x: 8 warps, each owning rows w, w + 8,
-// ..; lane l holds elements E l .. E l + E - 1 of a row (E = D / 32), so a warp
-// reads each row in one coalesced sweep and keeps its 16 rotated rows in
-// registers until the block's amax is known.
+// One CTA per (head, 128-row block) of x: 16 warps, each owning 8 rows; four
+// lanes share a row, lane l holding its elements E q .. E q + E - 1 (q = l mod
+// 4, E = D / 4), so that all but the two widest butterfly strides stay inside
+// a thread (the cross-lane strides go through shuffles, the unit that bounds
+// this kernel).  A warp reads its 8 rows in one coalesced sweep and keeps them
+// in registers until the block's amax is known.  The arithmetic per element
+// and the ascending order of the strides are those of any other layout, so the
+// codes do not depend on it.
 template <int D, bool BF16>
-__global__ void __launch_bounds__(256) attn_fp8_quantize_kernel(
+__global__ void __launch_bounds__(512) attn_fp8_quantize_kernel(
     const uint8_t* __restrict__ x, uint8_t* __restrict__ codes, float* __restrict__ scales,
     const int8_t* __restrict__ signs, int rotate, int N) {
-    constexpr int E = D / 32;
-    constexpr int RPW = 16;  // rows per warp
-    __shared__ float warp_max[8];
+    constexpr int E = D / 4;  // elements per lane
+    __shared__ float warp_max[16];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = lane & 3;  // quarter of the row this lane holds
     const int nb = (N + 127) / 128;
     const int bh = blockIdx.x / nb, blk = blockIdx.x % nb;
-    const int row0 = blk * 128;
-    float sgn[E];
+    const int r = blk * 128 + warp * 8 + (lane >> 2);
+    // bit e: the sign of element E q + e is negative (flipping the sign bit is
+    // the exact product with -1)
+    uint32_t neg = 0u;
+    if (signs != nullptr) {
 #pragma unroll
-    for (int e = 0; e < E; ++e) sgn[e] = (signs != nullptr && signs[lane * E + e] < 0) ? -1.f : 1.f;
-
-    // every row's load is issued before the first is used, so that a warp has
-    // all 16 in flight (the kernel is bound by HBM latency and bandwidth)
-    uint32_t raw[RPW][E / 2];
+        for (int e = 0; e < E; ++e) neg |= (signs[q * E + e] < 0 ? 1u : 0u) << e;
+    }
+    uint32_t raw[E / 2];
 #pragma unroll
-    for (int i = 0; i < RPW; ++i) {
-        const int r = row0 + warp + 8 * i;
+    for (int e = 0; e < E / 2; ++e) raw[e] = 0u;
+    if (r < N) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            x + ((static_cast<size_t>(bh) * N + r) * D + q * E) * 2);
 #pragma unroll
-        for (int e = 0; e < E / 2; ++e) raw[i][e] = 0u;
-        if (r < N) {
-            const size_t off = (static_cast<size_t>(bh) * N + r) * D + lane * E;  // elements
-            if constexpr (E == 4) {
-                const uint2 w = __ldg(reinterpret_cast<const uint2*>(x + off * 2));
-                raw[i][0] = w.x;
-                raw[i][1] = w.y;
-            } else {
-                raw[i][0] = __ldg(reinterpret_cast<const uint32_t*>(x + off * 2));
+        for (int w = 0; w < E / 8; ++w) {
+            const uint4 v = __ldg(src + w);
+            raw[4 * w] = v.x, raw[4 * w + 1] = v.y, raw[4 * w + 2] = v.z, raw[4 * w + 3] = v.w;
+        }
+    }
+    float y[E];
+#pragma unroll
+    for (int e = 0; e < E; e += 2) {
+        const float2 v = unpack2<BF16>(raw[e / 2]);
+        y[e] = __int_as_float(__float_as_int(v.x) ^ static_cast<int>(((neg >> e) & 1u) << 31));
+        y[e + 1] = __int_as_float(__float_as_int(v.y) ^ static_cast<int>(((neg >> (e + 1)) & 1u) << 31));
+    }
+    if (rotate) {
+        // butterflies of stride h < E inside the thread, then strides E and 2 E
+        // with the lane of the same row that differs in bit 0, then bit 1
+#pragma unroll
+        for (int h = 1; h < E; h *= 2)
+#pragma unroll
+            for (int b = 0; b < E; b += 2 * h)
+#pragma unroll
+                for (int j = b; j < b + h; ++j) {
+                    const float a = y[j], c = y[j + h];
+                    y[j] = __fadd_rn(a, c);
+                    y[j + h] = __fsub_rn(a, c);
+                }
+#pragma unroll
+        for (int m = 1; m < 4; m *= 2) {
+            const bool high = (q & m) != 0;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const float other = __shfl_xor_sync(0xffffffffu, y[e], m);
+                y[e] = high ? __fsub_rn(other, y[e]) : __fadd_rn(y[e], other);
             }
         }
     }
-    float y[RPW][E];
     float amax = 0.f;
 #pragma unroll
-    for (int i = 0; i < RPW; ++i) {
-#pragma unroll
-        for (int e = 0; e < E; e += 2) {
-            const float2 v = unpack2<BF16>(raw[i][e / 2]);
-            y[i][e] = v.x * sgn[e];
-            y[i][e + 1] = v.y * sgn[e + 1];
-        }
-        if (rotate) {
-            // butterflies of stride h < E inside the thread, then stride E m
-            // (m = 1 .. 16) with the lane that differs in bit m
-#pragma unroll
-            for (int h = 1; h < E; h *= 2)
-#pragma unroll
-                for (int b = 0; b < E; b += 2 * h)
-#pragma unroll
-                    for (int j = b; j < b + h; ++j) {
-                        const float a = y[i][j], c = y[i][j + h];
-                        y[i][j] = __fadd_rn(a, c);
-                        y[i][j + h] = __fsub_rn(a, c);
-                    }
-#pragma unroll
-            for (int m = 1; m < 32; m *= 2) {
-                const bool high = (lane & m) != 0;
-#pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    const float other = __shfl_xor_sync(0xffffffffu, y[i][e], m);
-                    y[i][e] = high ? __fsub_rn(other, y[i][e]) : __fadd_rn(y[i][e], other);
-                }
-            }
-        }
-#pragma unroll
-        for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(y[i][e]));
-    }
+    for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(y[e]));
 #pragma unroll
     for (int m = 16; m > 0; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
     if (lane == 0) warp_max[warp] = amax;
     __syncthreads();
     amax = warp_max[0];
 #pragma unroll
-    for (int w = 1; w < 8; ++w) amax = fmaxf(amax, warp_max[w]);
+    for (int w = 1; w < 16; ++w) amax = fmaxf(amax, warp_max[w]);
     const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
     if (threadIdx.x == 0) scales[static_cast<size_t>(bh) * nb + blk] = __fdiv_rn(amax, 448.f);
+    if (r >= N) return;
+    uint32_t packed[E / 4];
 #pragma unroll
-    for (int i = 0; i < RPW; ++i) {
-        const int r = row0 + warp + 8 * i;
-        if (r >= N) continue;
-        uint32_t packed = 0;
+    for (int w = 0; w < E / 4; ++w) {
+        uint32_t word = 0u;
 #pragma unroll
-        for (int e = 0; e < E; e += 2) {
+        for (int e = 0; e < 4; e += 2) {
             const __nv_fp8x2_storage_t c = __nv_cvt_float2_to_fp8x2(
-                make_float2(__fmul_rn(y[i][e], inv), __fmul_rn(y[i][e + 1], inv)),
+                make_float2(__fmul_rn(y[4 * w + e], inv), __fmul_rn(y[4 * w + e + 1], inv)),
                 __NV_SATFINITE, __NV_E4M3);
-            packed |= static_cast<uint32_t>(c) << (8 * e);
+            word |= static_cast<uint32_t>(c) << (8 * e);
         }
-        uint8_t* dst = codes + (static_cast<size_t>(bh) * N + r) * D + lane * E;
-        if constexpr (E == 4)
-            *reinterpret_cast<uint32_t*>(dst) = packed;
-        else
-            *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(packed);
+        packed[w] = word;
     }
+    uint4* dst = reinterpret_cast<uint4*>(codes + (static_cast<size_t>(bh) * N + r) * D + q * E);
+#pragma unroll
+    for (int w = 0; w < E / 16; ++w)
+        dst[w] = make_uint4(packed[4 * w], packed[4 * w + 1], packed[4 * w + 2], packed[4 * w + 3]);
 }
 
 }  // namespace attn
