@@ -441,6 +441,34 @@ __global__ void __launch_bounds__(480, 1)
                 reg_fence32(v[1]);
                 tc_fence_before();
                 mbar_arrive(BAR(C::B_DQE));  // the values are in registers: columns free
+                if constexpr (SPARSE) {
+                    // The block-sparse walk keeps the whole 32 KB tile and one
+                    // reduction per tile (measured faster there than the two
+                    // halves below, which are faster on the dense walk).  The
+                    // previous tile's reduction has finished reading the tile.
+                    if (g >= 1 && !(dq_ok = __all_sync(0xffffffffu,
+                                                       wait_bounded(BAR(C::B_STGE), (g - 1) & 1,
+                                                                    abort_flag))))
+                        break;
+#pragma unroll
+                    for (int e = 0; e < 64; ++e)
+                        st_shared_f32(stg + e * 512u, __uint_as_float(v[e >> 5][e & 31]) * p.scale);
+                    fence_proxy_async_smem();
+                    mbar_arrive(BAR(C::B_STGF));
+                    if (issuer) {
+                        if (!wait_bounded(BAR(C::B_STGF), g & 1, abort_flag)) {
+                            dq_ok = false;
+                        } else {
+                            const int nq = min(64, p.N - q0);
+                            bulk_reduce_add_f32(acc_head + static_cast<size_t>(q0) * D,
+                                                base + C::OFF_STG, static_cast<uint32_t>(nq) * 512u);
+                            bulk_commit();
+                            bulk_wait_read_all();
+                            mbar_arrive(BAR(C::B_STGE));
+                            if (it + 1 == n_it) mbar_arrive(BAR(C::B_DQD));  // item's staging done
+                        }
+                    }
+                } else {
                 // The staging tile goes out in two 16 KB halves of 32 queries, each
                 // by its own bulk reduction, so that half 1 is written while half
                 // 0's reduction reads: a half is rewritten once the previous tile's
@@ -480,6 +508,7 @@ __global__ void __launch_bounds__(480, 1)
                 if (dq_ok && issuer && it + 1 == n_it) {
                     bulk_wait_read_all();             // the staging tile is free for
                     mbar_arrive(BAR(C::B_DQD));       // the item's epilogue
+                }
                 }
                 dq_ok = __all_sync(0xffffffffu, dq_ok);
                 if (!dq_ok) break;

@@ -454,6 +454,23 @@ def dq_role(agent, plan, v):
             yield ("wait", [("DQF", g)])
             yield ("read", "DQ", g)
             yield ("arrive", "DQE", g)
+            if SINGLE_STAGING:
+                # the block-sparse instantiation: the whole 32 KB tile, one bulk
+                # reduction, whose read the issuing lane waits for at once
+                if g >= 1:
+                    yield ("wait", [("STGE0", g - 1)])
+                for h in range(2):
+                    yield ("write", ("STG", h), ("dQ", g))
+                yield ("arrive", "STGF0", g)
+                if agent == 0:
+                    yield ("wait", [("STGF0", g)])
+                    for h in range(2):
+                        yield ("read", ("STG", h), ("dQ", g))
+                    yield ("arrive", "STGE0", g)
+                    if it + 1 == n_it:
+                        yield ("arrive", "DQD", item)
+                g += 1
+                continue
             # the staging tile in two 16 KB halves (32 queries each), each sent by
             # its own bulk reduction; agent 0 (the issuing lane) releases a half
             # once the previous tile's reduction of it has read it
@@ -491,13 +508,18 @@ def dq_role(agent, plan, v):
 
 
 W = None  # the world of the schedule being run (the roles read it as a global)
+SINGLE_STAGING = False  # dQ staging as one 32 KB tile (block-sparse) or two halves
 
 
-def run_schedule(plan, seed, variant=None, max_steps=200000, in_order=False):
+def run_schedule(plan, seed, variant=None, max_steps=200000, in_order=False,
+                 single_staging=False):
     """Runs one random schedule of one CTA working through `plan`; raises
     ProtocolError on a violation or a deadlock.  in_order: complete each
-    unit's asynchronous work in issue order (a narrower set of schedules)."""
-    global W
+    unit's asynchronous work in issue order (a narrower set of schedules).
+    single_staging: the block-sparse instantiation's dQ staging (one 32 KB
+    tile per tile, one reduction) instead of the dense one's two halves."""
+    global W, SINGLE_STAGING
+    SINGLE_STAGING = single_staging
     v = variant or Variant()
     W = World()
     counts = {"KVE": 2, "ACCE": NCOMP, "PTF0": NCOMP, "PTF1": NCOMP, "DSF0": NCOMP,

@@ -16,10 +16,13 @@ PLANS = [[1], [2], [5], [3, 1, 4], [1, 1, 1, 1], [2, 2, 2], [4, 3, 2, 1],
          [0], [2, 0, 3], [0, 0, 1, 0], [1, 0, 0, 2, 0]]
 
 
+@pytest.mark.parametrize("single", [False, True], ids=["halves", "single"])
 @pytest.mark.parametrize("plan", PLANS, ids=lambda p: "-".join(map(str, p)))
-def test_protocol_holds_under_random_schedules(plan):
+def test_protocol_holds_under_random_schedules(plan, single):
+    # two dQ staging schemes: two 16 KB halves (dense) and one 32 KB tile
+    # (the block-sparse instantiation)
     for seed in range(120):
-        pm.run_schedule(plan, seed)
+        pm.run_schedule(plan, seed, single_staging=single)
 
 
 def test_earlier_correct_design_also_holds():
