@@ -157,14 +157,14 @@ struct BwdCfg {
     static constexpr int B_KV = 0, B_QF = 1, B_QE = B_QF + QST, B_DOF = B_QE + QST,
                          B_DOE = B_DOF + DOST, B_SF = B_DOE + DOST, B_DPF = B_SF + 1,
                          B_PTF = B_DPF + 1, B_DVD = B_PTF + 1, B_DSF = B_DVD + 1,
-                         B_DQF = B_DSF + 1, B_DQE = B_DQF + 1, B_FIN = B_DQE + 1,
+                         B_DQF = B_DSF + 1, B_DQE = B_DQF + 2, B_FIN = B_DQE + 2,
                          B_DR = B_FIN + 1, B_ENDA = B_DR + 1, B_ENDB = B_ENDA + 1,
                          B_SRD = B_ENDB + 1, NBAR = B_SRD + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
-    static constexpr uint32_t COL_DQ = 384;
+    static constexpr uint32_t COL_DQ = 384;  // two buffers: 384 and 448 (tile parity)
     static constexpr int NCOMPUTE = 256;             // 8 compute warps
     static constexpr int NTHREADS = NCOMPUTE + 64;   // + TMA warp + MMA warp
     static constexpr int WARP_TMA = NCOMPUTE / 32, WARP_MMA = WARP_TMA + 1;
@@ -224,8 +224,10 @@ __global__ void __launch_bounds__(320, 1)
         mbar_init(BAR(C::B_PTF), C::NCOMPUTE);
         mbar_init(BAR(C::B_DVD), 1);
         mbar_init(BAR(C::B_DSF), C::NCOMPUTE);
-        mbar_init(BAR(C::B_DQF), 1);
-        mbar_init(BAR(C::B_DQE), C::NCOMPUTE);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(BAR(C::B_DQF + b), 1);
+            mbar_init(BAR(C::B_DQE + b), C::NCOMPUTE);
+        }
         mbar_init(BAR(C::B_FIN), 1);
         mbar_init(BAR(C::B_DR), 1);
         mbar_init(BAR(C::B_ENDA), C::NCOMPUTE);
@@ -335,9 +337,12 @@ __global__ void __launch_bounds__(320, 1)
                            (it > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(BAR(C::B_DVD));
                 mma_commit(BAR(C::B_DOE + ds));
-                // dK += dS^T Q ; dQ partial
+                // dK += dS^T Q ; dQ partial into buffer it & 1, once its last
+                // contents, dQ(it-2), have been drained
                 if (!(ok = wait_bounded(BAR(C::B_DSF), ph, abort_flag))) break;
-                if (it > 0 && !(ok = wait_bounded(BAR(C::B_DQE), ph ^ 1, abort_flag))) break;
+                if (it >= 2 &&
+                    !(ok = wait_bounded(BAR(C::B_DQE + (it & 1)), ((it >> 1) - 1) & 1, abort_flag)))
+                    break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
@@ -347,11 +352,11 @@ __global__ void __launch_bounds__(320, 1)
                            (it > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)  // dQ = dS K: A = dS^T read MN-major, B = K MN-major
-                    mma_ss(tmem + C::COL_DQ, sdesc_sw128(sDST + kk * 2048u, 16384, 1024),
+                    mma_ss(tmem + C::COL_DQ + (it & 1) * 64u, sdesc_sw128(sDST + kk * 2048u, 16384, 1024),
                            sdesc_sw128(sK + kk * 2048u, 16384, 1024), ID_DQ,
                            kk > 0 ? 1u : 0u);
                 mma_commit(BAR(C::B_QE + qs));
-                mma_commit(BAR(C::B_DQF));
+                mma_commit(BAR(C::B_DQF + (it & 1)));
             }
             if (ok) mma_commit(BAR(C::B_FIN));
             if (*abort_flag) {
@@ -374,6 +379,28 @@ __global__ void __launch_bounds__(320, 1)
         const size_t head_row0 = static_cast<size_t>(bh) * p.N;
         const uint32_t sDST = base + C::OFF_DST;
         const int c0 = half * 64;  // first query column of this thread's half
+        // dQ of tile t (query rows q0p ..): lane r holds query row q0p + r; this
+        // half covers features 32 h .. 32 h + 31
+        auto drain_dq = [&](int t, int q0p) {
+            tc_fence_after();
+            const int qr = q0p + r;
+            float* row = p.dqacc + (head_row0 + qr) * D + half * 32;
+            uint32_t v[32];
+            tmem_ld32(lane_addr + C::COL_DQ + (t & 1) * 64u + half * 32u, v);
+            tmem_ld_wait();
+            reg_fence32(v);
+            tc_fence_before();
+            mbar_arrive(BAR(C::B_DQE + (t & 1)));  // in registers: the buffer is free
+            if (qr < p.N) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    red_add_v4_f32(row + 4 * e, __uint_as_float(v[4 * e]) * p.scale,
+                                   __uint_as_float(v[4 * e + 1]) * p.scale,
+                                   __uint_as_float(v[4 * e + 2]) * p.scale,
+                                   __uint_as_float(v[4 * e + 3]) * p.scale);
+            }
+        };
+        int prev_q0 = 0;
         bool ok = true;
         for (int it = 0, i = next_tile(i_begin); it < n_it; ++it, i = next_tile(i + 1)) {
             const int q0 = i * 128;
@@ -453,8 +480,13 @@ __global__ void __launch_bounds__(320, 1)
             tc_fence_before();
             mbar_arrive(BAR(C::B_PTF));
 
-            // ---- dS^T = P^T (dP^T - D), half, into shared memory
+            // ---- dS^T = P^T (dP^T - D), half, into shared memory, once dK and
+            // dQ of the previous tile have read it (implied by the dP^T commit,
+            // which follows them; kept as a guard)
             ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_DPF), ph, abort_flag));
+            if (ok && it >= 1)
+                ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_DQF + ((it - 1) & 1)),
+                                                          ((it - 1) >> 1) & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
@@ -490,27 +522,15 @@ __global__ void __launch_bounds__(320, 1)
             tc_fence_before();
             mbar_arrive(BAR(C::B_DSF));
 
-            // ---- dQ partial into the fp32 accumulator
-            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_DQF), ph, abort_flag));
-            if (!ok) break;
-            tc_fence_after();
-            // lane r holds query row q0 + r of dQ; this half covers features 32h .. 32h+31
-            const int qr = q0 + r;
-            float* row = p.dqacc + (head_row0 + qr) * D + half * 32;
-            uint32_t v[32];
-            tmem_ld32(lane_addr + C::COL_DQ + half * 32u, v);
-            tmem_ld_wait();
-            reg_fence32(v);
-            if (qr < p.N) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    red_add_v4_f32(row + 4 * e, __uint_as_float(v[4 * e]) * p.scale,
-                                   __uint_as_float(v[4 * e + 1]) * p.scale,
-                                   __uint_as_float(v[4 * e + 2]) * p.scale,
-                                   __uint_as_float(v[4 * e + 3]) * p.scale);
-            }
-            tc_fence_before();
-            mbar_arrive(BAR(C::B_DQE));
+            // ---- dQ of the previous tile into the fp32 accumulator: its product
+            // completed before dS^T(it) was written, so the drain no longer waits
+            if (it >= 1) drain_dq(it - 1, prev_q0);
+            prev_q0 = q0;
+        }
+        if (ok && n_it > 0) {  // the last tile's dQ
+            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_DQF + ((n_it - 1) & 1)),
+                                                      ((n_it - 1) >> 1) & 1, abort_flag));
+            if (ok) drain_dq(n_it - 1, prev_q0);
         }
         if (ok) ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_FIN), 0, abort_flag));
         if (ok) {  // dK_j, dV_j rows: lane r holds key row j*128 + r; this half, D/2 features

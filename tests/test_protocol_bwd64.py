@@ -1,6 +1,5 @@
 """The d = 64 backward kernel's mbarrier protocol on the CPU under random
-schedules (tests/protocol_model_bwd64.py mirrors the kernel's roles): the
-kernel as it is (one work item per CTA), the persistent design for it, and the
+schedules (tests/protocol_model_bwd64.py mirrors the kernel's roles), and the
 checker rejecting mistakes."""
 
 import pytest
@@ -8,40 +7,30 @@ import pytest
 import protocol_model_bwd64 as pm
 
 
-@pytest.mark.parametrize("n_it", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("n_it", [0, 1, 2, 3, 5, 8])
 def test_d64_protocol_holds_under_random_schedules(n_it):
     for seed in range(150):
         pm.run_schedule(n_it, seed)
 
 
-@pytest.mark.parametrize("plan", [[3, 1, 4], [1, 1, 1, 1], [2, 5, 2], [8, 1]],
-                         ids=lambda p: "-".join(map(str, p)))
-def test_persistent_d64_design_holds(plan):
-    for seed in range(100):
-        pm.run_schedule(plan, seed)
-
-
-def test_persistent_d64_static_item_order_holds():
-    # without the mask the items are dealt in a fixed order: no response slots
-    for seed in range(100):
-        pm.run_schedule([3, 1, 4, 2], seed, pm.Variant(static_items=True))
-
-
-def test_accumulator_release_is_implied_by_the_role_order():
-    for seed in range(150):
-        pm.run_schedule([3, 2, 4, 1], seed, pm.Variant(no_acce=True))
-
-
 @pytest.mark.parametrize("mistake", ["no_srd", "no_dsf_wait", "flag_without_endb"])
-@pytest.mark.parametrize("plan", [5, [3, 2, 4, 1]], ids=["one-item", "persistent"])
-def test_checker_rejects_d64_mistakes(mistake, plan):
+def test_checker_rejects_d64_mistakes(mistake):
     caught = 0
     for seed in range(300):
         try:
-            pm.run_schedule(plan, seed, pm.Variant(**{mistake: True}))
+            pm.run_schedule(5, seed, pm.Variant(**{mistake: True}))
         except pm.ProtocolError:
             caught += 1
-    assert caught > 0
+    assert caught > 0, f"{mistake} was never caught"
+
+
+@pytest.mark.parametrize("skipped", ["ds_without_dqf_wait", "dq_without_dqe_wait"])
+def test_two_waits_are_implied_by_the_issue_order(skipped):
+    """The kernel keeps two waits of the deferred dQ drain that the order makes
+    redundant (see Variant); skipping either alone is never caught.  They stay
+    as guards against a reordering."""
+    for seed in range(150):
+        pm.run_schedule(5, seed, pm.Variant(**{skipped: True}))
 
 
 def test_next_s_needs_the_dv_wait_although_issued_later():
