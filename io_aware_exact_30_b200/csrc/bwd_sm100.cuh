@@ -184,9 +184,13 @@ __global__ void __launch_bounds__(320, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Work item: head-major, the heaviest key tile (j = 0 under the causal mask) first.
-    const int bh = static_cast<int>(blockIdx.x) / p.n_ktiles;
-    const int j = static_cast<int>(blockIdx.x) % p.n_ktiles;
+    // Work item: under the causal mask key-tile-major, every head's heaviest key
+    // tile (j = 0) first, so that the CTAs launched last are the light ones;
+    // otherwise head-major.
+    const int bh = p.causal ? static_cast<int>(blockIdx.x) % p.BH
+                            : static_cast<int>(blockIdx.x) / p.n_ktiles;
+    const int j = p.causal ? static_cast<int>(blockIdx.x) / p.BH
+                           : static_cast<int>(blockIdx.x) % p.n_ktiles;
     const int i_begin = p.causal ? j : 0;
     // Query tiles i = i_begin .., and under a block mask only those marked for
     // key tile j; every role walks the same sequence (next_tile).
