@@ -464,10 +464,10 @@ int attn_linear_fwd(const void* q, const void* k, const void* v, void* o, void* 
         const unsigned gf = static_cast<unsigned>(2 * BH);
         if (dtype == ATTN_BF16)
             attn::linear_fused_kernel<true>
-                <<<gf, 320, attn::LinFusedCfg::SMEM_BYTES, st>>>(mq, mk, mv, p);
+                <<<gf, attn::LinFusedCfg::NTHREADS, attn::LinFusedCfg::SMEM_BYTES, st>>>(mq, mk, mv, p);
         else
             attn::linear_fused_kernel<false>
-                <<<gf, 320, attn::LinFusedCfg::SMEM_BYTES, st>>>(mq, mk, mv, p);
+                <<<gf, attn::LinFusedCfg::NTHREADS, attn::LinFusedCfg::SMEM_BYTES, st>>>(mq, mk, mv, p);
         return launch_ok() ? ATTN_OK : ATTN_ERR_LAUNCH;
     }
     if (!make_map(&ms, p.state, dtype, static_cast<int>(items), 128, 128)) return ATTN_ERR_LAUNCH;

@@ -301,16 +301,24 @@ __global__ void __launch_bounds__(192, 1)
 //   A_c  = Q_c K_c^T                tensor memory, two buffers (c % 2)
 //   KV_c = K_c^T V_c,h              tensor memory, two buffers
 //   P_c  = scale (A_c o M)          the row warps, written over A_c
-//   O_c  = Q_c S_{c-1} + P_c V_c,h  tensor memory; S_{c-1} from shared memory
+//   O_c  = Q_c S_{c-1} + P_c V_c,h  tensor memory, two buffers; S_{c-1} from
+//                                   shared memory
 // The state S_c = scale * sum_{c' <= c} KV_c' is kept in fp32 registers by the
 // state warps (thread = feature of K = tensor-memory lane), which add KV_c
 // and store S_c rounded to the 16-bit type into one of two shared buffers,
 // the B operand of the next chunk's Q S.  The sums are the ones the
 // three-kernel form makes, in the same order.
-// Roles (320 threads): warp 0 TMA producer, warp 1 tensor-memory owner and
-// MMA issuer, warps 2-5 mask/scale A into P and store O (thread = row of the
-// chunk), warps 6-9 the state.  Tensor memory: A at 0 and 128, O at 256, KV
-// at 320 and 384.
+// Issue order per chunk c: A_c and KV_c (once the chunk has landed), Q_c
+// S_{c-1}, then P_c V once P_c is written; the next chunk's loads have the
+// whole chunk to land.  O has two buffers and the row warps write P_c before
+// they read O_{c-1}, so no product waits for an output to be read.
+// Roles (448 threads): warp 0 TMA producer, warp 1 tensor-memory owner and
+// MMA issuer, warps 2-9 mask/scale A into P and store O (thread = row of the
+// chunk; warps 2-5 take keys 0-63 of P and features 0-31 of O, warps 6-9
+// keys 64-127 and features 32-63), warps 10-13 the state.  Each half of the
+// row warps packs its 64 keys of P over the first 32 of its own 64 columns
+// of A (columns 0-31 and 64-95), which it has read.  Tensor memory: A at 0
+// and 128, O at 256 and 320, KV at 384 and 448.
 // The fused form is chosen from this many heads (B H) on: with fewer, its
 // grid of 2 B H CTAs, each walking every chunk in turn, leaves most SMs idle
 // and the three chunk-parallel kernels are faster.
@@ -325,16 +333,19 @@ struct LinFusedCfg {
     static constexpr uint32_t OFF_BAR = OFF_S + 2 * VH;
     static constexpr int B_LD = 0, B_KE = B_LD + ST, B_AF = B_KE + ST, B_PF = B_AF + 2,
                          B_PVD = B_PF + 2, B_KVF = B_PVD + 2, B_KVE = B_KVF + 2,
-                         B_SSF = B_KVE + 2, B_SE = B_SSF + 2, B_OD = B_SE + 2, B_OE = B_OD + 1,
-                         B_DR = B_OE + 1, NBAR = B_DR + 1;
+                         B_SSF = B_KVE + 2, B_SE = B_SSF + 2, B_OD = B_SE + 2, B_OE = B_OD + 2,
+                         B_DR = B_OE + 2, NBAR = B_DR + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
-    static constexpr uint32_t COL_O = 256, COL_KV = 320;
+    static constexpr uint32_t COL_O = 256, COL_KV = 384;
+    static constexpr int NROW = 256, NSTATE = 128;    // row and state threads
+    static constexpr int NTHREADS = 64 + NROW + NSTATE;
+    static constexpr int WARP_STATE = 2 + NROW / 32;
     static_assert(SMEM_BYTES <= 232448u, "dynamic shared memory above the sm_100 per-block limit");
 };
 
 template <bool BF16>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(448, 1)
     linear_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const LinearParams p) {
     using C = LinFusedCfg;
@@ -356,15 +367,15 @@ __global__ void __launch_bounds__(320, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(LBAR(C::B_AF + b), 1);
-            mbar_init(LBAR(C::B_PF + b), 128);
+            mbar_init(LBAR(C::B_PF + b), C::NROW);
             mbar_init(LBAR(C::B_PVD + b), 1);
             mbar_init(LBAR(C::B_KVF + b), 1);
-            mbar_init(LBAR(C::B_KVE + b), 128);
-            mbar_init(LBAR(C::B_SSF + b), 128);
+            mbar_init(LBAR(C::B_KVE + b), C::NSTATE);
+            mbar_init(LBAR(C::B_SSF + b), C::NSTATE);
             mbar_init(LBAR(C::B_SE + b), 1);
+            mbar_init(LBAR(C::B_OD + b), 1);
+            mbar_init(LBAR(C::B_OE + b), C::NROW);
         }
-        mbar_init(LBAR(C::B_OD), 1);
-        mbar_init(LBAR(C::B_OE), 128);
         mbar_init(LBAR(C::B_DR), 1);
         *abort_flag = 0u;
         fence_mbar_init();
@@ -430,32 +441,33 @@ __global__ void __launch_bounds__(320, 1)
                     mma_ss(tmem + C::COL_KV + 64u * b, sdesc_sw128(sk + kk * 2048u, 16384, 1024),
                            sdesc_sw128(sv + kk * 2048u, 16384, 1024), ID_KV, kk > 0 ? 1u : 0u);
                 mma_commit(LBAR(C::B_KVF + b));
-                // O_c = Q_c S_{c-1}: the epilogue has read O_{c-1}, and the state
-                // warps have stored S_{c-1} (buffer (c - 1) & 1)
+                // O_c = Q_c S_{c-1} into O buffer b: the row warps have read O_{c-2}
+                // from it, and the state warps have stored S_{c-1} (buffer (c - 1) & 1)
                 if (c >= 1) {
                     const int bp = (c - 1) & 1, up = (c - 1) >> 1;
-                    if (!(ok = wait3(LBAR(C::B_OE), (c - 1) & 1, true, LBAR(C::B_SSF + bp), up & 1,
-                                     true, 0u, 0u, false, abort_flag)))
+                    if (!(ok = wait3(LBAR(C::B_OE + b), (u - 1) & 1, c >= 2, LBAR(C::B_SSF + bp),
+                                     up & 1, true, 0u, 0u, false, abort_flag)))
                         break;
                     tc_fence_after();
                     const uint32_t ss = base + C::OFF_S + bp * C::VH;
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {  // B = S rows (features of K)
                         const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                        mma_ss(tmem + C::COL_O, sdesc_sw128(sq + off, 16, 1024),
+                        mma_ss(tmem + C::COL_O + 64u * b, sdesc_sw128(sq + off, 16, 1024),
                                sdesc_sw128(ss + kk * 2048u, 16384, 1024), ID_O, kk > 0 ? 1u : 0u);
                     }
                     mma_commit(LBAR(C::B_SE + bp));  // S buffer bp may be rewritten
                 }
-                // O_c += P_c V_c,h once the row warps have written P_c
+                // O_c += P_c V_c,h once the row warps have written P_c: keys 0-63
+                // packed at columns 0-31 of A buffer b, keys 64-127 at 64-95
                 if (!(ok = wait_bounded(LBAR(C::B_PF + b), u & 1, abort_flag))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)  // K-dim: 16 tokens per step
-                    mma_ts(tmem + C::COL_O, tmem + 128u * b + kk * 8u,
+                    mma_ts(tmem + C::COL_O + 64u * b, tmem + 128u * b + kk * 8u + (kk >> 2) * 32u,
                            sdesc_sw128(sv + kk * 2048u, 16384, 1024), ID_O,
                            (c >= 1 || kk > 0) ? 1u : 0u);
-                mma_commit(LBAR(C::B_OD));
+                mma_commit(LBAR(C::B_OD + b));
                 mma_commit(LBAR(C::B_PVD + b));
                 mma_commit(LBAR(C::B_KE + s));
             }
@@ -465,10 +477,39 @@ __global__ void __launch_bounds__(320, 1)
             }
         }
         __syncwarp();
-    } else if (warp < 6) {
+    } else if (warp < C::WARP_STATE) {
         // ----------------------------------------- P and the output (rows)
+        const int hc = (warp - 2) >> 2;        // keys 64 hc.. of P, features 32 hc.. of O
         const int r = (warp & 3) * 32 + lane;  // row of the chunk == TMEM lane
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        // O_c (this half's 32 features) to the output rows; the buffer is
+        // released as soon as the values are in registers
+        auto store_o = [&](int c) -> bool {
+            const int b = c & 1;
+            if (!__all_sync(0xffffffffu, wait_bounded(LBAR(C::B_OD + b), (c >> 1) & 1, abort_flag)))
+                return false;
+            tc_fence_after();
+            uint32_t v[32];
+            tmem_ld32(lane_addr + C::COL_O + 64u * b + 32u * hc, v);
+            tmem_ld_wait();
+            reg_fence32(v);
+            tc_fence_before();
+            mbar_arrive(LBAR(C::B_OE + b));
+            const int row = c * 128 + r;
+            if (row < p.N) {
+                uint32_t o16[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    o16[e] = pack2<BF16>(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+                uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.o) +
+                                                      (static_cast<size_t>(bh) * p.N + row) * 256 +
+                                                      h * 128 + hc * 64);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    dst[e] = make_uint4(o16[4 * e], o16[4 * e + 1], o16[4 * e + 2], o16[4 * e + 3]);
+            }
+            return true;
+        };
         bool ok = true;
         for (int c = 0; ok && c < nc; ++c) {
             const int b = c & 1, u = c >> 1;
@@ -476,49 +517,27 @@ __global__ void __launch_bounds__(320, 1)
             if (!ok) break;
             tc_fence_after();
             // P_ij = scale A_ij for j <= i (rows and keys past N are zero already)
+            const uint32_t col = 128u * b + 64u * hc;
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
+            for (int cc = 0; cc < 2; ++cc) {
                 uint32_t v[32], pk[16];
-                tmem_ld32(lane_addr + 128u * b + cc * 32u, v);
+                tmem_ld32(lane_addr + col + cc * 32u, v);
                 tmem_ld_wait();
                 reg_fence32(v);
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const int j0 = cc * 32 + 2 * e;
+                    const int j0 = hc * 64 + cc * 32 + 2 * e;
                     pk[e] = pack2<BF16>(j0 <= r ? __uint_as_float(v[2 * e]) * p.scale : 0.f,
                                         j0 + 1 <= r ? __uint_as_float(v[2 * e + 1]) * p.scale : 0.f);
                 }
-                tmem_st16(lane_addr + 128u * b + cc * 16u, pk);  // over columns already read
+                tmem_st16(lane_addr + col + cc * 16u, pk);  // over columns already read
             }
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(LBAR(C::B_PF + b));
-            ok = __all_sync(0xffffffffu, wait_bounded(LBAR(C::B_OD), c & 1, abort_flag));
-            if (!ok) break;
-            tc_fence_after();
-            const int row = c * 128 + r;
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.o) +
-                                                  (static_cast<size_t>(bh) * p.N + row) * 256 + h * 128);
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                uint32_t v[32];
-                tmem_ld32(lane_addr + C::COL_O + cc * 32u, v);
-                tmem_ld_wait();
-                reg_fence32(v);
-                uint32_t o16[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    o16[e] = pack2<BF16>(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
-                if (row < p.N) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        dst[cc * 4 + e] =
-                            make_uint4(o16[4 * e], o16[4 * e + 1], o16[4 * e + 2], o16[4 * e + 3]);
-                }
-            }
-            tc_fence_before();
-            mbar_arrive(LBAR(C::B_OE));  // O_c has been read
+            if (c >= 1) ok = store_o(c - 1);
         }
+        if (ok && nc > 0) store_o(nc - 1);
     } else {
         // ------------------------------------------------------ the state
         const int a = (warp & 3) * 32 + lane;  // feature of K == TMEM lane == row of S

@@ -15,8 +15,17 @@ def test_linear_protocol_holds_under_random_schedules(nc):
         pl.run_schedule(nc, seed)
 
 
-@pytest.mark.parametrize("mistake", ["no_oe_wait", "no_ssf_wait"])
+@pytest.mark.parametrize("nc", [1, 2, 5])
+def test_linear_protocol_holds_in_issue_order(nc):
+    for seed in range(20):
+        pl.run_schedule(nc, seed, in_order=True)
+
+
+@pytest.mark.parametrize("mistake", ["no_oe_wait", "no_ssf_wait", "no_od_wait", "contiguous_p"])
 def test_checker_rejects_linear_mistakes(mistake):
+    """The output and state waits are needed, and so is the P layout: the
+    upper key half packing P next to the lower half's would overwrite columns
+    the lower half may not have read."""
     caught = 0
     for seed in range(300):
         try:
@@ -30,10 +39,11 @@ def test_checker_rejects_linear_mistakes(mistake):
 def test_three_waits_are_implied_by_the_issue_order(skipped):
     """The kernel keeps three waits that the current order makes redundant:
     the state warps' wait before overwriting a state buffer (the KV-full
-    commit they waited on follows the Q S that read it), the issuer's waits
-    for a KV buffer to be read (the state stored after that read was waited
-    for one chunk earlier) and for P V of two chunks back (the output read
-    after it was waited for one chunk earlier).  Skipping any of them alone
-    is never caught; they stay as a guard against a reordering."""
+    commit they waited on follows the Q S that read it), the issuer's wait for
+    a KV buffer to be read (the state stored after that read was waited for
+    one chunk earlier) and its wait for the P V of two chunks back (the same
+    commit released the Q/K/V stage whose new loads it waits for).  Skipping
+    any of them alone is never caught; they stay as a guard against a
+    reordering."""
     for seed in range(150):
         pl.run_schedule(6, seed, pl.Variant(**{skipped: True}))
