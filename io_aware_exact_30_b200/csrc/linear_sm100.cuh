@@ -311,7 +311,7 @@ __global__ void __launch_bounds__(192, 1)
 // Issue order per chunk c: A_c and KV_c (once the chunk has landed), Q_c
 // S_{c-1}, then P_c V once P_c is written; the next chunk's loads have the
 // whole chunk to land.  O has two buffers and the row warps write P_c before
-// they read O_{c-1}, so no product waits for an output to be read.
+// they read O_{c-1}, so Q_c S_{c-1} waits only for O_{c-2} to have been read.
 // Roles (448 threads): warp 0 TMA producer, warp 1 tensor-memory owner and
 // MMA issuer, warps 2-9 mask/scale A into P and store O (thread = row of the
 // chunk; warps 2-5 take keys 0-63 of P and features 0-31 of O, warps 6-9
