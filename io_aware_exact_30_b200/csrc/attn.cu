@@ -588,11 +588,11 @@ int attn_bwd_dropout(const void* q, const void* k, const void* v, const void* o,
                      int H, int N, int d, int causal, float scale, float dropout_p,
                      unsigned long long seed, attn_dtype_t dtype, void* stream) {
     const void* ptrs[10] = {q, k, v, o, lse, dout, dq, dk, dv, workspace};
-    int dev;
-    int rc = bwd_common_checks(ptrs, 10, workspace, B, H, N, d, dtype, scale, &dev);
+    attn::DropoutParams dp;  // the scalar first, as in attn_fwd_dropout
+    int rc = dropout_params(dropout_p, seed, &dp);
     if (rc) return rc;
-    attn::DropoutParams dp;
-    if ((rc = dropout_params(dropout_p, seed, &dp))) return rc;
+    int dev;
+    if ((rc = bwd_common_checks(ptrs, 10, workspace, B, H, N, d, dtype, scale, &dev))) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if ((rc = bwd_prep_dispatch(o, dout, lse, workspace, B, H, N, d, dtype, st))) return rc;
     return bwd_main_dispatch(q, k, v, dout, dq, dk, dv, workspace, B, H, N, d, causal, scale,
