@@ -113,3 +113,20 @@ def test_weak_scaling_helpers():
     # whole-job TFLOP/s: every rank's FLOPs over the slowest rank's time
     assert bench.job_tflops(1e12, 4, 2.0) == pytest.approx(2000.0)
     assert len({bench.rank_seed(7, r) for r in range(8)}) == 8
+
+
+def test_reference_arm_line():
+    """--impl reference: the oracle times a bounded sample on the host (rank 0
+    only) and the line carries the contract's keys."""
+    import argparse
+    args = argparse.Namespace(workload="tiny", passes=None, steps=1, warmup=3)
+    assert bench.run_reference(args, 1, 2) is None
+    line = bench.run_reference(args, 0, 1)
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["value"] > 0 and line["unit"] == "TFLOP/s" and line["higher_is_better"]
+    assert line["ms_per_step"] > 0 and line["sample_ms_per_step"] > 0
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"]
+    assert cb["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s",
+                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
