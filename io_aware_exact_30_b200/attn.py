@@ -484,3 +484,86 @@ def linear_forward(q, k, v, scale: float | None = None):
                      device=q.device)
     attn_linear_fwd(q, k, v, o, ws, scale)
     return o
+
+
+# ------------------------------------------------------------ several GPUs --
+# Every (batch, head) pair is independent in both passes, so one problem's heads
+# split across the ranks of a process group (one GPU each) with no exchange:
+# each rank runs the single-GPU calls above on a contiguous range of the
+# flattened B*H heads.  The one collective is an optional all-gather of the
+# outputs, for callers that want the whole tensors on every rank.  (Dropout is
+# not offered here: its random bytes are keyed by the head index within the
+# call, so a rank's slice would draw other bytes than the whole call.)
+
+def head_shard(BH: int, rank: int, world: int) -> tuple[int, int]:
+    """(first head, number of heads) of rank `rank` among `world` for B*H = BH
+    flattened heads: contiguous ranges, the first BH % world ranks one head more."""
+    if world < 1 or not 0 <= rank < world or BH < 0:
+        raise ValueError("need 0 <= rank < world and BH >= 0")
+    base, extra = divmod(BH, world)
+    return rank * base + min(rank, extra), base + (1 if rank < extra else 0)
+
+
+def _heads(x, s, n):
+    """Heads [s, s + n) of a (B, H, ...) tensor as a contiguous (1, n, ...) view."""
+    B, H = x.shape[0], x.shape[1]
+    return x.reshape(B * H, *x.shape[2:])[s:s + n].unsqueeze(0)
+
+
+def _gather_heads(parts, shape, s_n, group):
+    """All-gather every rank's (1, n_r, ...) slice into one (B, H, ...) tensor;
+    uneven counts are padded to the largest for the collective."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    m = max(n for _, n in s_n)
+    outs = []
+    for part in parts:
+        pad = part.new_zeros((1, m) + tuple(part.shape[2:]))
+        pad[:, :part.shape[1]] = part
+        bufs = [torch.empty_like(pad) for _ in range(world)]
+        dist.all_gather(bufs, pad, group=group)
+        full = torch.cat([b[0, :n] for b, (_, n) in zip(bufs, s_n)], dim=0)
+        outs.append(full.reshape(shape[:2] + tuple(part.shape[2:])))
+    return outs
+
+
+def forward_sharded(q, k, v, causal: bool = False, scale: float | None = None, group=None,
+                    gather: bool = True):
+    """The forward of (B, H, N, d) q, k, v (the same on every rank of `group`)
+    split by heads: this rank computes its head_shard() range with attn_fwd.
+    gather=True returns the whole (o, lse) on every rank (one all-gather each);
+    gather=False returns this rank's (o, lse) of shape (1, n, N, d) and (1, n, N)
+    and its (first head, count)."""
+    import torch.distributed as dist
+    B, H, N, d = _shape(q)
+    world, rank = dist.get_world_size(group), dist.get_rank(group)
+    s_n = [head_shard(B * H, r, world) for r in range(world)]
+    s, n = s_n[rank]
+    if n > 0:
+        o, lse = forward(_heads(q, s, n), _heads(k, s, n), _heads(v, s, n), causal, scale)
+    else:
+        o = q.new_empty((1, 0, N, d))
+        lse = torch.empty((1, 0, N), dtype=torch.float32, device=q.device)
+    if not gather:
+        return o, lse, (s, n)
+    o, lse = _gather_heads([o, lse], (B, H), s_n, group)
+    return o, lse
+
+
+def backward_sharded(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None,
+                     group=None, gather: bool = True):
+    """The backward split by heads as forward_sharded: this rank runs attn_bwd on
+    its head range; gather=True returns the whole (dq, dk, dv) on every rank,
+    gather=False this rank's slices and its (first head, count)."""
+    import torch.distributed as dist
+    B, H, N, d = _shape(q)
+    world, rank = dist.get_world_size(group), dist.get_rank(group)
+    s_n = [head_shard(B * H, r, world) for r in range(world)]
+    s, n = s_n[rank]
+    if n > 0:
+        grads = backward(*(_heads(x, s, n) for x in (q, k, v, o, lse, dout)), causal, scale)
+    else:
+        grads = tuple(x.new_empty((1, 0, N, d)) for x in (q, k, v))
+    if not gather:
+        return (*grads, (s, n))
+    return tuple(_gather_heads(list(grads), (B, H), s_n, group))
