@@ -490,7 +490,8 @@ def linear_forward(q, k, v, scale: float | None = None):
 # Every (batch, head) pair is independent in both passes, so one problem's heads
 # split across the ranks of a process group (one GPU each) with no exchange:
 # each rank runs the single-GPU calls above on a contiguous range of the
-# flattened B*H heads.  The one collective is an optional all-gather of the
+# flattened B*H heads (views of the inputs; an LSE slice that would not be
+# 16-byte aligned is copied).  The one collective is an optional all-gather of the
 # outputs, for callers that want the whole tensors on every rank.  (Dropout is
 # not offered here: its random bytes are keyed by the head index within the
 # call, so a rank's slice would draw other bytes than the whole call.)
@@ -505,9 +506,12 @@ def head_shard(BH: int, rank: int, world: int) -> tuple[int, int]:
 
 
 def _heads(x, s, n):
-    """Heads [s, s + n) of a (B, H, ...) tensor as a contiguous (1, n, ...) view."""
+    """Heads [s, s + n) of a (B, H, ...) tensor as a contiguous (1, n, ...) tensor:
+    a view, or a copy where the view would not start on the 16-byte boundary the
+    ABI requires (an fp32 LSE slice when s * N is not a multiple of 4)."""
     B, H = x.shape[0], x.shape[1]
-    return x.reshape(B * H, *x.shape[2:])[s:s + n].unsqueeze(0)
+    view = x.reshape(B * H, *x.shape[2:])[s:s + n].unsqueeze(0)
+    return view if view.data_ptr() % 16 == 0 else view.clone()
 
 
 def _gather_heads(parts, shape, s_n, group):

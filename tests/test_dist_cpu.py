@@ -63,13 +63,19 @@ def _sharded_worker(rank, world, port, out):
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        # stand-ins for the single-GPU calls (test doubles: no GPU here)
+        # stand-ins for the single-GPU calls (test doubles: no GPU here), which
+        # also hold the ABI's rule that every pointer is 16-byte aligned
+        def aligned(*xs):
+            assert all(x.data_ptr() % 16 == 0 and x.is_contiguous() for x in xs)
+
         def fwd(q, k, v, causal, scale):
+            aligned(q, k, v)
             o, lse = oracle.fwd(q.double().numpy(), k.double().numpy(), v.double().numpy(),
                                 causal, scale)
             return torch.from_numpy(o).float(), torch.from_numpy(lse).float()
 
         def bwd(q, k, v, o, lse, do, causal, scale):
+            aligned(q, k, v, o, lse, do)
             g = oracle.bwd(*(x.double().numpy() for x in (q, k, v, do)), causal, scale)
             return tuple(torch.from_numpy(x).float() for x in g)
 
