@@ -141,6 +141,32 @@ def kernel_traffic(kernels):
     return total
 
 
+def l2_text(working_set):
+    """How a workload keeps L2 from serving its inputs between timed steps."""
+    if working_set >= 2 * L2_BYTES:
+        return "inputs larger than L2 (working set %.0f MB)" % (working_set / 1e6)
+    return "L2 flushed between steps (256 MB write, outside the per-step events)"
+
+
+def run_config(workload, passes, world):
+    """The `config` object of a line, the same for both arms: the workload, its
+    FLOPs per step and how it is measured on the GPU."""
+    B, H, N, d, causal, _, _, default_passes = WORKLOADS[workload]
+    f_fwd, f_bwd = workload_flops(workload)
+    # device inputs (q, k, v, and dO for the backward) plus O, 16-bit each
+    working_set = ((4 if passes == "fwdbwd" else 3) + 1) * B * H * N * d * 2
+    return {
+        "workload": DESCRIPTION[workload] + ("" if passes == default_passes else f" ({passes} only)"),
+        "B": B, "H": H, "N": N, "d": d, "causal": causal, "passes": passes,
+        "flop_per_step": f_fwd + (f_bwd if passes == "fwdbwd" else 0.0),
+        "flop_convention": "fwd 4BHN^2d, bwd 10BHN^2d, halved when causal",
+        "l2": l2_text(working_set),
+        "timing": "ms_per_step = median over the timed steps of per-step CUDA events "
+                  "(max over ranks); ms_bracket_mean = barrier-to-barrier events / steps",
+        "parallelism": f"dp{world} (independent heads per rank, no collective)",
+    }
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -307,9 +333,7 @@ class DeviceRun:
         self.n_events = 4 if passes == "fwdbwd" else 2
 
     def l2_note(self):
-        if self.flush is None:
-            return "inputs larger than L2 (working set %.0f MB)" % (self.working_set / 1e6)
-        return "L2 flushed between steps (256 MB write, outside the per-step events)"
+        return l2_text(self.working_set)
 
     def step(self, evs=None):
         a, st = self.attn, self.stream
@@ -577,6 +601,8 @@ def run_ours(args, rank, world, local_rank):
 
     f_fwd, f_bwd = workload_flops(args.workload)
     f_step = f_fwd + (f_bwd if passes == "fwdbwd" else 0.0)
+    config = run_config(args.workload, passes, world)
+    config["l2"] = l2_note  # the run's own buffers (the same sizes run_config counts)
     value = job_tflops(f_step, world, max_step_ms)
     burst, sustained, hbm, src = peaks()
     roof, kern = roofline_entry(d, passes, f_fwd, f_bwd, fwd_ms, main_ms, None)
@@ -594,16 +620,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": dtype,
         "data": "synthetic (seeded splitmix64/Box-Muller, N(0, sigma^2), rounded to %s)" % dtype,
-        "config": {
-            "workload": DESCRIPTION[args.workload] + ("" if passes == WORKLOADS[args.workload][7] else f" ({passes} only)"),
-            "B": B, "H": H, "N": N, "d": d, "causal": causal, "passes": passes,
-            "flop_per_step": f_step,
-            "flop_convention": "fwd 4BHN^2d, bwd 10BHN^2d, halved when causal",
-            "l2": l2_note,
-            "timing": "ms_per_step = median over the timed steps of per-step CUDA events "
-                      "(max over ranks); ms_bracket_mean = barrier-to-barrier events / steps",
-            "parallelism": f"dp{world} (independent heads per rank, no collective)",
-        },
+        "config": config,
         "ms_bracket_mean": round(max_bracket_ms / args.steps, 4),
         "fwd_tflops": round(f_fwd / (fwd_ms * 1e-3) / 1e12, 2),
         "fwd_ms": round(fwd_ms, 4),
@@ -726,8 +743,7 @@ def run_reference(args, rank, world):
         "sample_ms_per_step": round(1e3 * statistics.mean(v["seconds"] for v in vals), 1),
         "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": DESCRIPTION[args.workload], "B": B, "H": H, "N": N, "d": d,
-                   "causal": causal, "passes": passes},
+        "config": run_config(args.workload, passes, world),
         "cpu_baseline": cb,
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},

@@ -130,3 +130,13 @@ def test_reference_arm_line():
     assert cb["value"] == line["value"]
     assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s",
                            "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    # the same config object as the GPU arm's line for this workload
+    assert line["config"] == bench.run_config("tiny", bench.WORKLOADS["tiny"][7], 1)
+
+
+def test_config_of_the_headline():
+    c = bench.run_config("large_head", "fwdbwd", 1)
+    assert (c["B"], c["H"], c["N"], c["d"], c["causal"]) == (4, 16, 4096, 128, True)
+    assert c["flop_per_step"] == sum(bench.flops(4, 16, 4096, 128, True))
+    assert c["l2"] == "inputs larger than L2 (working set 336 MB)"
+    assert bench.run_config("tiny", "fwd", 1)["l2"].startswith("L2 flushed")
