@@ -97,3 +97,20 @@ def test_every_entry_point_checks_its_arguments_before_device_work():
         assert calls["attn_fwd_dropout"]() == -9, bad
         assert calls["attn_bwd_dropout"]() == -9, bad
     assert L.attn_linear_fwd(p, p, p, p, p, 1, 1, 16, 64, 0.125, 0, None) == -3
+
+
+def test_linear_and_host_entry_sizes():
+    """Host-side size queries: linear attention keeps per (head, chunk of 128
+    rows) a 128 x 128 fp32 K^T V and a 16-bit state (d = 128 only); the host
+    entry's scratch grows with the chunk of heads and with the backward."""
+    def a256(x):
+        return (x + 255) // 256 * 256
+    for B, H, N in ((1, 1, 128), (1, 1, 1), (2, 3, 300), (4, 16, 4096)):
+        states = B * H * -(-N // 128) * 128 * 128
+        assert attn.attn_linear_workspace_bytes(B, H, N, 128) == a256(4 * states) + a256(2 * states)
+    assert attn.attn_linear_workspace_bytes(1, 1, 128, 64) == 0
+    assert attn.attn_linear_workspace_bytes(1, 0, 128, 128) == 0
+    f = attn.attn_sdpa_host_scratch_bytes
+    assert f(4, 16, 4096, 128, 1, 0) > f(4, 16, 4096, 128, 0, 0) > 0
+    assert f(4, 16, 4096, 128, 1, 16) > f(4, 16, 4096, 128, 1, 8) > f(4, 16, 4096, 128, 1, 1)
+    assert f(4, 16, 4096, 96, 1, 0) == 0 and f(0, 16, 4096, 128, 1, 0) == 0
